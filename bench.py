@@ -1,0 +1,366 @@
+"""Benchmark of the HySparse2 hybrid-block hot path on B200.
+
+One step = one decode step of a hybrid block for a batch of 32 sequences at a
+131,072-token bf16 MQA cache (16 query heads, head_dim 128): the full-attention
+layer with head-summed importance and token-level top-1024 + window-128
+selection, then 3 sparse-attention layers that reuse the cache and indices.
+Inputs are synthetic (seeded, planted needles) and resident in HBM; the 2 GiB
+cache per GPU is larger than L2, so no flush is needed between steps.
+
+`value` is sparse-attention decode queries per second over the whole step
+(batch x 3 sparse layers per step); the full-attention and sparse layers are
+also reported separately with their HBM roofline fractions.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch with torchrun: every rank runs an independent replica (the
+path has no exchange step), timing is the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "sparse-attn decode queries/s @128K ctx + prefill tokens/s; % HBM & TC roofline"
+FALLBACK_HBM_GBS = 6650.0
+# dram__bytes_read.sum + dram__bytes_write.sum of one hs2_full_attn_select call on the
+# decode workload, scaled from the ncu capture summarised in profiles/ (None until
+# captured for the current kernels).
+FULL_CALL_TRAFFIC_BYTES = None
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("bf16_tflops", 1590.0)), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def _barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def _max_over_ranks(ws, x):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+class DecodeBlock:
+    """Device buffers and C-ABI calls of one decode step of the hybrid block."""
+
+    def __init__(self, wl, seed):
+        import kv_shared_b200 as hs
+        self.hs = hs
+        self.wl = wl
+        inp = synth.make_inputs(wl, seed=seed, device="cuda")
+        self.q = inp.q_full.contiguous()
+        self.qs = [x.contiguous() for x in inp.q_sparse]
+        self.k, self.v = inp.k.contiguous(), inp.v.contiguous()
+        del inp
+        B, H, D = wl.batch, wl.heads, wl.head_dim
+        self.q_pos0 = torch.full((B,), wl.ctx - 1, dtype=torch.int32, device="cuda")
+        self.desc = hs.make_desc(B, 1, H, D, wl.window, wl.budget, max_ctx=wl.ctx)
+        self.ws = hs.alloc_workspace(self.desc, scores_in_workspace=True)
+        self.o = torch.empty_like(self.q)
+        self.o_sp = [torch.empty_like(self.q) for _ in self.qs]
+        self.idx = torch.empty(B, 1, self.desc.idx_stride, dtype=torch.int32, device="cuda")
+        self.cnt = torch.empty(B, 1, dtype=torch.int32, device="cuda")
+        self.launches_per_step = 3 + len(self.qs)       # qk, pv, select, one per sparse layer
+
+    def full(self):
+        self.hs.hs2_full_attn_select(self.desc, self.q, self.k, self.v, None, None, self.q_pos0, self.o,
+                                     None, self.idx, self.cnt, None, self.ws)
+
+    def sparse(self, l):
+        self.hs.hs2_sparse_attn(self.desc, self.qs[l], self.k, self.v, None, None, self.idx, self.cnt,
+                                self.o_sp[l], None, self.ws)
+
+    def step(self):
+        self.full()
+        for l in range(len(self.qs)):
+            self.sparse(l)
+
+    # bytes one call must move at minimum
+    def full_bytes(self):
+        wl = self.wl
+        return wl.batch * (wl.ctx * (2 * wl.head_dim * 2 + 4) + 2 * wl.heads * wl.head_dim * 2)
+
+    def sparse_bytes(self):
+        wl = self.wl
+        S = wl.window + wl.budget
+        return wl.batch * (S * (2 * wl.head_dim * 2 + 4) + 2 * wl.heads * wl.head_dim * 2)
+
+
+def run_ours(args, ws_, rank, local):
+    import kv_shared_b200 as hs
+    wl = synth.DECODE_128K
+    blk = DecodeBlock(wl, seed=1002 + rank)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        blk.step()
+    torch.cuda.synchronize()
+    st = hs.hs2_last_status(blk.ws)
+    if st != hs.HS2_OK:
+        raise RuntimeError("device status after warm-up: " + hs.status_string(st))
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + len(blk.qs))] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    _barrier(ws_)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for i in range(K):
+            ev[i][0].record(stream)
+            blk.full()
+            ev[i][1].record(stream)
+            for l in range(len(blk.qs)):
+                blk.sparse(l)
+                ev[i][2 + l].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+    _barrier(ws_)
+    total_ms = _max_over_ranks(ws_, start.elapsed_time(end))
+    full_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    sparse_ms = statistics.mean(e[1 + l].elapsed_time(e[2 + l]) for e in ev for l in range(len(blk.qs)))
+    st = hs.hs2_last_status(blk.ws)
+    if st != hs.HS2_OK:
+        raise RuntimeError("device status after timing: " + hs.status_string(st))
+
+    ms_per_step = total_ms / K
+    queries_per_step = wl.batch * len(blk.qs)
+    value = ws_ * queries_per_step / (ms_per_step / 1e3)
+
+    # end to end through the C ABI: per-step inputs (the 4 layers' queries and the new
+    # token's K/V row) come from pinned host memory, the last layer's output goes back
+    host_q = [torch.empty_like(x, device="cpu").pin_memory() for x in [blk.q] + blk.qs]
+    for h, d in zip(host_q, [blk.q] + blk.qs):
+        h.copy_(d)
+    host_kv = torch.empty(2, wl.batch, wl.head_dim, dtype=torch.bfloat16).pin_memory()
+    host_kv[0].copy_(blk.k[:, wl.ctx - 1])
+    host_kv[1].copy_(blk.v[:, wl.ctx - 1])
+    dev_kv = torch.empty(2, wl.batch, wl.head_dim, dtype=torch.bfloat16, device="cuda")
+    host_out = torch.empty_like(blk.o_sp[-1], device="cpu").pin_memory()
+    h2d = sum(h.numel() * h.element_size() for h in host_q) + host_kv.numel() * host_kv.element_size()
+    d2h = host_out.numel() * host_out.element_size()
+    _barrier(ws_)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(K):
+        for h, d in zip(host_q, [blk.q] + blk.qs):
+            d.copy_(h, non_blocking=True)
+        dev_kv.copy_(host_kv, non_blocking=True)
+        blk.k[:, wl.ctx - 1].copy_(dev_kv[0])
+        blk.v[:, wl.ctx - 1].copy_(dev_kv[1])
+        blk.step()
+        host_out.copy_(blk.o_sp[-1], non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = _max_over_ranks(ws_, e0.elapsed_time(e1)) / K
+    e2e_value = ws_ * queries_per_step / (e2e_ms / 1e3)
+
+    hbm, tf, peak_kind = _peaks()
+    full_gbs = blk.full_bytes() / (full_ms / 1e3) / 1e9
+    sparse_gbs = blk.sparse_bytes() / (sparse_ms / 1e3) / 1e9
+    out = {
+        "metric": METRIC, "value": value, "unit": "sparse-attn queries/s", "n_gpus": ws_,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx, "heads": wl.heads,
+                   "head_dim": wl.head_dim, "window": wl.window, "budget": wl.budget,
+                   "sparse_layers": len(blk.qs), "parallelism": f"replicas{ws_}",
+                   "l2": "inputs larger than L2 (2 GiB cache per GPU)",
+                   "step": "full attention + importance + top-1024/window-128 selection + 3 sparse layers"},
+        "layers": {
+            "full_attn_select": {"ms": full_ms, "GB/s": full_gbs, "hbm_frac": full_gbs / hbm,
+                                 "bytes_per_call": blk.full_bytes()},
+            "sparse_attn": {"ms": sparse_ms, "queries/s": wl.batch / (sparse_ms / 1e3),
+                            "GB/s": sparse_gbs, "hbm_frac": sparse_gbs / hbm,
+                            "bytes_per_call": blk.sparse_bytes()},
+        },
+        "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": full_gbs / hbm, "peak_source": peak_kind,
+                     "kernel": "hs2_full_attn_select (decode: QK pass, PV+importance pass, select)",
+                     "traffic": FULL_CALL_TRAFFIC_BYTES},
+        "e2e": {"value": e2e_value, "unit": "sparse-attn queries/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": K * blk.launches_per_step,
+        "clocks": clk.summary(),
+    }
+    if ws_ == 1 and rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(wl, seed=1002, sample_seqs=args.cpu_sample)
+    return out
+
+
+def _oracle_block(wl, inp, b):
+    import numpy as np
+    import oracle
+    q = inp.q_full[b].double().numpy()
+    k = inp.k[b].double().numpy()
+    v = inp.v[b].double().numpy()
+    pos = np.array([wl.ctx - 1])
+    _, _, sc = oracle.full_attn(q, k, v, pos)
+    idx, cnt = oracle.select_rows(sc, pos, wl.window, wl.budget)
+    for l in range(wl.n_sparse):
+        oracle.sparse_attn(inp.q_sparse[l][b].double().numpy(), k, v, idx, cnt)
+
+
+def cpu_baseline(wl, seed, sample_seqs):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload."""
+    from concurrent.futures import ThreadPoolExecutor
+    sub = synth.shrink(wl, batch=sample_seqs)
+    inp = synth.make_inputs(sub, seed=seed, device="cuda")
+    inp.q_full, inp.k, inp.v = inp.q_full.cpu(), inp.k.cpu(), inp.v.cpu()
+    inp.q_sparse = [x.cpu() for x in inp.q_sparse]
+    cores = min(sample_seqs, os.cpu_count() or 1)
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        list(ex.map(lambda b: _oracle_block(sub, inp, b), range(sample_seqs)))
+    dt = time.perf_counter() - t0
+    return {"value": sample_seqs * wl.n_sparse / dt, "unit": "sparse-attn queries/s", "cores": cores,
+            "kind": "oracle", "seconds": dt,
+            "sample": f"{sample_seqs} of the {wl.batch} sequences of {wl.name}, whole hybrid block "
+                      f"(full attention + selection + {wl.n_sparse} sparse layers), fp64, one thread per sequence"}
+
+
+def run_reference(args, ws_, rank):
+    """Reference arm: the CPU oracle timed on the host, each step a bounded sample."""
+    wl = synth.DECODE_128K
+    sample = args.cpu_sample
+    times = []
+    res = None
+    for _ in range(args.steps):
+        res = cpu_baseline(wl, seed=1002, sample_seqs=sample)
+        times.append(res["seconds"])
+    per_step = statistics.mean(times)
+    value = sample * wl.n_sparse / per_step
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "sparse-attn queries/s",
+            "n_gpus": ws_, "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": wl.name, "sample_sequences": sample, "parallelism": "host threads"},
+            "cpu_baseline": {"kind": "oracle", "cores": res["cores"], "sample": res["sample"], "value": value,
+                             "unit": "sparse-attn queries/s"},
+            "e2e": {"value": value, "unit": "sparse-attn queries/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-sample", type=int, default=16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        args.warmup = 3
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores only; other ranks exit without work
+        ws_ = int(os.environ.get("WORLD_SIZE", "1"))
+        if int(os.environ.get("RANK", "0")) == 0:
+            torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+            print(json.dumps(run_reference(args, ws_, 0)), flush=True)
+        return
+    ws_, rank, local = _dist()
+    out = run_ours(args, ws_, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws_ > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,476 @@
+// decode_attn.cu -- full-attention layer of a hybrid block for one new query
+// token per sequence (decode), with the per-key importance the selection needs.
+//
+// Importance of key j = sum over the 16 query heads of the softmax probability
+// P_h[j] = exp(s_h[j] - LSE_h) (the pages leave the rule open: "What HySparse2 is
+// actually optimizing", "What is not documented"), so every probability must be
+// normalized by the FINAL log-sum-exp.  Two streaming passes over the cache:
+//
+//   pass A  S = scale * K q^T for all heads (tensor cores, M = 16 heads), the
+//           scaled logits go to a [B][16][S_ld] fp32 buffer (64 B per key) and
+//           each CTA keeps a running (max, sum) per head -> per-split partials.
+//   pass B  every CTA merges the partials into LSE, re-reads its logits, forms
+//           P exactly normalized, writes importance = sum_h P and accumulates
+//           O = P V (no online rescaling is needed: LSE is final).  The last CTA
+//           of a sequence sums the split partials into O (semaphore, no spin).
+//
+// K is read once (pass A) and V once (pass B): 512 B of cache per key plus the
+// 64-B logit round trip.  Tiles of 64 keys stream through a 4-stage TMA pipeline
+// with 128-byte swizzle; e4m3 caches are converted to bf16 in shared memory
+// (exact) and the per-token scales are folded into the logits and into P.
+#include "common.cuh"
+#include "internal.h"
+
+namespace hs2 {
+namespace {
+
+constexpr int H = 16;
+constexpr int D = 128;
+constexpr int TILE = 64;
+constexpr int STAGES = 4;
+constexpr int NT = 128;            // 4 warps, each owns 16 keys of a tile
+
+struct Params {
+    int B;
+    int64_t cap;
+    int64_t max_ctx;
+    int splits, chunk, s_ld;
+    const int32_t* q_pos0;
+    const __nv_bfloat16* q;
+    const float* k_scale;
+    const float* v_scale;
+    float sc2;                      // softmax scale * log2(e)
+    float* S;                       // [B][H][s_ld] logits, log2 units
+    float2* part_ml;                // [B][splits][H]: (max, sum) in log2 units
+    float* part_o;                  // [B][splits][H][D]
+    int* counter;                   // [B]
+    __nv_bfloat16* o;               // [B][H][D]
+    float* lse;                     // [B][H] natural log, or null
+    float* scores;                  // [B][score_ld]
+    int64_t score_ld;
+    uint32_t* status;
+};
+
+template <bool KV8>
+struct Layout {
+    static constexpr int RAW = KV8 ? TILE * 128 : TILE * 256;   // one cache tile as loaded
+    static constexpr int CVT = KV8 ? TILE * 256 : 0;            // bf16 copy (e4m3 only)
+    static constexpr int STILE = 16 * 32 * 4 * 2;               // logits tile: 2 boxes 16x32 fp32
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Q A-fragments of the m16n8k16 tile: 16 heads x 128 dims, 8 k-steps.
+__device__ __forceinline__ void load_q_frags(const __nv_bfloat16* qb, int g, int t, uint32_t (&qa)[8][4]) {
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qb);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        qa[ks][0] = __ldg(q32 + (g * D + 16 * ks + 2 * t) / 2);
+        qa[ks][1] = __ldg(q32 + ((g + 8) * D + 16 * ks + 2 * t) / 2);
+        qa[ks][2] = __ldg(q32 + (g * D + 16 * ks + 2 * t + 8) / 2);
+        qa[ks][3] = __ldg(q32 + ((g + 8) * D + 16 * ks + 2 * t + 8) / 2);
+    }
+}
+
+// e4m3 tile (64 rows x 128 B, 128-byte swizzle) -> bf16 tile (swz_off layout),
+// rows whose key is past `last` are zeroed.
+__device__ __forceinline__ void convert_tile(const uint8_t* raw, uint8_t* cvt, int key0, int last, int tid) {
+#pragma unroll
+    for (int it = tid; it < TILE * 8; it += NT) {
+        const int r = it >> 3, c8 = it & 7;
+        uint4 in = *reinterpret_cast<const uint4*>(raw + r * 128 + ((c8 ^ (r & 7)) << 4));
+        uint4 lo, hi;
+        if (key0 + r <= last) {
+            const uint16_t* b = reinterpret_cast<const uint16_t*>(&in);
+            lo.x = e4m3x2_to_bf16x2(b[0]); lo.y = e4m3x2_to_bf16x2(b[1]);
+            lo.z = e4m3x2_to_bf16x2(b[2]); lo.w = e4m3x2_to_bf16x2(b[3]);
+            hi.x = e4m3x2_to_bf16x2(b[4]); hi.y = e4m3x2_to_bf16x2(b[5]);
+            hi.z = e4m3x2_to_bf16x2(b[6]); hi.w = e4m3x2_to_bf16x2(b[7]);
+        } else {
+            lo = make_uint4(0, 0, 0, 0); hi = lo;
+        }
+        *reinterpret_cast<uint4*>(cvt + swz_off<TILE>(r, 2 * c8)) = lo;
+        *reinterpret_cast<uint4*>(cvt + swz_off<TILE>(r, 2 * c8 + 1)) = hi;
+    }
+}
+
+__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
+    const float mn = fmaxf(m, m2);
+    if (mn == -INFINITY) return;
+    l = l * exp2f(m - mn) + l2 * exp2f(m2 - mn);
+    m = mn;
+}
+
+// ------------------------------------------------------------------ pass A
+template <bool KV8>
+__global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUtensorMap kmap, Params a) {
+    using L = Layout<KV8>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* raw = smem;
+    uint8_t* cvt = smem + STAGES * L::RAW;
+    uint64_t* full = reinterpret_cast<uint64_t*>(cvt + L::CVT);
+    __shared__ float red_m[4][H], red_l[4][H];
+
+    const int b = blockIdx.y, split = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int p = checked_pos(a.q_pos0[b], a.max_ctx, a.status);
+    const int k_begin = split * a.chunk;
+    const int k_end = min(p + 1, k_begin + a.chunk);
+    const int n_tiles = k_end > k_begin ? (k_end - k_begin + TILE - 1) / TILE : 0;
+
+    if (split == 0 && tid == 0) a.counter[b] = 0;     // consumed by pass B (stream order)
+    if (tid == 0) {
+        prefetch_tmap(&kmap);
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    auto issue = [&](int i, int s) {
+        const int row = static_cast<int>(b * a.cap) + k_begin + i * TILE;
+        mbar_arrive_expect_tx(&full[s], L::RAW);
+        if (KV8) {
+            tma_load_2d(raw + s * L::RAW, &kmap, &full[s], 0, row);
+        } else {
+            tma_load_2d(raw + s * L::RAW, &kmap, &full[s], 0, row);
+            tma_load_2d(raw + s * L::RAW + TILE * 128, &kmap, &full[s], 64, row);
+        }
+    };
+    if (tid == 0)
+        for (int s = 0; s < STAGES && s < n_tiles; ++s) issue(s, s);
+
+    uint32_t qa[8][4];
+    load_q_frags(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
+
+    float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
+    float* Sg = a.S + (static_cast<size_t>(b) * H + g) * a.s_ld;
+    float* Sg8 = Sg + static_cast<size_t>(8) * a.s_ld;
+    const float* ksc = KV8 ? a.k_scale + b * a.cap : nullptr;
+
+    for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % STAGES;
+        bool ok = mbar_wait(&full[s], (i / STAGES) & 1, a.status);
+        const int tile_key0 = k_begin + i * TILE;
+        const uint8_t* tile = raw + s * L::RAW;
+        if (KV8) {
+            convert_tile(tile, cvt, tile_key0, k_end - 1, tid);
+            __syncthreads();
+            tile = cvt;
+        }
+        const uint32_t tbase = smem_u32(tile);
+        float acc[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+            const int r = warp * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(tbase + swz_off<TILE>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+                mma_bf16(acc[nt], qa[2 * kk], b0, b1);
+                mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+            }
+        }
+        // logits (log2 units), masked past the last key
+        const int key0 = tile_key0 + warp * 16 + 2 * t;
+        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int key = key0 + nt * 8;
+            float f0 = a.sc2, f1 = a.sc2;
+            if (KV8) {
+                f0 *= (key < k_end) ? ksc[key] : 0.f;
+                f1 *= (key + 1 < k_end) ? ksc[key + 1] : 0.f;
+            }
+            acc[nt][0] = (key < k_end) ? acc[nt][0] * f0 : -INFINITY;
+            acc[nt][1] = (key + 1 < k_end) ? acc[nt][1] * f1 : -INFINITY;
+            acc[nt][2] = (key < k_end) ? acc[nt][2] * f0 : -INFINITY;
+            acc[nt][3] = (key + 1 < k_end) ? acc[nt][3] * f1 : -INFINITY;
+            if (key < k_end) {
+                *reinterpret_cast<float2*>(Sg + key) = make_float2(acc[nt][0], acc[nt][1]);
+                *reinterpret_cast<float2*>(Sg8 + key) = make_float2(acc[nt][2], acc[nt][3]);
+            }
+            mx[0] = fmaxf(mx[0], fmaxf(acc[nt][0], acc[nt][1]));
+            mx[1] = fmaxf(mx[1], fmaxf(acc[nt][2], acc[nt][3]));
+        }
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            const float mn = fmaxf(m2[hh], mx[hh]);
+            if (mn != -INFINITY) {
+                float sum = l2[hh] * exp2f(m2[hh] - mn);
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    sum += exp2f(acc[nt][2 * hh] - mn) + exp2f(acc[nt][2 * hh + 1] - mn);
+                l2[hh] = sum;
+                m2[hh] = mn;
+            }
+        }
+        if (__syncthreads_or(!ok)) break;
+        if (tid == 0 && i + STAGES < n_tiles) issue(i + STAGES, s);
+    }
+
+    // reduce (max, sum) over the quad, then over warps
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+        for (int off = 1; off <= 2; off <<= 1) {
+            const float om = __shfl_xor_sync(0xffffffffu, m2[hh], off);
+            const float ol = __shfl_xor_sync(0xffffffffu, l2[hh], off);
+            merge_ml(m2[hh], l2[hh], om, ol);
+        }
+    }
+    if (t == 0) {
+        red_m[warp][g] = m2[0]; red_l[warp][g] = l2[0];
+        red_m[warp][g + 8] = m2[1]; red_l[warp][g + 8] = l2[1];
+    }
+    __syncthreads();
+    if (tid < H) {
+        float m = red_m[0][tid], l = red_l[0][tid];
+        for (int w = 1; w < 4; ++w) merge_ml(m, l, red_m[w][tid], red_l[w][tid]);
+        a.part_ml[(static_cast<size_t>(b) * a.splits + split) * H + tid] = make_float2(m, l);
+    }
+}
+
+// ------------------------------------------------------------------ pass B
+template <bool KV8>
+__global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUtensorMap vmap,
+                                                    const __grid_constant__ CUtensorMap smap, Params a) {
+    using L = Layout<KV8>;
+    constexpr int STAGE = L::RAW + L::STILE;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* cvt = smem + STAGES * STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(cvt + L::CVT);
+    float* red_o = reinterpret_cast<float*>(full + STAGES);          // [H][D]
+    __shared__ int s_last;
+
+    const int b = blockIdx.y, split = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int p = checked_pos(a.q_pos0[b], a.max_ctx, a.status);
+    const int k_begin = split * a.chunk;
+    const int k_end = min(p + 1, k_begin + a.chunk);
+    const int n_tiles = k_end > k_begin ? (k_end - k_begin + TILE - 1) / TILE : 0;
+
+    if (tid == 0) {
+        prefetch_tmap(&vmap);
+        prefetch_tmap(&smap);
+        for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    for (int i = tid; i < H * D; i += NT) red_o[i] = 0.f;
+    __syncthreads();
+
+    auto issue = [&](int i, int s) {
+        uint8_t* st = smem + s * STAGE;
+        const int key = k_begin + i * TILE;
+        const int row = static_cast<int>(b * a.cap) + key;
+        mbar_arrive_expect_tx(&full[s], STAGE);
+        tma_load_2d(st, &vmap, &full[s], 0, row);
+        if (!KV8) tma_load_2d(st + TILE * 128, &vmap, &full[s], 64, row);
+        tma_load_2d(st + L::RAW, &smap, &full[s], key, b * H);
+        tma_load_2d(st + L::RAW + 2048, &smap, &full[s], key + 32, b * H);
+    };
+    if (tid == 0)
+        for (int s = 0; s < STAGES && s < n_tiles; ++s) issue(s, s);
+
+    // final log-sum-exp of this thread's two heads from all splits' partials
+    float lse2[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int h = g + 8 * hh;
+        float m = -INFINITY, l = 0.f;
+        for (int s = 0; s < a.splits; ++s) {
+            const float2 ml = a.part_ml[(static_cast<size_t>(b) * a.splits + s) * H + h];
+            merge_ml(m, l, ml.x, ml.y);
+        }
+        lse2[hh] = m + log2f(l);
+        if (split == 0 && warp == 0 && t == 0 && a.lse)
+            a.lse[static_cast<size_t>(b) * H + h] = lse2[hh] * kLn2;
+    }
+
+    float o[16][4];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
+    float* score_row = a.scores + b * a.score_ld;
+
+    for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % STAGES;
+        bool ok = mbar_wait(&full[s], (i / STAGES) & 1, a.status);
+        uint8_t* st = smem + s * STAGE;
+        const int tile_key0 = k_begin + i * TILE;
+        uint8_t* vt = st;
+        if (KV8) {
+            convert_tile(st, cvt, tile_key0, k_end - 1, tid);
+            vt = cvt;
+            __syncthreads();
+        } else if (tile_key0 + TILE > k_end) {
+            // tail tile: zero the V rows past the last key (cache rows there may hold
+            // anything, and 0 * NaN would poison the accumulators)
+            for (int it = tid; it < TILE * 16; it += NT) {
+                const int r = it >> 4, c = it & 15;
+                if (tile_key0 + r >= k_end)
+                    *reinterpret_cast<uint4*>(vt + swz_off<TILE>(r, c)) = make_uint4(0, 0, 0, 0);
+            }
+            __syncthreads();
+        }
+        // logits of this warp's 16 keys from the swizzled [16 heads][2 x 32 keys] tile
+        const uint8_t* stile = st + L::RAW;
+        const int c0 = 16 * (warp & 1) + 2 * t;
+        const uint8_t* half = stile + (warp >> 1) * 2048;
+        auto sld = [&](int hr, int c) {
+            return *reinterpret_cast<const float2*>(half + hr * 128 + (((c >> 2) ^ (hr & 7)) << 4) + (c & 3) * 4);
+        };
+        const float2 sgl = sld(g, c0), sg8l = sld(g + 8, c0), sgh = sld(g, c0 + 8), sg8h = sld(g + 8, c0 + 8);
+        const int kl = tile_key0 + warp * 16 + 2 * t, kh = kl + 8;
+        const bool v0 = kl < k_end, v1 = kl + 1 < k_end, v2 = kh < k_end, v3 = kh + 1 < k_end;
+        const float p00 = v0 ? exp2f(sgl.x - lse2[0]) : 0.f, p01 = v1 ? exp2f(sgl.y - lse2[0]) : 0.f;
+        const float p10 = v0 ? exp2f(sg8l.x - lse2[1]) : 0.f, p11 = v1 ? exp2f(sg8l.y - lse2[1]) : 0.f;
+        const float p02 = v2 ? exp2f(sgh.x - lse2[0]) : 0.f, p03 = v3 ? exp2f(sgh.y - lse2[0]) : 0.f;
+        const float p12 = v2 ? exp2f(sg8h.x - lse2[1]) : 0.f, p13 = v3 ? exp2f(sg8h.y - lse2[1]) : 0.f;
+        // importance: sum over the 16 heads (pair here, then across the 8 row groups)
+        float sc[4] = {p00 + p10, p01 + p11, p02 + p12, p03 + p13};
+#pragma unroll
+        for (int off = 4; off <= 16; off <<= 1)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) sc[e] += __shfl_xor_sync(0xffffffffu, sc[e], off);
+        if (g == 0) {
+            if (v0) score_row[kl] = sc[0];
+            if (v1) score_row[kl + 1] = sc[1];
+            if (v2) score_row[kh] = sc[2];
+            if (v3) score_row[kh + 1] = sc[3];
+        }
+        float f0 = 1.f, f1 = 1.f, f2 = 1.f, f3 = 1.f;
+        if (KV8) {
+            f0 = v0 ? vsc[kl] : 0.f; f1 = v1 ? vsc[kl + 1] : 0.f;
+            f2 = v2 ? vsc[kh] : 0.f; f3 = v3 ? vsc[kh + 1] : 0.f;
+        }
+        uint32_t pa[4];
+        pa[0] = pack_bf16(p00 * f0, p01 * f1);
+        pa[1] = pack_bf16(p10 * f0, p11 * f1);
+        pa[2] = pack_bf16(p02 * f2, p03 * f3);
+        pa[3] = pack_bf16(p12 * f2, p13 * f3);
+        const uint32_t vbase = smem_u32(vt);
+        const int vr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vbase + swz_off<TILE>(vr, 2 * c + (lane >> 4)), b0, b1, b2, b3);
+            mma_bf16(o[2 * c], pa, b0, b1);
+            mma_bf16(o[2 * c + 1], pa, b2, b3);
+        }
+        if (__syncthreads_or(!ok)) break;
+        if (tid == 0 && i + STAGES < n_tiles) issue(i + STAGES, s);
+    }
+
+    // CTA partial O = sum over warps
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        const int d = 8 * n + 2 * t;
+        atomicAdd(&red_o[g * D + d], o[n][0]);
+        atomicAdd(&red_o[g * D + d + 1], o[n][1]);
+        atomicAdd(&red_o[(g + 8) * D + d], o[n][2]);
+        atomicAdd(&red_o[(g + 8) * D + d + 1], o[n][3]);
+    }
+    __syncthreads();
+    float* my = a.part_o + (static_cast<size_t>(b) * a.splits + split) * H * D;
+    for (int i = tid; i < H * D; i += NT) my[i] = red_o[i];
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(&a.counter[b], 1) == a.splits - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const float* base = a.part_o + static_cast<size_t>(b) * a.splits * H * D;
+    for (int i = tid; i < H * D; i += NT) {
+        float acc = 0.f;
+        for (int s = 0; s < a.splits; ++s) acc += __ldcg(base + static_cast<size_t>(s) * H * D + i);
+        a.o[static_cast<size_t>(b) * H * D + i] = __float2bfloat16_rn(acc);
+    }
+}
+
+template <bool KV8>
+size_t smem_a() { return 1024 + STAGES * Layout<KV8>::RAW + Layout<KV8>::CVT + STAGES * 8; }
+template <bool KV8>
+size_t smem_b() {
+    return 1024 + STAGES * (Layout<KV8>::RAW + Layout<KV8>::STILE) + Layout<KV8>::CVT + STAGES * 8 + H * D * 4;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <bool KV8>
+cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
+    const DecodePlan pl = plan_decode(da.batch, da.max_ctx);
+    Params a{};
+    a.B = da.batch; a.cap = da.cap; a.max_ctx = da.max_ctx; a.splits = pl.splits; a.chunk = pl.chunk; a.s_ld = pl.s_ld;
+    a.q_pos0 = da.q_pos0;
+    a.q = static_cast<const __nv_bfloat16*>(da.q);
+    a.k_scale = da.k_scale; a.v_scale = da.v_scale;
+    a.sc2 = da.scale * kLog2e;
+    uint8_t* ws = static_cast<uint8_t*>(da.ws);
+    a.S = reinterpret_cast<float*>(ws);
+    ws += align256(sizeof(float) * da.batch * H * static_cast<size_t>(pl.s_ld));
+    a.part_ml = reinterpret_cast<float2*>(ws);
+    ws += align256(sizeof(float2) * da.batch * pl.splits * H);
+    a.part_o = reinterpret_cast<float*>(ws);
+    ws += align256(sizeof(float) * da.batch * pl.splits * H * D);
+    a.counter = reinterpret_cast<int*>(ws);
+    a.o = static_cast<__nv_bfloat16*>(da.o);
+    a.lse = da.lse;
+    a.scores = da.scores; a.score_ld = da.score_ld;
+    a.status = da.status;
+
+    CUtensorMap kmap, vmap, smap;
+    const uint64_t rows = static_cast<uint64_t>(da.batch) * da.cap;
+    const int eb = KV8 ? 1 : 2;
+    const CUtensorMapDataType dt = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const uint32_t box_cols = KV8 ? 128 : 64;
+    if (!make_tmap_2d(&kmap, da.k, dt, eb, D, rows, D * eb, box_cols, TILE, true)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&vmap, da.v, dt, eb, D, rows, D * eb, box_cols, TILE, true)) return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&smap, a.S, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, pl.s_ld,
+                      static_cast<uint64_t>(da.batch) * H, static_cast<uint64_t>(pl.s_ld) * 4, 32, 16, true))
+        return cudaErrorInvalidValue;
+
+    const dim3 grid(pl.splits, da.batch);
+    const size_t sa = smem_a<KV8>(), sb = smem_b<KV8>();
+    cudaError_t e = cudaFuncSetAttribute(dec_qk_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sa));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(dec_pv_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sb));
+    if (e != cudaSuccess) return e;
+    dec_qk_kernel<KV8><<<grid, NT, sa, st>>>(kmap, a);
+    dec_pv_kernel<KV8><<<grid, NT, sb, st>>>(vmap, smap, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+DecodePlan plan_decode(int batch, int64_t max_ctx) {
+    DecodePlan pl;
+    int splits = (2 * num_sms()) / (batch > 0 ? batch : 1);
+    if (splits < 1) splits = 1;
+    int64_t chunk = (max_ctx + splits - 1) / splits;
+    chunk = (chunk + TILE - 1) / TILE * TILE;
+    if (chunk < TILE) chunk = TILE;
+    pl.chunk = static_cast<int>(chunk);
+    pl.splits = static_cast<int>((max_ctx + chunk - 1) / chunk);
+    if (pl.splits < 1) pl.splits = 1;
+    pl.s_ld = static_cast<int>((max_ctx + TILE - 1) / TILE * TILE);
+    return pl;
+}
+
+size_t decode_ws_bytes(int batch, int64_t max_ctx) {
+    const DecodePlan pl = plan_decode(batch, max_ctx);
+    return align256(sizeof(float) * batch * H * static_cast<size_t>(pl.s_ld)) +
+           align256(sizeof(float2) * batch * pl.splits * H) +
+           align256(sizeof(float) * batch * pl.splits * H * D) + align256(sizeof(int) * batch);
+}
+
+cudaError_t launch_decode_full(const DecodeArgs& a, cudaStream_t st) {
+    return a.kv8 ? launch_impl<true>(a, st) : launch_impl<false>(a, st);
+}
+
+}  // namespace hs2

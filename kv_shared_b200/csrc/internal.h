@@ -1,0 +1,122 @@
+// internal.h -- launch interfaces between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace hs2 {
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+
+// Builds a 2-D tiled tensor map (row-major [rows][cols] of `elem_bytes` elements,
+// row pitch `row_bytes`), box [box_rows][box_cols], 128-byte swizzle when
+// `swizzle128` is set.  Returns false if the driver rejects it.
+bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                  uint64_t cols, uint64_t rows, uint64_t row_bytes, uint32_t box_cols,
+                  uint32_t box_rows, bool swizzle128);
+
+// ---------------------------------------------------------------- decode (n_q == 1)
+struct DecodePlan {
+    int splits;          // key splits per sequence
+    int chunk;           // keys per split (multiple of 64)
+    int s_ld;            // row pitch of the logit buffer (multiple of 64)
+};
+DecodePlan plan_decode(int batch, int64_t max_ctx);
+size_t decode_ws_bytes(int batch, int64_t max_ctx);   // logits + partials + counters
+
+struct DecodeArgs {
+    int batch;
+    int64_t cap;
+    int64_t max_ctx;
+    const int32_t* q_pos0;
+    const void* q;            // [B][16][128] bf16
+    const void* k;            // [B][cap][128] bf16 or e4m3
+    const void* v;
+    const float* k_scale;     // [B][cap] (e4m3)
+    const float* v_scale;
+    bool kv8;
+    float scale;
+    void* o;                  // [B][16][128] bf16
+    float* lse;               // [B][16] or null
+    float* scores;            // [B][score_ld]
+    int64_t score_ld;
+    void* ws;                 // decode scratch (decode_ws_bytes)
+    uint32_t* status;
+};
+cudaError_t launch_decode_full(const DecodeArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- selection
+struct SelectArgs {
+    int rows;                 // batch * n_q
+    int n_q;
+    const int32_t* q_pos0;
+    const float* scores;
+    int64_t score_ld;
+    int window, budget, block_size, idx_stride;
+    int32_t* idx;
+    int32_t* cnt;
+    int64_t max_ctx;          // positions are clamped below it (violations flag HS2_ERR_INDEX)
+    uint32_t* status;
+};
+cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- sparse attention
+struct SparsePlan {
+    int splits;
+    int chunk;               // selected entries per split (multiple of 64)
+};
+SparsePlan plan_sparse(int rows, int idx_stride);
+size_t sparse_ws_bytes(int rows, int idx_stride);
+
+struct SparseArgs {
+    int rows, n_q;
+    int64_t cap;
+    int idx_stride;
+    const void* q;            // [rows][16][128] bf16
+    const void* k;
+    const void* v;
+    const float* k_scale;
+    const float* v_scale;
+    bool kv8;
+    const int32_t* idx;
+    const int32_t* cnt;
+    float scale;
+    void* o;                  // [rows][16][128] bf16
+    float* lse;
+    void* ws;
+    uint32_t* status;
+};
+cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- fp32 SIMT path
+struct F32Args {
+    int batch, n_q, heads, head_dim;
+    int64_t cap;
+    int64_t max_ctx;
+    const int32_t* q_pos0;
+    const float* q;
+    const float* k;
+    const float* v;
+    float scale;
+    float* o;
+    float* lse;
+    float* scores;           // [rows][score_ld]
+    int64_t score_ld;
+    // sparse
+    const int32_t* idx;
+    const int32_t* cnt;
+    int idx_stride;
+    uint32_t* status;
+};
+cudaError_t launch_f32_full(const F32Args& a, cudaStream_t st);
+cudaError_t launch_f32_sparse(const F32Args& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- fp8 quantizer
+cudaError_t launch_fp8_quantize(const float* src, int64_t rows, int head_dim, uint8_t* codes,
+                                float* scales, cudaStream_t st);
+
+}  // namespace hs2
