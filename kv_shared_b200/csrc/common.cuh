@@ -20,10 +20,17 @@ namespace hs2 {
 // The first 256 bytes of every workspace hold the device status word.
 constexpr size_t kStatusBytes = 256;
 
-// Iteration cap of every spin on an mbarrier: a phase that has not completed
-// after this many polls (each poll may sleep in hardware) is reported as a
+// Bound of every wait on an mbarrier: a phase that has not completed within
+// kWaitNs nanoseconds of global time (or kWaitPolls polls) is reported as a
 // timeout instead of hanging the GPU.
-constexpr uint32_t kWaitPolls = 1u << 24;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr uint32_t kWaitPolls = 1u << 26;
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
 
 __device__ __forceinline__ void set_status(uint32_t* status, uint32_t code) {
     if (status) atomicCAS(status, 0u, code);
@@ -72,11 +79,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity; false (and the status word
-// set to HS2_ERR_TIMEOUT) if it did not complete within kWaitPolls polls.
+// set to HS2_ERR_TIMEOUT) if it did not complete in time.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
-                                          uint32_t polls = kWaitPolls) {
-    for (uint32_t i = 0; i < polls; ++i)
+                                          uint64_t limit_ns = kWaitNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > limit_ns) break;
+    }
     set_status(status, HS2_ERR_TIMEOUT);
     return false;
 }
