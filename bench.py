@@ -192,8 +192,25 @@ def run_ours(args, ws_, rank, local):
     if st != hs.HS2_OK:
         raise RuntimeError("device status after warm-up: " + hs.status_string(st))
 
+    # each C-ABI call of the step is captured once into a CUDA graph (the calls only
+    # enqueue kernels: no allocation, no synchronization) and replayed
+    graphs = []
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for fn in [blk.full] + [lambda l=l: blk.sparse(l) for l in range(len(blk.qs))]:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn()
+            graphs.append(g)
+    stream.wait_stream(side)
+    for _ in range(args.warmup):
+        for g in graphs:
+            g.replay()
+    torch.cuda.synchronize()
+
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2 + len(blk.qs))] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(K)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(ws_)
     torch.cuda.synchronize()
@@ -201,11 +218,9 @@ def run_ours(args, ws_, rank, local):
         start.record(stream)
         for i in range(K):
             ev[i][0].record(stream)
-            blk.full()
-            ev[i][1].record(stream)
-            for l in range(len(blk.qs)):
-                blk.sparse(l)
-                ev[i][2 + l].record(stream)
+            for j, g in enumerate(graphs):
+                g.replay()
+                ev[i][j + 1].record(stream)
         end.record(stream)
         torch.cuda.synchronize()
     _barrier(ws_)
@@ -242,7 +257,8 @@ def run_ours(args, ws_, rank, local):
         dev_kv.copy_(host_kv, non_blocking=True)
         blk.k[:, wl.ctx - 1].copy_(dev_kv[0])
         blk.v[:, wl.ctx - 1].copy_(dev_kv[1])
-        blk.step()
+        for g in graphs:
+            g.replay()
         host_out.copy_(blk.o_sp[-1], non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
@@ -339,7 +355,7 @@ def run_reference(args, ws_, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-sample", type=int, default=16)
