@@ -175,6 +175,36 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_attn_desc* desc, const void* q, con
                            size_t ws_bytes, hs2_stream_t stream);
 
 /*
+ * hs2_sparse_attn without a workspace argument, for callers that cannot
+ * allocate device memory at the point where they call the library: for example
+ * a plugin inside an inference engine that planned all of its memory up front,
+ * or code whose only device memory is the inputs and outputs it was handed.
+ * The pages have no counterpart; it exists for such callers only.
+ *
+ * Same arguments, kernel and results as hs2_sparse_attn with bf16 or e4m3
+ * caches (an f32 description returns HS2_ERR_UNSUPPORTED).  Its scratch (split
+ * partials, semaphore counters, status word) is a fixed 4 MiB array inside the
+ * library, held on every GPU that loads the library until the process exits.
+ *   - A problem whose scratch would exceed 4 MiB is rejected with
+ *     HS2_ERR_WORKSPACE before anything is enqueued (one 1,152-entry index row
+ *     per query needs at most about 2.7 MB at any batch size).
+ *   - The first call on each device looks up the array's device address with
+ *     the device current; make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; the
+ *     counters that must start at zero are cleared by every call.  Calls that
+ *     overlap on the GPU (different streams, or different host threads on one
+ *     device) race on the array and must be ordered by the caller.
+ *   - Conditions found on the device (an index outside the cache) are handled
+ *     as in hs2_sparse_attn (the entry is skipped) but are not reported: there
+ *     is no caller workspace to hold the status word.
+ * It calls no allocating routine.
+ */
+HS2_API hs2_status hs2_sparse_attn_noalloc(const hs2_attn_desc* desc, const void* q, const void* k,
+                                           const void* v, const float* k_scale, const float* v_scale,
+                                           const int32_t* idx, const int32_t* cnt, void* o, float* lse,
+                                           hs2_stream_t stream);
+
+/*
  * KV Bridging projection ([LB] "Two-Level KV Sharing": the cross-decoder's
  * full-attention caches are generated from the hidden states of the
  * self-decoder, each target layer with its own K/V projection; [AN]: the latter

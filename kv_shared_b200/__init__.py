@@ -19,7 +19,7 @@ HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUD
     HS2_ERR_TIMEOUT, HS2_ERR_INDEX = range(7)
 
 EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_topk_select",
-           "hs2_sparse_attn", "hs2_kv_bridge_proj", "hs2_kv_quantize_fp8", "hs2_last_status",
+           "hs2_sparse_attn", "hs2_sparse_attn_noalloc", "hs2_kv_bridge_proj", "hs2_kv_quantize_fp8", "hs2_last_status",
            "hs2_status_string")
 
 
@@ -55,6 +55,7 @@ def lib():
         L.hs2_full_attn_select.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.hs2_topk_select.argtypes = [dp, vp, i64, vp, i32, vp, vp, vp, sz, vp]
         L.hs2_sparse_attn.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.hs2_sparse_attn_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hs2_kv_bridge_proj.argtypes = [vp, vp, i32, i32, i32, i32, vp, i64, vp, vp, vp]
         L.hs2_kv_quantize_fp8.argtypes = [vp, i64, i32, vp, vp, vp]
         L.hs2_last_status.argtypes = [vp, vp]
@@ -127,6 +128,14 @@ def hs2_sparse_attn(desc, q, k, v, k_scale, v_scale, idx, cnt, o, lse, workspace
                                _p(idx), _p(cnt), _p(o), _p(lse), _p(workspace),
                                workspace.numel() * workspace.element_size(), _stream(stream))
     _check("hs2_sparse_attn", st)
+
+
+def hs2_sparse_attn_noalloc(desc, q, k, v, k_scale, v_scale, idx, cnt, o, lse, stream=None):
+    """hs2_sparse_attn without a workspace: for callers that cannot allocate device memory
+    where they call us; scratch is a fixed array inside the library (see include/hs2.h)."""
+    st = lib().hs2_sparse_attn_noalloc(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(k_scale), _p(v_scale),
+                                       _p(idx), _p(cnt), _p(o), _p(lse), _stream(stream))
+    _check("hs2_sparse_attn_noalloc", st)
 
 
 def hs2_kv_bridge_proj(hidden, w_kv, batch, n, d_model, head_dim, pos0, kv_capacity, k, v, stream=None):

@@ -245,6 +245,32 @@ hs2_status hs2_sparse_attn(const hs2_attn_desc* desc, const void* q, const void*
     return from_cuda(launch_sparse(a, st));
 }
 
+// Sparse attention without a caller workspace (see include/hs2.h): same checks
+// and kernel as hs2_sparse_attn, scratch taken from the library's fixed array.
+hs2_status hs2_sparse_attn_noalloc(const hs2_attn_desc* desc, const void* q, const void* k, const void* v,
+                                   const float* k_scale, const float* v_scale, const int32_t* idx,
+                                   const int32_t* cnt, void* o, float* lse, hs2_stream_t stream) {
+    Path path;
+    hs2_status s = check_desc(desc, &path);
+    if (s != HS2_OK) return s;
+    if (path != Path::TC) return HS2_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !idx || !cnt || !o) return HS2_ERR_INVALID_ARG;
+    const bool kv8 = desc->kv_dtype == HS2_E4M3;
+    if (kv8 && (!k_scale || !v_scale)) return HS2_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, idx, cnt, o};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return HS2_ERR_INVALID_ARG;
+    if (lse && !aligned16(lse)) return HS2_ERR_INVALID_ARG;
+    SparseArgs a{};
+    a.rows = desc->batch * desc->n_q; a.n_q = desc->n_q; a.cap = desc->kv_capacity; a.idx_stride = desc->idx_stride;
+    a.q = q; a.k = k; a.v = v; a.k_scale = k_scale; a.v_scale = v_scale; a.kv8 = kv8;
+    a.idx = idx; a.cnt = cnt; a.scale = eff_scale(desc); a.o = o; a.lse = lse;
+    bool too_large = false;
+    const cudaError_t e = launch_sparse_noalloc(a, reinterpret_cast<cudaStream_t>(stream), &too_large);
+    if (too_large) return HS2_ERR_WORKSPACE;
+    return from_cuda(e);
+}
+
 hs2_status hs2_kv_bridge_proj(const void* hidden, const void* w_kv, int32_t batch, int32_t n, int32_t d_model,
                               int32_t head_dim, const int32_t* pos0, int64_t kv_capacity, void* k, void* v,
                               hs2_stream_t stream) {

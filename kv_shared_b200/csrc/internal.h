@@ -92,6 +92,12 @@ struct SparseArgs {
 };
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t st);
 
+// Same kernel with its scratch in a fixed device array (no caller workspace);
+// *too_large is set, and nothing launched, when the problem needs more scratch
+// than sparse_noalloc_capacity() bytes.
+cudaError_t launch_sparse_noalloc(const SparseArgs& a, cudaStream_t st, bool* too_large);
+size_t sparse_noalloc_capacity();
+
 // ---------------------------------------------------------------- fp32 SIMT path
 struct F32Args {
     int batch, n_q, heads, head_dim;

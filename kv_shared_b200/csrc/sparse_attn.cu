@@ -13,6 +13,8 @@
 // (decode); split partials (max, sum, O) are merged by the last CTA of the row
 // (semaphore counter, no spin).  e4m3 rows are converted to bf16 in shared
 // memory (exact) and their per-token scales folded into the logits and into P.
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -405,6 +407,61 @@ size_t sparse_ws_bytes(int rows, int idx_stride) {
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t st) {
     if (a.rows <= 0) return cudaSuccess;
     return a.kv8 ? launch_impl<true>(a, st) : launch_impl<false>(a, st);
+}
+
+}  // namespace hs2
+
+// ---------------------------------------------------------------------------
+// Variant without a caller workspace, for callers that cannot allocate device
+// memory when they call us.  Its scratch (status word, split partials and the
+// semaphore counters) lives in one fixed file-scope device array that every GPU
+// loading this library keeps until the process exits.
+namespace hs2 {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;     // 4 MiB per device
+
+static __device__ __align__(256) uint8_t g_sparse_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mu;
+void* g_scratch_addr[64] = {nullptr};
+
+// Device address of g_sparse_scratch on the current device, looked up once per
+// device (host code cannot use the symbol itself as a device pointer).
+cudaError_t scratch_address(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_addr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_sparse_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_addr[dev] = p;
+    }
+    *out = g_scratch_addr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t sparse_noalloc_capacity() { return kNoAllocScratchBytes; }
+
+cudaError_t launch_sparse_noalloc(const SparseArgs& in, cudaStream_t st, bool* too_large) {
+    *too_large = false;
+    if (in.rows <= 0) return cudaSuccess;
+    if (kStatusBytes + sparse_ws_bytes(in.rows, in.idx_stride) > kNoAllocScratchBytes) {
+        *too_large = true;
+        return cudaSuccess;
+    }
+    void* base = nullptr;
+    const cudaError_t e = scratch_address(&base);
+    if (e != cudaSuccess) return e;
+    SparseArgs a = in;
+    a.status = static_cast<uint32_t*>(base);
+    a.ws = static_cast<uint8_t*>(base) + kStatusBytes;
+    return launch_sparse(a, st);
 }
 
 }  // namespace hs2
