@@ -180,6 +180,119 @@ class DecodeBlock:
         return wl.batch * (S * (2 * wl.head_dim * 2 + 4) + 2 * wl.heads * wl.head_dim * 2)
 
 
+class PrefillBlock:
+    """Device buffers and C-ABI calls of one agent-round prefill step: KV bridging of the
+    new rows, full attention with importance and selection over cached + new rows, and
+    the sparse layers."""
+
+    def __init__(self, wl, seed):
+        import kv_shared_b200 as hs
+        self.hs = hs
+        self.wl = wl
+        inp = synth.make_inputs(wl, seed=seed, device="cuda")
+        self.q = inp.q_full.contiguous()
+        self.qs = [x.contiguous() for x in inp.q_sparse]
+        self.k, self.v = inp.k.contiguous(), inp.v.contiguous()
+        self.hidden, self.w_kv = inp.hidden.contiguous(), inp.w_kv.contiguous()
+        del inp
+        B = wl.batch
+        self.q_pos0 = torch.full((B,), wl.q_pos0, dtype=torch.int32, device="cuda")
+        self.pos0_new = torch.full((B,), wl.ctx - wl.n_new, dtype=torch.int32, device="cuda")
+        self.desc = hs.make_desc(B, wl.n_q, wl.heads, wl.head_dim, wl.window, wl.budget, max_ctx=wl.ctx)
+        self.ws = hs.alloc_workspace(self.desc, scores_in_workspace=True)
+        self.o = torch.empty_like(self.q)
+        self.o_sp = [torch.empty_like(self.q) for _ in self.qs]
+        self.idx = torch.empty(B, wl.n_q, self.desc.idx_stride, dtype=torch.int32, device="cuda")
+        self.cnt = torch.empty(B, wl.n_q, dtype=torch.int32, device="cuda")
+        self.launches_per_step = 1 + 3 + len(self.qs)   # bridge, lse, out, select, sparse layers
+
+    def bridge(self):
+        wl = self.wl
+        self.hs.hs2_kv_bridge_proj(self.hidden, self.w_kv, wl.batch, wl.n_new, wl.d_model, wl.head_dim,
+                                   self.pos0_new, wl.ctx, self.k, self.v)
+
+    def full(self):
+        self.hs.hs2_full_attn_select(self.desc, self.q, self.k, self.v, None, None, self.q_pos0, self.o,
+                                     None, self.idx, self.cnt, None, self.ws)
+
+    def sparse(self, l):
+        self.hs.hs2_sparse_attn(self.desc, self.qs[l], self.k, self.v, None, None, self.idx, self.cnt,
+                                self.o_sp[l], None, self.ws)
+
+    def pairs(self):
+        wl = self.wl
+        return wl.batch * sum(wl.q_pos0 + r + 1 for r in range(wl.n_q))
+
+    def full_flops(self):
+        # QK^T and PV over every causal (row, key) pair, all heads
+        wl = self.wl
+        return self.pairs() * wl.heads * wl.head_dim * 4
+
+
+def _capture(fns, stream):
+    graphs = []
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        for fn in fns:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn()
+            graphs.append(g)
+    stream.wait_stream(side)
+    return graphs
+
+
+def run_prefill(args, ws_):
+    """Agent-round prefill: times the graph-replayed step and its full-attention call."""
+    import kv_shared_b200 as hs
+    wl = synth.PREFILL_AGENT
+    blk = PrefillBlock(wl, seed=1003)
+    stream = torch.cuda.current_stream()
+    blk.bridge(); blk.full(); [blk.sparse(l) for l in range(len(blk.qs))]
+    torch.cuda.synchronize()
+    st = hs.hs2_last_status(blk.ws)
+    if st != hs.HS2_OK:
+        raise RuntimeError("prefill device status: " + hs.status_string(st))
+    graphs = _capture([blk.bridge, blk.full] + [lambda l=l: blk.sparse(l) for l in range(len(blk.qs))], stream)
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    K = max(3, args.prefill_steps)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(K)]
+    _barrier(ws_)
+    torch.cuda.synchronize()
+    for i in range(K):
+        ev[i][0].record(stream)
+        for j, g in enumerate(graphs):
+            g.replay()
+            ev[i][j + 1].record(stream)
+    torch.cuda.synchronize()
+    step_ms = _max_over_ranks(ws_, statistics.mean(e[0].elapsed_time(e[-1]) for e in ev))
+    bridge_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    full_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    sparse_ms = statistics.mean(e[2 + l].elapsed_time(e[3 + l]) for e in ev for l in range(len(blk.qs)))
+    _, tf, peak_kind = _peaks()
+    full_tflops = blk.full_flops() / (full_ms / 1e3) / 1e12
+    bridge_flops = 2 * wl.batch * wl.n_new * wl.d_model * 2 * wl.head_dim
+    bridge_bytes = 2 * wl.batch * wl.n_new * (wl.d_model + 2 * wl.head_dim) + wl.d_model * 2 * wl.head_dim * 2
+    hbm, _, _ = _peaks()
+    return {
+        "workload": wl.name, "tokens/s": ws_ * wl.batch * wl.n_q / (step_ms / 1e3), "ms_per_step": step_ms,
+        "steps": K,
+        "step": "KV bridging of the 8192 new rows + full attention with importance over 65536+8192 keys "
+                "+ top-1024/window-128 selection per row + 3 sparse layers",
+        "full_attn_select": {"ms": full_ms, "algorithmic_tflop": blk.full_flops() / 1e12,
+                             "TFLOP/s": full_tflops, "tc_frac": full_tflops * 1e3 / tf,
+                             "peak_source": peak_kind},
+        "kv_bridge": {"ms": bridge_ms, "TFLOP/s": bridge_flops / (bridge_ms / 1e3) / 1e12,
+                      "GB/s": bridge_bytes / (bridge_ms / 1e3) / 1e9,
+                      "hbm_frac": bridge_bytes / (bridge_ms / 1e3) / 1e9 / hbm},
+        "sparse_attn": {"ms": sparse_ms},
+        "gpu_launches": K * blk.launches_per_step,
+    }
+
+
 def run_ours(args, ws_, rank, local):
     import kv_shared_b200 as hs
     wl = synth.DECODE_128K
@@ -194,16 +307,7 @@ def run_ours(args, ws_, rank, local):
 
     # each C-ABI call of the step is captured once into a CUDA graph (the calls only
     # enqueue kernels: no allocation, no synchronization) and replayed
-    graphs = []
-    side = torch.cuda.Stream()
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        for fn in [blk.full] + [lambda l=l: blk.sparse(l) for l in range(len(blk.qs))]:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=side):
-                fn()
-            graphs.append(g)
-    stream.wait_stream(side)
+    graphs = _capture([blk.full] + [lambda l=l: blk.sparse(l) for l in range(len(blk.qs))], stream)
     for _ in range(args.warmup):
         for g in graphs:
             g.replay()
@@ -293,6 +397,11 @@ def run_ours(args, ws_, rank, local):
         "gpu_launches": K * blk.launches_per_step,
         "clocks": clk.summary(),
     }
+    del blk, graphs
+    torch.cuda.empty_cache()
+    if not args.no_prefill:
+        out["prefill"] = run_prefill(args, ws_)
+        out["gpu_launches"] += out["prefill"]["gpu_launches"]
     if ws_ == 1 and rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, seed=1002, sample_seqs=args.cpu_sample)
     return out
@@ -360,6 +469,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-sample", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=10)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3

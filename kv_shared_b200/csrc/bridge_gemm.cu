@@ -1,0 +1,186 @@
+// bridge_gemm.cu -- KV Bridging projection on the fifth-generation tensor cores.
+//
+// "Xiaomi Unveils HySparse2 Architecture for MiMo-V3", section "Two-Level KV
+// Sharing: Enabling Prefill Early Exit": the KV cache of the cross-decoder's
+// full-attention layers is generated directly from the self-decoder's hidden
+// states, each target layer with its own K/V projection.  Here:
+//   [K | V] = hidden [rows x d_model] * W_kv [d_model x 2D],  bf16 in, fp32
+//   accumulation, rounded to bf16 and written to cache rows pos0[b] + t.
+//
+// One CTA computes a 128-row x 256-column tile (all of K and V for 128 tokens):
+//   warp 0        TMA producer: A tile [128 x 64] (K-major, 128-byte swizzle) and
+//                 B tile [64 x 256] as four [64 x 64] boxes of W_kv, which is
+//                 row-major (d_model x 2D) and therefore an MN-major B operand
+//   warp 1        allocates 256 TMEM columns; one thread issues tcgen05.mma
+//                 (M=128, N=256, K=16) and commits each stage back to the producer
+//   warps 2..5    epilogue: tcgen05.ld of the fp32 accumulator rows (one TMEM lane
+//                 quarter per warp), bf16 rounding, stores into the cache
+// A 4-stage mbarrier pipeline (48 KB per stage) keeps TMA and MMA overlapped.
+#include "common.cuh"
+#include "internal.h"
+#include "tcgen05.cuh"
+
+namespace hs2 {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int BK = 64;                       // one 128-byte swizzle atom of bf16
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr int B_BYTES = BK * BN * 2;         // 32 KB (four 64x64 boxes)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NT = 192;
+
+struct Params {
+    int rows;                                // batch * n
+    int n;                                   // tokens per sequence
+    int d_model;
+    int64_t cap;
+    const int32_t* pos0;
+    __nv_bfloat16* k;
+    __nv_bfloat16* v;
+    uint32_t* status;                        // may be null
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ CUtensorMap amap,
+                                                      const __grid_constant__ CUtensorMap bmap, Params a) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    __shared__ uint64_t full[STAGES], empty[STAGES], acc_ready;
+    __shared__ uint32_t tmem_base;
+    __shared__ int abort_flag;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.x * BM;
+    const int nk = a.d_model / BK;
+
+    if (threadIdx.x == 0) {
+        prefetch_tmap(&amap);
+        prefetch_tmap(&bmap);
+        for (int s = 0; s < STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+        mbar_init(&acc_ready, 1);
+        fence_mbar_init();
+        abort_flag = 0;
+    }
+    if (warp == 1) umma::tmem_alloc(&tmem_base, 256);
+    umma::fence_before();
+    __syncthreads();
+    umma::fence_after();
+    const uint32_t tmem = tmem_base;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            for (int kb = 0; kb < nk; ++kb) {
+                const int s = kb % STAGES;
+                if (kb >= STAGES && !mbar_wait(&empty[s], ((kb / STAGES) - 1) & 1, a.status)) {
+                    abort_flag = 1;
+                    break;
+                }
+                uint8_t* st = smem + s * STAGE_BYTES;
+                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
+                tma_load_2d(st, &amap, &full[s], kb * BK, m0);
+#pragma unroll
+                for (int nb = 0; nb < BN / 64; ++nb)
+                    tma_load_2d(st + A_BYTES + nb * (BK * 128), &bmap, &full[s], nb * 64, kb * BK);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma::idesc_bf16(BM, BN, false, true);
+            bool ok = true;
+            for (int kb = 0; kb < nk && ok; ++kb) {
+                const int s = kb % STAGES;
+                ok = mbar_wait(&full[s], (kb / STAGES) & 1, a.status);
+                if (!ok) break;
+                umma::fence_after();
+                const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
+                const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk) {
+                    // A: K-major rows of 128 B; step 16 elements = 32 B inside the atom
+                    const uint64_t ad = umma::sdesc_sw128(sa + kk * 32, 16, 1024);
+                    // B: MN-major; 64-column groups 8 KB apart, 8-row K groups 1 KB apart;
+                    // step 16 K-rows = 2 KB
+                    const uint64_t bd = umma::sdesc_sw128(sb + kk * 2048, BK * 128, 1024);
+                    umma::mma_bf16_ss(tmem, ad, bd, idesc, (kb | kk) != 0);
+                }
+                umma::commit(&empty[s]);
+            }
+            if (!ok) abort_flag = 1;
+            umma::commit(&acc_ready);
+        }
+    } else {
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
+        const int q = warp & 3;
+        const int row = m0 + q * 32 + lane;
+        const bool ok = mbar_wait(&acc_ready, 0, a.status);
+        umma::fence_after();
+        __nv_bfloat16* dk = nullptr;
+        __nv_bfloat16* dv = nullptr;
+        if (row < a.rows) {
+            const int b = row / a.n, t = row % a.n;
+            const int p0 = a.pos0[b];
+            if (p0 < 0 || static_cast<int64_t>(p0) + a.n > a.cap) {
+                set_status(a.status, HS2_ERR_INDEX);         // destination outside the cache
+            } else {
+                const int64_t crow = static_cast<int64_t>(b) * a.cap + p0 + t;
+                dk = a.k + crow * 128;
+                dv = a.v + crow * 128;
+            }
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            umma::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, r);
+            umma::tmem_ld_wait();
+            if (dk && ok) {
+                __nv_bfloat16* dst = (c < 4 ? dk : dv) + (c & 3) * 32;
+#pragma unroll
+                for (int j = 0; j < 32; j += 8) {
+                    uint4 pk;
+                    pk.x = pack_bf16(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]));
+                    pk.y = pack_bf16(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                    pk.z = pack_bf16(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+                    pk.w = pack_bf16(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+                    *reinterpret_cast<uint4*>(dst + j) = pk;
+                }
+            }
+        }
+    }
+    umma::fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        umma::fence_after();
+        umma::tmem_dealloc(tmem, 256);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_bridge(const BridgeArgs& ba, cudaStream_t st) {
+    const int rows = ba.batch * ba.n;
+    if (rows <= 0) return cudaSuccess;
+    CUtensorMap amap, bmap;
+    if (!make_tmap_2d(&amap, ba.hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, ba.d_model, rows,
+                      static_cast<uint64_t>(ba.d_model) * 2, BK, BM, true))
+        return cudaErrorInvalidValue;
+    if (!make_tmap_2d(&bmap, ba.w_kv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BN, ba.d_model, BN * 2, 64, BK, true))
+        return cudaErrorInvalidValue;
+    Params a{};
+    a.rows = rows; a.n = ba.n; a.d_model = ba.d_model; a.cap = ba.cap; a.pos0 = ba.pos0;
+    a.k = static_cast<__nv_bfloat16*>(ba.k);
+    a.v = static_cast<__nv_bfloat16*>(ba.v);
+    a.status = ba.status;
+    const size_t smem = 1024 + STAGES * STAGE_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(bridge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    bridge_kernel<<<(rows + BM - 1) / BM, NT, smem, st>>>(amap, bmap, a);
+    return cudaGetLastError();
+}
+
+}  // namespace hs2

@@ -277,20 +277,30 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     if (tid == 0)
         for (int s = 0; s < STAGES && s < n_tiles; ++s) issue(s, s);
 
-    // final log-sum-exp of this thread's two heads from all splits' partials
-    float lse2[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int h = g + 8 * hh;
+    // final log-sum-exp per head: all splits' partials are read in parallel (thread t
+    // takes head t % 16 and every 8th split), then the 8 groups are combined
+    __shared__ float2 lse_part[NT / H][H];
+    __shared__ float lse_s[H];
+    {
+        const int h = tid & (H - 1), grp = tid >> 4;
         float m = -INFINITY, l = 0.f;
-        for (int s = 0; s < a.splits; ++s) {
-            const float2 ml = a.part_ml[(static_cast<size_t>(b) * a.splits + s) * H + h];
+        const float2* pml = a.part_ml + static_cast<size_t>(b) * a.splits * H;
+#pragma unroll 4
+        for (int s = grp; s < a.splits; s += NT / H) {
+            const float2 ml = pml[s * H + h];
             merge_ml(m, l, ml.x, ml.y);
         }
-        lse2[hh] = m + log2f(l);
-        if (split == 0 && warp == 0 && t == 0 && a.lse)
-            a.lse[static_cast<size_t>(b) * H + h] = lse2[hh] * kLn2;
+        lse_part[grp][h] = make_float2(m, l);
+        __syncthreads();
+        if (tid < H) {
+            float mm = -INFINITY, ll = 0.f;
+            for (int q = 0; q < NT / H; ++q) merge_ml(mm, ll, lse_part[q][tid].x, lse_part[q][tid].y);
+            lse_s[tid] = mm + log2f(ll);
+            if (split == 0 && a.lse) a.lse[static_cast<size_t>(b) * H + tid] = lse_s[tid] * kLn2;
+        }
+        __syncthreads();
     }
+    float lse2[2] = {lse_s[g], lse_s[g + 8]};
 
     float o[16][4];
 #pragma unroll
@@ -385,11 +395,29 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const float* base = a.part_o + static_cast<size_t>(b) * a.splits * H * D;
-    for (int i = tid; i < H * D; i += NT) {
-        float acc = 0.f;
-        for (int s = 0; s < a.splits; ++s) acc += __ldcg(base + static_cast<size_t>(s) * H * D + i);
-        a.o[static_cast<size_t>(b) * H * D + i] = __float2bfloat16_rn(acc);
+    // sum of the split partials with independent 16-byte loads (4 per thread per split)
+    const float4* base4 = reinterpret_cast<const float4*>(a.part_o + static_cast<size_t>(b) * a.splits * H * D);
+    constexpr int F4 = H * D / 4;
+    constexpr int PER = F4 / NT;
+    float4 acc[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = 0; s < a.splits; ++s) {
+        float4 v[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) v[k] = __ldcg(base4 + static_cast<size_t>(s) * F4 + tid + k * NT);
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            acc[k].x += v[k].x; acc[k].y += v[k].y; acc[k].z += v[k].z; acc[k].w += v[k].w;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        uint2 packed;
+        packed.x = pack_bf16(acc[k].x, acc[k].y);
+        packed.y = pack_bf16(acc[k].z, acc[k].w);
+        *reinterpret_cast<uint2*>(a.o + static_cast<size_t>(b) * H * D + 4 * (tid + k * NT)) = packed;
     }
 }
 

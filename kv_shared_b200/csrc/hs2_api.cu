@@ -103,6 +103,7 @@ size_t full_region(const hs2_attn_desc* d, Path path, bool scores_in_ws) {
     const size_t rows = static_cast<size_t>(d->batch) * d->n_q;
     size_t n = 0;
     if (path == Path::TC && d->n_q == 1) n += a256(decode_ws_bytes(d->batch, d->max_ctx));
+    if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q));
     if (scores_in_ws) n += a256(sizeof(float) * rows * static_cast<size_t>(score_pitch(d)));
     return n;
 }
@@ -145,7 +146,7 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     for (const void* p : ptrs)
         if (!aligned16(p)) return HS2_ERR_INVALID_ARG;
     if ((lse && !aligned16(lse)) || (scores && !aligned16(scores)) || !aligned16(q_pos0)) return HS2_ERR_INVALID_ARG;
-    if (path == Path::TC && desc->n_q != 1) return HS2_ERR_UNSUPPORTED;
+    if (path == Path::TC && desc->n_q > 1 && desc->kv_dtype != HS2_BF16) return HS2_ERR_UNSUPPORTED;
     if (ws_bytes < hs2_workspace_size(desc, scores == nullptr)) return HS2_ERR_WORKSPACE;
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -156,7 +157,9 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     float* score_buf = scores;
     int64_t score_ld = desc->max_ctx;
     size_t used = 0;
-    if (path == Path::TC) used = a256(decode_ws_bytes(desc->batch, desc->max_ctx));
+    if (path == Path::TC)
+        used = desc->n_q == 1 ? a256(decode_ws_bytes(desc->batch, desc->max_ctx))
+                              : a256(prefill_ws_bytes(desc->batch, desc->n_q));
     if (!score_buf) {
         score_buf = reinterpret_cast<float*>(region + used);
         score_ld = score_pitch(desc);
@@ -172,6 +175,12 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
         a.scale = scale; a.o = static_cast<float*>(o); a.lse = lse;
         a.scores = score_buf; a.score_ld = score_ld; a.status = status;
         e = launch_f32_full(a, st);
+    } else if (desc->n_q > 1) {
+        PrefillArgs a{};
+        a.batch = desc->batch; a.n_q = desc->n_q; a.cap = desc->kv_capacity; a.max_ctx = desc->max_ctx;
+        a.q_pos0 = q_pos0; a.q = q; a.k = k; a.v = v; a.scale = scale; a.o = o; a.lse = lse;
+        a.scores = score_buf; a.score_ld = score_ld; a.ws = region; a.status = status;
+        e = launch_prefill_full(a, st);
     } else {
         DecodeArgs a{};
         a.batch = desc->batch; a.cap = desc->kv_capacity; a.max_ctx = desc->max_ctx; a.q_pos0 = q_pos0;
@@ -276,8 +285,16 @@ hs2_status hs2_kv_bridge_proj(const void* hidden, const void* w_kv, int32_t batc
                               hs2_stream_t stream) {
     if (!hidden || !w_kv || !pos0 || !k || !v || batch < 1 || n < 1 || d_model < 1 || kv_capacity < n)
         return HS2_ERR_INVALID_ARG;
-    (void)head_dim; (void)stream;
-    return HS2_ERR_UNSUPPORTED;
+    const void* ptrs[] = {hidden, w_kv, pos0, k, v};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return HS2_ERR_INVALID_ARG;
+    if (head_dim != 128 || d_model % 64 != 0) return HS2_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(batch) * n >= (int64_t(1) << 31) || static_cast<int64_t>(batch) * kv_capacity >= (int64_t(1) << 31))
+        return HS2_ERR_UNSUPPORTED;
+    BridgeArgs a{};
+    a.hidden = hidden; a.w_kv = w_kv; a.batch = batch; a.n = n; a.d_model = d_model;
+    a.pos0 = pos0; a.cap = kv_capacity; a.k = k; a.v = v; a.status = nullptr;
+    return from_cuda(launch_bridge(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hs2_status hs2_kv_quantize_fp8(const float* src, int64_t rows, int32_t head_dim, uint8_t* codes, float* scales,

@@ -49,6 +49,25 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode_full(const DecodeArgs& a, cudaStream_t st);
 
+// ---------------------------------------------------------------- prefill (n_q > 1), tcgen05
+struct PrefillArgs {
+    int batch, n_q;
+    int64_t cap, max_ctx;
+    const int32_t* q_pos0;
+    const void* q;            // [B][n_q][16][128] bf16
+    const void* k;            // [B][cap][128] bf16
+    const void* v;
+    float scale;
+    void* o;                  // [B][n_q][16][128] bf16
+    float* lse;               // [B][n_q][16] natural log, or null
+    float* scores;            // [B][n_q][score_ld]
+    int64_t score_ld;
+    void* ws;                 // prefill_ws_bytes: per-(row, head) log-sum-exp
+    uint32_t* status;
+};
+size_t prefill_ws_bytes(int batch, int n_q);
+cudaError_t launch_prefill_full(const PrefillArgs& a, cudaStream_t st);
+
 // ---------------------------------------------------------------- selection
 struct SelectArgs {
     int rows;                 // batch * n_q
@@ -120,6 +139,19 @@ struct F32Args {
 };
 cudaError_t launch_f32_full(const F32Args& a, cudaStream_t st);
 cudaError_t launch_f32_sparse(const F32Args& a, cudaStream_t st);
+
+// ---------------------------------------------------------------- KV bridge GEMM
+struct BridgeArgs {
+    const void* hidden;      // [batch][n][d_model] bf16
+    const void* w_kv;        // [d_model][256] bf16
+    int batch, n, d_model;
+    const int32_t* pos0;     // [batch] device
+    int64_t cap;
+    void* k;                 // [batch][cap][128] bf16
+    void* v;
+    uint32_t* status;        // may be null
+};
+cudaError_t launch_bridge(const BridgeArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- fp8 quantizer
 cudaError_t launch_fp8_quantize(const float* src, int64_t rows, int head_dim, uint8_t* codes,

@@ -25,6 +25,7 @@ constexpr int H = 16;
 constexpr int D = 128;
 constexpr int SUB = 64;            // gathered rows per pipeline stage
 constexpr int NT = 128;            // 4 warps x 16 rows
+constexpr int kMaxSplits = 32;     // bound of the split count (shared-memory merge tables)
 
 struct Params {
     int rows, n_q, idx_stride, splits, chunk;
@@ -314,27 +315,53 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     if (!s_last) return;
     __threadfence();
     if (tid == 0) a.counter[row] = 0;          // ready for the next launch
-    // merge the splits
-    __shared__ float fm[H], fl[H];
+    // merge the splits: every split's (max, sum) is staged in shared memory by one
+    // parallel round of loads, then the partial outputs are weighted and summed with
+    // independent 16-byte loads (4 per thread per split)
+    __shared__ float2 sml[kMaxSplits][H];
+    __shared__ float sw[kMaxSplits][H];
+    __shared__ float fm[H], finv[H];
+    const float2* pml = a.part_ml + static_cast<size_t>(row) * a.splits * H;
+    for (int i = tid; i < a.splits * H; i += NT) sml[i / H][i % H] = __ldcg(pml + i);
+    __syncthreads();
     if (tid < H) {
         float m = -INFINITY, l = 0.f;
-        for (int sp = 0; sp < a.splits; ++sp) {
-            const float2 ml = __ldcg(&a.part_ml[(static_cast<size_t>(row) * a.splits + sp) * H + tid]);
-            merge_ml(m, l, ml.x, ml.y);
-        }
-        fm[tid] = m; fl[tid] = l;
+        for (int sp = 0; sp < a.splits; ++sp) merge_ml(m, l, sml[sp][tid].x, sml[sp][tid].y);
+        fm[tid] = m;
+        finv[tid] = l > 0.f ? 1.f / l : 0.f;
         if (a.lse) a.lse[static_cast<size_t>(row) * H + tid] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
     __syncthreads();
-    const float* base = a.part_o + static_cast<size_t>(row) * a.splits * H * D;
-    for (int i = tid; i < H * D; i += NT) {
-        const int h = i / D;
-        float acc = 0.f;
-        for (int sp = 0; sp < a.splits; ++sp) {
-            const float2 ml = __ldcg(&a.part_ml[(static_cast<size_t>(row) * a.splits + sp) * H + h]);
-            if (ml.x != -INFINITY) acc += __ldcg(base + static_cast<size_t>(sp) * H * D + i) * exp2f(ml.x - fm[h]);
+    for (int i = tid; i < a.splits * H; i += NT) {
+        const int sp = i / H, h = i % H;
+        const float mm = sml[sp][h].x;
+        sw[sp][h] = (mm == -INFINITY) ? 0.f : exp2f(mm - fm[h]) * finv[h];
+    }
+    __syncthreads();
+    const float4* base4 = reinterpret_cast<const float4*>(a.part_o + static_cast<size_t>(row) * a.splits * H * D);
+    constexpr int F4 = H * D / 4;                  // float4 per split partial
+    constexpr int PER = F4 / NT;                   // 4 per thread
+    float4 acc[PER];
+#pragma unroll
+    for (int k = 0; k < PER; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 3
+    for (int sp = 0; sp < a.splits; ++sp) {
+        float4 v[PER];
+#pragma unroll
+        for (int k = 0; k < PER; ++k) v[k] = __ldcg(base4 + static_cast<size_t>(sp) * F4 + tid + k * NT);
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const float w = sw[sp][(tid + k * NT) / (D / 4)];
+            acc[k].x += w * v[k].x; acc[k].y += w * v[k].y; acc[k].z += w * v[k].z; acc[k].w += w * v[k].w;
         }
-        a.o[static_cast<size_t>(row) * H * D + i] = __float2bfloat16_rn(fl[h] > 0.f ? acc / fl[h] : 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int f = tid + k * NT;
+        uint2 packed;
+        packed.x = pack_bf16(acc[k].x, acc[k].y);
+        packed.y = pack_bf16(acc[k].z, acc[k].w);
+        *reinterpret_cast<uint2*>(a.o + static_cast<size_t>(row) * H * D + 4 * f) = packed;
     }
 }
 
@@ -386,7 +413,8 @@ SparsePlan plan_sparse(int rows, int idx_stride) {
     SparsePlan pl;
     // enough CTAs to cover the SMs twice; one CTA per row when rows alone do
     int splits = (2 * num_sms() + rows - 1) / (rows > 0 ? rows : 1);
-    const int max_splits = (idx_stride + SUB - 1) / SUB;
+    int max_splits = (idx_stride + SUB - 1) / SUB;
+    if (max_splits > kMaxSplits) max_splits = kMaxSplits;
     if (splits > max_splits) splits = max_splits;
     if (splits < 1) splits = 1;
     int chunk = (idx_stride + splits - 1) / splits;

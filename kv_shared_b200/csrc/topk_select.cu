@@ -10,28 +10,47 @@
 // kept whole if any of its tokens is important): blocks of `bs` positions from
 // 0, block importance = max, floor(K/bs) best blocks (lower block on ties).
 //
-// One CTA per row.  The K-th best key is found exactly by a three-digit radix
-// select (11 + 11 + 10 bits) on order-preserving uint32 images of the fp32
-// values; then one ascending pass writes every candidate above the threshold
-// and the first (K - #above) candidates equal to it, which is the lower-index
-// tie rule, already in ascending order.  Integer work only after the key map.
+// A row is handled by a cluster of CS CTAs (CS = 1..8); CTA r owns a contiguous
+// slice of the candidates and keeps their order-preserving uint32 images in
+// shared memory when they fit.  The K-th best key is found exactly by a
+// three-digit radix select (11 + 11 + 10 bits): per digit every CTA builds a
+// histogram of its slice, the cluster's histograms are summed over distributed
+// shared memory and each CTA takes the same decision.  Then every CTA writes,
+// in ascending order, its keys above the threshold and its share of the first
+// (K - #above) keys equal to it (the lower-index tie rule), at offsets from a
+// cluster-wide prefix of the counts.  Integer work only after the key map.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace hs2 {
 namespace {
 
-constexpr int NT = 1024;
+constexpr int NT = 512;
 constexpr int NW = NT / 32;
+constexpr int NBINS = 2048;
+constexpr int kMaxCluster = 8;
+constexpr int kSmemKeys = 32768;          // keys cached per CTA (128 KB)
 
 __device__ __forceinline__ uint32_t ord_key(float f) {
     const uint32_t u = __float_as_uint(f);
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Block-wide exclusive scan of one int per thread; returns the exclusive prefix
-// and writes the total to *total.  All threads must call it.
-__device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total) {
+struct Smem {
+    int hist[NBINS];
+    int warp_tot[NW];
+    int total;
+    int found_bin;
+    int found_above;
+    int counts[2];              // this CTA's (#above, #equal) for the compaction
+};
+
+// Block-wide exclusive scan of one int per thread; *total receives the sum.
+__device__ __forceinline__ int block_excl_scan(int v, Smem& sm) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
 #pragma unroll
@@ -39,197 +58,246 @@ __device__ __forceinline__ int block_excl_scan(int v, int* warp_tot, int* total)
         const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
-    if (lane == 31) warp_tot[warp] = x;
+    if (lane == 31) sm.warp_tot[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        int w = lane < NW ? warp_tot[lane] : 0;
+        const int w = lane < NW ? sm.warp_tot[lane] : 0;
         int s = w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const int y = __shfl_up_sync(0xffffffffu, s, o);
             if (lane >= o) s += y;
         }
-        if (lane < NW) warp_tot[lane] = s - w;      // exclusive warp offsets
-        if (lane == NW - 1) *total = s;
+        if (lane < NW) sm.warp_tot[lane] = s - w;
+        if (lane == NW - 1) sm.total = s;
     }
     __syncthreads();
-    const int r = warp_tot[warp] + x - v;
+    const int r = sm.warp_tot[warp] + x - v;
     __syncthreads();
     return r;
 }
 
-struct Smem {
-    int hist[2048];
-    int warp_tot[NW];
-    int total;
-    int found_bin;
-    int found_above;
+// Keys of this CTA's slice: cached in shared memory or recomputed from global.
+struct Slice {
+    const float* s;            // row scores
+    int bs;                    // 1 = token keys, >1 = block maxima
+    int n_cand;                // candidates of the row
+    int begin, end;            // this CTA's key range (tokens or blocks)
+    uint32_t* cache;           // shared-memory copy or nullptr
+    __device__ __forceinline__ uint32_t compute(int i) const {
+        if (bs == 1) return ord_key(s[i]);
+        float m = -INFINITY;
+        const int e = min((i + 1) * bs, n_cand);
+        for (int j = i * bs; j < e; ++j) m = fmaxf(m, s[j]);
+        return ord_key(m);
+    }
+    __device__ __forceinline__ uint32_t key(int i) const { return cache ? cache[i - begin] : compute(i); }
 };
 
-// Exact K-th largest key among n keys given by get(i) (K in [1, n-1]).
-// Returns the threshold key; *need_eq = how many keys equal to it are taken.
-template <typename Get>
-__device__ uint32_t radix_threshold(Get get, int n, int K, Smem& sm, int* need_eq) {
-    uint32_t prefix = 0, mask = 0;
-    int k_rem = K;
-    const int shifts[3] = {21, 10, 0};
-    const int widths[3] = {11, 11, 10};
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = shifts[pass], nb = 1 << widths[pass];
-        for (int i = threadIdx.x; i < nb; i += NT) sm.hist[i] = 0;
-        __syncthreads();
-        for (int i = threadIdx.x; i < n; i += NT) {
-            const uint32_t key = get(i);
-            if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (nb - 1)], 1);
-        }
-        __syncthreads();
-        // suffix counts from the top: thread j owns bins [j*per, (j+1)*per) counted from the top
-        const int per = nb / NT;                       // 2 (first two passes) or 1
-        int local = 0;
-        for (int q = 0; q < per; ++q) local += sm.hist[nb - 1 - (threadIdx.x * per + q)];
-        const int above = block_excl_scan(local, sm.warp_tot, &sm.total);
-        if (above < k_rem && above + local >= k_rem) {
-            int acc = above;
-            for (int q = 0; q < per; ++q) {
-                const int bin = nb - 1 - (threadIdx.x * per + q);
-                const int c = sm.hist[bin];
-                if (acc + c >= k_rem) { sm.found_bin = bin; sm.found_above = acc; break; }
-                acc += c;
-            }
-        }
-        __syncthreads();
-        prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
-        mask |= static_cast<uint32_t>(nb - 1) << shift;
-        k_rem -= sm.found_above;
-        __syncthreads();
-    }
-    *need_eq = k_rem;
-    return prefix;
-}
-
-__global__ void __launch_bounds__(NT) select_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int cache_keys) {
+    extern __shared__ uint32_t key_cache[];
     __shared__ Smem sm;
-    const int row = blockIdx.x;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int row = blockIdx.x / cs;
     const int b = row / a.n_q, r = row % a.n_q;
     const int p = checked_pos(a.q_pos0[b] + r, a.max_ctx, a.status);
-    const float* s = a.scores + static_cast<size_t>(row) * a.score_ld;
     int32_t* out = a.idx + static_cast<size_t>(row) * a.idx_stride;
     const int W = a.window;
     const int n_cand = max(p - W + 1, 0);
-    const int w0 = max(p - W + 1, 0);
-    int written = 0;
+    const int w0 = n_cand;
+    const int bs = a.block_size < 1 ? 1 : a.block_size;
+    const int n_keys = (n_cand + bs - 1) / bs;                    // tokens or blocks
+    const int K = bs == 1 ? min(a.budget, n_cand) : min(a.budget / bs, n_keys);
 
-    if (a.block_size <= 1) {
-        const int K = min(a.budget, n_cand);
-        if (K > 0) {
-            uint32_t tau = 0;
-            int need_eq = 0;
-            if (K < n_cand) {
-                tau = radix_threshold([&](int i) { return ord_key(s[i]); }, n_cand, K, sm, &need_eq);
+    Slice sl;
+    sl.s = a.scores + static_cast<size_t>(row) * a.score_ld;
+    sl.bs = bs;
+    sl.n_cand = n_cand;
+    const int per = ((n_keys + cs - 1) / cs + 3) & ~3;
+    sl.begin = min(rank * per, n_keys);
+    sl.end = min(sl.begin + per, n_keys);
+    sl.cache = (per <= cache_keys) ? key_cache : nullptr;
+    if (sl.cache)
+        for (int i = sl.begin + threadIdx.x; i < sl.end; i += NT) sl.cache[i - sl.begin] = sl.compute(i);
+    __syncthreads();
+
+    uint32_t tau = 0;
+    int need_eq = 0;
+    const bool take_all = (K >= n_keys);
+    const bool take_none = (K <= 0);
+    if (!take_all && K > 0) {
+        uint32_t prefix = 0, mask = 0;
+        int k_rem = K;
+        const int shifts[3] = {21, 10, 0};
+        const int widths[3] = {11, 11, 10};
+#pragma unroll 1
+        for (int pass = 0; pass < 3; ++pass) {
+            const int shift = shifts[pass], nb = 1 << widths[pass];
+            for (int i = threadIdx.x; i < nb; i += NT) sm.hist[i] = 0;
+            __syncthreads();
+            for (int i = sl.begin + threadIdx.x; i < sl.end; i += NT) {
+                const uint32_t key = sl.key(i);
+                if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (nb - 1)], 1);
             }
-            // ascending compaction: 4 consecutive candidates per thread per round
-            int eq_seen = 0;
-            for (int base = 0; base < n_cand; base += 4 * NT) {
-                const int j0 = base + 4 * threadIdx.x;
-                int gt = 0, eq = 0;
-                uint32_t keys[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j = j0 + u;
-                    keys[u] = (j < n_cand) ? ord_key(s[j]) : 0u;
-                    if (j < n_cand && K < n_cand) {
-                        gt += keys[u] > tau;
-                        eq += keys[u] == tau;
+            cluster.sync();
+            // counts of the whole row: sum of the cluster's histograms (from the top bin)
+            const int bins_per = nb / NT;                               // 4 or 2
+            int local[NBINS / NT];
+            int tot = 0;
+            for (int q = 0; q < bins_per; ++q) {
+                const int bin = nb - 1 - (threadIdx.x * bins_per + q);
+                int c = 0;
+                for (int rr = 0; rr < cs; ++rr) c += cluster.map_shared_rank(sm.hist, rr)[bin];
+                local[q] = c;
+                tot += c;
+            }
+            cluster.sync();                    // every CTA has read every histogram
+            const int above = block_excl_scan(tot, sm);
+            if (above < k_rem && above + tot >= k_rem) {
+                int acc = above;
+                for (int q = 0; q < bins_per; ++q) {
+                    if (acc + local[q] >= k_rem) {
+                        sm.found_bin = nb - 1 - (threadIdx.x * bins_per + q);
+                        sm.found_above = acc;
+                        break;
                     }
+                    acc += local[q];
                 }
-                const int eq_before = block_excl_scan(eq, sm.warp_tot, &sm.total);
-                const int eq_round = sm.total;
-                // number selected by this thread
-                int rank = eq_seen + eq_before, mine = 0;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j = j0 + u;
-                    if (j >= n_cand) break;
-                    bool sel;
-                    if (K == n_cand) sel = true;
-                    else if (keys[u] > tau) sel = true;
-                    else if (keys[u] == tau) { sel = rank < need_eq; ++rank; }
-                    else sel = false;
-                    mine += sel;
-                }
-                (void)gt;
-                const int pos = block_excl_scan(mine, sm.warp_tot, &sm.total);
-                const int round_total = sm.total;
-                rank = eq_seen + eq_before;
-                int o = written + pos;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int j = j0 + u;
-                    if (j >= n_cand) break;
-                    bool sel;
-                    if (K == n_cand) sel = true;
-                    else if (keys[u] > tau) sel = true;
-                    else if (keys[u] == tau) { sel = rank < need_eq; ++rank; }
-                    else sel = false;
-                    if (sel) out[o++] = j;
-                }
-                written += round_total;
-                eq_seen += eq_round;
-                __syncthreads();
             }
+            __syncthreads();
+            prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
+            mask |= static_cast<uint32_t>(nb - 1) << shift;
+            k_rem -= sm.found_above;
+            __syncthreads();
         }
-    } else {
-        // block arm: block importance = max over its tokens inside the candidates,
-        // recomputed on every pass (no scratch)
-        const int bs = a.block_size;
-        const int nb = (n_cand + bs - 1) / bs;
-        const int Kb = min(a.budget / bs, nb);
-        auto bkey = [&](int bb) {
-            float m = -INFINITY;
-            const int e = min((bb + 1) * bs, n_cand);
-            for (int j = bb * bs; j < e; ++j) m = fmaxf(m, s[j]);
-            return ord_key(m);
-        };
-        if (Kb > 0) {
-            uint32_t tau = 0;
-            int need_eq = 0;
-            if (Kb < nb) tau = radix_threshold(bkey, nb, Kb, sm, &need_eq);
-            int eq_seen = 0;
-            for (int base = 0; base < nb; base += NT) {
-                const int bb = base + threadIdx.x;
-                const uint32_t key = bb < nb ? bkey(bb) : 0u;
-                const int eq = (bb < nb && Kb < nb && key == tau) ? 1 : 0;
-                const int eq_before = block_excl_scan(eq, sm.warp_tot, &sm.total);
-                const int eq_round = sm.total;
-                bool sel = false;
-                if (bb < nb) {
-                    if (Kb == nb || key > tau) sel = true;
-                    else if (key == tau) sel = (eq_seen + eq_before) < need_eq;
-                }
-                const int ntok = sel ? (min((bb + 1) * bs, n_cand) - bb * bs) : 0;
-                const int pos = block_excl_scan(ntok, sm.warp_tot, &sm.total);
-                const int round_total = sm.total;
-                for (int u = 0; u < ntok; ++u) out[written + pos + u] = bb * bs + u;
-                written += round_total;
-                eq_seen += eq_round;
-                __syncthreads();
-            }
+        tau = prefix;
+        need_eq = k_rem;
+    }
+
+    // this CTA's counts, then cluster-wide offsets
+    int gt = 0, eq = 0;
+    if (!take_all && K > 0) {
+        for (int i = sl.begin + threadIdx.x; i < sl.end; i += NT) {
+            const uint32_t key = sl.key(i);
+            gt += key > tau;
+            eq += key == tau;
         }
     }
-    // forced window after the global picks (all window positions exceed every candidate)
-    for (int j = w0 + threadIdx.x; j <= p; j += NT) out[written + (j - w0)] = j;
-    const int total = written + (p - w0 + 1);
-    for (int i = total + threadIdx.x; i < a.idx_stride; i += NT) out[i] = -1;
-    if (threadIdx.x == 0) a.cnt[row] = total;
+    int t_gt = block_excl_scan(gt, sm);
+    t_gt = sm.total;
+    int t_eq = block_excl_scan(eq, sm);
+    t_eq = sm.total;
+    (void)t_gt;
+    if (threadIdx.x == 0) { sm.counts[0] = t_gt; sm.counts[1] = t_eq; }
+    cluster.sync();
+    int out_base = 0, eq_base = 0;                   // tokens written / equal keys seen before this CTA
+    for (int rr = 0; rr < rank; ++rr) {
+        const int* c = cluster.map_shared_rank(sm.counts, rr);
+        const int e_before = eq_base;
+        const int take_eq = take_all ? 0 : max(0, min(c[1], need_eq - e_before));
+        int keys_sel;
+        if (take_all) {
+            const int rb = min(rr * per, n_keys), re = min(rb + per, n_keys);
+            keys_sel = re - rb;
+        } else {
+            keys_sel = c[0] + take_eq;
+        }
+        // tokens: blocks expand to bs tokens (only the row's last block is partial, and it
+        // belongs to the last CTA, never to a lower rank)
+        out_base += keys_sel * bs;
+        eq_base += c[1];
+    }
+    cluster.sync();                                  // remote counts read: they may be reused
+
+    // ascending compaction of this CTA's slice, 4 consecutive keys per thread per round
+    int eq_seen = eq_base;
+    int written = out_base;
+    for (int base = sl.begin; base < (take_none ? sl.begin : sl.end); base += 4 * NT) {
+        const int i0 = base + 4 * threadIdx.x;
+        uint32_t keys[4];
+        int e_cnt = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            keys[u] = (i < sl.end) ? sl.key(i) : 0u;
+            if (i < sl.end && !take_all) e_cnt += keys[u] == tau;
+        }
+        const int eq_before = block_excl_scan(e_cnt, sm);
+        const int eq_round = sm.total;
+        int rank_eq = eq_seen + eq_before, ntok = 0;
+        bool sel[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = i0 + u;
+            sel[u] = false;
+            if (i >= sl.end) continue;
+            if (take_all || keys[u] > tau) sel[u] = true;
+            else if (keys[u] == tau) { sel[u] = rank_eq < need_eq; ++rank_eq; }
+            if (sel[u]) ntok += min((i + 1) * bs, n_cand) - i * bs;
+        }
+        const int pos = block_excl_scan(ntok, sm);
+        const int round_total = sm.total;
+        int o = written + pos;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (!sel[u]) continue;
+            const int i = i0 + u;
+            const int e = min((i + 1) * bs, n_cand);
+            for (int j = i * bs; j < e; ++j) out[o++] = j;
+        }
+        written += round_total;
+        eq_seen += eq_round;
+    }
+
+    // the forced window after all global picks (every window position exceeds every
+    // candidate), written by the CTA owning the last candidate key: its running count
+    // is exact (a partial last block is counted with its true length)
+    const int writer = n_keys > 0 ? min((n_keys - 1) / per, cs - 1) : 0;
+    if (rank == writer) {
+        for (int j = w0 + threadIdx.x; j <= p; j += NT) out[written + (j - w0)] = j;
+        const int total = written + (p - w0 + 1);
+        for (int i = total + threadIdx.x; i < a.idx_stride; i += NT) out[i] = -1;
+        if (threadIdx.x == 0) a.cnt[row] = total;
+    }
+    cluster.sync();                                  // no CTA leaves while its memory may be read
+}
+
+int pick_cluster(int rows, int64_t max_keys) {
+    int cs = 1;
+    while (cs < kMaxCluster && (max_keys + cs - 1) / cs > kSmemKeys) cs *= 2;
+    const int target = 2 * num_sms();
+    while (cs < kMaxCluster && static_cast<int64_t>(rows) * cs * 2 <= target && max_keys / (cs * 2) >= 1024)
+        cs *= 2;
+    return cs;
 }
 
 }  // namespace
 
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
     if (a.rows <= 0) return cudaSuccess;
-    select_kernel<<<a.rows, NT, 0, st>>>(a);
-    return cudaGetLastError();
+    const int bs = a.block_size < 1 ? 1 : a.block_size;
+    const int64_t max_keys = (a.max_ctx + bs - 1) / bs;
+    const int cs = pick_cluster(a.rows, max_keys);
+    const int64_t per = ((max_keys + cs - 1) / cs + 3) & ~int64_t(3);
+    const int cache_keys = per <= kSmemKeys ? static_cast<int>(per) : 0;
+    const size_t smem = static_cast<size_t>(cache_keys) * sizeof(uint32_t);
+    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(a.rows) * cs);
+    cfg.blockDim = dim3(NT);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, select_kernel, a, cs, cache_keys);
 }
 
 }  // namespace hs2

@@ -42,13 +42,22 @@ def compare_out(gpu, ref, kv_dtype, what="O"):
     return float(err.max()), float(rel)
 
 
-def compare_scores(gpu, ref, pos):
-    """gpu/ref [rows, >= p+1]; only entries 0..p of each row are defined."""
+def compare_scores(gpu, ref, pos, bridged_from=None):
+    """gpu/ref [rows, >= p+1]; only entries 0..p of each row are defined.
+
+    Keys at positions >= bridged_from come from the KV-bridge projection, whose GPU
+    result may differ from the oracle's by one bf16 ulp in an element (fp32 versus
+    exact accumulation before rounding); one ulp (<= 2^-7 relative) moves that key's
+    logit by <= scale * sum_d |q_d| |k_d| 2^-7, i.e. up to ~1e-2 relative in its
+    probabilities at these magnitudes, so those keys get rtol 1e-2."""
     worst = 0.0
     for r, p in enumerate(pos):
         g = np.asarray(gpu[r, :p + 1], dtype=np.float64)
         o = ref[r, :p + 1]
-        bad = np.abs(g - o) > 1e-4 * np.abs(o) + 1e-8
+        rtol = np.full(p + 1, 1e-4)
+        if bridged_from is not None:
+            rtol[bridged_from:] = 1e-2
+        bad = np.abs(g - o) > rtol * np.abs(o) + 1e-8
         assert not bad.any(), f"row {r}: {bad.sum()} scores out of tolerance, e.g. j={np.flatnonzero(bad)[:5]}"
         worst = max(worst, float((np.abs(g - o) / (np.abs(o) + 1e-30)).max()))
     return worst
@@ -134,6 +143,7 @@ class Dev:
 
     # ---- oracle inputs: the generator's bytes; an e4m3 cache is quantized by the oracle itself
     def kv_f64(self, b):
+        """Oracle K/V of sequence b (fp64) from the generator's bytes."""
         if self.wl.kv_dtype == "e4m3":
             out = []
             for src in (self.k_src, self.v_src):
@@ -141,3 +151,86 @@ class Dev:
                 out.append(oracle.fp8_dequantize(codes, scales))
             return out[0], out[1]
         return f64(self.k_in[b]), f64(self.v_in[b])
+
+
+def _dev_bridge(self):
+    """KV bridging on the GPU: rows [ctx - n_new, ctx) of every sequence's cache."""
+    wl = self.wl
+    self.pos0_new = torch.full((wl.batch,), wl.ctx - wl.n_new, dtype=torch.int32, device="cuda")
+    hs.hs2_kv_bridge_proj(self.hidden, self.w_kv, wl.batch, wl.n_new, wl.d_model, wl.head_dim,
+                          self.pos0_new, wl.ctx, self.k, self.v)
+
+
+def _oracle_bridged_kv(self, b, k, v):
+    """The oracle's own bridge rows (fp64 product rounded to bf16) replace the placeholders."""
+    wl = self.wl
+    kk, vv = oracle.bridge(f64(self.hidden_in[b]), f64(self.w_in), wl.head_dim)
+    k = k.copy()
+    v = v.copy()
+    k[wl.ctx - wl.n_new:] = oracle.bf16_to_f64(oracle.round_bf16(kk))
+    v[wl.ctx - wl.n_new:] = oracle.bf16_to_f64(oracle.round_bf16(vv))
+    return k, v
+
+
+Dev.bridge = _dev_bridge
+Dev.oracle_bridged_kv = _oracle_bridged_kv
+
+
+def block_parity(wl, seed, seqs=None, device="cpu", rows=None):
+    """Runs the hybrid block through the C ABI and checks it against the oracle on the
+    given sequences and query rows (all by default)."""
+    import synth
+    inp = synth.make_inputs(wl, seed=seed, device=device)
+    dev = Dev(inp)
+    if wl.n_new:
+        dev.hidden_in, dev.w_in = inp.hidden, inp.w_kv
+        dev.hidden = inp.hidden.to("cuda").contiguous()
+        dev.w_kv = inp.w_kv.to("cuda").contiguous()
+        dev.bridge()
+    dev.full()
+    for l in range(wl.n_sparse):
+        dev.sparse(l)
+    assert dev.status() == hs.HS2_OK
+    seqs = range(wl.batch) if seqs is None else seqs
+    rows = np.arange(wl.n_q) if rows is None else np.asarray(rows)
+    pos = wl.q_pos0 + rows
+    report = {"differing_rows": 0, "rows": 0}
+    for b in seqs:
+        k, v = dev.kv_f64(b)
+        if wl.n_new:
+            k, v = dev.oracle_bridged_kv(b, k, v)
+        qf = f64(inp.q_full[b])[rows]
+        o_ref, lse_ref, sc_ref = oracle.full_attn(qf, k, v, pos)
+        compare_out(f64(dev.o_full[b])[rows], o_ref, wl.kv_dtype, "O_full")
+        np.testing.assert_allclose(dev.lse[b].cpu().numpy()[rows], lse_ref, rtol=1e-4, atol=1e-4)
+        compare_scores(dev.scores[b, torch.from_numpy(rows).cuda()].cpu().numpy(), sc_ref, pos,
+                       bridged_from=(wl.ctx - wl.n_new) if wl.n_new else None)
+        o_idx, o_cnt = oracle.select_rows(sc_ref, pos, wl.window, wl.budget, block_size=wl.block_size)
+        g_idx = dev.idx[b].cpu().numpy()[rows]
+        g_cnt = dev.cnt[b].cpu().numpy()[rows]
+        report["differing_rows"] += check_selection(g_idx, g_cnt, o_idx, o_cnt, sc_ref, pos, wl.window)
+        report["rows"] += len(rows)
+        if inp.needle_pos is not None and wl.block_size == 1:
+            sel = set(g_idx[-1, :g_cnt[-1]].tolist())
+            assert set(inp.needle_pos[b].tolist()) <= sel, "planted key not selected"
+        same = np.array([np.array_equal(g_idx[r], o_idx[r]) for r in range(len(rows))])
+        oi = torch.from_numpy(o_idx[None]).cuda()
+        oc = torch.from_numpy(o_cnt[None]).cuda()
+        rsel = torch.from_numpy(rows).cuda()
+        for l in range(wl.n_sparse):
+            o_sp_ref = oracle.sparse_attn(f64(inp.q_sparse[l][b])[rows], k, v, o_idx, o_cnt)
+            # end to end (GPU indices) where the index sets agree
+            if same.any():
+                compare_out(f64(dev.o_sparse[l][b])[rows][same], o_sp_ref[same], wl.kv_dtype, f"O_sparse{l}")
+            # and the kernel alone on the oracle's selection, every sampled row
+            desc1 = hs.make_desc(1, len(rows), wl.heads, wl.head_dim, wl.window, wl.budget,
+                                 q_dtype=dev.desc.q_dtype, kv_dtype=dev.desc.kv_dtype, max_ctx=wl.ctx)
+            q1 = dev.q_sparse[l][b][rsel].unsqueeze(0).contiguous()
+            o1 = torch.empty_like(q1)
+            ws1 = hs.alloc_workspace(desc1)
+            ks = dev.k_scale[b:b + 1] if dev.k_scale is not None else None
+            vs = dev.v_scale[b:b + 1] if dev.v_scale is not None else None
+            hs.hs2_sparse_attn(desc1, q1, dev.k[b:b + 1].contiguous(), dev.v[b:b + 1].contiguous(), ks, vs,
+                               oi, oc, o1, None, ws1)
+            compare_out(f64(o1[0]), o_sp_ref, wl.kv_dtype, f"O_sparse{l}_oracle_idx")
+    return report

@@ -13,7 +13,8 @@ import torch
 import kv_shared_b200 as hs
 import oracle
 import synth
-from hs2_check import (Dev, check_selection, compare_out, compare_scores, f64)
+from hs2_check import (Dev, block_parity as _block_parity, check_selection, compare_out,
+                       compare_scores, f64)
 
 pytestmark = pytest.mark.gpu
 
@@ -135,52 +136,6 @@ def test_sparse_attn_bad_index_reports_status():
 
 
 # ------------------------------------------------------------------ whole hybrid block
-def _block_parity(wl, seed, seqs=None, device="cpu"):
-    inp = synth.make_inputs(wl, seed=seed, device=device)
-    dev = Dev(inp)
-    dev.full()
-    for l in range(wl.n_sparse):
-        dev.sparse(l)
-    assert dev.status() == hs.HS2_OK
-    seqs = range(wl.batch) if seqs is None else seqs
-    pos = np.arange(wl.q_pos0, wl.ctx)
-    report = {"differing_rows": 0}
-    for b in seqs:
-        k, v = dev.kv_f64(b)
-        qf = f64(inp.q_full[b])
-        o_ref, lse_ref, sc_ref = oracle.full_attn(qf, k, v, pos)
-        compare_out(f64(dev.o_full[b]), o_ref, wl.kv_dtype, "O_full")
-        np.testing.assert_allclose(dev.lse[b].cpu().numpy(), lse_ref, rtol=1e-4, atol=1e-4)
-        compare_scores(dev.scores[b].cpu().numpy(), sc_ref, pos)
-        o_idx, o_cnt = oracle.select_rows(sc_ref, pos, wl.window, wl.budget, block_size=wl.block_size)
-        g_idx = dev.idx[b].cpu().numpy()
-        g_cnt = dev.cnt[b].cpu().numpy()
-        report["differing_rows"] += check_selection(g_idx, g_cnt, o_idx, o_cnt, sc_ref, pos, wl.window)
-        if inp.needle_pos is not None and wl.block_size == 1:
-            sel = set(g_idx[-1, :g_cnt[-1]].tolist())
-            assert set(inp.needle_pos[b].tolist()) <= sel, "planted key not selected"
-        # sparse layers: the GPU kernel on the oracle's indices vs the oracle (no tie leakage)
-        oi = torch.from_numpy(o_idx[None]).cuda()
-        oc = torch.from_numpy(o_cnt[None]).cuda()
-        for l in range(wl.n_sparse):
-            o_sp_ref = oracle.sparse_attn(f64(inp.q_sparse[l][b]), k, v, o_idx, o_cnt)
-            # end to end (GPU indices) where the index sets agree
-            same = np.array([np.array_equal(g_idx[r], o_idx[r]) for r in range(len(pos))])
-            if same.any():
-                compare_out(f64(dev.o_sparse[l][b])[same], o_sp_ref[same], wl.kv_dtype, f"O_sparse{l}")
-            # and the kernel alone on the oracle's selection, every row
-            desc1 = hs.make_desc(1, wl.n_q, wl.heads, wl.head_dim, wl.window, wl.budget,
-                                 q_dtype=dev.desc.q_dtype, kv_dtype=dev.desc.kv_dtype, max_ctx=wl.ctx)
-            o1 = torch.empty_like(dev.o_sparse[l][b:b + 1])
-            ws1 = hs.alloc_workspace(desc1)
-            ks = dev.k_scale[b:b + 1] if dev.k_scale is not None else None
-            vs = dev.v_scale[b:b + 1] if dev.v_scale is not None else None
-            hs.hs2_sparse_attn(desc1, dev.q_sparse[l][b:b + 1].contiguous(), dev.k[b:b + 1].contiguous(),
-                               dev.v[b:b + 1].contiguous(), ks, vs, oi, oc, o1, None, ws1)
-            compare_out(f64(o1[0]), o_sp_ref, wl.kv_dtype, f"O_sparse{l}_oracle_idx")
-    return report
-
-
 def test_tiny_f32_block_all_rows():
     rep = _block_parity(synth.TINY, seed=1001)
     assert rep["differing_rows"] <= 2
