@@ -243,10 +243,24 @@ def _capture(fns, stream):
     return graphs
 
 
+def _prefill_workload(args):
+    wl = synth.PREFILL_AGENT
+    if args.small:   # profiling shape: same kernels, a few hundred MB on the device
+        wl = synth.shrink(wl, batch=1, n_q=1024, ctx=16384 + 1024, n_new=1024)
+    return wl
+
+
+def _decode_workload(args):
+    wl = synth.DECODE_128K
+    if args.small:
+        wl = synth.shrink(wl, ctx=32768)
+    return wl
+
+
 def run_prefill(args, ws_):
     """Agent-round prefill: times the graph-replayed step and its full-attention call."""
     import kv_shared_b200 as hs
-    wl = synth.PREFILL_AGENT
+    wl = _prefill_workload(args)
     blk = PrefillBlock(wl, seed=1003)
     stream = torch.cuda.current_stream()
     blk.bridge(); blk.full(); [blk.sparse(l) for l in range(len(blk.qs))]
@@ -283,7 +297,7 @@ def run_prefill(args, ws_):
         "step": "KV bridging of the 8192 new rows + full attention with importance over 65536+8192 keys "
                 "+ top-1024/window-128 selection per row + 3 sparse layers",
         "full_attn_select": {"ms": full_ms, "algorithmic_tflop": blk.full_flops() / 1e12,
-                             "TFLOP/s": full_tflops, "tc_frac": full_tflops * 1e3 / tf,
+                             "TFLOP/s": full_tflops, "tc_frac": full_tflops / tf,
                              "peak_source": peak_kind},
         "kv_bridge": {"ms": bridge_ms, "TFLOP/s": bridge_flops / (bridge_ms / 1e3) / 1e12,
                       "GB/s": bridge_bytes / (bridge_ms / 1e3) / 1e9,
@@ -295,7 +309,10 @@ def run_prefill(args, ws_):
 
 def run_ours(args, ws_, rank, local):
     import kv_shared_b200 as hs
-    wl = synth.DECODE_128K
+    if args.workload == "prefill":
+        out = {"metric": METRIC, "prefill": run_prefill(args, ws_), "n_gpus": ws_, "data": "synthetic"}
+        return out
+    wl = _decode_workload(args)
     blk = DecodeBlock(wl, seed=1002 + rank)
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):
@@ -399,7 +416,7 @@ def run_ours(args, ws_, rank, local):
     }
     del blk, graphs
     torch.cuda.empty_cache()
-    if not args.no_prefill:
+    if not args.no_prefill and args.workload == "all":
         out["prefill"] = run_prefill(args, ws_)
         out["gpu_launches"] += out["prefill"]["gpu_launches"]
     if ws_ == 1 and rank == 0 and not args.no_cpu_baseline:
@@ -470,6 +487,10 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--workload", choices=["all", "decode", "prefill"], default="all",
+                    help="all: decode headline + prefill leg")
+    ap.add_argument("--small", action="store_true",
+                    help="reduced shapes of the same kernels (for profiler captures; not a bench value)")
     ap.add_argument("--prefill-steps", type=int, default=10)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -79,14 +79,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity; false (and the status word
-// set to HS2_ERR_TIMEOUT) if it did not complete in time.
+// set to HS2_ERR_TIMEOUT) if it did not complete in time.  The clock is read only
+// every 64 polls so that a phase completing soon costs nothing but the polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status,
                                           uint64_t limit_ns = kWaitNs) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 64; ++i)
+        if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
+#pragma unroll 1
     for (uint32_t i = 0; i < kWaitPolls; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (global_ns() - t0 > limit_ns) break;
+        if ((i & 63) == 63 && global_ns() - t0 > limit_ns) break;
     }
     set_status(status, HS2_ERR_TIMEOUT);
     return false;
@@ -177,6 +181,14 @@ __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
     for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// 2^x by the hardware approximation (one MUFU op; subnormal results flush to 0,
+// which only affects probabilities below 2^-126).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -99,7 +99,7 @@ __device__ __forceinline__ void convert_tile(const uint8_t* raw, uint8_t* cvt, i
 __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
     const float mn = fmaxf(m, m2);
     if (mn == -INFINITY) return;
-    l = l * exp2f(m - mn) + l2 * exp2f(m2 - mn);
+    l = l * ex2(m - mn) + l2 * ex2(m2 - mn);
     m = mn;
 }
 
@@ -201,10 +201,10 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
         for (int hh = 0; hh < 2; ++hh) {
             const float mn = fmaxf(m2[hh], mx[hh]);
             if (mn != -INFINITY) {
-                float sum = l2[hh] * exp2f(m2[hh] - mn);
+                float sum = l2[hh] * ex2(m2[hh] - mn);
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
-                    sum += exp2f(acc[nt][2 * hh] - mn) + exp2f(acc[nt][2 * hh + 1] - mn);
+                    sum += ex2(acc[nt][2 * hh] - mn) + ex2(acc[nt][2 * hh + 1] - mn);
                 l2[hh] = sum;
                 m2[hh] = mn;
             }
@@ -338,10 +338,10 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
         const float2 sgl = sld(g, c0), sg8l = sld(g + 8, c0), sgh = sld(g, c0 + 8), sg8h = sld(g + 8, c0 + 8);
         const int kl = tile_key0 + warp * 16 + 2 * t, kh = kl + 8;
         const bool v0 = kl < k_end, v1 = kl + 1 < k_end, v2 = kh < k_end, v3 = kh + 1 < k_end;
-        const float p00 = v0 ? exp2f(sgl.x - lse2[0]) : 0.f, p01 = v1 ? exp2f(sgl.y - lse2[0]) : 0.f;
-        const float p10 = v0 ? exp2f(sg8l.x - lse2[1]) : 0.f, p11 = v1 ? exp2f(sg8l.y - lse2[1]) : 0.f;
-        const float p02 = v2 ? exp2f(sgh.x - lse2[0]) : 0.f, p03 = v3 ? exp2f(sgh.y - lse2[0]) : 0.f;
-        const float p12 = v2 ? exp2f(sg8h.x - lse2[1]) : 0.f, p13 = v3 ? exp2f(sg8h.y - lse2[1]) : 0.f;
+        const float p00 = v0 ? ex2(sgl.x - lse2[0]) : 0.f, p01 = v1 ? ex2(sgl.y - lse2[0]) : 0.f;
+        const float p10 = v0 ? ex2(sg8l.x - lse2[1]) : 0.f, p11 = v1 ? ex2(sg8l.y - lse2[1]) : 0.f;
+        const float p02 = v2 ? ex2(sgh.x - lse2[0]) : 0.f, p03 = v3 ? ex2(sgh.y - lse2[0]) : 0.f;
+        const float p12 = v2 ? ex2(sg8h.x - lse2[1]) : 0.f, p13 = v3 ? ex2(sg8h.y - lse2[1]) : 0.f;
         // importance: sum over the 16 heads (pair here, then across the 8 row groups)
         float sc[4] = {p00 + p10, p01 + p11, p02 + p12, p03 + p13};
 #pragma unroll

@@ -16,8 +16,9 @@
 //           MN-major A operand of O += P V (V is MN-major straight from the
 //           cache); O stays in tensor memory for the whole key loop.
 //
-// Roles (192 threads): warp 0 issues TMA loads, one thread of warp 1 issues the
-// MMAs (and warp 1 owns the tensor memory), warps 2..5 do the softmax work.
+// Roles (320 threads): warp 0 issues TMA loads, one thread of warp 1 issues the
+// MMAs (and warp 1 owns the tensor memory), warps 2..9 do the softmax work: two
+// warps per tensor-memory lane quarter, each owning 64 of the 128 columns.
 // Every wait is bounded; a wait that gives up flags the status word and makes
 // all roles leave their loops.
 #include "common.cuh"
@@ -32,7 +33,8 @@ constexpr int D = 128;
 constexpr int ROWS = 8;                         // query rows per CTA
 constexpr int MT = ROWS * H;                    // 128 (row, head) pairs
 constexpr int KT = 128;                         // keys per tile
-constexpr int NT = 192;
+constexpr int NT = 320;
+constexpr int NSOFT = 256;                      // softmax threads (warps 2..9)
 constexpr int TILE_BYTES = KT * D * 2;          // 32 KB: two 128-row x 64-col swizzled boxes
 constexpr int BOX_BYTES = TILE_BYTES / 2;
 
@@ -103,7 +105,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         prefetch_tmap(&kmap);
         mbar_init(&q_full, 1);
         for (int s = 0; s < P1_STAGES; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 128); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], NSOFT); }
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -149,8 +151,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
             }
         }
     } else {
-        // softmax: this thread owns TMEM lane m = (row, head) of the S tile
-        const int quarter = warp & 3;
+        // softmax: this thread owns TMEM lane m = (row, head) of the S tile and one half
+        // (64 keys) of every key tile
+        const int quarter = warp & 3, hf = (warp - 2) >> 2;
         const int m = quarter * 32 + lane;
         const int row = r0 + (m >> 4);
         const int p = pos_base + (m >> 4);
@@ -159,43 +162,50 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
             const int buf = i & 1;
             if (!wait_or_abort(&s_full[buf], (i >> 1) & 1, &abort_flag, a.status)) break;
             umma::fence_after();
-            const int key0 = i * KT;
-            const bool need_mask = key0 + KT - 1 > p;
-#pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[2][32];
-                const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128 + half * 64;
-                umma::tmem_ld32(ta, r[0]);
-                umma::tmem_ld32(ta + 32, r[1]);
-                umma::tmem_ld_wait();
-                if (half == 1) {
-                    umma::fence_before();
-                    mbar_arrive(&s_empty[buf]);
-                }
-                float v[64];
-                float mx = -INFINITY;
+            const int key0 = i * KT + hf * 64;
+            uint32_t r[2][32];
+            const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128 + hf * 64;
+            umma::tmem_ld32(ta, r[0]);
+            umma::tmem_ld32(ta + 32, r[1]);
+            umma::tmem_ld_wait();
+            umma::fence_before();
+            mbar_arrive(&s_empty[buf]);
+            const bool need_mask = key0 + 63 > p;
+            float v[64];
+            float mx = -INFINITY;
 #pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    float x = __uint_as_float(r[c >> 5][c & 31]) * a.sc2;
-                    if (need_mask && key0 + half * 64 + c > p) x = -INFINITY;
-                    v[c] = x;
-                    mx = fmaxf(mx, x);
-                }
-                const float mn = fmaxf(run_m, mx);
-                if (mn != -INFINITY) {
-                    float sum = 0.f;
+            for (int c = 0; c < 64; ++c) {
+                float x = __uint_as_float(r[c >> 5][c & 31]) * a.sc2;
+                if (need_mask && key0 + c > p) x = -INFINITY;
+                v[c] = x;
+                mx = fmaxf(mx, x);
+            }
+            const float mn = fmaxf(run_m, mx);
+            if (mn != -INFINITY) {
+                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) sum += exp2f(v[c] - mn);
-                    run_l = run_l * exp2f(run_m - mn) + sum;
-                    run_m = mn;
+                for (int c = 0; c < 64; c += 4) {
+                    s0 += ex2(v[c] - mn);
+                    s1 += ex2(v[c + 1] - mn);
+                    s2 += ex2(v[c + 2] - mn);
+                    s3 += ex2(v[c + 3] - mn);
                 }
+                run_l = run_l * ex2(run_m - mn) + ((s0 + s1) + (s2 + s3));
+                run_m = mn;
             }
         }
-        if (row < a.n_q && !abort_flag) {
-            const float l2 = run_m + log2f(run_l);
-            const size_t o = (static_cast<size_t>(b) * a.n_q + row) * H + (m & 15);
-            a.lse2[o] = l2;
-            if (a.lse_user) a.lse_user[o] = l2 * kLn2;
+        // combine the two halves of the key range
+        __shared__ float2 part[2][MT];
+        part[hf][m] = make_float2(run_m, run_l);
+        named_sync(1, NSOFT);
+        if (hf == 0 && row < a.n_q && !abort_flag) {
+            const float2 o = part[1][m];
+            const float mn = fmaxf(run_m, o.x);
+            const float l = run_l * ex2(run_m - mn) + o.y * ex2(o.x - mn);
+            const float l2 = mn + log2f(l);
+            const size_t oi = (static_cast<size_t>(b) * a.n_q + row) * H + (m & 15);
+            a.lse2[oi] = l2;
+            if (a.lse_user) a.lse_user[oi] = l2 * kLn2;
         }
     }
     umma::fence_before();
@@ -217,9 +227,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     uint8_t* smem = align1024(smem_raw);
     uint8_t* qs = smem;
     uint8_t* kv = smem + TILE_BYTES;
-    uint8_t* ps = kv + P2_STAGES * KV_BYTES;    // P tile, MN-major A operand
+    uint8_t* ps = kv + P2_STAGES * KV_BYTES;    // two P tiles, MN-major A operands
     __shared__ uint64_t q_full, kv_full[P2_STAGES], kv_empty[P2_STAGES], s_full[2], s_empty[2];
-    __shared__ uint64_t p_full, p_empty, o_full;
+    __shared__ uint64_t p_full[2], p_empty[2], o_full;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     __shared__ __align__(16) float lse_s[MT];
@@ -239,9 +249,10 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         prefetch_tmap(&vmap);
         mbar_init(&q_full, 1);
         for (int s = 0; s < P2_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 128); }
-        mbar_init(&p_full, 128);
-        mbar_init(&p_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], NSOFT);
+            mbar_init(&p_full[s], NSOFT); mbar_init(&p_empty[s], 1);
+        }
         mbar_init(&o_full, 1);
         fence_mbar_init();
         abort_flag = 0;
@@ -289,100 +300,101 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
                     umma::commit(&s_full[buf]);
                 }
                 if (i >= 1) {                   // O += P(j) V(j), j = i - 1
-                    const int j = i - 1, s = j % P2_STAGES;
-                    if (!(ok = wait_or_abort(&p_full, j & 1, &abort_flag, a.status))) break;
+                    const int j = i - 1, s = j % P2_STAGES, pbuf = j & 1;
+                    if (!(ok = wait_or_abort(&p_full[pbuf], (j >> 1) & 1, &abort_flag, a.status))) break;
                     umma::fence_after();
                     const uint32_t vb = smem_u32(kv + s * KV_BYTES + TILE_BYTES);
+                    const uint32_t pbj = pb + pbuf * TILE_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < KT / 16; ++kk)
-                        umma::mma_bf16_ss(tmem + 256, mnmajor_desc(pb, kk), mnmajor_desc(vb, kk), idesc_o,
+                        umma::mma_bf16_ss(tmem + 256, mnmajor_desc(pbj, kk), mnmajor_desc(vb, kk), idesc_o,
                                           (j > 0 || kk > 0) ? 1u : 0u);
-                    umma::commit(&p_empty);
+                    umma::commit(&p_empty[pbuf]);
                     umma::commit(&kv_empty[s]);
                 }
             }
             umma::commit(&o_full);
         }
     } else {
-        const int quarter = warp & 3;
-        const int st = threadIdx.x - 64;        // 0..127
+        const int quarter = warp & 3, hf = (warp - 2) >> 2;
+        const int st = threadIdx.x - 64;        // 0..255
         // log-sum-exp of the 128 (row, head) columns; rows past n_q get +inf (P = 0)
-        {
+        if (st < MT) {
             const int row = r0 + (st >> 4);
             lse_s[st] = row < a.n_q ? a.lse2[(static_cast<size_t>(b) * a.n_q + row) * H + (st & 15)] : INFINITY;
         }
-        named_sync(1, 128);
+        named_sync(1, NSOFT);
         const int kl = quarter * 32 + lane;     // the key lane this thread owns in S'
-        float* srow0 = a.scores + (static_cast<size_t>(b) * a.n_q + r0) * a.score_ld;
+        // this thread's half: columns hf*64 .. hf*64+63 = rows 4hf .. 4hf+3, all heads
+        float* srow0 = a.scores + (static_cast<size_t>(b) * a.n_q + r0 + 4 * hf) * a.score_ld;
+        const float* lse_h = lse_s + hf * 64;
         for (int i = 0; i < n_kt; ++i) {
             const int buf = i & 1;
             if (!wait_or_abort(&s_full[buf], (i >> 1) & 1, &abort_flag, a.status)) break;
             umma::fence_after();
-            uint32_t r[4][32];
-            const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128;
+            uint32_t r[2][32];
+            const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128 + hf * 64;
             umma::tmem_ld32(ta, r[0]);
             umma::tmem_ld32(ta + 32, r[1]);
-            umma::tmem_ld32(ta + 64, r[2]);
-            umma::tmem_ld32(ta + 96, r[3]);
             umma::tmem_ld_wait();
             umma::fence_before();
             mbar_arrive(&s_empty[buf]);
             const int key = i * KT + kl;
             // probabilities, head sums, bf16 pairs for the P tile
-            uint32_t pk[64];
-            float sc[ROWS];
+            uint32_t pk[32];
+            float sc[4];
 #pragma unroll
-            for (int rr = 0; rr < ROWS; ++rr) {
-                const bool valid = key <= pos_base + rr;
-                float acc = 0.f;
+            for (int rr = 0; rr < 4; ++rr) {
+                const bool valid = key <= pos_base + 4 * hf + rr;
+                float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
                 for (int h = 0; h < H; h += 2) {
                     const int c = rr * H + h;
-                    const float2 l2 = *reinterpret_cast<const float2*>(&lse_s[c]);
-                    float p0 = exp2f(__uint_as_float(r[c >> 5][c & 31]) * a.sc2 - l2.x);
-                    float p1 = exp2f(__uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]) * a.sc2 - l2.y);
+                    const float2 l2 = *reinterpret_cast<const float2*>(&lse_h[c]);
+                    float p0 = ex2(__uint_as_float(r[c >> 5][c & 31]) * a.sc2 - l2.x);
+                    float p1 = ex2(__uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]) * a.sc2 - l2.y);
                     if (!valid) { p0 = 0.f; p1 = 0.f; }
-                    acc += p0 + p1;
+                    acc0 += p0;
+                    acc1 += p1;
                     pk[c >> 1] = pack_bf16(p0, p1);
                 }
-                sc[rr] = acc;
+                sc[rr] = acc0 + acc1;
             }
 #pragma unroll
-            for (int rr = 0; rr < ROWS; ++rr)
-                if (key <= pos_base + rr && r0 + rr < a.n_q) srow0[rr * a.score_ld + key] = sc[rr];
+            for (int rr = 0; rr < 4; ++rr)
+                if (key <= pos_base + 4 * hf + rr && r0 + 4 * hf + rr < a.n_q) srow0[rr * a.score_ld + key] = sc[rr];
             // last tile: cache rows past the last query position may hold anything, and
-            // 0 * NaN would poison O, so this key's V row is zeroed (the K row only feeds
-            // probabilities that are forced to 0 above)
+            // 0 * NaN would poison O, so this key's V row (this half) is zeroed (the K row
+            // only feeds probabilities that are forced to 0 above)
             if (i == n_kt - 1 && key > p_max) {
-                uint8_t* vrow = kv + (i % P2_STAGES) * KV_BYTES + TILE_BYTES + kl * 128;
+                uint8_t* vrow = kv + (i % P2_STAGES) * KV_BYTES + TILE_BYTES + hf * BOX_BYTES + kl * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
-                    *reinterpret_cast<uint4*>(vrow + BOX_BYTES + c * 16) = make_uint4(0, 0, 0, 0);
-                }
+                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
             }
-            // the P tile is free once the previous O MMA has completed
-            if (i >= 1 && !wait_or_abort(&p_empty, (i - 1) & 1, &abort_flag, a.status)) break;
-            // row `kl` of the MN-major P tile: m = (row, head) 0..127 in two 64-wide groups
-            uint8_t* prow = ps + (kl >> 3) * 1024 + (kl & 7) * 128;
+            // P tile i%2 is free once the O MMA of tile i-2 has completed
+            const int pbuf = i & 1;
+            if (i >= 2 && !wait_or_abort(&p_empty[pbuf], ((i >> 1) - 1) & 1, &abort_flag, a.status)) break;
+            // row `kl` of the MN-major P tile, m-group hf (m = 64 hf .. 64 hf + 63)
+            uint8_t* prow = ps + pbuf * TILE_BYTES + hf * BOX_BYTES + (kl >> 3) * 1024 + (kl & 7) * 128;
 #pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
+            for (int cc = 0; cc < 8; ++cc) {
                 const uint4 w = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-                *reinterpret_cast<uint4*>(prow + (cc >> 3) * BOX_BYTES + (((cc & 7) ^ (kl & 7)) << 4)) = w;
+                *reinterpret_cast<uint4*>(prow + ((cc ^ (kl & 7)) << 4)) = w;
             }
             umma::fence_proxy_async();
-            mbar_arrive(&p_full);
+            mbar_arrive(&p_full[pbuf]);
         }
-        // O epilogue: this thread owns TMEM lane m = (row, head) of the O accumulator
+        // O epilogue: this thread owns TMEM lane m = (row, head) of the O accumulator and
+        // columns 64 hf .. 64 hf + 63
         if (wait_or_abort(&o_full, 0, &abort_flag, a.status)) {
             umma::fence_after();
             const int m = quarter * 32 + lane;
             const int row = r0 + (m >> 4);
-            __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + row) * H + (m & 15)) * D;
+            __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + row) * H + (m & 15)) * D + hf * 64;
 #pragma unroll 1
-            for (int c = 0; c < D; c += 32) {
+            for (int c = 0; c < 64; c += 32) {
                 uint32_t r[32];
-                umma::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 256 + c, r);
+                umma::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 256 + hf * 64 + c, r);
                 umma::tmem_ld_wait();
                 if (row < a.n_q) {
 #pragma unroll
@@ -431,7 +443,7 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     a.status = pa.status;
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
     const size_t s1 = 1024 + TILE_BYTES + P1_STAGES * TILE_BYTES;
-    const size_t s2 = 1024 + TILE_BYTES + P2_STAGES * KV_BYTES + TILE_BYTES;
+    const size_t s2 = 1024 + TILE_BYTES + P2_STAGES * KV_BYTES + 2 * TILE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(prefill_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(prefill_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));

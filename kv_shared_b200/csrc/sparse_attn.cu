@@ -60,7 +60,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
     const float mn = fmaxf(m, m2);
     if (mn == -INFINITY) return;
-    l = l * exp2f(m - mn) + l2 * exp2f(m2 - mn);
+    l = l * ex2(m - mn) + l2 * ex2(m2 - mn);
     m = mn;
 }
 
@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
             mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
             mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
             const float mn = fmaxf(m2[hh], mx[hh]);
-            alpha[hh] = (mn == -INFINITY) ? 1.f : exp2f(m2[hh] - mn);
+            alpha[hh] = (mn == -INFINITY) ? 1.f : ex2(m2[hh] - mn);
             m2[hh] = mn;
         }
         float pr[2][4];
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int hh = e >> 1;
-                pr[nt][e] = (m2[hh] == -INFINITY) ? 0.f : exp2f(acc[nt][e] - m2[hh]);
+                pr[nt][e] = (m2[hh] == -INFINITY) ? 0.f : ex2(acc[nt][e] - m2[hh]);
             }
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
@@ -273,7 +273,7 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     for (int hh = 0; hh < 2; ++hh) {
         const int h = g + 8 * hh;
         M[hh] = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
-        f[hh] = (M[hh] == -INFINITY) ? 0.f : exp2f(m2[hh] - M[hh]);
+        f[hh] = (M[hh] == -INFINITY) ? 0.f : ex2(m2[hh] - M[hh]);
     }
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
         const float Mh = fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid]));
         float Lh = 0.f;
         if (Mh != -INFINITY)
-            for (int w = 0; w < 4; ++w) Lh += wl[w][tid] * exp2f(wm[w][tid] - Mh);
+            for (int w = 0; w < 4; ++w) Lh += wl[w][tid] * ex2(wm[w][tid] - Mh);
         cm[tid] = Mh; cl[tid] = Lh;
     }
     __syncthreads();
@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     for (int i = tid; i < a.splits * H; i += NT) {
         const int sp = i / H, h = i % H;
         const float mm = sml[sp][h].x;
-        sw[sp][h] = (mm == -INFINITY) ? 0.f : exp2f(mm - fm[h]) * finv[h];
+        sw[sp][h] = (mm == -INFINITY) ? 0.f : ex2(mm - fm[h]) * finv[h];
     }
     __syncthreads();
     const float4* base4 = reinterpret_cast<const float4*>(a.part_o + static_cast<size_t>(row) * a.splits * H * D);

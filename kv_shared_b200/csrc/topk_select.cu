@@ -12,10 +12,11 @@
 //
 // A row is handled by a cluster of CS CTAs (CS = 1..8); CTA r owns a contiguous
 // slice of the candidates and keeps their order-preserving uint32 images in
-// shared memory when they fit.  The K-th best key is found exactly by a
-// three-digit radix select (11 + 11 + 10 bits): per digit every CTA builds a
-// histogram of its slice, the cluster's histograms are summed over distributed
-// shared memory and each CTA takes the same decision.  Then every CTA writes,
+// shared memory when they fit.  The K-th best key is found exactly by a radix
+// select over the bits below those every key of the row shares (from the row's
+// key range), at most 11 bits per digit: per digit every CTA builds a histogram
+// of its slice, the cluster's histograms are summed over distributed shared
+// memory and each CTA takes the same decision.  Then every CTA writes,
 // in ascending order, its keys above the threshold and its share of the first
 // (K - #above) keys equal to it (the lower-index tie rule), at offsets from a
 // cluster-wide prefix of the counts.  Integer work only after the key map.
@@ -47,6 +48,8 @@ struct Smem {
     int found_bin;
     int found_above;
     int counts[2];              // this CTA's (#above, #equal) for the compaction
+    uint32_t wlo[NW], whi[NW];  // per-warp key range
+    uint32_t range[2];          // this CTA's key range (read by the cluster)
 };
 
 // Block-wide exclusive scan of one int per thread; *total receives the sum.
@@ -94,6 +97,27 @@ struct Slice {
     __device__ __forceinline__ uint32_t key(int i) const { return cache ? cache[i - begin] : compute(i); }
 };
 
+// Visits every key of the slice as f(i, key, valid) with 8 independent loads in
+// flight per thread; all threads of the block make the same number of calls (keys
+// past the slice come with valid = false), so f may use warp-wide primitives.
+constexpr int kBatch = 8;
+template <typename F>
+__device__ __forceinline__ void for_keys(const Slice& sl, F f) {
+    for (int base = sl.begin; base < sl.end; base += NT * kBatch) {
+        uint32_t k[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = base + u * NT + threadIdx.x;
+            k[u] = i < sl.end ? sl.key(i) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int i = base + u * NT + threadIdx.x;
+            f(i, k[u], i < sl.end);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int cache_keys) {
     extern __shared__ uint32_t key_cache[];
     __shared__ Smem sm;
@@ -117,9 +141,24 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int ca
     const int per = ((n_keys + cs - 1) / cs + 3) & ~3;
     sl.begin = min(rank * per, n_keys);
     sl.end = min(sl.begin + per, n_keys);
-    sl.cache = (per <= cache_keys) ? key_cache : nullptr;
-    if (sl.cache)
-        for (int i = sl.begin + threadIdx.x; i < sl.end; i += NT) sl.cache[i - sl.begin] = sl.compute(i);
+    sl.cache = nullptr;
+    if (per <= cache_keys) {
+        if (bs == 1) {
+            // token keys: 8 coalesced loads in flight per thread
+            for_keys(sl, [&](int i, uint32_t key, bool valid) { if (valid) key_cache[i - sl.begin] = key; });
+        } else {
+            // block keys: one warp per block, max over its tokens by shuffles
+            const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+            for (int bb = sl.begin + warp; bb < sl.end; bb += NW) {
+                const int e = min((bb + 1) * bs, n_cand);
+                float m = -INFINITY;
+                for (int j = bb * bs + lane; j < e; j += 32) m = fmaxf(m, sl.s[j]);
+                m = warp_max(m);
+                if (lane == 0) key_cache[bb - sl.begin] = ord_key(m);
+            }
+        }
+        sl.cache = key_cache;
+    }
     __syncthreads();
 
     uint32_t tau = 0;
@@ -127,62 +166,92 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int ca
     const bool take_all = (K >= n_keys);
     const bool take_none = (K <= 0);
     if (!take_all && K > 0) {
-        uint32_t prefix = 0, mask = 0;
-        int k_rem = K;
-        const int shifts[3] = {21, 10, 0};
-        const int widths[3] = {11, 11, 10};
-#pragma unroll 1
-        for (int pass = 0; pass < 3; ++pass) {
-            const int shift = shifts[pass], nb = 1 << widths[pass];
-            for (int i = threadIdx.x; i < nb; i += NT) sm.hist[i] = 0;
-            __syncthreads();
-            for (int i = sl.begin + threadIdx.x; i < sl.end; i += NT) {
-                const uint32_t key = sl.key(i);
-                if ((key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (nb - 1)], 1);
-            }
-            cluster.sync();
-            // counts of the whole row: sum of the cluster's histograms (from the top bin)
-            const int bins_per = nb / NT;                               // 4 or 2
-            int local[NBINS / NT];
-            int tot = 0;
-            for (int q = 0; q < bins_per; ++q) {
-                const int bin = nb - 1 - (threadIdx.x * bins_per + q);
-                int c = 0;
-                for (int rr = 0; rr < cs; ++rr) c += cluster.map_shared_rank(sm.hist, rr)[bin];
-                local[q] = c;
-                tot += c;
-            }
-            cluster.sync();                    // every CTA has read every histogram
-            const int above = block_excl_scan(tot, sm);
-            if (above < k_rem && above + tot >= k_rem) {
-                int acc = above;
-                for (int q = 0; q < bins_per; ++q) {
-                    if (acc + local[q] >= k_rem) {
-                        sm.found_bin = nb - 1 - (threadIdx.x * bins_per + q);
-                        sm.found_above = acc;
-                        break;
-                    }
-                    acc += local[q];
-                }
-            }
-            __syncthreads();
-            prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
-            mask |= static_cast<uint32_t>(nb - 1) << shift;
-            k_rem -= sm.found_above;
-            __syncthreads();
+        // key range of the row: the digits start right below the bits every key shares
+        // (importance values crowd into a few binades; a fixed top digit would put them
+        // into a handful of bins)
+        uint32_t lo = 0xffffffffu, hi = 0u;
+        for_keys(sl, [&](int, uint32_t key, bool valid) {
+            if (valid) { lo = min(lo, key); hi = max(hi, key); }
+        });
+        lo = __reduce_min_sync(0xffffffffu, lo);
+        hi = __reduce_max_sync(0xffffffffu, hi);
+        if ((threadIdx.x & 31) == 0) { sm.wlo[threadIdx.x >> 5] = lo; sm.whi[threadIdx.x >> 5] = hi; }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            uint32_t l = sm.wlo[0], h = sm.whi[0];
+            for (int w = 1; w < NW; ++w) { l = min(l, sm.wlo[w]); h = max(h, sm.whi[w]); }
+            sm.range[0] = l; sm.range[1] = h;
         }
-        tau = prefix;
-        need_eq = k_rem;
+        cluster.sync();
+        lo = 0xffffffffu; hi = 0u;
+        for (int rr = 0; rr < cs; ++rr) {
+            const uint32_t* rg = cluster.map_shared_rank(sm.range, rr);
+            lo = min(lo, rg[0]);
+            hi = max(hi, rg[1]);
+        }
+        cluster.sync();
+        if (lo == hi) {                         // every candidate key is the same value
+            tau = hi;
+            need_eq = K;
+        } else {
+            const int hb = 31 - __clz(lo ^ hi); // highest bit where the keys differ
+            uint32_t mask = ~((2u << hb) - 1u); // (hb == 31 gives 0: nothing shared)
+            uint32_t prefix = hi & mask;
+            int k_rem = K;
+#pragma unroll 1
+            for (int top = hb; top >= 0;) {
+                const int width = min(11, top + 1);
+                const int shift = top - width + 1, nb = 1 << width;
+                for (int i = threadIdx.x; i < nb; i += NT) sm.hist[i] = 0;
+                __syncthreads();
+                for_keys(sl, [&](int, uint32_t key, bool valid) {
+                    if (valid && (key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (nb - 1)], 1);
+                });
+                cluster.sync();
+                // counts of the whole row: sum of the cluster's histograms, from the top bin
+                const int bins_per = (nb + NT - 1) / NT;               // 1..4
+                int local[NBINS / NT];
+                int tot = 0;
+                for (int q = 0; q < bins_per; ++q) {
+                    const int bin = nb - 1 - (threadIdx.x * bins_per + q);
+                    int c = 0;
+                    if (bin >= 0)
+                        for (int rr = 0; rr < cs; ++rr) c += cluster.map_shared_rank(sm.hist, rr)[bin];
+                    local[q] = c;
+                    tot += c;
+                }
+                cluster.sync();                 // every CTA has read every histogram
+                const int above = block_excl_scan(tot, sm);
+                if (above < k_rem && above + tot >= k_rem) {
+                    int acc = above;
+                    for (int q = 0; q < bins_per; ++q) {
+                        if (acc + local[q] >= k_rem) {
+                            sm.found_bin = nb - 1 - (threadIdx.x * bins_per + q);
+                            sm.found_above = acc;
+                            break;
+                        }
+                        acc += local[q];
+                    }
+                }
+                __syncthreads();
+                prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
+                mask |= static_cast<uint32_t>(nb - 1) << shift;
+                k_rem -= sm.found_above;
+                __syncthreads();
+                top = shift - 1;
+            }
+            tau = prefix;
+            need_eq = k_rem;
+        }
     }
 
     // this CTA's counts, then cluster-wide offsets
     int gt = 0, eq = 0;
     if (!take_all && K > 0) {
-        for (int i = sl.begin + threadIdx.x; i < sl.end; i += NT) {
-            const uint32_t key = sl.key(i);
-            gt += key > tau;
-            eq += key == tau;
-        }
+        for_keys(sl, [&](int, uint32_t key, bool valid) {
+            gt += valid && key > tau;
+            eq += valid && key == tau;
+        });
     }
     int t_gt = block_excl_scan(gt, sm);
     t_gt = sm.total;
