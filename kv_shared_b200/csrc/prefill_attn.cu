@@ -78,6 +78,10 @@ __device__ __forceinline__ void named_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Tensor-memory S buffers: three 128-column tiles in flight, so that the MMA can
+// run ahead while the two softmax warpgroups each work on their own key tile.
+constexpr int NSB = 3;
+
 // ------------------------------------------------------------------ pass 1: LSE
 constexpr int P1_STAGES = 4;
 
@@ -87,9 +91,10 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
     uint8_t* smem = align1024(smem_raw);
     uint8_t* qs = smem;
     uint8_t* ks = smem + TILE_BYTES;
-    __shared__ uint64_t q_full, k_full[P1_STAGES], k_empty[P1_STAGES], s_full[2], s_empty[2];
+    __shared__ uint64_t q_full, k_full[P1_STAGES], k_empty[P1_STAGES], s_full[NSB], s_empty[NSB];
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
+    __shared__ float2 part[2][MT];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int blocks_per_seq = (a.n_q + ROWS - 1) / ROWS;
@@ -105,11 +110,11 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         prefetch_tmap(&kmap);
         mbar_init(&q_full, 1);
         for (int s = 0; s < P1_STAGES; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], NSOFT); }
+        for (int s = 0; s < NSB; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 128); }
         fence_mbar_init();
         abort_flag = 0;
     }
-    if (warp == 1) umma::tmem_alloc(&tmem_base, 256);
+    if (warp == 1) umma::tmem_alloc(&tmem_base, 512);
     umma::fence_before();
     __syncthreads();
     umma::fence_after();
@@ -137,45 +142,36 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
             const uint32_t qb = smem_u32(qs);
             if (wait_or_abort(&q_full, 0, &abort_flag, a.status)) {
                 for (int i = 0; i < n_kt; ++i) {
-                    const int s = i % P1_STAGES, buf = i & 1;
+                    const int s = i % P1_STAGES, sb = i % NSB;
                     if (!wait_or_abort(&k_full[s], (i / P1_STAGES) & 1, &abort_flag, a.status)) break;
-                    if (i >= 2 && !wait_or_abort(&s_empty[buf], ((i >> 1) - 1) & 1, &abort_flag, a.status)) break;
+                    if (i >= NSB && !wait_or_abort(&s_empty[sb], ((i / NSB) - 1) & 1, &abort_flag, a.status)) break;
                     umma::fence_after();
                     const uint32_t kb = smem_u32(ks + s * TILE_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
-                        umma::mma_bf16_ss(tmem + buf * 128, kmajor_desc(qb, kk), kmajor_desc(kb, kk), idesc, kk > 0);
+                        umma::mma_bf16_ss(tmem + sb * 128, kmajor_desc(qb, kk), kmajor_desc(kb, kk), idesc, kk > 0);
                     umma::commit(&k_empty[s]);
-                    umma::commit(&s_full[buf]);
+                    umma::commit(&s_full[sb]);
                 }
             }
         }
     } else {
-        // softmax: this thread owns TMEM lane m = (row, head) of the S tile and one half
-        // (64 keys) of every key tile
-        const int quarter = warp & 3, hf = (warp - 2) >> 2;
+        // softmax warpgroup g takes key tiles i = g, g+2, ...; each thread owns TMEM lane
+        // m = (row, head) and all 128 columns of a tile, read in 32-column chunks with the
+        // next chunk's load in flight while the current one is reduced
+        const int quarter = warp & 3, g = (warp - 2) >> 2;
         const int m = quarter * 32 + lane;
         const int row = r0 + (m >> 4);
         const int p = pos_base + (m >> 4);
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         float run_m = -INFINITY, run_l = 0.f;
-        for (int i = 0; i < n_kt; ++i) {
-            const int buf = i & 1;
-            if (!wait_or_abort(&s_full[buf], (i >> 1) & 1, &abort_flag, a.status)) break;
-            umma::fence_after();
-            const int key0 = i * KT + hf * 64;
-            uint32_t r[2][32];
-            const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128 + hf * 64;
-            umma::tmem_ld32(ta, r[0]);
-            umma::tmem_ld32(ta + 32, r[1]);
-            umma::tmem_ld_wait();
-            umma::fence_before();
-            mbar_arrive(&s_empty[buf]);
-            const bool need_mask = key0 + 63 > p;
-            float v[64];
+        auto reduce_chunk = [&](const uint32_t (&r)[32], int key0) {
+            float v[32];
             float mx = -INFINITY;
+            const bool need_mask = key0 + 31 > p;
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float x = __uint_as_float(r[c >> 5][c & 31]) * a.sc2;
+            for (int c = 0; c < 32; ++c) {
+                float x = __uint_as_float(r[c]) * a.sc2;
                 if (need_mask && key0 + c > p) x = -INFINITY;
                 v[c] = x;
                 mx = fmaxf(mx, x);
@@ -184,7 +180,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
             if (mn != -INFINITY) {
                 float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
 #pragma unroll
-                for (int c = 0; c < 64; c += 4) {
+                for (int c = 0; c < 32; c += 4) {
                     s0 += ex2(v[c] - mn);
                     s1 += ex2(v[c + 1] - mn);
                     s2 += ex2(v[c + 2] - mn);
@@ -193,15 +189,37 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
                 run_l = run_l * ex2(run_m - mn) + ((s0 + s1) + (s2 + s3));
                 run_m = mn;
             }
+        };
+        for (int i = g; i < n_kt; i += 2) {
+            const int sb = i % NSB;
+            if (!wait_or_abort(&s_full[sb], (i / NSB) & 1, &abort_flag, a.status)) break;
+            umma::fence_after();
+            const uint32_t ta = tmem + lane_base + sb * 128;
+            const int key0 = i * KT;
+            uint32_t ra[32], rb[32];
+            umma::tmem_ld32(ta, ra);
+            umma::tmem_ld_wait();
+            umma::tmem_ld32(ta + 32, rb);
+            reduce_chunk(ra, key0);
+            umma::tmem_ld_wait();
+            umma::tmem_ld32(ta + 64, ra);
+            reduce_chunk(rb, key0 + 32);
+            umma::tmem_ld_wait();
+            umma::tmem_ld32(ta + 96, rb);
+            reduce_chunk(ra, key0 + 64);
+            umma::tmem_ld_wait();
+            umma::fence_before();
+            mbar_arrive(&s_empty[sb]);
+            reduce_chunk(rb, key0 + 96);
         }
-        // combine the two halves of the key range
-        __shared__ float2 part[2][MT];
-        part[hf][m] = make_float2(run_m, run_l);
+        // combine the two warpgroups' key tiles
+        part[g][m] = make_float2(run_m, run_l);
         named_sync(1, NSOFT);
-        if (hf == 0 && row < a.n_q && !abort_flag) {
+        if (g == 0 && row < a.n_q && !abort_flag) {
             const float2 o = part[1][m];
             const float mn = fmaxf(run_m, o.x);
-            const float l = run_l * ex2(run_m - mn) + o.y * ex2(o.x - mn);
+            const float l = (run_m == -INFINITY ? 0.f : run_l * ex2(run_m - mn)) +
+                            (o.x == -INFINITY ? 0.f : o.y * ex2(o.x - mn));
             const float l2 = mn + log2f(l);
             const size_t oi = (static_cast<size_t>(b) * a.n_q + row) * H + (m & 15);
             a.lse2[oi] = l2;
@@ -212,13 +230,39 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
     __syncthreads();
     if (warp == 1) {
         umma::fence_after();
-        umma::tmem_dealloc(tmem, 256);
+        umma::tmem_dealloc(tmem, 512);
+    }
+}
+
+// One 32-column chunk of an S' row (pass 2): columns = rows 2C, 2C+1 x 16 heads.
+// Probabilities P = 2^(S' sc2 - LSE2), the two rows' importance (written to the score
+// rows), and bf16 pairs of P into pk[16 C .. 16 C + 15].
+template <int C>
+__device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], int key, int pos_base, int r0, int n_q,
+                                         float sc2, const float* lse_s, float* srow0, int64_t score_ld,
+                                         uint32_t (&pk)[64]) {
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+        const int row = 2 * C + rr;
+        const bool valid = key <= pos_base + row;
+        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+        for (int h = 0; h < H; h += 2) {
+            const int col = rr * H + h;
+            const float2 l2 = *reinterpret_cast<const float2*>(&lse_s[C * 32 + col]);
+            float p0 = ex2(__uint_as_float(r[col]) * sc2 - l2.x);
+            float p1 = ex2(__uint_as_float(r[col + 1]) * sc2 - l2.y);
+            if (!valid) { p0 = 0.f; p1 = 0.f; }
+            acc0 += p0;
+            acc1 += p1;
+            pk[C * 16 + (col >> 1)] = pack_bf16(p0, p1);
+        }
+        if (valid && r0 + row < n_q) srow0[row * score_ld + key] = acc0 + acc1;
     }
 }
 
 // ------------------------------------------------------------------ pass 2: P, importance, O
-constexpr int P2_STAGES = 2;
-constexpr int KV_BYTES = 2 * TILE_BYTES;        // K tile then V tile
+constexpr int P2_STAGES = 2;                    // K and V tiles each double-buffered
 
 __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constant__ CUtensorMap qmap,
                                                            const __grid_constant__ CUtensorMap kmap,
@@ -226,10 +270,11 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* qs = smem;
-    uint8_t* kv = smem + TILE_BYTES;
-    uint8_t* ps = kv + P2_STAGES * KV_BYTES;    // two P tiles, MN-major A operands
-    __shared__ uint64_t q_full, kv_full[P2_STAGES], kv_empty[P2_STAGES], s_full[2], s_empty[2];
-    __shared__ uint64_t p_full[2], p_empty[2], o_full;
+    uint8_t* kst = smem + TILE_BYTES;                         // K stages
+    uint8_t* vst = kst + P2_STAGES * TILE_BYTES;              // V stages
+    uint8_t* ps = vst + P2_STAGES * TILE_BYTES;               // P tiles (one per warpgroup)
+    __shared__ uint64_t q_full, k_full[P2_STAGES], k_empty[P2_STAGES], v_full[P2_STAGES], v_empty[P2_STAGES];
+    __shared__ uint64_t s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_full;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     __shared__ __align__(16) float lse_s[MT];
@@ -248,11 +293,12 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         prefetch_tmap(&kmap);
         prefetch_tmap(&vmap);
         mbar_init(&q_full, 1);
-        for (int s = 0; s < P2_STAGES; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], NSOFT);
-            mbar_init(&p_full[s], NSOFT); mbar_init(&p_empty[s], 1);
+        for (int s = 0; s < P2_STAGES; ++s) {
+            mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
+            mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
         }
+        for (int s = 0; s < NSB; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 128); }
+        for (int s = 0; s < 2; ++s) { mbar_init(&p_full[s], 128); mbar_init(&p_empty[s], 1); }
         mbar_init(&o_full, 1);
         fence_mbar_init();
         abort_flag = 0;
@@ -261,7 +307,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     umma::fence_before();
     __syncthreads();
     umma::fence_after();
-    const uint32_t tmem = tmem_base;            // S' buffers at columns 0 and 128, O at 256
+    const uint32_t tmem = tmem_base;            // S' buffers at columns 0, 128, 256; O at 384
+    constexpr uint32_t kOcol = NSB * 128;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -269,16 +316,24 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             mbar_arrive_expect_tx(&q_full, TILE_BYTES);
             tma_load_2d(qs, &qmap, &q_full, 0, qrow);
             tma_load_2d(qs + BOX_BYTES, &qmap, &q_full, 64, qrow);
-            for (int i = 0; i < n_kt; ++i) {
-                const int s = i % P2_STAGES;
-                if (i >= P2_STAGES && !wait_or_abort(&kv_empty[s], ((i / P2_STAGES) - 1) & 1, &abort_flag, a.status)) break;
-                uint8_t* dst = kv + s * KV_BYTES;
-                const int krow = static_cast<int>(b * a.cap) + i * KT;
-                mbar_arrive_expect_tx(&kv_full[s], KV_BYTES);
-                tma_load_2d(dst, &kmap, &kv_full[s], 0, krow);
-                tma_load_2d(dst + BOX_BYTES, &kmap, &kv_full[s], 64, krow);
-                tma_load_2d(dst + TILE_BYTES, &vmap, &kv_full[s], 0, krow);
-                tma_load_2d(dst + TILE_BYTES + BOX_BYTES, &vmap, &kv_full[s], 64, krow);
+            // K runs one tile ahead of V: K(t) is needed by S'(t), V(t) only by O after P(t)
+            for (int t = 0; t <= n_kt; ++t) {
+                if (t < n_kt) {
+                    const int s = t % P2_STAGES;
+                    if (t >= P2_STAGES && !wait_or_abort(&k_empty[s], ((t / P2_STAGES) - 1) & 1, &abort_flag, a.status)) break;
+                    const int krow = static_cast<int>(b * a.cap) + t * KT;
+                    mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
+                    tma_load_2d(kst + s * TILE_BYTES, &kmap, &k_full[s], 0, krow);
+                    tma_load_2d(kst + s * TILE_BYTES + BOX_BYTES, &kmap, &k_full[s], 64, krow);
+                }
+                if (t >= 1) {
+                    const int j = t - 1, s = j % P2_STAGES;
+                    if (j >= P2_STAGES && !wait_or_abort(&v_empty[s], ((j / P2_STAGES) - 1) & 1, &abort_flag, a.status)) break;
+                    const int vrow = static_cast<int>(b * a.cap) + j * KT;
+                    mbar_arrive_expect_tx(&v_full[s], TILE_BYTES);
+                    tma_load_2d(vst + s * TILE_BYTES, &vmap, &v_full[s], 0, vrow);
+                    tma_load_2d(vst + s * TILE_BYTES + BOX_BYTES, &vmap, &v_full[s], 64, vrow);
+                }
             }
         }
     } else if (warp == 1) {
@@ -287,36 +342,39 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             constexpr uint32_t idesc_o = umma::idesc_bf16(128, 128, true, true);
             const uint32_t qb = smem_u32(qs), pb = smem_u32(ps);
             bool ok = wait_or_abort(&q_full, 0, &abort_flag, a.status);
-            for (int i = 0; ok && i <= n_kt; ++i) {
+            // S'(i) runs two tiles ahead of O += P(i-2) V(i-2)
+            for (int i = 0; ok && i < n_kt + 2; ++i) {
                 if (i < n_kt) {                 // S'(i) = K(i) Q^T
-                    const int s = i % P2_STAGES, buf = i & 1;
-                    if (!(ok = wait_or_abort(&kv_full[s], (i / P2_STAGES) & 1, &abort_flag, a.status))) break;
-                    if (i >= 2 && !(ok = wait_or_abort(&s_empty[buf], ((i >> 1) - 1) & 1, &abort_flag, a.status))) break;
+                    const int s = i % P2_STAGES, sb = i % NSB;
+                    if (!(ok = wait_or_abort(&k_full[s], (i / P2_STAGES) & 1, &abort_flag, a.status))) break;
+                    if (i >= NSB && !(ok = wait_or_abort(&s_empty[sb], ((i / NSB) - 1) & 1, &abort_flag, a.status))) break;
                     umma::fence_after();
-                    const uint32_t kb = smem_u32(kv + s * KV_BYTES);
+                    const uint32_t kb = smem_u32(kst + s * TILE_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
-                        umma::mma_bf16_ss(tmem + buf * 128, kmajor_desc(kb, kk), kmajor_desc(qb, kk), idesc_s, kk > 0);
-                    umma::commit(&s_full[buf]);
+                        umma::mma_bf16_ss(tmem + sb * 128, kmajor_desc(kb, kk), kmajor_desc(qb, kk), idesc_s, kk > 0);
+                    umma::commit(&k_empty[s]);
+                    umma::commit(&s_full[sb]);
                 }
-                if (i >= 1) {                   // O += P(j) V(j), j = i - 1
-                    const int j = i - 1, s = j % P2_STAGES, pbuf = j & 1;
-                    if (!(ok = wait_or_abort(&p_full[pbuf], (j >> 1) & 1, &abort_flag, a.status))) break;
+                if (i >= 2) {                   // O += P(j) V(j), j = i - 2
+                    const int j = i - 2, s = j % P2_STAGES, pg = j & 1;
+                    if (!(ok = wait_or_abort(&p_full[pg], (j >> 1) & 1, &abort_flag, a.status))) break;
+                    if (!(ok = wait_or_abort(&v_full[s], (j / P2_STAGES) & 1, &abort_flag, a.status))) break;
                     umma::fence_after();
-                    const uint32_t vb = smem_u32(kv + s * KV_BYTES + TILE_BYTES);
-                    const uint32_t pbj = pb + pbuf * TILE_BYTES;
+                    const uint32_t vb = smem_u32(vst + s * TILE_BYTES);
+                    const uint32_t pbj = pb + pg * TILE_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < KT / 16; ++kk)
-                        umma::mma_bf16_ss(tmem + 256, mnmajor_desc(pbj, kk), mnmajor_desc(vb, kk), idesc_o,
+                        umma::mma_bf16_ss(tmem + kOcol, mnmajor_desc(pbj, kk), mnmajor_desc(vb, kk), idesc_o,
                                           (j > 0 || kk > 0) ? 1u : 0u);
-                    umma::commit(&p_empty[pbuf]);
-                    umma::commit(&kv_empty[s]);
+                    umma::commit(&p_empty[pg]);
+                    umma::commit(&v_empty[s]);
                 }
             }
             umma::commit(&o_full);
         }
     } else {
-        const int quarter = warp & 3, hf = (warp - 2) >> 2;
+        const int quarter = warp & 3, g = (warp - 2) >> 2;
         const int st = threadIdx.x - 64;        // 0..255
         // log-sum-exp of the 128 (row, head) columns; rows past n_q get +inf (P = 0)
         if (st < MT) {
@@ -325,76 +383,69 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         }
         named_sync(1, NSOFT);
         const int kl = quarter * 32 + lane;     // the key lane this thread owns in S'
-        // this thread's half: columns hf*64 .. hf*64+63 = rows 4hf .. 4hf+3, all heads
-        float* srow0 = a.scores + (static_cast<size_t>(b) * a.n_q + r0 + 4 * hf) * a.score_ld;
-        const float* lse_h = lse_s + hf * 64;
-        for (int i = 0; i < n_kt; ++i) {
-            const int buf = i & 1;
-            if (!wait_or_abort(&s_full[buf], (i >> 1) & 1, &abort_flag, a.status)) break;
+        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+        float* srow0 = a.scores + (static_cast<size_t>(b) * a.n_q + r0) * a.score_ld;
+        uint8_t* pg_tile = ps + g * TILE_BYTES;
+        // one 32-column chunk = rows 2c, 2c+1 x 16 heads: probabilities, the two rows'
+        // importance, bf16 pairs for the P tile
+        uint32_t pk[64];
+        for (int i = g; i < n_kt; i += 2) {
+            const int sb = i % NSB;
+            if (!wait_or_abort(&s_full[sb], (i / NSB) & 1, &abort_flag, a.status)) break;
             umma::fence_after();
-            uint32_t r[2][32];
-            const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + buf * 128 + hf * 64;
-            umma::tmem_ld32(ta, r[0]);
-            umma::tmem_ld32(ta + 32, r[1]);
+            const uint32_t ta = tmem + lane_base + sb * 128;
+            const int key = i * KT + kl;
+            uint32_t ra[32], rb[32];
+            umma::tmem_ld32(ta, ra);
+            umma::tmem_ld_wait();
+            umma::tmem_ld32(ta + 32, rb);
+            p2_chunk<0>(ra, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
+            umma::tmem_ld_wait();
+            umma::tmem_ld32(ta + 64, ra);
+            p2_chunk<1>(rb, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
+            umma::tmem_ld_wait();
+            umma::tmem_ld32(ta + 96, rb);
+            p2_chunk<2>(ra, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
             umma::tmem_ld_wait();
             umma::fence_before();
-            mbar_arrive(&s_empty[buf]);
-            const int key = i * KT + kl;
-            // probabilities, head sums, bf16 pairs for the P tile
-            uint32_t pk[32];
-            float sc[4];
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-                const bool valid = key <= pos_base + 4 * hf + rr;
-                float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                for (int h = 0; h < H; h += 2) {
-                    const int c = rr * H + h;
-                    const float2 l2 = *reinterpret_cast<const float2*>(&lse_h[c]);
-                    float p0 = ex2(__uint_as_float(r[c >> 5][c & 31]) * a.sc2 - l2.x);
-                    float p1 = ex2(__uint_as_float(r[(c + 1) >> 5][(c + 1) & 31]) * a.sc2 - l2.y);
-                    if (!valid) { p0 = 0.f; p1 = 0.f; }
-                    acc0 += p0;
-                    acc1 += p1;
-                    pk[c >> 1] = pack_bf16(p0, p1);
-                }
-                sc[rr] = acc0 + acc1;
-            }
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr)
-                if (key <= pos_base + 4 * hf + rr && r0 + 4 * hf + rr < a.n_q) srow0[rr * a.score_ld + key] = sc[rr];
+            mbar_arrive(&s_empty[sb]);
+            p2_chunk<3>(rb, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
             // last tile: cache rows past the last query position may hold anything, and
-            // 0 * NaN would poison O, so this key's V row (this half) is zeroed (the K row
-            // only feeds probabilities that are forced to 0 above)
+            // 0 * NaN would poison O, so this key's V row is zeroed (the K row only feeds
+            // probabilities that are forced to 0 above).  V(i) is resident: S'(i) was
+            // computed, and V(i) is loaded before K(i + 1).
             if (i == n_kt - 1 && key > p_max) {
-                uint8_t* vrow = kv + (i % P2_STAGES) * KV_BYTES + TILE_BYTES + hf * BOX_BYTES + kl * 128;
+                if (!wait_or_abort(&v_full[i % P2_STAGES], (i / P2_STAGES) & 1, &abort_flag, a.status)) break;
+                uint8_t* vrow = vst + (i % P2_STAGES) * TILE_BYTES + kl * 128;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+                for (int c = 0; c < 8; ++c) {
+                    *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(vrow + BOX_BYTES + c * 16) = make_uint4(0, 0, 0, 0);
+                }
             }
-            // P tile i%2 is free once the O MMA of tile i-2 has completed
-            const int pbuf = i & 1;
-            if (i >= 2 && !wait_or_abort(&p_empty[pbuf], ((i >> 1) - 1) & 1, &abort_flag, a.status)) break;
-            // row `kl` of the MN-major P tile, m-group hf (m = 64 hf .. 64 hf + 63)
-            uint8_t* prow = ps + pbuf * TILE_BYTES + hf * BOX_BYTES + (kl >> 3) * 1024 + (kl & 7) * 128;
+            // this warpgroup's P tile is free once O += P(i-2) V(i-2) has completed
+            if (i >= 2 && !wait_or_abort(&p_empty[g], ((i >> 1) - 1) & 1, &abort_flag, a.status)) break;
+            // row `kl` of the MN-major P tile: m = (row, head) 0..127 in two 64-wide groups
+            uint8_t* prow = pg_tile + (kl >> 3) * 1024 + (kl & 7) * 128;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
+            for (int cc = 0; cc < 16; ++cc) {
                 const uint4 w = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-                *reinterpret_cast<uint4*>(prow + ((cc ^ (kl & 7)) << 4)) = w;
+                *reinterpret_cast<uint4*>(prow + (cc >> 3) * BOX_BYTES + (((cc & 7) ^ (kl & 7)) << 4)) = w;
             }
             umma::fence_proxy_async();
-            mbar_arrive(&p_full[pbuf]);
+            mbar_arrive(&p_full[g]);
         }
         // O epilogue: this thread owns TMEM lane m = (row, head) of the O accumulator and
-        // columns 64 hf .. 64 hf + 63
+        // columns 64 g .. 64 g + 63
         if (wait_or_abort(&o_full, 0, &abort_flag, a.status)) {
             umma::fence_after();
             const int m = quarter * 32 + lane;
             const int row = r0 + (m >> 4);
-            __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + row) * H + (m & 15)) * D + hf * 64;
+            __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + row) * H + (m & 15)) * D + g * 64;
 #pragma unroll 1
             for (int c = 0; c < 64; c += 32) {
                 uint32_t r[32];
-                umma::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + 256 + hf * 64 + c, r);
+                umma::tmem_ld32(tmem + lane_base + kOcol + g * 64 + c, r);
                 umma::tmem_ld_wait();
                 if (row < a.n_q) {
 #pragma unroll
@@ -443,7 +494,7 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     a.status = pa.status;
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
     const size_t s1 = 1024 + TILE_BYTES + P1_STAGES * TILE_BYTES;
-    const size_t s2 = 1024 + TILE_BYTES + P2_STAGES * KV_BYTES + 2 * TILE_BYTES;
+    const size_t s2 = 1024 + TILE_BYTES + 2 * P2_STAGES * TILE_BYTES + 2 * TILE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(prefill_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(prefill_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));

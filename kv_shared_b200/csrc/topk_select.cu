@@ -10,16 +10,23 @@
 // kept whole if any of its tokens is important): blocks of `bs` positions from
 // 0, block importance = max, floor(K/bs) best blocks (lower block on ties).
 //
-// A row is handled by a cluster of CS CTAs (CS = 1..8); CTA r owns a contiguous
-// slice of the candidates and keeps their order-preserving uint32 images in
-// shared memory when they fit.  The K-th best key is found exactly by a radix
-// select over the bits below those every key of the row shares (from the row's
-// key range), at most 11 bits per digit: per digit every CTA builds a histogram
-// of its slice, the cluster's histograms are summed over distributed shared
-// memory and each CTA takes the same decision.  Then every CTA writes,
-// in ascending order, its keys above the threshold and its share of the first
-// (K - #above) keys equal to it (the lower-index tie rule), at offsets from a
-// cluster-wide prefix of the counts.  Integer work only after the key map.
+// Exact selection on order-preserving uint32 images of the fp32 values.  A row
+// is handled by a cluster of CS CTAs (CS = 1..8), CTA r owning a contiguous
+// slice of the keys, cached in shared memory when it fits.
+//   1. the row's key range (reduced over the cluster) gives the bits all keys
+//      share; the first radix digit (<= 11 bits) is taken right below them
+//   2. one histogram of that digit over every key (summed over the cluster by
+//      distributed shared memory) locates the bin b1 holding the K-th best key
+//   3. every CTA compacts, in position order, its keys in bins >= b1 into a
+//      short candidate list (about K plus the few keys of bin b1 per row)
+//   4. the remaining digits are resolved on the candidate lists only -> the exact
+//      threshold key tau and how many keys equal to it are taken (need_eq)
+//   5. each CTA writes its candidates above tau and its share of the first
+//      need_eq equal to tau (the lower-position tie rule), already ascending, at
+//      offsets from a cluster-wide prefix of the counts.
+// If a candidate list would overflow its buffer (adversarial value
+// distributions), the cluster falls back to resolving every digit over all keys.
+// Integer work only after the key map.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -34,7 +41,8 @@ constexpr int NT = 512;
 constexpr int NW = NT / 32;
 constexpr int NBINS = 2048;
 constexpr int kMaxCluster = 8;
-constexpr int kSmemKeys = 32768;          // keys cached per CTA (128 KB)
+constexpr int kSmemKeys = 24576;          // keys cached per CTA (96 KB)
+constexpr int kCandCap = 2048;            // candidates per CTA (16 KB)
 
 __device__ __forceinline__ uint32_t ord_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -42,17 +50,19 @@ __device__ __forceinline__ uint32_t ord_key(float f) {
 }
 
 struct Smem {
-    int hist[NBINS];
+    int hist[2][NBINS];         // double-buffered: a digit's histogram may still be read
+                                // by the cluster while the next digit's is built
     int warp_tot[NW];
     int total;
     int found_bin;
     int found_above;
-    int counts[2];              // this CTA's (#above, #equal) for the compaction
-    uint32_t wlo[NW], whi[NW];  // per-warp key range
+    uint32_t wlo[NW], whi[NW];
     uint32_t range[2];          // this CTA's key range (read by the cluster)
+    int counts[3];              // published to the cluster: #above, #equal, overflow flag
+    int wcnt[NW];               // per-warp candidate counts
 };
 
-// Block-wide exclusive scan of one int per thread; *total receives the sum.
+// Block-wide exclusive scan of one int per thread; sm.total receives the sum.
 __device__ __forceinline__ int block_excl_scan(int v, Smem& sm) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int x = v;
@@ -84,9 +94,9 @@ __device__ __forceinline__ int block_excl_scan(int v, Smem& sm) {
 struct Slice {
     const float* s;            // row scores
     int bs;                    // 1 = token keys, >1 = block maxima
-    int n_cand;                // candidates of the row
+    int n_cand;                // candidate tokens of the row
     int begin, end;            // this CTA's key range (tokens or blocks)
-    uint32_t* cache;           // shared-memory copy or nullptr
+    const uint32_t* cache;     // shared-memory copy or nullptr
     __device__ __forceinline__ uint32_t compute(int i) const {
         if (bs == 1) return ord_key(s[i]);
         float m = -INFINITY;
@@ -95,11 +105,12 @@ struct Slice {
         return ord_key(m);
     }
     __device__ __forceinline__ uint32_t key(int i) const { return cache ? cache[i - begin] : compute(i); }
+    // tokens a selected key expands to
+    __device__ __forceinline__ int tokens(int i) const { return min((i + 1) * bs, n_cand) - i * bs; }
 };
 
 // Visits every key of the slice as f(i, key, valid) with 8 independent loads in
-// flight per thread; all threads of the block make the same number of calls (keys
-// past the slice come with valid = false), so f may use warp-wide primitives.
+// flight per thread; all threads make the same number of calls.
 constexpr int kBatch = 8;
 template <typename F>
 __device__ __forceinline__ void for_keys(const Slice& sl, F f) {
@@ -118,11 +129,111 @@ __device__ __forceinline__ void for_keys(const Slice& sl, F f) {
     }
 }
 
-__global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int cache_keys) {
-    extern __shared__ uint32_t key_cache[];
+// One radix digit: histogram of bits [shift, shift+width) of the keys that `visit`
+// offers and that match prefix under mask, summed over the cluster; leaves the bin
+// holding the k_rem-th largest and the count above it in sm.found_bin/found_above.
+// Histogram buffer `hb` alternates between digits, so one cluster barrier per digit
+// suffices (a buffer is rebuilt only after every CTA has passed the next barrier).
+template <int CS, typename Visit>
+__device__ __forceinline__ void radix_digit(cg::cluster_group& cluster, Smem& sm, int hbuf, int shift, int width,
+                                            uint32_t prefix, uint32_t mask, int k_rem, Visit visit) {
+    const int nb = 1 << width;
+    int* hist = sm.hist[hbuf];
+    for (int i = threadIdx.x; i < nb; i += NT) hist[i] = 0;
+    __syncthreads();
+    visit([&](uint32_t key) {
+        if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1);
+    });
+    cluster.sync();
+    const int bins_per = (nb + NT - 1) / NT;                   // 1..4
+    int local[NBINS / NT];
+    int tot = 0;
+#pragma unroll
+    for (int q = 0; q < NBINS / NT; ++q) {
+        const int bin = nb - 1 - (threadIdx.x * bins_per + q);
+        int c = 0;
+        if (q < bins_per && bin >= 0) {
+            int v[CS];
+#pragma unroll
+            for (int rr = 0; rr < CS; ++rr) v[rr] = CS == 1 ? hist[bin] : cluster.map_shared_rank(hist, rr)[bin];
+#pragma unroll
+            for (int rr = 0; rr < CS; ++rr) c += v[rr];
+        }
+        local[q] = c;
+        tot += c;
+    }
+    const int above = block_excl_scan(tot, sm);
+    if (above < k_rem && above + tot >= k_rem) {
+        int acc = above;
+        for (int q = 0; q < bins_per; ++q) {
+            if (acc + local[q] >= k_rem) {
+                sm.found_bin = nb - 1 - (threadIdx.x * bins_per + q);
+                sm.found_above = acc;
+                break;
+            }
+            acc += local[q];
+        }
+    }
+    __syncthreads();
+}
+
+// Writes, in ascending order from out + written, the selected keys among n entries
+// (position pos(e), key keyf(e), already ascending): key > tau, or key == tau while
+// the running rank of equal keys (starting at eq_seen) is below need_eq; take_all
+// selects every entry.  Returns the new written count.
+template <typename Pos, typename Key>
+__device__ __forceinline__ int ordered_write(Smem& sm, const Slice& sl, int n, Pos pos, Key keyf, uint32_t tau,
+                                             int need_eq, bool take_all, int eq_seen, int written, int32_t* out) {
+    for (int base = 0; base < n; base += 4 * NT) {
+        const int e0 = base + 4 * threadIdx.x;
+        uint32_t keys[4];
+        int e_cnt = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u;
+            keys[u] = (e < n) ? keyf(e) : 0u;
+            if (e < n && !take_all) e_cnt += keys[u] == tau;
+        }
+        const int eq_before = block_excl_scan(e_cnt, sm);
+        const int eq_round = sm.total;
+        int rank_eq = eq_seen + eq_before, ntok = 0;
+        bool sel[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u;
+            sel[u] = false;
+            if (e >= n) continue;
+            if (take_all || keys[u] > tau) sel[u] = true;
+            else if (keys[u] == tau) { sel[u] = rank_eq < need_eq; ++rank_eq; }
+            if (sel[u]) ntok += sl.tokens(pos(e));
+        }
+        const int at = block_excl_scan(ntok, sm);
+        const int round_total = sm.total;
+        int o = written + at;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (!sel[u]) continue;
+            const int i = pos(e0 + u);
+            const int e = min((i + 1) * sl.bs, sl.n_cand);
+            for (int j = i * sl.bs; j < e; ++j) out[o++] = j;
+        }
+        written += round_total;
+        eq_seen += eq_round;
+    }
+    return written;
+}
+
+template <int CS>
+__global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys) {
+    constexpr int cs = CS;
+    extern __shared__ uint32_t dsm[];
+    uint32_t* key_cache = dsm;                                 // [cache_keys]
+    uint32_t* cand_key = dsm + cache_keys;                     // [kCandCap]
+    int* cand_pos = reinterpret_cast<int*>(cand_key + kCandCap);
     __shared__ Smem sm;
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int row = blockIdx.x / cs;
     const int b = row / a.n_q, r = row % a.n_q;
     const int p = checked_pos(a.q_pos0[b] + r, a.max_ctx, a.status);
@@ -133,6 +244,8 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int ca
     const int bs = a.block_size < 1 ? 1 : a.block_size;
     const int n_keys = (n_cand + bs - 1) / bs;                    // tokens or blocks
     const int K = bs == 1 ? min(a.budget, n_cand) : min(a.budget / bs, n_keys);
+    const bool take_all = (K >= n_keys);
+    const bool take_none = (K <= 0);
 
     Slice sl;
     sl.s = a.scores + static_cast<size_t>(row) * a.score_ld;
@@ -142,100 +255,150 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int ca
     sl.begin = min(rank * per, n_keys);
     sl.end = min(sl.begin + per, n_keys);
     sl.cache = nullptr;
-    if (per <= cache_keys) {
-        if (bs == 1) {
-            // token keys: 8 coalesced loads in flight per thread
-            for_keys(sl, [&](int i, uint32_t key, bool valid) { if (valid) key_cache[i - sl.begin] = key; });
-        } else {
+
+    // ---- 1. cache the slice's keys (when they fit) and find its key range
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    const bool cached = per <= cache_keys;
+    if (!take_all && !take_none) {
+        if (cached && bs > 1) {
             // block keys: one warp per block, max over its tokens by shuffles
-            const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
             for (int bb = sl.begin + warp; bb < sl.end; bb += NW) {
                 const int e = min((bb + 1) * bs, n_cand);
                 float m = -INFINITY;
                 for (int j = bb * bs + lane; j < e; j += 32) m = fmaxf(m, sl.s[j]);
                 m = warp_max(m);
-                if (lane == 0) key_cache[bb - sl.begin] = ord_key(m);
+                const uint32_t k = ord_key(m);
+                if (lane == 0) key_cache[bb - sl.begin] = k;
+                lo = min(lo, k);
+                hi = max(hi, k);
             }
+        } else {
+            for_keys(sl, [&](int i, uint32_t key, bool valid) {
+                if (!valid) return;
+                if (cached) key_cache[i - sl.begin] = key;
+                lo = min(lo, key);
+                hi = max(hi, key);
+            });
         }
-        sl.cache = key_cache;
-    }
-    __syncthreads();
-
-    uint32_t tau = 0;
-    int need_eq = 0;
-    const bool take_all = (K >= n_keys);
-    const bool take_none = (K <= 0);
-    if (!take_all && K > 0) {
-        // key range of the row: the digits start right below the bits every key shares
-        // (importance values crowd into a few binades; a fixed top digit would put them
-        // into a handful of bins)
-        uint32_t lo = 0xffffffffu, hi = 0u;
-        for_keys(sl, [&](int, uint32_t key, bool valid) {
-            if (valid) { lo = min(lo, key); hi = max(hi, key); }
-        });
+        if (cached) sl.cache = key_cache;
         lo = __reduce_min_sync(0xffffffffu, lo);
         hi = __reduce_max_sync(0xffffffffu, hi);
-        if ((threadIdx.x & 31) == 0) { sm.wlo[threadIdx.x >> 5] = lo; sm.whi[threadIdx.x >> 5] = hi; }
+        if (lane == 0) { sm.wlo[warp] = lo; sm.whi[warp] = hi; }
         __syncthreads();
         if (threadIdx.x == 0) {
             uint32_t l = sm.wlo[0], h = sm.whi[0];
             for (int w = 1; w < NW; ++w) { l = min(l, sm.wlo[w]); h = max(h, sm.whi[w]); }
             sm.range[0] = l; sm.range[1] = h;
         }
-        cluster.sync();
+        cluster.sync();                            // sm.range is written once: no barrier after
         lo = 0xffffffffu; hi = 0u;
+#pragma unroll
         for (int rr = 0; rr < cs; ++rr) {
-            const uint32_t* rg = cluster.map_shared_rank(sm.range, rr);
+            const uint32_t* rg = cs == 1 ? sm.range : cluster.map_shared_rank(sm.range, rr);
             lo = min(lo, rg[0]);
             hi = max(hi, rg[1]);
         }
-        cluster.sync();
-        if (lo == hi) {                         // every candidate key is the same value
+    }
+
+    uint32_t tau = 0;
+    int need_eq = 0;
+    int written = 0;
+    bool use_cands = false;
+    int n_my = 0;                                  // this CTA's candidate count
+    if (!take_all && !take_none) {
+        if (lo == hi) {                            // every key has the same value
             tau = hi;
             need_eq = K;
         } else {
-            const int hb = 31 - __clz(lo ^ hi); // highest bit where the keys differ
-            uint32_t mask = ~((2u << hb) - 1u); // (hb == 31 gives 0: nothing shared)
+            const int hb = 31 - __clz(lo ^ hi);    // highest bit where the keys differ
+            uint32_t mask = ~((2u << hb) - 1u);    // (hb == 31 gives 0: nothing shared)
             uint32_t prefix = hi & mask;
             int k_rem = K;
-#pragma unroll 1
-            for (int top = hb; top >= 0;) {
-                const int width = min(11, top + 1);
-                const int shift = top - width + 1, nb = 1 << width;
-                for (int i = threadIdx.x; i < nb; i += NT) sm.hist[i] = 0;
-                __syncthreads();
-                for_keys(sl, [&](int, uint32_t key, bool valid) {
-                    if (valid && (key & mask) == prefix) atomicAdd(&sm.hist[(key >> shift) & (nb - 1)], 1);
-                });
-                cluster.sync();
-                // counts of the whole row: sum of the cluster's histograms, from the top bin
-                const int bins_per = (nb + NT - 1) / NT;               // 1..4
-                int local[NBINS / NT];
-                int tot = 0;
-                for (int q = 0; q < bins_per; ++q) {
-                    const int bin = nb - 1 - (threadIdx.x * bins_per + q);
-                    int c = 0;
-                    if (bin >= 0)
-                        for (int rr = 0; rr < cs; ++rr) c += cluster.map_shared_rank(sm.hist, rr)[bin];
-                    local[q] = c;
-                    tot += c;
-                }
-                cluster.sync();                 // every CTA has read every histogram
-                const int above = block_excl_scan(tot, sm);
-                if (above < k_rem && above + tot >= k_rem) {
-                    int acc = above;
-                    for (int q = 0; q < bins_per; ++q) {
-                        if (acc + local[q] >= k_rem) {
-                            sm.found_bin = nb - 1 - (threadIdx.x * bins_per + q);
-                            sm.found_above = acc;
-                            break;
-                        }
-                        acc += local[q];
+            // ---- 2. first digit over every key
+            int width = min(11, hb + 1);
+            int shift = hb - width + 1;
+            int hbuf = 0;
+            radix_digit<CS>(cluster, sm, hbuf, shift, width, prefix, mask, k_rem, [&](auto add) {
+                for_keys(sl, [&](int, uint32_t key, bool valid) { if (valid) add(key); });
+            });
+            hbuf ^= 1;
+            prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
+            mask |= static_cast<uint32_t>((1 << width) - 1) << shift;
+            k_rem -= sm.found_above;
+            __syncthreads();
+            // ---- 3. candidates: keys >= prefix (bins >= b1), in position order
+            {
+                const int seg = (((sl.end - sl.begin) + NW - 1) / NW + 31) & ~31;
+                const int s0 = min(sl.begin + warp * seg, sl.end), s1 = min(s0 + seg, sl.end);
+                int c = 0;
+                for (int i = s0; i < s1; i += 32 * kBatch) {
+                    uint32_t k[kBatch];
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u) {
+                        const int ii = i + u * 32 + lane;
+                        k[u] = ii < s1 ? sl.key(ii) : 0u;
                     }
+#pragma unroll
+                    for (int u = 0; u < kBatch; ++u)
+                        c += __popc(__ballot_sync(0xffffffffu, (i + u * 32 + lane < s1) && k[u] >= prefix));
                 }
+                if (lane == 0) sm.wcnt[warp] = c;
                 __syncthreads();
+                if (threadIdx.x == 0) {
+                    int acc = 0;
+                    for (int w = 0; w < NW; ++w) { const int t = sm.wcnt[w]; sm.wcnt[w] = acc; acc += t; }
+                    sm.counts[2] = acc > kCandCap ? 1 : 0;
+                    sm.total = acc;
+                }
+                cluster.sync();                    // the flag is written once: no barrier after
+                int overflow = 0;
+#pragma unroll
+                for (int rr = 0; rr < cs; ++rr) overflow |= (cs == 1 ? sm.counts : cluster.map_shared_rank(sm.counts, rr))[2];
+                n_my = sm.total;
+                __syncthreads();                   // sm.total is reused by the scans below
+                use_cands = overflow == 0;
+                if (use_cands) {
+                    int at = sm.wcnt[warp];
+                    for (int i = s0; i < s1; i += 32 * kBatch) {
+                        uint32_t k[kBatch];
+#pragma unroll
+                        for (int u = 0; u < kBatch; ++u) {
+                            const int ii = i + u * 32 + lane;
+                            k[u] = ii < s1 ? sl.key(ii) : 0u;
+                        }
+#pragma unroll
+                        for (int u = 0; u < kBatch; ++u) {
+                            const int ii = i + u * 32 + lane;
+                            const bool q = (ii < s1) && k[u] >= prefix;
+                            const unsigned bal = __ballot_sync(0xffffffffu, q);
+                            if (q) {
+                                const int o = at + __popc(bal & ((1u << lane) - 1u));
+                                cand_key[o] = k[u];
+                                cand_pos[o] = ii;
+                            }
+                            at += __popc(bal);
+                        }
+                    }
+                    __syncthreads();
+                }
+            }
+            // ---- 4. remaining digits on the candidates (or, after an overflow, on every key)
+#pragma unroll 1
+            for (int top = shift - 1; top >= 0;) {
+                width = min(11, top + 1);
+                shift = top - width + 1;
+                if (use_cands) {
+                    radix_digit<CS>(cluster, sm, hbuf, shift, width, prefix, mask, k_rem, [&](auto add) {
+                        for (int e = threadIdx.x; e < n_my; e += NT) add(cand_key[e]);
+                    });
+                } else {
+                    radix_digit<CS>(cluster, sm, hbuf, shift, width, prefix, mask, k_rem, [&](auto add) {
+                        for_keys(sl, [&](int, uint32_t key, bool valid) { if (valid) add(key); });
+                    });
+                }
+                hbuf ^= 1;
                 prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
-                mask |= static_cast<uint32_t>(nb - 1) << shift;
+                mask |= static_cast<uint32_t>((1 << width) - 1) << shift;
                 k_rem -= sm.found_above;
                 __syncthreads();
                 top = shift - 1;
@@ -245,78 +408,57 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int ca
         }
     }
 
-    // this CTA's counts, then cluster-wide offsets
+    // ---- 5. counts of this CTA, cluster-wide offsets, ordered write
     int gt = 0, eq = 0;
-    if (!take_all && K > 0) {
-        for_keys(sl, [&](int, uint32_t key, bool valid) {
-            gt += valid && key > tau;
-            eq += valid && key == tau;
-        });
+    if (!take_all && !take_none) {
+        if (use_cands) {
+            for (int e = threadIdx.x; e < n_my; e += NT) {
+                gt += cand_key[e] > tau;
+                eq += cand_key[e] == tau;
+            }
+        } else {
+            for_keys(sl, [&](int, uint32_t key, bool valid) {
+                gt += valid && key > tau;
+                eq += valid && key == tau;
+            });
+        }
     }
-    int t_gt = block_excl_scan(gt, sm);
-    t_gt = sm.total;
-    int t_eq = block_excl_scan(eq, sm);
-    t_eq = sm.total;
-    (void)t_gt;
+    block_excl_scan(gt, sm);
+    const int t_gt = sm.total;
+    block_excl_scan(eq, sm);
+    const int t_eq = sm.total;
     if (threadIdx.x == 0) { sm.counts[0] = t_gt; sm.counts[1] = t_eq; }
-    cluster.sync();
-    int out_base = 0, eq_base = 0;                   // tokens written / equal keys seen before this CTA
+    cluster.sync();                                // counts are written once: the final barrier
+                                                   // keeps them alive while they are read
+    int out_base = 0, eq_base = 0;                 // tokens written / equal keys before this CTA
     for (int rr = 0; rr < rank; ++rr) {
         const int* c = cluster.map_shared_rank(sm.counts, rr);
-        const int e_before = eq_base;
-        const int take_eq = take_all ? 0 : max(0, min(c[1], need_eq - e_before));
         int keys_sel;
         if (take_all) {
             const int rb = min(rr * per, n_keys), re = min(rb + per, n_keys);
             keys_sel = re - rb;
+        } else if (take_none) {
+            keys_sel = 0;
         } else {
-            keys_sel = c[0] + take_eq;
+            keys_sel = c[0] + max(0, min(c[1], need_eq - eq_base));
         }
-        // tokens: blocks expand to bs tokens (only the row's last block is partial, and it
-        // belongs to the last CTA, never to a lower rank)
+        // lower ranks own only whole blocks (a partial last block belongs to the CTA
+        // owning the row's last key, and never precedes another CTA's keys)
         out_base += keys_sel * bs;
         eq_base += c[1];
     }
-    cluster.sync();                                  // remote counts read: they may be reused
 
-    // ascending compaction of this CTA's slice, 4 consecutive keys per thread per round
-    int eq_seen = eq_base;
-    int written = out_base;
-    for (int base = sl.begin; base < (take_none ? sl.begin : sl.end); base += 4 * NT) {
-        const int i0 = base + 4 * threadIdx.x;
-        uint32_t keys[4];
-        int e_cnt = 0;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u;
-            keys[u] = (i < sl.end) ? sl.key(i) : 0u;
-            if (i < sl.end && !take_all) e_cnt += keys[u] == tau;
+    written = out_base;
+    if (!take_none) {
+        if (use_cands) {
+            written = ordered_write(
+                sm, sl, n_my, [&](int e) { return cand_pos[e]; }, [&](int e) { return cand_key[e]; }, tau, need_eq,
+                false, eq_base, written, out);
+        } else {
+            written = ordered_write(
+                sm, sl, sl.end - sl.begin, [&](int e) { return sl.begin + e; },
+                [&](int e) { return sl.key(sl.begin + e); }, tau, need_eq, take_all, eq_base, written, out);
         }
-        const int eq_before = block_excl_scan(e_cnt, sm);
-        const int eq_round = sm.total;
-        int rank_eq = eq_seen + eq_before, ntok = 0;
-        bool sel[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = i0 + u;
-            sel[u] = false;
-            if (i >= sl.end) continue;
-            if (take_all || keys[u] > tau) sel[u] = true;
-            else if (keys[u] == tau) { sel[u] = rank_eq < need_eq; ++rank_eq; }
-            if (sel[u]) ntok += min((i + 1) * bs, n_cand) - i * bs;
-        }
-        const int pos = block_excl_scan(ntok, sm);
-        const int round_total = sm.total;
-        int o = written + pos;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            if (!sel[u]) continue;
-            const int i = i0 + u;
-            const int e = min((i + 1) * bs, n_cand);
-            for (int j = i * bs; j < e; ++j) out[o++] = j;
-        }
-        written += round_total;
-        eq_seen += eq_round;
     }
 
     // the forced window after all global picks (every window position exceeds every
@@ -329,10 +471,12 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cs, int ca
         for (int i = total + threadIdx.x; i < a.idx_stride; i += NT) out[i] = -1;
         if (threadIdx.x == 0) a.cnt[row] = total;
     }
-    cluster.sync();                                  // no CTA leaves while its memory may be read
+    cluster.sync();                                // no CTA leaves while its memory may be read
 }
 
 int pick_cluster(int rows, int64_t max_keys) {
+    // enough rows to fill the GPU: one CTA per row (keys streamed when they do not fit)
+    if (rows >= 2 * num_sms()) return 1;
     int cs = 1;
     while (cs < kMaxCluster && (max_keys + cs - 1) / cs > kSmemKeys) cs *= 2;
     const int target = 2 * num_sms();
@@ -350,10 +494,7 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
     const int cs = pick_cluster(a.rows, max_keys);
     const int64_t per = ((max_keys + cs - 1) / cs + 3) & ~int64_t(3);
     const int cache_keys = per <= kSmemKeys ? static_cast<int>(per) : 0;
-    const size_t smem = static_cast<size_t>(cache_keys) * sizeof(uint32_t);
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
+    const size_t smem = (static_cast<size_t>(cache_keys) + 2 * kCandCap) * sizeof(uint32_t);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(a.rows) * cs);
     cfg.blockDim = dim3(NT);
@@ -366,7 +507,17 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, select_kernel, a, cs, cache_keys);
+    auto launch = [&](auto kern) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        return cudaLaunchKernelEx(&cfg, kern, a, cache_keys);
+    };
+    switch (cs) {
+        case 1: return launch(select_kernel<1>);
+        case 2: return launch(select_kernel<2>);
+        case 4: return launch(select_kernel<4>);
+        default: return launch(select_kernel<8>);
+    }
 }
 
 }  // namespace hs2
