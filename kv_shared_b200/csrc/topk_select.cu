@@ -42,7 +42,7 @@ constexpr int NW = NT / 32;
 constexpr int NBINS = 2048;
 constexpr int kMaxCluster = 8;
 constexpr int kSmemKeys = 24576;          // keys cached per CTA (96 KB)
-constexpr int kCandCap = 2048;            // candidates per CTA (16 KB)
+constexpr int kCandCap = 2048;            // candidates per CTA (16 KB), a power of two
 
 __device__ __forceinline__ uint32_t ord_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -58,8 +58,13 @@ struct Smem {
     int found_above;
     uint32_t wlo[NW], whi[NW];
     uint32_t range[2];          // this CTA's key range (read by the cluster)
-    int counts[3];              // published to the cluster: #above, #equal, overflow flag
-    int wcnt[NW];               // per-warp candidate counts
+    int counts[2];              // published to the cluster: #above, #equal (fallback paths)
+    int dec[8];                 // rank 0's decisions: first-digit bin, count above, bin size,
+                                // candidate mode; threshold key and equal keys to take
+    int pub[2];                 // this CTA's candidate count (read by rank 0)
+    int table[kMaxCluster][2];  // rank 0: output offset and equal-key rank base per CTA
+    int cnt_gt[kMaxCluster], cnt_eq[kMaxCluster];
+    int ncand, ncand2;
 };
 
 // Block-wide exclusive scan of one int per thread; sm.total receives the sum.
@@ -223,13 +228,75 @@ __device__ __forceinline__ int ordered_write(Smem& sm, const Slice& sl, int n, P
     return written;
 }
 
+// Visits every key of the slice as f(i, key) (any order).  Token keys go through
+// 16-byte loads, 4 keys each and 4 loads in flight per thread, whenever the slice
+// start is 16-byte aligned (shared-memory cache or score row); otherwise for_keys.
+template <typename F>
+__device__ __forceinline__ void for_keys_fast(const Slice& sl, F f) {
+    const void* base_ptr = sl.cache ? static_cast<const void*>(sl.cache) : static_cast<const void*>(sl.s + sl.begin);
+    if (sl.bs != 1 || (reinterpret_cast<uintptr_t>(base_ptr) & 15u) != 0) {
+        for_keys(sl, [&](int i, uint32_t key, bool valid) { if (valid) f(i, key); });
+        return;
+    }
+    const int n = sl.end - sl.begin, n4 = n >> 2;
+    for (int base = 0; base < n4; base += NT * 4) {
+        uint4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int q = base + u * NT + threadIdx.x;
+            if (q < n4) {
+                if (sl.cache) {
+                    v[u] = reinterpret_cast<const uint4*>(sl.cache)[q];
+                } else {
+                    const float4 x = __ldg(reinterpret_cast<const float4*>(sl.s + sl.begin) + q);
+                    v[u] = make_uint4(ord_key(x.x), ord_key(x.y), ord_key(x.z), ord_key(x.w));
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int q = base + u * NT + threadIdx.x;
+            if (q < n4) {
+                const int i = sl.begin + 4 * q;
+                f(i, v[u].x); f(i + 1, v[u].y); f(i + 2, v[u].z); f(i + 3, v[u].w);
+            }
+        }
+    }
+    for (int i = sl.begin + 4 * n4 + threadIdx.x; i < sl.end; i += NT) f(i, sl.key(i));
+}
+
+// Bitonic sort of n (<= cap, cap a power of two) (a, b) pairs in shared memory,
+// ascending by a when `ascending`, else descending; entries [n, N) are padding.
+__device__ __forceinline__ void bitonic_sort(uint32_t* a, uint32_t* bvals, int n, bool ascending) {
+    int N = 1;
+    while (N < n) N <<= 1;
+    const uint32_t pad = ascending ? 0xffffffffu : 0u;
+    for (int i = n + threadIdx.x; i < N; i += NT) { a[i] = pad; if (bvals) bvals[i] = 0u; }
+    __syncthreads();
+    for (int k = 2; k <= N; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int t = threadIdx.x; t < N / 2; t += NT) {
+                const int i = (t / j) * 2 * j + (t % j);
+                const int l = i + j;
+                const bool up = ((i & k) == 0) == ascending;
+                const uint32_t x = a[i], y = a[l];
+                if ((x > y) == up && x != y) {
+                    a[i] = y; a[l] = x;
+                    if (bvals) { const uint32_t t2 = bvals[i]; bvals[i] = bvals[l]; bvals[l] = t2; }
+                }
+            }
+            __syncthreads();
+        }
+    }
+}
+
 template <int CS>
 __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys) {
     constexpr int cs = CS;
     extern __shared__ uint32_t dsm[];
     uint32_t* key_cache = dsm;                                 // [cache_keys]
     uint32_t* cand_key = dsm + cache_keys;                     // [kCandCap]
-    int* cand_pos = reinterpret_cast<int*>(cand_key + kCandCap);
+    uint32_t* cand_pos = cand_key + kCandCap;                  // [kCandCap]
     __shared__ Smem sm;
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
@@ -246,6 +313,7 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
     const int K = bs == 1 ? min(a.budget, n_cand) : min(a.budget / bs, n_keys);
     const bool take_all = (K >= n_keys);
     const bool take_none = (K <= 0);
+    auto remote = [&](auto* ptr, int rr) { return cs == 1 ? ptr : cluster.map_shared_rank(ptr, rr); };
 
     Slice sl;
     sl.s = a.scores + static_cast<size_t>(row) * a.score_ld;
@@ -256,7 +324,7 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
     sl.end = min(sl.begin + per, n_keys);
     sl.cache = nullptr;
 
-    // ---- 1. cache the slice's keys (when they fit) and find its key range
+    // ---- 1. cache the slice's keys (when they fit) and find the row's key range
     uint32_t lo = 0xffffffffu, hi = 0u;
     const bool cached = per <= cache_keys;
     if (!take_all && !take_none) {
@@ -273,8 +341,7 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
                 hi = max(hi, k);
             }
         } else {
-            for_keys(sl, [&](int i, uint32_t key, bool valid) {
-                if (!valid) return;
+            for_keys_fast(sl, [&](int i, uint32_t key) {
                 if (cached) key_cache[i - sl.begin] = key;
                 lo = min(lo, key);
                 hi = max(hi, key);
@@ -290,11 +357,11 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
             for (int w = 1; w < NW; ++w) { l = min(l, sm.wlo[w]); h = max(h, sm.whi[w]); }
             sm.range[0] = l; sm.range[1] = h;
         }
-        cluster.sync();                            // sm.range is written once: no barrier after
+        cluster.sync();                            // [barrier 1] ranges written once
         lo = 0xffffffffu; hi = 0u;
 #pragma unroll
         for (int rr = 0; rr < cs; ++rr) {
-            const uint32_t* rg = cs == 1 ? sm.range : cluster.map_shared_rank(sm.range, rr);
+            const uint32_t* rg = remote(sm.range, rr);
             lo = min(lo, rg[0]);
             hi = max(hi, rg[1]);
         }
@@ -302,9 +369,10 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
 
     uint32_t tau = 0;
     int need_eq = 0;
-    int written = 0;
     bool use_cands = false;
     int n_my = 0;                                  // this CTA's candidate count
+    int out_base = 0, eq_base = 0;                 // tokens / equal keys before this CTA's
+    bool offsets_known = false;
     if (!take_all && !take_none) {
         if (lo == hi) {                            // every key has the same value
             tau = hi;
@@ -314,146 +382,194 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
             uint32_t mask = ~((2u << hb) - 1u);    // (hb == 31 gives 0: nothing shared)
             uint32_t prefix = hi & mask;
             int k_rem = K;
-            // ---- 2. first digit over every key
             int width = min(11, hb + 1);
             int shift = hb - width + 1;
-            int hbuf = 0;
-            radix_digit<CS>(cluster, sm, hbuf, shift, width, prefix, mask, k_rem, [&](auto add) {
-                for_keys(sl, [&](int, uint32_t key, bool valid) { if (valid) add(key); });
-            });
-            hbuf ^= 1;
-            prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
-            mask |= static_cast<uint32_t>((1 << width) - 1) << shift;
-            k_rem -= sm.found_above;
+            const int nb = 1 << width;
+            // ---- 2. first digit over every key; rank 0 sums the cluster's histograms
+            int* hist = sm.hist[0];
+            for (int i = threadIdx.x; i < nb; i += NT) hist[i] = 0;
             __syncthreads();
-            // ---- 3. candidates: keys >= prefix (bins >= b1), in position order
-            {
-                const int seg = (((sl.end - sl.begin) + NW - 1) / NW + 31) & ~31;
-                const int s0 = min(sl.begin + warp * seg, sl.end), s1 = min(s0 + seg, sl.end);
-                int c = 0;
-                for (int i = s0; i < s1; i += 32 * kBatch) {
-                    uint32_t k[kBatch];
+            for_keys_fast(sl, [&](int, uint32_t key) { atomicAdd(&hist[(key >> shift) & (nb - 1)], 1); });
+            cluster.sync();                        // [barrier 2] histograms complete
+            if (rank == 0) {
+                const int bins_per = (nb + NT - 1) / NT;
+                int local[NBINS / NT];
+                int tot = 0;
 #pragma unroll
-                    for (int u = 0; u < kBatch; ++u) {
-                        const int ii = i + u * 32 + lane;
-                        k[u] = ii < s1 ? sl.key(ii) : 0u;
+                for (int q = 0; q < NBINS / NT; ++q) {
+                    const int bin = nb - 1 - (threadIdx.x * bins_per + q);
+                    int c = 0;
+                    if (q < bins_per && bin >= 0) {
+                        int v[CS];
+#pragma unroll
+                        for (int rr = 0; rr < CS; ++rr) v[rr] = remote(hist, rr)[bin];
+#pragma unroll
+                        for (int rr = 0; rr < CS; ++rr) c += v[rr];
                     }
-#pragma unroll
-                    for (int u = 0; u < kBatch; ++u)
-                        c += __popc(__ballot_sync(0xffffffffu, (i + u * 32 + lane < s1) && k[u] >= prefix));
+                    local[q] = c;
+                    tot += c;
                 }
-                if (lane == 0) sm.wcnt[warp] = c;
-                __syncthreads();
-                if (threadIdx.x == 0) {
-                    int acc = 0;
-                    for (int w = 0; w < NW; ++w) { const int t = sm.wcnt[w]; sm.wcnt[w] = acc; acc += t; }
-                    sm.counts[2] = acc > kCandCap ? 1 : 0;
-                    sm.total = acc;
-                }
-                cluster.sync();                    // the flag is written once: no barrier after
-                int overflow = 0;
-#pragma unroll
-                for (int rr = 0; rr < cs; ++rr) overflow |= (cs == 1 ? sm.counts : cluster.map_shared_rank(sm.counts, rr))[2];
-                n_my = sm.total;
-                __syncthreads();                   // sm.total is reused by the scans below
-                use_cands = overflow == 0;
-                if (use_cands) {
-                    int at = sm.wcnt[warp];
-                    for (int i = s0; i < s1; i += 32 * kBatch) {
-                        uint32_t k[kBatch];
-#pragma unroll
-                        for (int u = 0; u < kBatch; ++u) {
-                            const int ii = i + u * 32 + lane;
-                            k[u] = ii < s1 ? sl.key(ii) : 0u;
+                const int above = block_excl_scan(tot, sm);
+                if (above < k_rem && above + tot >= k_rem) {
+                    int acc = above;
+                    for (int q = 0; q < bins_per; ++q) {
+                        if (acc + local[q] >= k_rem) {
+                            sm.dec[0] = nb - 1 - (threadIdx.x * bins_per + q);
+                            sm.dec[1] = acc;
+                            sm.dec[2] = local[q];
+                            break;
                         }
-#pragma unroll
-                        for (int u = 0; u < kBatch; ++u) {
-                            const int ii = i + u * 32 + lane;
-                            const bool q = (ii < s1) && k[u] >= prefix;
-                            const unsigned bal = __ballot_sync(0xffffffffu, q);
-                            if (q) {
-                                const int o = at + __popc(bal & ((1u << lane) - 1u));
-                                cand_key[o] = k[u];
-                                cand_pos[o] = ii;
-                            }
-                            at += __popc(bal);
+                        acc += local[q];
+                    }
+                }
+                __syncthreads();
+                // candidate lists fit when K + |bin b1| <= kCandCap (a CTA holds at most the
+                // row's keys above b1 (< K) plus those in b1); the gather buffer holds |b1|
+                if (threadIdx.x == 0) sm.dec[3] = (K + sm.dec[2] <= kCandCap && sm.dec[2] <= 2 * NBINS) ? 1 : 0;
+            }
+            cluster.sync();                        // [barrier 3] decision published
+            const int* d0 = remote(sm.dec, 0);
+            const int b1 = d0[0], above1 = d0[1];
+            use_cands = d0[3] != 0;
+            prefix |= static_cast<uint32_t>(b1) << shift;
+            mask |= static_cast<uint32_t>(nb - 1) << shift;
+            k_rem -= above1;
+            if (use_cands) {
+                // ---- 3. candidates: this CTA's keys at or above bin b1, sorted by position
+                if (threadIdx.x == 0) { sm.ncand = 0; sm.ncand2 = 0; }
+                __syncthreads();
+                for_keys_fast(sl, [&](int i, uint32_t key) {
+                    if (key >= prefix) {
+                        const int o = atomicAdd(&sm.ncand, 1);
+                        cand_key[o] = key;
+                        cand_pos[o] = static_cast<uint32_t>(i);
+                    }
+                });
+                __syncthreads();
+                n_my = sm.ncand;
+                bitonic_sort(cand_pos, cand_key, n_my, true);
+                if (threadIdx.x == 0) sm.pub[0] = n_my;
+                cluster.sync();                    // [barrier 4] candidate lists complete
+                // ---- 4. rank 0: the bin-b1 keys of the whole cluster, sorted descending, give
+                // tau exactly; then every CTA's counts and output offsets
+                if (rank == 0) {
+                    uint32_t* g = reinterpret_cast<uint32_t*>(&sm.hist[0][0]);    // 2 * NBINS keys
+                    for (int rr = 0; rr < cs; ++rr) {
+                        const int n_rr = remote(sm.pub, rr)[0];
+                        const uint32_t* ck = remote(cand_key, rr);
+                        for (int e = threadIdx.x; e < n_rr; e += NT) {
+                            const uint32_t key = ck[e];
+                            if ((key & mask) == prefix) g[atomicAdd(&sm.ncand2, 1)] = key;
+                        }
+                    }
+                    if (threadIdx.x < kMaxCluster) { sm.cnt_gt[threadIdx.x] = 0; sm.cnt_eq[threadIdx.x] = 0; }
+                    __syncthreads();
+                    const int n1 = sm.ncand2;
+                    bitonic_sort(g, nullptr, n1, false);
+                    const uint32_t t = g[k_rem - 1];
+                    for (int rr = 0; rr < cs; ++rr) {
+                        const int n_rr = remote(sm.pub, rr)[0];
+                        const uint32_t* ck = remote(cand_key, rr);
+                        int cg_ = 0, ce = 0;
+                        for (int e = threadIdx.x; e < n_rr; e += NT) {
+                            const uint32_t key = ck[e];
+                            cg_ += key > t;
+                            ce += key == t;
+                        }
+                        cg_ = __reduce_add_sync(0xffffffffu, cg_);
+                        ce = __reduce_add_sync(0xffffffffu, ce);
+                        if (lane == 0) {
+                            if (cg_) atomicAdd(&sm.cnt_gt[rr], cg_);
+                            if (ce) atomicAdd(&sm.cnt_eq[rr], ce);
                         }
                     }
                     __syncthreads();
+                    if (threadIdx.x == 0) {
+                        int total_gt = 0;
+                        for (int rr = 0; rr < cs; ++rr) total_gt += sm.cnt_gt[rr];
+                        const int neq = K - total_gt;          // equal keys still to take
+                        int ob = 0, eb = 0;
+                        for (int rr = 0; rr < cs; ++rr) {
+                            sm.table[rr][0] = ob;
+                            sm.table[rr][1] = eb;
+                            ob += (sm.cnt_gt[rr] + max(0, min(sm.cnt_eq[rr], neq - eb))) * bs;
+                            eb += sm.cnt_eq[rr];
+                        }
+                        sm.dec[4] = static_cast<int>(t);
+                        sm.dec[5] = neq;
+                    }
                 }
-            }
-            // ---- 4. remaining digits on the candidates (or, after an overflow, on every key)
+                cluster.sync();                    // [barrier 5] threshold and offsets published
+                const int* d1 = remote(sm.dec, 0);
+                tau = static_cast<uint32_t>(d1[4]);
+                need_eq = d1[5];
+                const int* tb = remote(&sm.table[0][0], 0);
+                out_base = tb[2 * rank];
+                eq_base = tb[2 * rank + 1];
+                offsets_known = true;
+            } else {
+                // ---- 4'. candidate lists would not fit: remaining digits over every key
+                int hbuf = 1;
 #pragma unroll 1
-            for (int top = shift - 1; top >= 0;) {
-                width = min(11, top + 1);
-                shift = top - width + 1;
-                if (use_cands) {
-                    radix_digit<CS>(cluster, sm, hbuf, shift, width, prefix, mask, k_rem, [&](auto add) {
-                        for (int e = threadIdx.x; e < n_my; e += NT) add(cand_key[e]);
-                    });
-                } else {
+                for (int top = shift - 1; top >= 0;) {
+                    width = min(11, top + 1);
+                    shift = top - width + 1;
                     radix_digit<CS>(cluster, sm, hbuf, shift, width, prefix, mask, k_rem, [&](auto add) {
                         for_keys(sl, [&](int, uint32_t key, bool valid) { if (valid) add(key); });
                     });
+                    hbuf ^= 1;
+                    prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
+                    mask |= static_cast<uint32_t>((1 << width) - 1) << shift;
+                    k_rem -= sm.found_above;
+                    __syncthreads();
+                    top = shift - 1;
                 }
-                hbuf ^= 1;
-                prefix |= static_cast<uint32_t>(sm.found_bin) << shift;
-                mask |= static_cast<uint32_t>((1 << width) - 1) << shift;
-                k_rem -= sm.found_above;
-                __syncthreads();
-                top = shift - 1;
+                tau = prefix;
+                need_eq = k_rem;
             }
-            tau = prefix;
-            need_eq = k_rem;
         }
     }
 
-    // ---- 5. counts of this CTA, cluster-wide offsets, ordered write
-    int gt = 0, eq = 0;
-    if (!take_all && !take_none) {
-        if (use_cands) {
-            for (int e = threadIdx.x; e < n_my; e += NT) {
-                gt += cand_key[e] > tau;
-                eq += cand_key[e] == tau;
-            }
-        } else {
+    // ---- 5. (all-equal and fallback paths) this CTA's counts and cluster-wide offsets
+    if (!offsets_known) {
+        int gt = 0, eq = 0;
+        if (!take_all && !take_none)
             for_keys(sl, [&](int, uint32_t key, bool valid) {
                 gt += valid && key > tau;
                 eq += valid && key == tau;
             });
-        }
-    }
-    block_excl_scan(gt, sm);
-    const int t_gt = sm.total;
-    block_excl_scan(eq, sm);
-    const int t_eq = sm.total;
-    if (threadIdx.x == 0) { sm.counts[0] = t_gt; sm.counts[1] = t_eq; }
-    cluster.sync();                                // counts are written once: the final barrier
+        block_excl_scan(gt, sm);
+        const int t_gt = sm.total;
+        block_excl_scan(eq, sm);
+        const int t_eq = sm.total;
+        if (threadIdx.x == 0) { sm.counts[0] = t_gt; sm.counts[1] = t_eq; }
+        cluster.sync();                            // counts written once; the final barrier
                                                    // keeps them alive while they are read
-    int out_base = 0, eq_base = 0;                 // tokens written / equal keys before this CTA
-    for (int rr = 0; rr < rank; ++rr) {
-        const int* c = cluster.map_shared_rank(sm.counts, rr);
-        int keys_sel;
-        if (take_all) {
-            const int rb = min(rr * per, n_keys), re = min(rb + per, n_keys);
-            keys_sel = re - rb;
-        } else if (take_none) {
-            keys_sel = 0;
-        } else {
-            keys_sel = c[0] + max(0, min(c[1], need_eq - eq_base));
+        for (int rr = 0; rr < rank; ++rr) {
+            const int* c = cluster.map_shared_rank(sm.counts, rr);
+            int keys_sel;
+            if (take_all) {
+                const int rb = min(rr * per, n_keys), re = min(rb + per, n_keys);
+                keys_sel = re - rb;
+            } else if (take_none) {
+                keys_sel = 0;
+            } else {
+                keys_sel = c[0] + max(0, min(c[1], need_eq - eq_base));
+            }
+            // lower ranks own only whole blocks (a partial last block belongs to the CTA
+            // owning the row's last key, and never precedes another CTA's keys)
+            out_base += keys_sel * bs;
+            eq_base += c[1];
         }
-        // lower ranks own only whole blocks (a partial last block belongs to the CTA
-        // owning the row's last key, and never precedes another CTA's keys)
-        out_base += keys_sel * bs;
-        eq_base += c[1];
     }
 
-    written = out_base;
+    // ---- 6. ordered write of this CTA's selection
+    int written = out_base;
     if (!take_none) {
         if (use_cands) {
             written = ordered_write(
-                sm, sl, n_my, [&](int e) { return cand_pos[e]; }, [&](int e) { return cand_key[e]; }, tau, need_eq,
-                false, eq_base, written, out);
+                sm, sl, n_my, [&](int e) { return static_cast<int>(cand_pos[e]); },
+                [&](int e) { return cand_key[e]; }, tau, need_eq, false, eq_base, written, out);
         } else {
             written = ordered_write(
                 sm, sl, sl.end - sl.begin, [&](int e) { return sl.begin + e; },
