@@ -112,8 +112,9 @@ typedef struct {
 HS2_API size_t hs2_workspace_size(const hs2_attn_desc* desc, int32_t scores_in_workspace);
 
 /*
- * Clears the device status word at the start of `workspace` (enqueued on
- * `stream`).  Call once on a newly allocated workspace before its first use.
+ * Clears the status block at the start of `workspace` (the device status word and
+ * the merge counters, 4 KB; enqueued on `stream`).  Call once on a newly
+ * allocated workspace before its first use.
  */
 HS2_API hs2_status hs2_workspace_init(void* workspace, hs2_stream_t stream);
 

@@ -17,8 +17,13 @@
 namespace hs2 {
 
 // ---------------------------------------------------------------- status word
-// The first 256 bytes of every workspace hold the device status word.
-constexpr size_t kStatusBytes = 256;
+// The first 4 KB of every workspace are the status block: the device status word
+// at offset 0 and, from byte 256, the semaphore counters of split-K merges (zero
+// when idle: hs2_workspace_init clears the block, the last CTA of a merge resets
+// its counter).
+constexpr size_t kStatusBytes = 4096;
+constexpr int kCounterOffsetInts = 64;
+constexpr int kMaxCounters = static_cast<int>(kStatusBytes / 4) - kCounterOffsetInts;
 
 // Bound of every wait on an mbarrier: a phase that has not completed within
 // kWaitNs nanoseconds of global time (or kWaitPolls polls) is reported as a

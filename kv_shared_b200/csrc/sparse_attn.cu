@@ -70,10 +70,10 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* cvt = smem + 2 * L::STAGE;                    // e4m3 only: K bf16 then V bf16
-    int* sidx = reinterpret_cast<int*>(cvt + L::CVT);      // [2][SUB] row index per stage (-1 invalid)
-    float* sks = reinterpret_cast<float*>(sidx + 2 * SUB); // [2][SUB] k scales
-    float* svs = sks + 2 * SUB;                            // [2][SUB] v scales
-    float* red_o = svs + 2 * SUB;                          // [H][D]
+    float* red_o = reinterpret_cast<float*>(cvt + L::CVT); // [H][D]
+    int* sidx = reinterpret_cast<int*>(red_o + H * D);     // [chunk] cache row per entry (-1 invalid)
+    float* sks = reinterpret_cast<float*>(sidx + a.chunk); // [chunk] k scales (e4m3)
+    float* svs = sks + a.chunk;                            // [chunk] v scales (e4m3)
     __shared__ float wm[4][H], wl[4][H];
     __shared__ int s_last;
 
@@ -91,30 +91,29 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     const int32_t* irow = a.idx + static_cast<size_t>(row) * a.idx_stride;
     const size_t seq_base = static_cast<size_t>(b) * a.cap;
 
-    for (int i = tid; i < H * D; i += NT) red_o[i] = 0.f;
+    // every index (and scale) of this CTA's entries, loaded once up front
+    for (int e = tid; e < a.chunk; e += NT) {
+        int j = -1;
+        if (e_begin + e < e_end) {
+            j = irow[e_begin + e];
+            if (j < 0 || j >= a.cap) { set_status(a.status, HS2_ERR_INDEX); j = -1; }
+        }
+        sidx[e] = j;
+        if (KV8) {
+            sks[e] = j >= 0 ? a.k_scale[seq_base + j] : 0.f;
+            svs[e] = j >= 0 ? a.v_scale[seq_base + j] : 0.f;
+        }
+    }
+    __syncthreads();
 
     // gather sub-tile i into stage s (cp.async, zero-filled past the end)
     auto gather = [&](int i, int s) {
         uint8_t* st = smem + s * L::STAGE;
-        const int e0 = e_begin + i * SUB;
-        if (tid < SUB) {
-            const int e = e0 + tid;
-            int j = -1;
-            if (e < e_end) {
-                j = irow[e];
-                if (j < 0 || j >= a.cap) { set_status(a.status, HS2_ERR_INDEX); j = -1; }
-            }
-            sidx[s * SUB + tid] = j;
-            if (KV8) {
-                sks[s * SUB + tid] = j >= 0 ? a.k_scale[seq_base + j] : 0.f;
-                svs[s * SUB + tid] = j >= 0 ? a.v_scale[seq_base + j] : 0.f;
-            }
-        }
-        __syncthreads();
+        const int* si = sidx + i * SUB;
         constexpr int CH = L::ROWB / 16;                   // 16-byte chunks per row
         for (int it = tid; it < SUB * CH; it += NT) {
             const int r = it / CH, ch = it % CH;
-            const int j = sidx[s * SUB + r];
+            const int j = si[r];
             const size_t off = (seq_base + (j >= 0 ? j : 0)) * L::ROWB + ch * 16;
             uint32_t dk, dv;
             if (KV8) {
@@ -193,7 +192,7 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
                 mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
             }
         }
-        const int* si = sidx + s * SUB;
+        const int* si = sidx + i * SUB;
         float vf[2][2];
         float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
@@ -202,8 +201,8 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
             const bool ok0 = si[r0] >= 0, ok1 = si[r0 + 1] >= 0;
             float f0 = a.sc2, f1 = a.sc2;
             if (KV8) {
-                f0 *= sks[s * SUB + r0]; f1 *= sks[s * SUB + r0 + 1];
-                vf[nt][0] = svs[s * SUB + r0]; vf[nt][1] = svs[s * SUB + r0 + 1];
+                f0 *= sks[i * SUB + r0]; f1 *= sks[i * SUB + r0 + 1];
+                vf[nt][0] = svs[i * SUB + r0]; vf[nt][1] = svs[i * SUB + r0 + 1];
             } else {
                 vf[nt][0] = vf[nt][1] = 1.f;
             }
@@ -275,13 +274,23 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
         M[hh] = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
         f[hh] = (M[hh] == -INFINITY) ? 0.f : ex2(m2[hh] - M[hh]);
     }
+    // each warp's rescaled O goes to its own padded slab in the drained stage buffers,
+    // then the four slabs are summed (no shared atomics)
+    constexpr int RP = D + 4;                              // padded row (floats)
+    float* slab = reinterpret_cast<float*>(smem) + warp * H * RP;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
         const int d = 8 * n + 2 * t;
-        atomicAdd(&red_o[g * D + d], o[n][0] * f[0]);
-        atomicAdd(&red_o[g * D + d + 1], o[n][1] * f[0]);
-        atomicAdd(&red_o[(g + 8) * D + d], o[n][2] * f[1]);
-        atomicAdd(&red_o[(g + 8) * D + d + 1], o[n][3] * f[1]);
+        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(o[n][0] * f[0], o[n][1] * f[0]);
+        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(o[n][2] * f[1], o[n][3] * f[1]);
+    }
+    __syncthreads();
+    {
+        const float* sb = reinterpret_cast<const float*>(smem);
+        for (int i = tid; i < H * D; i += NT) {
+            const int h = i / D, d = i % D;
+            red_o[i] = sb[h * RP + d] + sb[H * RP + h * RP + d] + sb[2 * H * RP + h * RP + d] + sb[3 * H * RP + h * RP + d];
+        }
     }
     __syncthreads();
     // per-head CTA (max, sum); threads 0..15 own head tid
@@ -368,9 +377,9 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <bool KV8>
-size_t smem_bytes() {
+size_t smem_bytes(int chunk) {
     using L = Layout<KV8>;
-    return 1024 + 2 * L::STAGE + L::CVT + 2 * SUB * 4 * 3 + H * D * 4;
+    return 1024 + 2 * L::STAGE + L::CVT + H * D * 4 + static_cast<size_t>(chunk) * 4 * (KV8 ? 3 : 1);
 }
 
 template <bool KV8>
@@ -390,17 +399,14 @@ cudaError_t launch_impl(const SparseArgs& sa, cudaStream_t st) {
     ws += align256(sizeof(float2) * sa.rows * pl.splits * H);
     a.part_o = reinterpret_cast<float*>(ws);
     ws += align256(sizeof(float) * static_cast<size_t>(sa.rows) * pl.splits * H * D);
-    a.counter = reinterpret_cast<int*>(ws);
+    // semaphore counters live in the status block (zeroed by hs2_workspace_init; the
+    // last CTA of a row resets its counter)
+    a.counter = reinterpret_cast<int*>(sa.status) + kCounterOffsetInts;
     a.o = static_cast<__nv_bfloat16*>(sa.o);
     a.lse = sa.lse;
     a.status = sa.status;
-    const size_t sm = smem_bytes<KV8>();
+    const size_t sm = smem_bytes<KV8>(pl.chunk);
     cudaError_t e;
-    if (pl.splits > 1) {
-        // the semaphore counters must start at zero; the last CTA of a row resets its own
-        e = cudaMemsetAsync(a.counter, 0, sizeof(int) * sa.rows, st);
-        if (e != cudaSuccess) return e;
-    }
     e = cudaFuncSetAttribute(sparse_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
     if (e != cudaSuccess) return e;
     sparse_kernel<KV8><<<dim3(pl.splits, sa.rows), NT, sm, st>>>(a);
@@ -413,6 +419,7 @@ SparsePlan plan_sparse(int rows, int idx_stride) {
     SparsePlan pl;
     // enough CTAs to cover the SMs twice; one CTA per row when rows alone do
     int splits = (2 * num_sms() + rows - 1) / (rows > 0 ? rows : 1);
+    if (rows > kMaxCounters) splits = 1;           // semaphore counters exist for kMaxCounters rows
     int max_splits = (idx_stride + SUB - 1) / SUB;
     if (max_splits > kMaxSplits) max_splits = kMaxSplits;
     if (splits > max_splits) splits = max_splits;
@@ -465,6 +472,10 @@ cudaError_t scratch_address(void** out) {
     if (!g_scratch_addr[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_sparse_scratch);
+        if (e != cudaSuccess) return e;
+        // status word and semaphore counters start at zero (the counters return to
+        // zero at the end of every call)
+        e = cudaMemset(p, 0, kStatusBytes);
         if (e != cudaSuccess) return e;
         g_scratch_addr[dev] = p;
     }
