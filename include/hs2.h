@@ -2,11 +2,11 @@
  * hs2.h -- C ABI of the B200 (sm_100a) HySparse2 hybrid-block attention library.
  *
  * The hybrid block described by the pages: one causal full-attention layer over
- * a single shared MQA K/V cache, which on completion selects important positions
- * per query (token level, the 1,024 best earlier positions plus a forced window
- * of the 128 most recent), followed by sparse-attention layers that reuse that
- * cache and those indices; the cross-decoder caches are built by projecting
- * self-decoder hidden states (KV Bridging).
+ * a single shared MQA K/V cache that, having run, decides per query which
+ * positions the next layers see (individual tokens: 1,024 chosen earlier
+ * positions plus a compulsory window of the latest 128), then sparse-attention
+ * layers that read that same cache at those same positions; the cross-decoder
+ * caches come from a projection of self-decoder activations (KV Bridging).
  *
  * Sources, cited by page title and section:
  *   [NF] "Xiaomi's MiMo-V3 Architecture Reduces Prefill Compute by 80%" (news flash)
@@ -121,9 +121,9 @@ HS2_API hs2_status hs2_workspace_init(void* workspace, hs2_stream_t stream);
 /*
  * Full-attention layer of a hybrid block plus its token-level selection.
  *
- * [LB] "Two-Level KV Sharing" (KV Reuse): the full-attention layer selects
- * important positions upon completion; [NF]: these layers select the 1,024 most
- * relevant tokens and later layers always keep the most recent 128.
+ * [LB] "Two-Level KV Sharing" (KV Reuse): the full layer, having run, chooses
+ * the positions for the layers after it; [NF]: a budget of 1,024 chosen tokens,
+ * and the latest 128 are kept by the later layers no matter what.
  * The pages give no scoring rule ([AX] "What is not documented"); this library
  * scores key j for query row i as sum over heads h of the softmax probability
  * P_h[i][j] = exp(scale * q_h.k_j - LSE_h[i]) computed in fp32, and breaks ties
@@ -150,8 +150,8 @@ HS2_API hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q
  * Selection alone, from a caller-given importance array.
  *
  * block_size 1: token level as above ([LB] "Token-Level Sparse Selection").
- * block_size > 1: the first-generation rule ([NF]: tokens grouped in sets of 64,
- * a group is kept whole if any of its tokens is important): blocks of block_size
+ * block_size > 1: the first-generation rule ([NF]: importance decided per group
+ * of 64 tokens, a group with one important member kept in full): blocks of block_size
  * positions tile [0, p - W] from position 0, a block scores the max of its
  * tokens, the floor(K_sel / block_size) best blocks (ties to the lower block) are
  * kept, plus the window.  idx_stride must then be >= W + K_sel.
@@ -163,10 +163,10 @@ HS2_API hs2_status hs2_topk_select(const hs2_attn_desc* desc, const float* score
                            hs2_stream_t stream);
 
 /*
- * One sparse-attention layer with KV Reuse ([AX] section 2: sparse layers reuse
- * the preceding full-attention layer's KV cache and selection indices; [AX]
- * section 3: local and global tokens share one cache, so one softmax runs over
- * the whole selected set).  q is this layer's own query; idx/cnt as produced by
+ * One sparse-attention layer with KV Reuse ([AX] section 2: a sparse layer keeps
+ * no cache and no selector of its own, it reads the full layer's cache at the
+ * full layer's chosen positions; [AX] section 3: window and global positions sit
+ * in one cache, so a single softmax covers the whole chosen set).  q is this layer's own query; idx/cnt as produced by
  * hs2_full_attn_select (positions must lie in [0, kv_capacity)).
  * o: [batch][n_q][heads][head_dim] in q_dtype; lse optional.
  */
@@ -206,10 +206,10 @@ HS2_API hs2_status hs2_sparse_attn_noalloc(const hs2_attn_desc* desc, const void
                                            hs2_stream_t stream);
 
 /*
- * KV Bridging projection ([LB] "Two-Level KV Sharing": the cross-decoder's
- * full-attention caches are generated from the hidden states of the
- * self-decoder, each target layer with its own K/V projection; [AN]: the latter
- * half projects its key-value caches from the first half's hidden states).
+ * KV Bridging projection ([LB] "Two-Level KV Sharing": the caches of the
+ * cross-decoder's full layers are projections of self-decoder activations, a
+ * separate K/V weight per target layer; [AN]: the second half of the model
+ * obtains its caches this way from the first half).
  *
  * hidden [batch][n][d_model] bf16, w_kv [d_model][2*head_dim] bf16 (columns
  * 0..D-1 give K, D..2D-1 give V; no bias).  Rows t = 0..n-1 of sequence b are

@@ -1,9 +1,9 @@
 // sparse_attn.cu -- sparse-attention layer of a hybrid block (KV Reuse).
 //
-// "What HySparse2 is actually optimizing", section 2: sparse layers reuse the
-// preceding full-attention layer's KV cache and selection indices; section 3:
-// local and global tokens share one cache, so one softmax runs over the whole
-// selected set (window plus global picks).
+// "What HySparse2 is actually optimizing", section 2: a sparse layer keeps no
+// cache or selector of its own and reads the full layer's cache at the full
+// layer's chosen positions; section 3: window and global positions sit in one
+// cache, so a single softmax covers the whole chosen set.
 //
 // For each query row (16 heads) the selected cache rows are gathered by index
 // with 16-byte cp.async copies into shared memory (swizzled so ldmatrix reads

@@ -2,7 +2,7 @@
 //
 // Per query row at position p ("Xiaomi Unveils HySparse2 Architecture for
 // MiMo-V3", section "Token-Level Sparse Selection: Precision and Efficiency
-// Balance": the most recent 128 tokens are forced, plus 1,024 global tokens):
+// Balance": a compulsory window of the latest 128 tokens and 1,024 global picks):
 //   window = [max(0, p-W+1), p], candidates = [0, p-W],
 //   global = the K best candidates by (importance desc, position asc),
 //   idx    = ascending union, -1 padded; cnt = |idx|.

@@ -46,9 +46,9 @@
 /* ------------------------------------------------------------------------- */
 /* Full causal MQA attention with per-key importance.                         */
 /*                                                                           */
-/* [LB] "Two-Level KV Sharing" (KV Reuse paragraph): the full-attention layer */
-/* selects important positions upon completion.  [AN]: the configuration     */
-/* switches from GQA to MQA, so all query heads share one K/V head.          */
+/* [LB] "Two-Level KV Sharing" (KV Reuse paragraph): once the full layer has */
+/* run, it picks the positions that matter for the later layers.  [AN]: the  */
+/* compared configuration uses MQA: every query head reads one K/V head.     */
 /*                                                                           */
 /* q     [n_rows][H][D]   query rows of one sequence                          */
 /* k, v  [n_keys][D]      the sequence's shared cache                         */
@@ -105,11 +105,11 @@ EXPORT void oracle_full_attn(int n_rows, int H, int D, int64_t n_keys,
 /* ------------------------------------------------------------------------- */
 /* Selection.                                                                 */
 /*                                                                           */
-/* [NF]: the full layers first pick the 1,024 most relevant tokens; later     */
-/* layers reuse that pick and always keep the 128 most recent tokens.        */
-/* [LB] "Token-Level Sparse Selection": a local window forcing the most       */
-/* recent 128 tokens plus an additional 1,024 global tokens; selection is     */
-/* per token ([AX] section 3).  Output: ascending positions, count returned. */
+/* [NF]: a budget of 1,024 picked tokens, and the latest 128 tokens are kept */
+/* unconditionally by the layers that reuse the pick.  [LB] "Token-Level     */
+/* Sparse Selection": a 128-token local window on top of 1,024 global picks; */
+/* picks are individual tokens ([AX] section 3).  Output: ascending          */
+/* positions, count returned.                                                */
 /* ------------------------------------------------------------------------- */
 typedef struct { double key; int64_t id; } ranked_t;
 
@@ -149,8 +149,8 @@ EXPORT int oracle_select_tokens(int64_t p, int W, int K_sel, const double* score
     return c;
 }
 
-/* Block level (the first-generation rule, [NF]: tokens grouped in sets of 64; if
- * any token in a group is important the whole group is kept): blocks of size bs
+/* Block level (the first-generation rule, [NF]: importance was decided per group
+ * of 64 tokens, and a group with one important member was kept in full): blocks of size bs
  * tile Cand from position 0, a block's score is the max of its tokens' scores,
  * the floor(K_sel/bs) best blocks by (block score desc, block asc) are kept
  * (only their positions inside Cand), plus the window.  Returns the count. */
@@ -181,9 +181,9 @@ EXPORT int oracle_select_blocks(int64_t p, int W, int K_sel, int bs, const doubl
 /* ------------------------------------------------------------------------- */
 /* Sparse attention with KV Reuse.                                            */
 /*                                                                           */
-/* [AX] section 2: sparse layers reuse the preceding full-attention layer's   */
-/* KV cache and selection indices; [AX] section 3: local and global tokens    */
-/* share one KV cache -> one softmax over the selected set.                   */
+/* [AX] section 2: a sparse layer has no cache or selector of its own; it    */
+/* reads the full layer's cache at the full layer's picks.  [AX] section 3:  */
+/* window and global picks live in the same cache -> one softmax over both.  */
 /* q [n_rows][H][D]; k, v [n_keys][D]; idx [n_rows][idx_stride]; cnt [n_rows] */
 /* ------------------------------------------------------------------------- */
 EXPORT void oracle_sparse_attn(int n_rows, int H, int D, const double* q, const double* k,
@@ -222,9 +222,9 @@ EXPORT void oracle_sparse_attn(int n_rows, int H, int D, const double* q, const 
 /* ------------------------------------------------------------------------- */
 /* KV Bridging projection.                                                    */
 /*                                                                           */
-/* [LB] "Two-Level KV Sharing": the second half's full-attention KV cache is  */
-/* generated directly from the hidden states of the first half, each target   */
-/* layer with its own K/V projection.  Reading: one matrix W [dm][2D], K from */
+/* [LB] "Two-Level KV Sharing": the caches of the cross-decoder's full layers */
+/* are projections of self-decoder activations, with a separate K/V weight    */
+/* per target layer.  Reading: one matrix W [dm][2D], K from                  */
 /* columns 0..D-1 and V from columns D..2D-1, no bias, no norm.               */
 /* x [n][dm]; w [dm][2D]; kout, vout [n][D] (exact fp64 products)             */
 /* ------------------------------------------------------------------------- */
