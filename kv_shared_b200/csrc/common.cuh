@@ -101,6 +101,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
     return false;
 }
 
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// As mbar_wait, but polling with the non-blocking test_wait, so that the thread
+// never sleeps and reacts to the phase change at once.  For a single thread whose
+// reaction time is on the critical path (the MMA issuer).
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, uint32_t* status,
+                                               uint64_t limit_ns = kWaitNs) {
+    const uint64_t t0 = global_ns();
+#pragma unroll 1
+    for (uint64_t i = 0; i < static_cast<uint64_t>(kWaitPolls) * 64u; ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 255) == 255 && global_ns() - t0 > limit_ns) break;
+    }
+    set_status(status, HS2_ERR_TIMEOUT);
+    return false;
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar,
                                             int32_t x, int32_t y) {

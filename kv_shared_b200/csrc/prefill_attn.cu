@@ -5,22 +5,28 @@
 // P_h[i][j] = exp(s_h[i][j] - LSE_h[i]) (the pages leave the rule open: "What
 // HySparse2 is actually optimizing", "What is not documented").  The final
 // log-sum-exp is needed before any probability is formed, hence two passes
-// over the causal key range of each block of 8 query rows:
+// over the causal key range of each block of 16 query rows.
 //
-//   pass 1  S = Q K^T with M = 8 rows x 16 heads = 128 (all query heads share the
-//           one K/V head, so stacking them in M reuses every K tile 128 times);
-//           one thread per (row, head) keeps a running max and sum -> LSE.
-//   pass 2  S' = K Q^T (M = 128 keys, N = 128 (row, head)): one thread per key
-//           owns all 128 probabilities of its key, so the 16-head sum of the
-//           importance is plain register adds.  P goes to shared memory as the
-//           MN-major A operand of O += P V (V is MN-major straight from the
-//           cache); O stays in tensor memory for the whole key loop.
+// All 16 query heads share the one K/V head, so a CTA stacks (row, head) pairs
+// in the MMA's M dimension: 16 rows x 16 heads = 256 pairs, as two 128-lane
+// halves that both consume every K (and V) tile the CTA loads.  Each tile is
+// fetched from L2 once per 256 pairs; with fewer pairs per tile the kernels are
+// bound by the L2-to-SM traffic rather than by the tensor or exponential units.
 //
-// Roles (320 threads): warp 0 issues TMA loads, one thread of warp 1 issues the
-// MMAs (and warp 1 owns the tensor memory), warps 2..9 do the softmax work: two
-// warps per tensor-memory lane quarter, each owning 64 of the 128 columns.
-// Every wait is bounded; a wait that gives up flags the status word and makes
-// all roles leave their loops.
+//   pass 1  S_h = Q_h K^T per half h; one thread per (row, head) keeps a
+//           running max and sum -> LSE.
+//   pass 2  S_h = Q_h K^T; P_h = exp2(S_h sc2 - LSE2) is written back into the
+//           same tensor-memory columns as packed bf16 and used from there as
+//           the A operand of O_h += P_h V, so P never touches shared memory.
+//           The importance sums P over the 16 lanes (heads) of each row with a
+//           warp-shuffle transpose-reduction.
+//
+// Roles (576 threads): warp 0 issues TMA loads, one thread of warp 1 issues the
+// MMAs (warp 1 owns the tensor memory), warps 2..9 work on half 0 and warps
+// 10..17 on half 1, two warps per tensor-memory lane quarter (a warp may only
+// touch its quarter, warp % 4), so that four softmax warps per SM sub-partition
+// hide the tensor-memory and exponential latencies.  Every wait is bounded; a
+// wait that gives up flags the status word and makes all roles leave their loops.
 #include "common.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -30,11 +36,11 @@ namespace {
 
 constexpr int H = 16;
 constexpr int D = 128;
-constexpr int ROWS = 8;                         // query rows per CTA
-constexpr int MT = ROWS * H;                    // 128 (row, head) pairs
+constexpr int ROWS = 16;                        // query rows per CTA
+constexpr int HALF_ROWS = ROWS / 2;             // rows per 128-lane half
 constexpr int KT = 128;                         // keys per tile
-constexpr int NT = 320;
-constexpr int NSOFT = 256;                      // softmax threads (warps 2..9)
+constexpr int NT = 576;
+constexpr int NSOFT = 512;                      // softmax threads (warps 2..17)
 constexpr int TILE_BYTES = KT * D * 2;          // 32 KB: two 128-row x 64-col swizzled boxes
 constexpr int BOX_BYTES = TILE_BYTES / 2;
 
@@ -42,7 +48,7 @@ struct Params {
     int B, n_q;
     int64_t cap, max_ctx;
     const int32_t* q_pos0;
-    float sc2;                                  // scale * log2(e)
+    float sc2;                                  // scale * log2(e), > 0
     float* lse2;                                // [B][n_q][H] log2 units (pass 1 out, pass 2 in)
     float* lse_user;                            // [B][n_q][H] natural log or null
     float* scores;                              // [B][n_q][score_ld]
@@ -67,6 +73,10 @@ __device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int kk) {
     return umma::sdesc_sw128(base + kk * 2048, BOX_BYTES, 1024);
 }
 
+__device__ __forceinline__ void named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               uint32_t* status) {
     if (*abort_flag) return false;
@@ -74,13 +84,48 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return true;
 }
 
-__device__ __forceinline__ void named_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+// the MMA issuer's waits: it sits on the critical path of every handoff, so it polls
+// without ever being suspended
+__device__ __forceinline__ bool spin_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              uint32_t* status) {
+    if (*abort_flag) return false;
+    if (!mbar_wait_spin(bar, parity, status)) { *abort_flag = 1; return false; }
+    return true;
 }
 
-// Tensor-memory S buffers: three 128-column tiles in flight, so that the MMA can
-// run ahead while the two softmax warpgroups each work on their own key tile.
-constexpr int NSB = 3;
+// one arrival per warp, after every lane's tensor-memory accesses are ordered before it
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+    umma::fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+}
+
+// ---- packed fp32 pairs (one instruction for two lanes of arithmetic on sm_100)
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("{\n\t.reg .b64 ra, rb, rc;\n\t"
+        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\tmov.b64 rc, {%5, %6};\n\t"
+        "fma.rn.f32x2 %0, ra, rb, rc;\n\t}"
+        : "=l"(d) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+    uint64_t d;
+    asm("{\n\t.reg .b64 ra, rb;\n\t"
+        "mov.b64 ra, {%1, %2};\n\tmov.b64 rb, {%3, %4};\n\t"
+        "add.rn.f32x2 %0, ra, rb;\n\t}"
+        : "=l"(d) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
 
 // ------------------------------------------------------------------ pass 1: LSE
 constexpr int P1_STAGES = 4;
@@ -89,12 +134,12 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
                                                            const __grid_constant__ CUtensorMap kmap, Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* qs = smem;
-    uint8_t* ks = smem + TILE_BYTES;
-    __shared__ uint64_t q_full, k_full[P1_STAGES], k_empty[P1_STAGES], s_full[NSB], s_empty[NSB];
+    uint8_t* qs = smem;                                       // Q halves 0, 1
+    uint8_t* ks = smem + 2 * TILE_BYTES;
+    __shared__ uint64_t q_full, k_full[P1_STAGES], k_empty[P1_STAGES], s_full[2][2], s_empty[2][2];
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
-    __shared__ float2 part[2][MT];
+    __shared__ float2 part[NSOFT];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int blocks_per_seq = (a.n_q + ROWS - 1) / ROWS;
@@ -110,7 +155,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         prefetch_tmap(&kmap);
         mbar_init(&q_full, 1);
         for (int s = 0; s < P1_STAGES; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
-        for (int s = 0; s < NSB; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 128); }
+        for (int s = 0; s < 2; ++s)
+            for (int h = 0; h < 2; ++h) { mbar_init(&s_full[s][h], 1); mbar_init(&s_empty[s][h], 8); }
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -118,14 +164,16 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
     umma::fence_before();
     __syncthreads();
     umma::fence_after();
-    const uint32_t tmem = tmem_base;
+    const uint32_t tmem = tmem_base;            // S of (buffer u, half h) at column (2u + h) * 128
 
     if (warp == 0) {
         if (lane == 0) {
             const int qrow = (b * a.n_q + r0) * H;
-            mbar_arrive_expect_tx(&q_full, TILE_BYTES);
-            tma_load_2d(qs, &qmap, &q_full, 0, qrow);
-            tma_load_2d(qs + BOX_BYTES, &qmap, &q_full, 64, qrow);
+            mbar_arrive_expect_tx(&q_full, 2 * TILE_BYTES);
+            for (int h = 0; h < 2; ++h) {
+                tma_load_2d(qs + h * TILE_BYTES, &qmap, &q_full, 0, qrow + h * 128);
+                tma_load_2d(qs + h * TILE_BYTES + BOX_BYTES, &qmap, &q_full, 64, qrow + h * 128);
+            }
             for (int i = 0; i < n_kt; ++i) {
                 const int s = i % P1_STAGES;
                 if (i >= P1_STAGES && !wait_or_abort(&k_empty[s], ((i / P1_STAGES) - 1) & 1, &abort_flag, a.status)) break;
@@ -140,83 +188,89 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         if (lane == 0) {
             constexpr uint32_t idesc = umma::idesc_bf16(128, 128, false, false);
             const uint32_t qb = smem_u32(qs);
-            if (wait_or_abort(&q_full, 0, &abort_flag, a.status)) {
-                for (int i = 0; i < n_kt; ++i) {
-                    const int s = i % P1_STAGES, sb = i % NSB;
-                    if (!wait_or_abort(&k_full[s], (i / P1_STAGES) & 1, &abort_flag, a.status)) break;
-                    if (i >= NSB && !wait_or_abort(&s_empty[sb], ((i / NSB) - 1) & 1, &abort_flag, a.status)) break;
+            bool ok = spin_or_abort(&q_full, 0, &abort_flag, a.status);
+            for (int i = 0; ok && i < n_kt; ++i) {
+                const int s = i % P1_STAGES, u = i & 1;
+                if (!(ok = spin_or_abort(&k_full[s], (i / P1_STAGES) & 1, &abort_flag, a.status))) break;
+                const uint32_t kb = smem_u32(ks + s * TILE_BYTES);
+                for (int h = 0; h < 2; ++h) {
+                    if (i >= 2 && !(ok = spin_or_abort(&s_empty[u][h], ((i >> 1) - 1) & 1, &abort_flag, a.status))) break;
                     umma::fence_after();
-                    const uint32_t kb = smem_u32(ks + s * TILE_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk)
-                        umma::mma_bf16_ss(tmem + sb * 128, kmajor_desc(qb, kk), kmajor_desc(kb, kk), idesc, kk > 0);
-                    umma::commit(&k_empty[s]);
-                    umma::commit(&s_full[sb]);
+                        umma::mma_bf16_ss(tmem + (2 * u + h) * 128, kmajor_desc(qb + h * TILE_BYTES, kk),
+                                          kmajor_desc(kb, kk), idesc, kk > 0);
+                    umma::commit(&s_full[u][h]);
                 }
+                umma::commit(&k_empty[s]);
             }
         }
     } else {
-        // softmax warpgroup g takes key tiles i = g, g+2, ...; each thread owns TMEM lane
-        // m = (row, head) and all 128 columns of a tile, read in 32-column chunks with the
-        // next chunk's load in flight while the current one is reduced
-        const int quarter = warp & 3, g = (warp - 2) >> 2;
+        // half h, key-column half c of every tile: each thread owns TMEM lane m =
+        // (row, head) of its half and columns 64 c .. 64 c + 63 of each tile, read in two
+        // 32-column chunks (the second in flight while the first is reduced); the two
+        // column halves' running (max, sum) are merged at the end
+        const int sw = warp - 2, quarter = warp & 3;
+        const int h = sw >> 3, c = (sw >> 2) & 1;
         const int m = quarter * 32 + lane;
-        const int row = r0 + (m >> 4);
-        const int p = pos_base + (m >> 4);
+        const int lrow = h * HALF_ROWS + (m >> 4);
+        const int row = r0 + lrow;
+        const int p = pos_base + lrow;
+        const float sc2 = a.sc2;
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         float run_m = -INFINITY, run_l = 0.f;
+        // scale > 0, so the row maximum of S sc2 is sc2 times the maximum of S
         auto reduce_chunk = [&](const uint32_t (&r)[32], int key0) {
             float v[32];
-            float mx = -INFINITY;
-            const bool need_mask = key0 + 31 > p;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                float x = __uint_as_float(r[c]) * a.sc2;
-                if (need_mask && key0 + c > p) x = -INFINITY;
-                v[c] = x;
-                mx = fmaxf(mx, x);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (key0 + 31 > p) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    if (key0 + j > p) v[j] = -INFINITY;
             }
-            const float mn = fmaxf(run_m, mx);
-            if (mn != -INFINITY) {
-                float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+            float m0 = max3(v[0], v[1], v[2]), m1 = max3(v[3], v[4], v[5]);
 #pragma unroll
-                for (int c = 0; c < 32; c += 4) {
-                    s0 += ex2(v[c] - mn);
-                    s1 += ex2(v[c + 1] - mn);
-                    s2 += ex2(v[c + 2] - mn);
-                    s3 += ex2(v[c + 3] - mn);
+            for (int j = 6; j < 30; j += 4) {
+                m0 = max3(m0, v[j], v[j + 1]);
+                m1 = max3(m1, v[j + 2], v[j + 3]);
+            }
+            const float mx = max3(m0, m1, fmaxf(v[30], v[31]));
+            const float mn = fmaxf(run_m, mx * sc2);
+            if (mn != -INFINITY) {
+                const float2 s2 = make_float2(sc2, sc2), nm = make_float2(-mn, -mn);
+                float2 acc0 = make_float2(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float2 x0 = fma2(make_float2(v[j], v[j + 1]), s2, nm);
+                    const float2 x1 = fma2(make_float2(v[j + 2], v[j + 3]), s2, nm);
+                    acc0 = add2(acc0, make_float2(ex2(x0.x), ex2(x0.y)));
+                    acc1 = add2(acc1, make_float2(ex2(x1.x), ex2(x1.y)));
                 }
-                run_l = run_l * ex2(run_m - mn) + ((s0 + s1) + (s2 + s3));
+                const float2 acc = add2(acc0, acc1);
+                run_l = run_l * ex2(run_m - mn) + (acc.x + acc.y);
                 run_m = mn;
             }
         };
-        for (int i = g; i < n_kt; i += 2) {
-            const int sb = i % NSB;
-            if (!wait_or_abort(&s_full[sb], (i / NSB) & 1, &abort_flag, a.status)) break;
+        for (int i = 0; i < n_kt; ++i) {
+            const int u = i & 1;
+            if (!wait_or_abort(&s_full[u][h], (i >> 1) & 1, &abort_flag, a.status)) break;
             umma::fence_after();
-            const uint32_t ta = tmem + lane_base + sb * 128;
-            const int key0 = i * KT;
+            const uint32_t ta = tmem + lane_base + (2 * u + h) * 128 + 64 * c;
+            const int key0 = i * KT + 64 * c;
             uint32_t ra[32], rb[32];
             umma::tmem_ld32(ta, ra);
             umma::tmem_ld_wait();
             umma::tmem_ld32(ta + 32, rb);
             reduce_chunk(ra, key0);
             umma::tmem_ld_wait();
-            umma::tmem_ld32(ta + 64, ra);
+            warp_arrive(&s_empty[u][h]);
             reduce_chunk(rb, key0 + 32);
-            umma::tmem_ld_wait();
-            umma::tmem_ld32(ta + 96, rb);
-            reduce_chunk(ra, key0 + 64);
-            umma::tmem_ld_wait();
-            umma::fence_before();
-            mbar_arrive(&s_empty[sb]);
-            reduce_chunk(rb, key0 + 96);
         }
-        // combine the two warpgroups' key tiles
-        part[g][m] = make_float2(run_m, run_l);
+        part[sw * 32 + lane] = make_float2(run_m, run_l);
         named_sync(1, NSOFT);
-        if (g == 0 && row < a.n_q && !abort_flag) {
-            const float2 o = part[1][m];
+        if (c == 0 && row < a.n_q && !abort_flag) {
+            const float2 o = part[(sw + 4) * 32 + lane];          // the other column half, same lane
             const float mn = fmaxf(run_m, o.x);
             const float l = (run_m == -INFINITY ? 0.f : run_l * ex2(run_m - mn)) +
                             (o.x == -INFINITY ? 0.f : o.y * ex2(o.x - mn));
@@ -234,50 +288,84 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
     }
 }
 
-// One 32-column chunk of an S' row (pass 2): columns = rows 2C, 2C+1 x 16 heads.
-// Probabilities P = 2^(S' sc2 - LSE2), the two rows' importance (written to the score
-// rows), and bf16 pairs of P into pk[16 C .. 16 C + 15].
-template <int C>
-__device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], int key, int pos_base, int r0, int n_q,
-                                         float sc2, const float* lse_s, float* srow0, int64_t score_ld,
-                                         uint32_t (&pk)[64]) {
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        const int row = 2 * C + rr;
-        const bool valid = key <= pos_base + row;
-        float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-        for (int h = 0; h < H; h += 2) {
-            const int col = rr * H + h;
-            const float2 l2 = *reinterpret_cast<const float2*>(&lse_s[C * 32 + col]);
-            float p0 = ex2(__uint_as_float(r[col]) * sc2 - l2.x);
-            float p1 = ex2(__uint_as_float(r[col + 1]) * sc2 - l2.y);
-            if (!valid) { p0 = 0.f; p1 = 0.f; }
-            acc0 += p0;
-            acc1 += p1;
-            pk[C * 16 + (col >> 1)] = pack_bf16(p0, p1);
-        }
-        if (valid && r0 + row < n_q) srow0[row * score_ld + key] = acc0 + acc1;
-    }
-}
-
 // ------------------------------------------------------------------ pass 2: P, importance, O
 constexpr int P2_STAGES = 2;                    // K and V tiles each double-buffered
+
+// Sum over the 8 lanes that share t % 4 (lane bits 2..4) of eight float2 values, one
+// per 16x256b repetition j; afterwards lane t holds in v[0] the sum for repetition t / 4.
+__device__ __forceinline__ float2 transpose_reduce8(float2 (&v)[8], int t) {
+    const bool b4 = t & 16, b3 = t & 8, b2 = t & 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 lo = v[j], hi = v[j + 4];
+        const float2 send = b4 ? lo : hi, keep = b4 ? hi : lo;
+        v[j] = add2(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 16),
+                                      __shfl_xor_sync(0xffffffffu, send.y, 16)));
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float2 lo = v[j], hi = v[j + 2];
+        const float2 send = b3 ? lo : hi, keep = b3 ? hi : lo;
+        v[j] = add2(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 8),
+                                      __shfl_xor_sync(0xffffffffu, send.y, 8)));
+    }
+    const float2 lo = v[0], hi = v[1];
+    const float2 send = b2 ? lo : hi, keep = b2 ? hi : lo;
+    return add2(keep, make_float2(__shfl_xor_sync(0xffffffffu, send.x, 4),
+                                  __shfl_xor_sync(0xffffffffu, send.y, 4)));
+}
+
+// One 64-key chunk of one row (16 lanes = the row's 16 heads) of S_h, read with the
+// 16x256b shape: thread t holds heads t/4 (A) and t/4 + 8 (B) at keys
+// key_base + 8j + 2(t%4) + {0, 1}.  Forms P, writes it back as packed bf16 (16x128b
+// shape, key pair -> one column) and stores the row's importance for its keys
+// key_base + 2t, key_base + 2t + 1.
+__device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_taddr, int key_base, int p, float sc2,
+                                         float lse_a, float lse_b, float* srow, bool vec2, int t) {
+    const float2 s2 = make_float2(sc2, sc2);
+    const float2 na = make_float2(-lse_a, -lse_a), nb = make_float2(-lse_b, -lse_b);
+    const bool need_mask = key_base + 63 > p;
+    uint32_t pk[16];
+    float2 imp[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const float2 xa = fma2(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s2, na);
+        const float2 xb = fma2(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s2, nb);
+        float2 pa = make_float2(ex2(xa.x), ex2(xa.y)), pb = make_float2(ex2(xb.x), ex2(xb.y));
+        if (need_mask) {
+            const int k0 = key_base + 8 * j + 2 * (t & 3);
+            if (k0 > p) { pa.x = 0.f; pb.x = 0.f; }
+            if (k0 + 1 > p) { pa.y = 0.f; pb.y = 0.f; }
+        }
+        pk[2 * j] = pack_bf16(pa.x, pa.y);
+        pk[2 * j + 1] = pack_bf16(pb.x, pb.y);
+        imp[j] = add2(pa, pb);
+    }
+    umma::tmem_st16x128_x8(p_taddr, pk);
+    const float2 s = transpose_reduce8(imp, t);
+    if (srow) {
+        const int k = key_base + 2 * t;
+        if (vec2 && k + 1 <= p) {
+            *reinterpret_cast<float2*>(srow + k) = s;
+        } else {
+            if (k <= p) srow[k] = s.x;
+            if (k + 1 <= p) srow[k + 1] = s.y;
+        }
+    }
+}
 
 __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constant__ CUtensorMap qmap,
                                                            const __grid_constant__ CUtensorMap kmap,
                                                            const __grid_constant__ CUtensorMap vmap, Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* qs = smem;
-    uint8_t* kst = smem + TILE_BYTES;                         // K stages
+    uint8_t* qs = smem;                                       // Q halves 0, 1
+    uint8_t* kst = smem + 2 * TILE_BYTES;                     // K stages
     uint8_t* vst = kst + P2_STAGES * TILE_BYTES;              // V stages
-    uint8_t* ps = vst + P2_STAGES * TILE_BYTES;               // P tiles (one per warpgroup)
     __shared__ uint64_t q_full, k_full[P2_STAGES], k_empty[P2_STAGES], v_full[P2_STAGES], v_empty[P2_STAGES];
-    __shared__ uint64_t s_full[NSB], s_empty[NSB], p_full[2], p_empty[2], o_full;
+    __shared__ uint64_t s_full[2], p_full[2], o_full;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
-    __shared__ __align__(16) float lse_s[MT];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int blocks_per_seq = (a.n_q + ROWS - 1) / ROWS;
@@ -297,8 +385,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
         }
-        for (int s = 0; s < NSB; ++s) { mbar_init(&s_full[s], 1); mbar_init(&s_empty[s], 128); }
-        for (int s = 0; s < 2; ++s) { mbar_init(&p_full[s], 128); mbar_init(&p_empty[s], 1); }
+        for (int h = 0; h < 2; ++h) { mbar_init(&s_full[h], 1); mbar_init(&p_full[h], 8); }
         mbar_init(&o_full, 1);
         fence_mbar_init();
         abort_flag = 0;
@@ -307,16 +394,18 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     umma::fence_before();
     __syncthreads();
     umma::fence_after();
-    const uint32_t tmem = tmem_base;            // S' buffers at columns 0, 128, 256; O at 384
-    constexpr uint32_t kOcol = NSB * 128;
+    const uint32_t tmem = tmem_base;            // S/P of half h at column 128 h, O of half h at 256 + 128 h
+    constexpr uint32_t kOcol = 256;
 
     if (warp == 0) {
         if (lane == 0) {
             const int qrow = (b * a.n_q + r0) * H;
-            mbar_arrive_expect_tx(&q_full, TILE_BYTES);
-            tma_load_2d(qs, &qmap, &q_full, 0, qrow);
-            tma_load_2d(qs + BOX_BYTES, &qmap, &q_full, 64, qrow);
-            // K runs one tile ahead of V: K(t) is needed by S'(t), V(t) only by O after P(t)
+            mbar_arrive_expect_tx(&q_full, 2 * TILE_BYTES);
+            for (int h = 0; h < 2; ++h) {
+                tma_load_2d(qs + h * TILE_BYTES, &qmap, &q_full, 0, qrow + h * 128);
+                tma_load_2d(qs + h * TILE_BYTES + BOX_BYTES, &qmap, &q_full, 64, qrow + h * 128);
+            }
+            // K runs one tile ahead of V: K(t) is needed by S(t), V(t) only after P(t)
             for (int t = 0; t <= n_kt; ++t) {
                 if (t < n_kt) {
                     const int s = t % P2_STAGES;
@@ -339,115 +428,108 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma::idesc_bf16(128, 128, false, false);
-            constexpr uint32_t idesc_o = umma::idesc_bf16(128, 128, true, true);
-            const uint32_t qb = smem_u32(qs), pb = smem_u32(ps);
-            bool ok = wait_or_abort(&q_full, 0, &abort_flag, a.status);
-            // S'(i) runs two tiles ahead of O += P(i-2) V(i-2)
-            for (int i = 0; ok && i < n_kt + 2; ++i) {
-                if (i < n_kt) {                 // S'(i) = K(i) Q^T
-                    const int s = i % P2_STAGES, sb = i % NSB;
-                    if (!(ok = wait_or_abort(&k_full[s], (i / P2_STAGES) & 1, &abort_flag, a.status))) break;
-                    if (i >= NSB && !(ok = wait_or_abort(&s_empty[sb], ((i / NSB) - 1) & 1, &abort_flag, a.status))) break;
-                    umma::fence_after();
-                    const uint32_t kb = smem_u32(kst + s * TILE_BYTES);
+            constexpr uint32_t idesc_o = umma::idesc_bf16(128, 128, false, true);
+            const uint32_t qb = smem_u32(qs);
+            auto issue_s = [&](int h, int s) {          // S_h = Q_h K^T from K stage s
+                const uint32_t kb = smem_u32(kst + s * TILE_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk)
-                        umma::mma_bf16_ss(tmem + sb * 128, kmajor_desc(kb, kk), kmajor_desc(qb, kk), idesc_s, kk > 0);
-                    umma::commit(&k_empty[s]);
-                    umma::commit(&s_full[sb]);
-                }
-                if (i >= 2) {                   // O += P(j) V(j), j = i - 2
-                    const int j = i - 2, s = j % P2_STAGES, pg = j & 1;
-                    if (!(ok = wait_or_abort(&p_full[pg], (j >> 1) & 1, &abort_flag, a.status))) break;
-                    if (!(ok = wait_or_abort(&v_full[s], (j / P2_STAGES) & 1, &abort_flag, a.status))) break;
+                for (int kk = 0; kk < D / 16; ++kk)
+                    umma::mma_bf16_ss(tmem + h * 128, kmajor_desc(qb + h * TILE_BYTES, kk), kmajor_desc(kb, kk),
+                                      idesc_s, kk > 0);
+                umma::commit(&s_full[h]);
+            };
+            bool ok = spin_or_abort(&q_full, 0, &abort_flag, a.status) &&
+                      spin_or_abort(&k_full[0], 0, &abort_flag, a.status);
+            if (ok) {
+                umma::fence_after();
+                issue_s(0, 0);
+                issue_s(1, 0);
+                umma::commit(&k_empty[0]);
+            }
+            // per tile i and half h: O_h += P_h(i) V(i), then at once S_h(i + 1) into the
+            // columns that this PV MMA reads P_h from.  The tensor pipe executes one thread's
+            // MMAs in issue order, so the PV read of P_h precedes the S write; waiting for the
+            // PV to complete instead would drain the pipe twice per tile.
+            for (int i = 0; ok && i < n_kt; ++i) {
+                const int vs = i % P2_STAGES, ks1 = (i + 1) % P2_STAGES;
+                const uint32_t vb = smem_u32(vst + vs * TILE_BYTES);
+                for (int h = 0; h < 2; ++h) {
+                    if (!(ok = spin_or_abort(&p_full[h], i & 1, &abort_flag, a.status))) break;
+                    if (h == 0 && !(ok = spin_or_abort(&v_full[vs], (i / P2_STAGES) & 1, &abort_flag, a.status))) break;
                     umma::fence_after();
-                    const uint32_t vb = smem_u32(vst + s * TILE_BYTES);
-                    const uint32_t pbj = pb + pg * TILE_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < KT / 16; ++kk)
-                        umma::mma_bf16_ss(tmem + kOcol, mnmajor_desc(pbj, kk), mnmajor_desc(vb, kk), idesc_o,
-                                          (j > 0 || kk > 0) ? 1u : 0u);
-                    umma::commit(&p_empty[pg]);
-                    umma::commit(&v_empty[s]);
+                        umma::mma_bf16_ts(tmem + kOcol + h * 128, tmem + h * 128 + kk * 8, mnmajor_desc(vb, kk),
+                                          idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+                    if (h == 1) umma::commit(&v_empty[vs]);
+                    if (i + 1 < n_kt) {
+                        if (h == 0 && !(ok = spin_or_abort(&k_full[ks1], ((i + 1) / P2_STAGES) & 1, &abort_flag, a.status))) break;
+                        issue_s(h, ks1);
+                        if (h == 1) umma::commit(&k_empty[ks1]);
+                    }
                 }
             }
             umma::commit(&o_full);
         }
     } else {
-        const int quarter = warp & 3, g = (warp - 2) >> 2;
-        const int st = threadIdx.x - 64;        // 0..255
-        // log-sum-exp of the 128 (row, head) columns; rows past n_q get +inf (P = 0)
-        if (st < MT) {
-            const int row = r0 + (st >> 4);
-            lse_s[st] = row < a.n_q ? a.lse2[(static_cast<size_t>(b) * a.n_q + row) * H + (st & 15)] : INFINITY;
-        }
-        named_sync(1, NSOFT);
-        const int kl = quarter * 32 + lane;     // the key lane this thread owns in S'
-        const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-        float* srow0 = a.scores + (static_cast<size_t>(b) * a.n_q + r0) * a.score_ld;
-        uint8_t* pg_tile = ps + g * TILE_BYTES;
-        // one 32-column chunk = rows 2c, 2c+1 x 16 heads: probabilities, the two rows'
-        // importance, bf16 pairs for the P tile
-        uint32_t pk[64];
-        for (int i = g; i < n_kt; i += 2) {
-            const int sb = i % NSB;
-            if (!wait_or_abort(&s_full[sb], (i / NSB) & 1, &abort_flag, a.status)) break;
+        // half h, row s of lane quarter `quarter`: local row h*8 + 2*quarter + s, TMEM
+        // lanes 32 quarter + 16 s (the row's 16 heads)
+        const int sw = warp - 2, quarter = warp & 3;
+        const int h = sw >> 3, s = (sw >> 2) & 1;
+        const int wt = (sw & 7) * 32 + lane;                  // thread index within the half
+        const int lrow = h * HALF_ROWS + 2 * quarter + s;
+        const int row = r0 + lrow;
+        const int p = pos_base + lrow;
+        const bool row_ok = row < a.n_q;
+        const size_t li = (static_cast<size_t>(b) * a.n_q + row) * H;
+        const float lse_a = row_ok ? a.lse2[li + (lane >> 2)] : INFINITY;      // P = 0 for rows past n_q
+        const float lse_b = row_ok ? a.lse2[li + (lane >> 2) + 8] : INFINITY;
+        float* srow = row_ok ? a.scores + (static_cast<size_t>(b) * a.n_q + row) * a.score_ld : nullptr;
+        const bool vec2 = (a.score_ld & 1) == 0;
+        const float sc2 = a.sc2;
+        const uint32_t tbase = tmem + h * 128 + (static_cast<uint32_t>(32 * quarter + 16 * s) << 16);
+        for (int i = 0; i < n_kt; ++i) {
+            if (!wait_or_abort(&s_full[h], i & 1, &abort_flag, a.status)) break;
             umma::fence_after();
-            const uint32_t ta = tmem + lane_base + sb * 128;
-            const int key = i * KT + kl;
-            uint32_t ra[32], rb[32];
-            umma::tmem_ld32(ta, ra);
-            umma::tmem_ld_wait();
-            umma::tmem_ld32(ta + 32, rb);
-            p2_chunk<0>(ra, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
-            umma::tmem_ld_wait();
-            umma::tmem_ld32(ta + 64, ra);
-            p2_chunk<1>(rb, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
-            umma::tmem_ld_wait();
-            umma::tmem_ld32(ta + 96, rb);
-            p2_chunk<2>(ra, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
-            umma::tmem_ld_wait();
-            umma::fence_before();
-            mbar_arrive(&s_empty[sb]);
-            p2_chunk<3>(rb, key, pos_base, r0, a.n_q, a.sc2, lse_s, srow0, a.score_ld, pk);
             // last tile: cache rows past the last query position may hold anything, and
-            // 0 * NaN would poison O, so this key's V row is zeroed (the K row only feeds
-            // probabilities that are forced to 0 above).  V(i) is resident: S'(i) was
-            // computed, and V(i) is loaded before K(i + 1).
-            if (i == n_kt - 1 && key > p_max) {
-                if (!wait_or_abort(&v_full[i % P2_STAGES], (i / P2_STAGES) & 1, &abort_flag, a.status)) break;
-                uint8_t* vrow = vst + (i % P2_STAGES) * TILE_BYTES + kl * 128;
+            // 0 * NaN would poison O, so those V rows are zeroed before P(i) is released
+            // (the K rows only feed probabilities that are forced to 0)
+            // (no early exit here: every lane must reach the warp's arrival below)
+            if (h == 0 && i == n_kt - 1 && wt < KT && i * KT + wt > p_max &&
+                wait_or_abort(&v_full[i % P2_STAGES], (i / P2_STAGES) & 1, &abort_flag, a.status)) {
+                uint8_t* vrow = vst + (i % P2_STAGES) * TILE_BYTES + wt * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
                     *reinterpret_cast<uint4*>(vrow + BOX_BYTES + c * 16) = make_uint4(0, 0, 0, 0);
                 }
+                umma::fence_proxy_async();
             }
-            // this warpgroup's P tile is free once O += P(i-2) V(i-2) has completed
-            if (i >= 2 && !wait_or_abort(&p_empty[g], ((i >> 1) - 1) & 1, &abort_flag, a.status)) break;
-            // row `kl` of the MN-major P tile: m = (row, head) 0..127 in two 64-wide groups
-            uint8_t* prow = pg_tile + (kl >> 3) * 1024 + (kl & 7) * 128;
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-                const uint4 w = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-                *reinterpret_cast<uint4*>(prow + (cc >> 3) * BOX_BYTES + (((cc & 7) ^ (kl & 7)) << 4)) = w;
-            }
-            umma::fence_proxy_async();
-            mbar_arrive(&p_full[g]);
+            const int kb = i * KT;
+            uint32_t r[32];
+            umma::tmem_ld16x256_x8(tbase, r);                  // keys kb .. kb + 63
+            umma::tmem_ld_wait();
+            p2_chunk(r, tbase, kb, p, sc2, lse_a, lse_b, srow, vec2, lane);
+            umma::tmem_ld16x256_x8(tbase + 64, r);             // keys kb + 64 .. kb + 127
+            umma::tmem_ld_wait();
+            p2_chunk(r, tbase + 32, kb + 64, p, sc2, lse_a, lse_b, srow, vec2, lane);
+            umma::tmem_st_wait();
+            warp_arrive(&p_full[h]);
         }
-        // O epilogue: this thread owns TMEM lane m = (row, head) of the O accumulator and
-        // columns 64 g .. 64 g + 63
-        if (wait_or_abort(&o_full, 0, &abort_flag, a.status)) {
+        // O epilogue: this thread owns TMEM lane m = (row, head) of O_h, columns 64 s .. 64 s + 63
+        // warp-uniform decision: the tensor-memory loads below are warp-collective
+        if (__all_sync(0xffffffffu, wait_or_abort(&o_full, 0, &abort_flag, a.status))) {
             umma::fence_after();
             const int m = quarter * 32 + lane;
-            const int row = r0 + (m >> 4);
-            __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + row) * H + (m & 15)) * D + g * 64;
+            const int orow_i = r0 + h * HALF_ROWS + (m >> 4);
+            __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + orow_i) * H + (m & 15)) * D + 64 * s;
+            const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
 #pragma unroll 1
             for (int c = 0; c < 64; c += 32) {
                 uint32_t r[32];
-                umma::tmem_ld32(tmem + lane_base + kOcol + g * 64 + c, r);
+                umma::tmem_ld32(tmem + lane_base + kOcol + h * 128 + 64 * s + c, r);
                 umma::tmem_ld_wait();
-                if (row < a.n_q) {
+                if (orow_i < a.n_q) {
 #pragma unroll
                     for (int j = 0; j < 32; j += 8) {
                         uint4 w;
@@ -493,8 +575,8 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     a.o = static_cast<__nv_bfloat16*>(pa.o);
     a.status = pa.status;
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
-    const size_t s1 = 1024 + TILE_BYTES + P1_STAGES * TILE_BYTES;
-    const size_t s2 = 1024 + TILE_BYTES + 2 * P2_STAGES * TILE_BYTES + 2 * TILE_BYTES;
+    const size_t s1 = 1024 + 2 * TILE_BYTES + P1_STAGES * TILE_BYTES;
+    const size_t s2 = 1024 + 2 * TILE_BYTES + 2 * P2_STAGES * TILE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(prefill_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(prefill_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));
