@@ -86,7 +86,8 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 // ---------------------------------------------------------------- sparse attention
 struct SparsePlan {
     int splits;
-    int chunk;               // selected entries per split (multiple of 64)
+    int chunk;               // selected entries per split (multiple of 64; of 16 in cluster mode)
+    bool cluster;            // one cluster of CTAs per row, partials merged on chip
 };
 SparsePlan plan_sparse(int rows, int idx_stride);
 size_t sparse_ws_bytes(int rows, int idx_stride);

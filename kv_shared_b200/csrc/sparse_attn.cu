@@ -15,17 +15,29 @@
 // memory (exact) and their per-token scales folded into the logits and into P.
 #include <mutex>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "internal.h"
+#include "sparse_core.cuh"
+
+namespace cg = cooperative_groups;
 
 namespace hs2 {
 namespace {
 
-constexpr int H = 16;
-constexpr int D = 128;
-constexpr int SUB = 64;            // gathered rows per pipeline stage
-constexpr int NT = 128;            // 4 warps x 16 rows
+using sparse::D;
+using sparse::H;
+using sparse::Layout;
+using sparse::NT;
+using sparse::SUB;
 constexpr int kMaxSplits = 32;     // bound of the split count (shared-memory merge tables)
+constexpr int kCluster = 8;        // CTAs per query row in the cluster kernel
+constexpr int kWT = 16;            // selected entries per warp tile (cluster kernel)
+constexpr int kCW = 9;             // warps (= warp tiles) per CTA of the cluster kernel
+constexpr int kCEntries = kWT * kCW;               // 144 entries per CTA
+constexpr int kCNT = 32 * kCW;                     // 288 threads
+static_assert(H == 2 * kCluster, "each CTA of a cluster finalizes two heads");
 
 struct Params {
     int rows, n_q, idx_stride, splits, chunk;
@@ -46,263 +58,84 @@ struct Params {
     uint32_t* status;
 };
 
-template <bool KV8>
-struct Layout {
-    static constexpr int ROWB = KV8 ? 128 : 256;      // bytes per gathered cache row
-    static constexpr int STAGE = 2 * SUB * ROWB;       // K rows then V rows
-    static constexpr int CVT = KV8 ? 2 * SUB * 256 : 0;
-};
-
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
-    const float mn = fmaxf(m, m2);
-    if (mn == -INFINITY) return;
-    l = l * ex2(m - mn) + l2 * ex2(m2 - mn);
-    m = mn;
-}
-
-template <bool KV8>
-__global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
-    using L = Layout<KV8>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = align1024(smem_raw);
-    uint8_t* cvt = smem + 2 * L::STAGE;                    // e4m3 only: K bf16 then V bf16
-    float* red_o = reinterpret_cast<float*>(cvt + L::CVT); // [H][D]
-    int* sidx = reinterpret_cast<int*>(red_o + H * D);     // [chunk] cache row per entry (-1 invalid)
-    float* sks = reinterpret_cast<float*>(sidx + a.chunk); // [chunk] k scales (e4m3)
-    float* svs = sks + a.chunk;                            // [chunk] v scales (e4m3)
-    __shared__ float wm[4][H], wl[4][H];
-    __shared__ int s_last;
-
-    const int row = blockIdx.y, split = blockIdx.x;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
-    const int b = row / a.n_q;
+// The selected count of `row`, clamped to what the index row can hold (flagged).
+__device__ __forceinline__ int checked_count(const Params& a, int row) {
     int c = a.cnt[row];
-    if (c < 0 || c > a.idx_stride) {                       // a count the index row cannot hold
-        if (tid == 0) set_status(a.status, HS2_ERR_INDEX);
+    if (c < 0 || c > a.idx_stride) {
+        if (threadIdx.x == 0) set_status(a.status, HS2_ERR_INDEX);
         c = c < 0 ? 0 : a.idx_stride;
     }
-    const int e_begin = split * a.chunk;
-    const int e_end = min(c, e_begin + a.chunk);
-    const int n_sub = e_end > e_begin ? (e_end - e_begin + SUB - 1) / SUB : 0;
-    const int32_t* irow = a.idx + static_cast<size_t>(row) * a.idx_stride;
-    const size_t seq_base = static_cast<size_t>(b) * a.cap;
+    return c;
+}
 
-    // every index (and scale) of this CTA's entries, loaded once up front
-    for (int e = tid; e < a.chunk; e += NT) {
-        int j = -1;
-        if (e_begin + e < e_end) {
-            j = irow[e_begin + e];
-            if (j < 0 || j >= a.cap) { set_status(a.status, HS2_ERR_INDEX); j = -1; }
-        }
+// Entries [e_begin, e_begin + n) of the row's index list into sidx (and their e4m3
+// scales into sks/svs); entries at or past `c`, and out-of-range rows (flagged),
+// become -1.  The index loads do not wait for the count.
+// Slots [n, n_alloc) (padding up to whole sub-tiles) become -1 as well.
+template <bool KV8>
+__device__ __forceinline__ void load_entries(const Params& a, int row, int e_begin, int n, int n_alloc, int c,
+                                             int* sidx, float* sks, float* svs, size_t seq_base) {
+    const int32_t* irow = a.idx + static_cast<size_t>(row) * a.idx_stride;
+    for (int e = threadIdx.x; e < n_alloc; e += NT) {
+        const int ge = e_begin + e;
+        int j = (e < n && ge < a.idx_stride) ? irow[ge] : -1;
+        if (e >= n || ge >= c) j = -1;
+        else if (j < 0 || j >= a.cap) { set_status(a.status, HS2_ERR_INDEX); j = -1; }
         sidx[e] = j;
         if (KV8) {
             sks[e] = j >= 0 ? a.k_scale[seq_base + j] : 0.f;
             svs[e] = j >= 0 ? a.v_scale[seq_base + j] : 0.f;
         }
     }
+}
+
+template <bool KV8>
+__global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
+    using L = Layout<KV8>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = sparse::align1024(smem_raw);
+    uint8_t* cvt = smem + 2 * L::STAGE;                    // e4m3 only: K bf16 then V bf16
+    float* red_o = reinterpret_cast<float*>(cvt + L::CVT); // [H][D]
+    int* sidx = reinterpret_cast<int*>(red_o + H * D);     // [chunk] cache row per entry (-1 invalid)
+    float* sks = reinterpret_cast<float*>(sidx + a.chunk); // [chunk] k scales (e4m3)
+    float* svs = sks + a.chunk;                            // [chunk] v scales (e4m3)
+    __shared__ float wm[4][H], wl[4][H], cm[H], cl[H];
+    __shared__ int s_last;
+
+    const int row = blockIdx.y, split = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int b = row / a.n_q;
+    const int c = checked_count(a, row);
+    const int e_begin = split * a.chunk;
+    const int e_end = min(c, e_begin + a.chunk);
+    const int n_sub = e_end > e_begin ? (e_end - e_begin + SUB - 1) / SUB : 0;
+    const size_t seq_base = static_cast<size_t>(b) * a.cap;
+
+    // every index (and scale) of this CTA's entries, loaded once up front
+    load_entries<KV8>(a, row, e_begin, a.chunk, a.chunk, c, sidx, sks, svs, seq_base);
     __syncthreads();
 
-    // gather sub-tile i into stage s (cp.async, zero-filled past the end)
-    auto gather = [&](int i, int s) {
-        uint8_t* st = smem + s * L::STAGE;
-        const int* si = sidx + i * SUB;
-        constexpr int CH = L::ROWB / 16;                   // 16-byte chunks per row
-        for (int it = tid; it < SUB * CH; it += NT) {
-            const int r = it / CH, ch = it % CH;
-            const int j = si[r];
-            const size_t off = (seq_base + (j >= 0 ? j : 0)) * L::ROWB + ch * 16;
-            uint32_t dk, dv;
-            if (KV8) {
-                dk = r * 128 + ((ch ^ (r & 7)) << 4);
-                dv = SUB * 128 + dk;
-            } else {
-                dk = swz_off<SUB>(r, ch);
-                dv = SUB * 256 + dk;
-            }
-            cp_async16_zfill(st + dk, a.k + off, j >= 0);
-            cp_async16_zfill(st + dv, a.v + off, j >= 0);
-        }
+    uint32_t qa[8][4];
+    sparse::load_q(a.q + static_cast<size_t>(row) * H * D, qa, lane >> 2, lane & 3);
+    auto gather = [&](int i, int st) {
+        sparse::gather_rows<KV8>(smem + st * L::STAGE, sidx + i * SUB, a.k, a.v, seq_base, tid);
         cp_async_commit();
     };
-
-    uint32_t qa[8][4];
-    {
-        const uint32_t* q32 = reinterpret_cast<const uint32_t*>(a.q + static_cast<size_t>(row) * H * D);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            qa[ks][0] = __ldg(q32 + (g * D + 16 * ks + 2 * t) / 2);
-            qa[ks][1] = __ldg(q32 + ((g + 8) * D + 16 * ks + 2 * t) / 2);
-            qa[ks][2] = __ldg(q32 + (g * D + 16 * ks + 2 * t + 8) / 2);
-            qa[ks][3] = __ldg(q32 + ((g + 8) * D + 16 * ks + 2 * t + 8) / 2);
-        }
-    }
-
     if (n_sub > 0) gather(0, 0);
     if (n_sub > 1) gather(1, 1);
 
-    float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
-    float o[16][4];
-#pragma unroll
-    for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-
+    sparse::State stt;
+    stt.init();
     for (int i = 0; i < n_sub; ++i) {
-        const int s = i & 1;
+        const int st = i & 1;
         if (i + 1 < n_sub) cp_async_wait<1>(); else cp_async_wait<0>();
         __syncthreads();
-        uint8_t* st = smem + s * L::STAGE;
-        const uint8_t* kt = st;
-        const uint8_t* vt = st + SUB * L::ROWB;
-        if (KV8) {
-            // e4m3 rows (128-byte swizzle) -> bf16 tiles (swz_off layout), exact
-            for (int it = tid; it < 2 * SUB * 8; it += NT) {
-                const int half = it / (SUB * 8), rr = (it / 8) % SUB, c8 = it & 7;
-                const uint8_t* src = st + half * SUB * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4);
-                uint8_t* dst = cvt + half * SUB * 256;
-                const uint4 in = *reinterpret_cast<const uint4*>(src);
-                const uint16_t* bb = reinterpret_cast<const uint16_t*>(&in);
-                uint4 lo, hi;
-                lo.x = e4m3x2_to_bf16x2(bb[0]); lo.y = e4m3x2_to_bf16x2(bb[1]);
-                lo.z = e4m3x2_to_bf16x2(bb[2]); lo.w = e4m3x2_to_bf16x2(bb[3]);
-                hi.x = e4m3x2_to_bf16x2(bb[4]); hi.y = e4m3x2_to_bf16x2(bb[5]);
-                hi.z = e4m3x2_to_bf16x2(bb[6]); hi.w = e4m3x2_to_bf16x2(bb[7]);
-                *reinterpret_cast<uint4*>(dst + swz_off<SUB>(rr, 2 * c8)) = lo;
-                *reinterpret_cast<uint4*>(dst + swz_off<SUB>(rr, 2 * c8 + 1)) = hi;
-            }
-            __syncthreads();
-            kt = cvt;
-            vt = cvt + SUB * 256;
-        }
-        // S = Q K^T for this warp's 16 gathered rows
-        float acc[2][4];
-        const uint32_t kb = smem_u32(kt);
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-            const int r = warp * 16 + nt * 8 + (lane & 7);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kb + swz_off<SUB>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
-                mma_bf16(acc[nt], qa[2 * kk], b0, b1);
-                mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
-            }
-        }
-        const int* si = sidx + i * SUB;
-        float vf[2][2];
-        float mx[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int r0 = warp * 16 + nt * 8 + 2 * t;
-            const bool ok0 = si[r0] >= 0, ok1 = si[r0 + 1] >= 0;
-            float f0 = a.sc2, f1 = a.sc2;
-            if (KV8) {
-                f0 *= sks[i * SUB + r0]; f1 *= sks[i * SUB + r0 + 1];
-                vf[nt][0] = svs[i * SUB + r0]; vf[nt][1] = svs[i * SUB + r0 + 1];
-            } else {
-                vf[nt][0] = vf[nt][1] = 1.f;
-            }
-            acc[nt][0] = ok0 ? acc[nt][0] * f0 : -INFINITY;
-            acc[nt][1] = ok1 ? acc[nt][1] * f1 : -INFINITY;
-            acc[nt][2] = ok0 ? acc[nt][2] * f0 : -INFINITY;
-            acc[nt][3] = ok1 ? acc[nt][3] * f1 : -INFINITY;
-            mx[0] = fmaxf(mx[0], fmaxf(acc[nt][0], acc[nt][1]));
-            mx[1] = fmaxf(mx[1], fmaxf(acc[nt][2], acc[nt][3]));
-        }
-        float alpha[2];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
-            mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
-            const float mn = fmaxf(m2[hh], mx[hh]);
-            alpha[hh] = (mn == -INFINITY) ? 1.f : ex2(m2[hh] - mn);
-            m2[hh] = mn;
-        }
-        float pr[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int hh = e >> 1;
-                pr[nt][e] = (m2[hh] == -INFINITY) ? 0.f : ex2(acc[nt][e] - m2[hh]);
-            }
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-            l2[hh] = l2[hh] * alpha[hh] + pr[0][2 * hh] + pr[0][2 * hh + 1] + pr[1][2 * hh] + pr[1][2 * hh + 1];
-#pragma unroll
-        for (int n = 0; n < 16; ++n) {
-            o[n][0] *= alpha[0]; o[n][1] *= alpha[0];
-            o[n][2] *= alpha[1]; o[n][3] *= alpha[1];
-        }
-        uint32_t pa[4];
-        pa[0] = pack_bf16(pr[0][0] * vf[0][0], pr[0][1] * vf[0][1]);
-        pa[1] = pack_bf16(pr[0][2] * vf[0][0], pr[0][3] * vf[0][1]);
-        pa[2] = pack_bf16(pr[1][0] * vf[1][0], pr[1][1] * vf[1][1]);
-        pa[3] = pack_bf16(pr[1][2] * vf[1][0], pr[1][3] * vf[1][1]);
-        const uint32_t vb = smem_u32(vt);
-        const int vr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vb + swz_off<SUB>(vr, 2 * cc + (lane >> 4)), b0, b1, b2, b3);
-            mma_bf16(o[2 * cc], pa, b0, b1);
-            mma_bf16(o[2 * cc + 1], pa, b2, b3);
-        }
+        sparse::attend_subtile<KV8>(smem + st * L::STAGE, cvt, sidx + i * SUB, sks + i * SUB, svs + i * SUB, qa,
+                                    a.sc2, stt, tid, warp, lane);
         __syncthreads();
-        if (i + 2 < n_sub) gather(i + 2, s);
+        if (i + 2 < n_sub) gather(i + 2, st);
     }
-
-    // merge the 4 warps: quad-reduce l, then a common max per head
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        l2[hh] += __shfl_xor_sync(0xffffffffu, l2[hh], 1);
-        l2[hh] += __shfl_xor_sync(0xffffffffu, l2[hh], 2);
-    }
-    if (t == 0) {
-        wm[warp][g] = m2[0]; wl[warp][g] = l2[0];
-        wm[warp][g + 8] = m2[1]; wl[warp][g + 8] = l2[1];
-    }
-    __syncthreads();
-    float M[2], f[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int h = g + 8 * hh;
-        M[hh] = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
-        f[hh] = (M[hh] == -INFINITY) ? 0.f : ex2(m2[hh] - M[hh]);
-    }
-    // each warp's rescaled O goes to its own padded slab in the drained stage buffers,
-    // then the four slabs are summed (no shared atomics)
-    constexpr int RP = D + 4;                              // padded row (floats)
-    float* slab = reinterpret_cast<float*>(smem) + warp * H * RP;
-#pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        const int d = 8 * n + 2 * t;
-        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(o[n][0] * f[0], o[n][1] * f[0]);
-        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(o[n][2] * f[1], o[n][3] * f[1]);
-    }
-    __syncthreads();
-    {
-        const float* sb = reinterpret_cast<const float*>(smem);
-        for (int i = tid; i < H * D; i += NT) {
-            const int h = i / D, d = i % D;
-            red_o[i] = sb[h * RP + d] + sb[H * RP + h * RP + d] + sb[2 * H * RP + h * RP + d] + sb[3 * H * RP + h * RP + d];
-        }
-    }
-    __syncthreads();
-    // per-head CTA (max, sum); threads 0..15 own head tid
-    __shared__ float cm[H], cl[H];
-    if (tid < H) {
-        const float Mh = fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid]));
-        float Lh = 0.f;
-        if (Mh != -INFINITY)
-            for (int w = 0; w < 4; ++w) Lh += wl[w][tid] * ex2(wm[w][tid] - Mh);
-        cm[tid] = Mh; cl[tid] = Lh;
-    }
-    __syncthreads();
+    sparse::cta_reduce(stt, reinterpret_cast<float*>(smem), red_o, wm, wl, cm, cl, tid, warp, lane);
 
     if (a.splits == 1) {
         for (int i = tid; i < H * D; i += NT) {
@@ -335,7 +168,7 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     __syncthreads();
     if (tid < H) {
         float m = -INFINITY, l = 0.f;
-        for (int sp = 0; sp < a.splits; ++sp) merge_ml(m, l, sml[sp][tid].x, sml[sp][tid].y);
+        for (int sp = 0; sp < a.splits; ++sp) sparse::merge_ml(m, l, sml[sp][tid].x, sml[sp][tid].y);
         fm[tid] = m;
         finv[tid] = l > 0.f ? 1.f / l : 0.f;
         if (a.lse) a.lse[static_cast<size_t>(row) * H + tid] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
@@ -374,6 +207,279 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     }
 }
 
+// ---------------------------------------------------------------- cluster kernel
+// Few rows (decode): the kCluster CTAs of a cluster share one query row, CTA r taking
+// entries [r kCEntries, (r + 1) kCEntries).  Every warp owns one 16-entry warp tile:
+// it loads its indices, gathers its K/V rows (16-byte cp.async into its own swizzled
+// slice of shared memory), scores them against the 16 heads and forms its partial
+// (max, sum, O) with no CTA-wide barrier on the way.  The warps' partials are folded
+// into one per CTA with shared-memory float atomics, each CTA pushes its partial of
+// heads 2p, 2p + 1 into CTA p's shared memory (distributed shared memory stores),
+// and after one cluster barrier CTA p finalizes heads 2p, 2p + 1 from its own memory.
+template <bool KV8>
+struct CLayout {
+    static constexpr int ROWB = KV8 ? 128 : 256;          // bytes per gathered row
+    static constexpr int RAW = 2 * kWT * ROWB;            // one warp's gathered K then V rows
+    static constexpr int TILE = 2 * kWT * 256;            // one warp's bf16 K then V tiles
+    static constexpr int RAW_OFF = 0;
+    static constexpr int BF_OFF = KV8 ? kCW * RAW : 0;    // e4m3: converted copies after the raw rows
+    static constexpr int GATHER_END = BF_OFF + kCW * TILE;
+    static constexpr int SLAB_BYTES = kCW * H * sparse::RP * 4;   // the warps' rescaled O, after the compute
+    static constexpr int Q_OFF = GATHER_END > SLAB_BYTES ? GATHER_END : SLAB_BYTES;
+    static constexpr int RECV_OFF = Q_OFF + H * D * 2;    // [kCluster][2][D] f32 pushed partials
+    static constexpr int BYTES = RECV_OFF + kCluster * 2 * D * 4;
+};
+
+// This warp's 16 gathered rows against the 16 heads: state `s` receives the tile's
+// own (max, sum, O) (no prior state).  `ok0/ok1`: validity of rows 2t, 2t + 1 of each
+// 8-row half; fk/fv: per-row logit and value factors (e4m3 scales; 1 for bf16).
+__device__ __forceinline__ void attend_warp_tile(const uint8_t* kt, const uint8_t* vt, const uint8_t* qs,
+                                                 const bool (&ok)[2][2], const float (&fk)[2][2],
+                                                 const float (&fv)[2][2], float sc2, sparse::State& s, int lane) {
+    float acc[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+    const uint32_t kb = smem_u32(kt), qb = smem_u32(qs);
+    const int qr = (lane & 7) + ((lane >> 3) & 1) * 8;     // A fragments: matrices (rows 0-7 | 8-15) x (k lo | hi)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        uint32_t qa[2][4];
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+            ldsm_x4(qb + swz_off<kWT>(qr, 2 * (2 * kk + u) + (lane >> 4)), qa[u][0], qa[u][1], qa[u][2], qa[u][3]);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kb + swz_off<kWT>(nt * 8 + (lane & 7), 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+            mma_bf16(acc[nt], qa[0], b0, b1);
+            mma_bf16(acc[nt], qa[1], b2, b3);
+        }
+    }
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        acc[nt][0] = ok[nt][0] ? acc[nt][0] * (sc2 * fk[nt][0]) : -INFINITY;
+        acc[nt][1] = ok[nt][1] ? acc[nt][1] * (sc2 * fk[nt][1]) : -INFINITY;
+        acc[nt][2] = ok[nt][0] ? acc[nt][2] * (sc2 * fk[nt][0]) : -INFINITY;
+        acc[nt][3] = ok[nt][1] ? acc[nt][3] * (sc2 * fk[nt][1]) : -INFINITY;
+        mx[0] = fmaxf(mx[0], fmaxf(acc[nt][0], acc[nt][1]));
+        mx[1] = fmaxf(mx[1], fmaxf(acc[nt][2], acc[nt][3]));
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
+        s.m2[hh] = mx[hh];
+    }
+    float pr[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int hh = e >> 1;
+            pr[nt][e] = (mx[hh] == -INFINITY) ? 0.f : ex2(acc[nt][e] - mx[hh]);
+        }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        float l = pr[0][2 * hh] + pr[0][2 * hh + 1] + pr[1][2 * hh] + pr[1][2 * hh + 1];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        s.l2[hh] = l;
+    }
+    uint32_t pa[4];
+    pa[0] = pack_bf16(pr[0][0] * fv[0][0], pr[0][1] * fv[0][1]);
+    pa[1] = pack_bf16(pr[0][2] * fv[0][0], pr[0][3] * fv[0][1]);
+    pa[2] = pack_bf16(pr[1][0] * fv[1][0], pr[1][1] * fv[1][1]);
+    pa[3] = pack_bf16(pr[1][2] * fv[1][0], pr[1][3] * fv[1][1]);
+    const uint32_t vb = smem_u32(vt);
+    const int vr = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + swz_off<kWT>(vr, 2 * cc + (lane >> 4)), b0, b1, b2, b3);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s.o[2 * cc][e] = 0.f, s.o[2 * cc + 1][e] = 0.f;
+        mma_bf16(s.o[2 * cc], pa, b0, b1);
+        mma_bf16(s.o[2 * cc + 1], pa, b2, b3);
+    }
+}
+
+template <bool KV8>
+__global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
+    using CL = CLayout<KV8>;
+    extern __shared__ uint8_t csm_raw[];
+    uint8_t* csm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(csm_raw) + 127) & ~uintptr_t(127));
+    uint8_t* qs = csm + CL::Q_OFF;                                    // [H][D] bf16, swz_off<16>
+    float* recv_o = reinterpret_cast<float*>(csm + CL::RECV_OFF);    // [kCluster][2][D]
+    __shared__ float wm[kCW][H], wl[kCW][H], cmx[H], csum[H];
+    __shared__ float2 recv_ml[kCluster][2];
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int row = blockIdx.y;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int b = row / a.n_q;
+    const size_t seq_base = static_cast<size_t>(b) * a.cap;
+    // a peer's shared memory may be written only once the peer runs: arrive now, wait
+    // just before the pushes
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+    // the row's queries (16 heads x 128) into shared memory, one 16-byte chunk per thread
+    if (tid < H * 16) {
+        const int r = tid >> 4, ch = tid & 15;
+        cp_async16(qs + swz_off<kWT>(r, ch), reinterpret_cast<const uint8_t*>(a.q + static_cast<size_t>(row) * H * D) +
+                                                 r * 256 + ch * 16);
+    }
+    cp_async_commit();
+
+    // ---- this warp's 16 entries: lane l < 16 holds entry e0 + l (the index load does not
+    // wait for the count)
+    const int e0 = rank * kCEntries + warp * kWT;
+    int j = -1;
+    if (lane < kWT && e0 + lane < a.idx_stride) j = a.idx[static_cast<size_t>(row) * a.idx_stride + e0 + lane];
+    const int c = checked_count(a, row);
+    float ksc = 0.f, vsc = 0.f;
+    if (lane < kWT) {
+        if (e0 + lane >= c) j = -1;
+        else if (j < 0 || j >= a.cap) { set_status(a.status, HS2_ERR_INDEX); j = -1; }
+        if (KV8 && j >= 0) { ksc = a.k_scale[seq_base + j]; vsc = a.v_scale[seq_base + j]; }
+    } else {
+        j = -1;
+    }
+    // ---- gather: a row's 16-byte chunks on consecutive lanes (whole rows per instruction)
+    uint8_t* raw = csm + CL::RAW_OFF + warp * CL::RAW;
+    {
+        constexpr int CH = CL::ROWB / 16;                   // chunks per row: 16 (bf16) or 8 (e4m3)
+        constexpr int RPI = 32 / CH;                        // rows per instruction
+        const int ch = lane % CH;
+#pragma unroll
+        for (int u = 0; u < kWT / RPI; ++u) {
+            const int r = u * RPI + lane / CH;
+            const int jr = __shfl_sync(0xffffffffu, j, r);
+            const size_t off = (seq_base + (jr >= 0 ? jr : 0)) * CL::ROWB + ch * 16;
+            uint32_t dk;
+            if (KV8) dk = r * 128 + ((ch ^ (r & 7)) << 4);
+            else dk = swz_off<kWT>(r, ch);
+            cp_async16_zfill(raw + dk, a.k + off, jr >= 0);
+            cp_async16_zfill(raw + kWT * CL::ROWB + dk, a.v + off, jr >= 0);
+        }
+        cp_async_commit();
+    }
+    // per-lane row facts for the fragment layout: rows 8 nt + 2t and 8 nt + 2t + 1
+    bool ok[2][2];
+    float fk[2][2], fv[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int r = nt * 8 + 2 * t + e;
+            ok[nt][e] = __shfl_sync(0xffffffffu, j, r) >= 0;
+            fk[nt][e] = KV8 ? __shfl_sync(0xffffffffu, ksc, r) : 1.f;
+            fv[nt][e] = KV8 ? __shfl_sync(0xffffffffu, vsc, r) : 1.f;
+        }
+    cp_async_wait<1>();                                  // the queries (committed first) have landed
+    __syncthreads();
+    cp_async_wait<0>();                                  // and this warp's rows
+    __syncwarp();
+    const uint8_t* kt = raw;
+    const uint8_t* vt = raw + kWT * CL::ROWB;
+    if (KV8) {
+        // e4m3 rows (128-byte swizzle) -> bf16 tiles of this warp (swz_off<16> layout), exact
+        uint8_t* bf = csm + CL::BF_OFF + warp * CL::TILE;
+        for (int it = lane; it < 2 * kWT * 8; it += 32) {
+            const int half = it / (kWT * 8), rr = (it / 8) % kWT, c8 = it & 7;
+            const uint8_t* src = raw + half * kWT * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4);
+            uint8_t* dst = bf + half * kWT * 256;
+            const uint4 in = *reinterpret_cast<const uint4*>(src);
+            const uint16_t* bb = reinterpret_cast<const uint16_t*>(&in);
+            uint4 lo, hi;
+            lo.x = e4m3x2_to_bf16x2(bb[0]); lo.y = e4m3x2_to_bf16x2(bb[1]);
+            lo.z = e4m3x2_to_bf16x2(bb[2]); lo.w = e4m3x2_to_bf16x2(bb[3]);
+            hi.x = e4m3x2_to_bf16x2(bb[4]); hi.y = e4m3x2_to_bf16x2(bb[5]);
+            hi.z = e4m3x2_to_bf16x2(bb[6]); hi.w = e4m3x2_to_bf16x2(bb[7]);
+            *reinterpret_cast<uint4*>(dst + swz_off<kWT>(rr, 2 * c8)) = lo;
+            *reinterpret_cast<uint4*>(dst + swz_off<kWT>(rr, 2 * c8 + 1)) = hi;
+        }
+        __syncwarp();
+        kt = bf;
+        vt = bf + kWT * 256;
+    }
+    sparse::State st;
+    attend_warp_tile(kt, vt, qs, ok, fk, fv, a.sc2, st, lane);
+
+    // ---- fold the warps: per-head CTA max; each warp writes its rescaled O to its own
+    // padded slab (the gather area is free once every warp has computed)
+    if (t == 0) {
+        wm[warp][g] = st.m2[0]; wl[warp][g] = st.l2[0];
+        wm[warp][g + 8] = st.m2[1]; wl[warp][g + 8] = st.l2[1];
+    }
+    __syncthreads();
+    float f[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int h = g + 8 * hh;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kCW; ++w) M = fmaxf(M, wm[w][h]);
+        f[hh] = (st.m2[hh] == -INFINITY) ? 0.f : ex2(st.m2[hh] - M);
+    }
+    constexpr int RP = sparse::RP;
+    float* slabs = reinterpret_cast<float*>(csm);
+    float* slab = slabs + warp * H * RP;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        const int d = 8 * n + 2 * t;
+        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(st.o[n][0] * f[0], st.o[n][1] * f[0]);
+        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(st.o[n][2] * f[1], st.o[n][3] * f[1]);
+    }
+    if (tid < H) {
+        float M = -INFINITY;
+        for (int w = 0; w < kCW; ++w) M = fmaxf(M, wm[w][tid]);
+        float L = 0.f;
+        if (M != -INFINITY)
+            for (int w = 0; w < kCW; ++w) L += wl[w][tid] * ex2(wm[w][tid] - M);
+        cmx[tid] = M; csum[tid] = L;
+    }
+    __syncthreads();
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    // ---- push heads 2p, 2p + 1 of this CTA's partial (the slab sum) to CTA p
+    for (int i = tid; i < H * D / 4; i += kCNT) {
+        const int h = (4 * i) / D, d = (4 * i) % D;
+        float4 v = *reinterpret_cast<const float4*>(slabs + h * RP + d);
+#pragma unroll
+        for (int w = 1; w < kCW; ++w) {
+            const float4 u = *reinterpret_cast<const float4*>(slabs + w * H * RP + h * RP + d);
+            v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+        }
+        float* dst = cluster.map_shared_rank(recv_o, h >> 1) + (rank * 2 + (h & 1)) * D + d;
+        *reinterpret_cast<float4*>(dst) = v;
+    }
+    if (tid < H) *cluster.map_shared_rank(&recv_ml[rank][tid & 1], tid >> 1) = make_float2(cmx[tid], csum[tid]);
+    cluster.sync();                                      // pushes complete and visible; none after it
+    // ---- finalize heads 2 rank, 2 rank + 1 from this CTA's own memory
+    if (tid < 2 * D) {
+        const int hh = tid / D, d = tid % D, h = 2 * rank + hh;
+        float M = -INFINITY;
+#pragma unroll
+        for (int cc = 0; cc < kCluster; ++cc) M = fmaxf(M, recv_ml[cc][hh].x);
+        float L = 0.f;
+        if (M != -INFINITY)
+#pragma unroll
+            for (int cc = 0; cc < kCluster; ++cc) L += recv_ml[cc][hh].y * ex2(recv_ml[cc][hh].x - M);
+        const float inv = L > 0.f ? 1.f / L : 0.f;
+        float acc = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < kCluster; ++cc) {
+            const float mc = recv_ml[cc][hh].x;
+            if (mc != -INFINITY) acc += ex2(mc - M) * inv * recv_o[(cc * 2 + hh) * D + d];
+        }
+        a.o[(static_cast<size_t>(row) * H + h) * D + d] = __float2bfloat16_rn(acc);
+        if (a.lse && d == 0)
+            a.lse[static_cast<size_t>(row) * H + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
+    }
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <bool KV8>
@@ -405,8 +511,27 @@ cudaError_t launch_impl(const SparseArgs& sa, cudaStream_t st) {
     a.o = static_cast<__nv_bfloat16*>(sa.o);
     a.lse = sa.lse;
     a.status = sa.status;
-    const size_t sm = smem_bytes<KV8>(pl.chunk);
     cudaError_t e;
+    if (pl.cluster) {
+        const size_t sm = CLayout<KV8>::BYTES + 128;
+        e = cudaFuncSetAttribute(sparse_cluster_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(sm));
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(kCluster, sa.rows);
+        cfg.blockDim = dim3(kCNT);
+        cfg.dynamicSmemBytes = sm;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = kCluster;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, sparse_cluster_kernel<KV8>, a);
+    }
+    const size_t sm = smem_bytes<KV8>(pl.chunk);
     e = cudaFuncSetAttribute(sparse_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
     if (e != cudaSuccess) return e;
     sparse_kernel<KV8><<<dim3(pl.splits, sa.rows), NT, sm, st>>>(a);
@@ -417,6 +542,14 @@ cudaError_t launch_impl(const SparseArgs& sa, cudaStream_t st) {
 
 SparsePlan plan_sparse(int rows, int idx_stride) {
     SparsePlan pl;
+    pl.cluster = false;
+    // few rows: one cluster of kCluster CTAs per row, merged on chip
+    if (rows <= num_sms() && idx_stride <= kCluster * kCEntries) {
+        pl.cluster = true;
+        pl.splits = kCluster;
+        pl.chunk = kCEntries;
+        return pl;
+    }
     // enough CTAs to cover the SMs twice; one CTA per row when rows alone do
     int splits = (2 * num_sms() + rows - 1) / (rows > 0 ? rows : 1);
     if (rows > kMaxCounters) splits = 1;           // semaphore counters exist for kMaxCounters rows
@@ -433,7 +566,7 @@ SparsePlan plan_sparse(int rows, int idx_stride) {
 
 size_t sparse_ws_bytes(int rows, int idx_stride) {
     const SparsePlan pl = plan_sparse(rows, idx_stride);
-    if (pl.splits == 1) return 0;
+    if (pl.splits == 1 || pl.cluster) return 0;
     return align256(sizeof(float2) * rows * pl.splits * H) +
            align256(sizeof(float) * static_cast<size_t>(rows) * pl.splits * H * D) +
            align256(sizeof(int) * rows);

@@ -1,0 +1,244 @@
+// sparse_core.cuh -- the per-CTA arithmetic of the sparse-attention layer, shared
+// by the split kernel (global-memory merge) and the cluster kernel (merge through
+// distributed shared memory): one 64-row gathered sub-tile against the 16 query
+// heads (mma.sync m16n8k16, M = the heads, online softmax in registers), and the
+// reduction of the four warps' states to one (max, sum, O) per head.
+#pragma once
+
+#include "common.cuh"
+
+namespace hs2 {
+namespace sparse {
+
+constexpr int H = 16;
+constexpr int D = 128;
+constexpr int SUB = 64;            // gathered rows per sub-tile
+constexpr int NT = 128;            // 4 warps x 16 rows
+constexpr int RP = D + 4;          // padded slab row (floats) of the warp merge
+
+template <bool KV8>
+struct Layout {
+    static constexpr int ROWB = KV8 ? 128 : 256;      // bytes per gathered cache row
+    static constexpr int STAGE = 2 * SUB * ROWB;       // K rows then V rows
+    static constexpr int CVT = KV8 ? 2 * SUB * 256 : 0;
+    static constexpr int SLABS = 4 * H * RP * 4;       // warp-merge slabs (bytes)
+};
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
+    const float mn = fmaxf(m, m2);
+    if (mn == -INFINITY) return;
+    l = l * ex2(m - mn) + l2 * ex2(m2 - mn);
+    m = mn;
+}
+
+// Per-thread softmax state: rows g and g + 8 of the 16 heads (m2, l2 per head
+// half), O fragments of 16 column blocks of 8.
+struct State {
+    float m2[2], l2[2];
+    float o[16][4];
+    __device__ __forceinline__ void init() {
+        m2[0] = m2[1] = -INFINITY;
+        l2[0] = l2[1] = 0.f;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+    }
+};
+
+// Q fragments (A operand, 16 heads x 128) of one query row, straight from global.
+__device__ __forceinline__ void load_q(const __nv_bfloat16* qrow, uint32_t (&qa)[8][4], int g, int t) {
+    const uint32_t* q32 = reinterpret_cast<const uint32_t*>(qrow);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        qa[ks][0] = __ldg(q32 + (g * D + 16 * ks + 2 * t) / 2);
+        qa[ks][1] = __ldg(q32 + ((g + 8) * D + 16 * ks + 2 * t) / 2);
+        qa[ks][2] = __ldg(q32 + (g * D + 16 * ks + 2 * t + 8) / 2);
+        qa[ks][3] = __ldg(q32 + ((g + 8) * D + 16 * ks + 2 * t + 8) / 2);
+    }
+}
+
+// Issues the 16-byte cp.async copies of the SUB gathered rows `si` (cache row per
+// entry, -1 = none: zero-filled) into stage `st` (K rows, then V rows); no commit.
+template <bool KV8>
+__device__ __forceinline__ void gather_rows(uint8_t* st, const int* si, const uint8_t* k, const uint8_t* v,
+                                            size_t seq_base, int tid) {
+    using L = Layout<KV8>;
+    constexpr int CH = L::ROWB / 16;                   // 16-byte chunks per row
+    for (int it = tid; it < SUB * CH; it += NT) {
+        const int r = it / CH, ch = it % CH;
+        const int j = si[r];
+        const size_t off = (seq_base + (j >= 0 ? j : 0)) * L::ROWB + ch * 16;
+        uint32_t dk, dv;
+        if (KV8) {
+            dk = r * 128 + ((ch ^ (r & 7)) << 4);
+            dv = SUB * 128 + dk;
+        } else {
+            dk = swz_off<SUB>(r, ch);
+            dv = SUB * 256 + dk;
+        }
+        cp_async16_zfill(st + dk, k + off, j >= 0);
+        cp_async16_zfill(st + dv, v + off, j >= 0);
+    }
+}
+
+// One landed sub-tile (stage `st`): e4m3 rows are first converted to bf16 in `cvt`
+// (exact; contains a CTA barrier, so every thread calls this), then this warp's 16
+// rows are scored against the 16 heads, the online softmax advanced and P V added.
+// `si` / `sks` / `svs`: the sub-tile's cache rows and (e4m3) per-token scales.
+template <bool KV8>
+__device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, const int* si, const float* sks,
+                                               const float* svs, const uint32_t (&qa)[8][4], float sc2, State& s,
+                                               int tid, int warp, int lane) {
+    const int t = lane & 3;
+    const uint8_t* kt = st;
+    const uint8_t* vt = st + SUB * Layout<KV8>::ROWB;
+    if (KV8) {
+        // e4m3 rows (128-byte swizzle) -> bf16 tiles (swz_off layout), exact
+        for (int it = tid; it < 2 * SUB * 8; it += NT) {
+            const int half = it / (SUB * 8), rr = (it / 8) % SUB, c8 = it & 7;
+            const uint8_t* src = st + half * SUB * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4);
+            uint8_t* dst = cvt + half * SUB * 256;
+            const uint4 in = *reinterpret_cast<const uint4*>(src);
+            const uint16_t* bb = reinterpret_cast<const uint16_t*>(&in);
+            uint4 lo, hi;
+            lo.x = e4m3x2_to_bf16x2(bb[0]); lo.y = e4m3x2_to_bf16x2(bb[1]);
+            lo.z = e4m3x2_to_bf16x2(bb[2]); lo.w = e4m3x2_to_bf16x2(bb[3]);
+            hi.x = e4m3x2_to_bf16x2(bb[4]); hi.y = e4m3x2_to_bf16x2(bb[5]);
+            hi.z = e4m3x2_to_bf16x2(bb[6]); hi.w = e4m3x2_to_bf16x2(bb[7]);
+            *reinterpret_cast<uint4*>(dst + swz_off<SUB>(rr, 2 * c8)) = lo;
+            *reinterpret_cast<uint4*>(dst + swz_off<SUB>(rr, 2 * c8 + 1)) = hi;
+        }
+        __syncthreads();
+        kt = cvt;
+        vt = cvt + SUB * 256;
+    }
+    // S = Q K^T for this warp's 16 gathered rows
+    float acc[2][4];
+    const uint32_t kb = smem_u32(kt);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+        const int r = warp * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kb + swz_off<SUB>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+            mma_bf16(acc[nt], qa[2 * kk], b0, b1);
+            mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+        }
+    }
+    float vf[2][2];
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int r0 = warp * 16 + nt * 8 + 2 * t;
+        const bool ok0 = si[r0] >= 0, ok1 = si[r0 + 1] >= 0;
+        float f0 = sc2, f1 = sc2;
+        if (KV8) {
+            f0 *= sks[r0]; f1 *= sks[r0 + 1];
+            vf[nt][0] = svs[r0]; vf[nt][1] = svs[r0 + 1];
+        } else {
+            vf[nt][0] = vf[nt][1] = 1.f;
+        }
+        acc[nt][0] = ok0 ? acc[nt][0] * f0 : -INFINITY;
+        acc[nt][1] = ok1 ? acc[nt][1] * f1 : -INFINITY;
+        acc[nt][2] = ok0 ? acc[nt][2] * f0 : -INFINITY;
+        acc[nt][3] = ok1 ? acc[nt][3] * f1 : -INFINITY;
+        mx[0] = fmaxf(mx[0], fmaxf(acc[nt][0], acc[nt][1]));
+        mx[1] = fmaxf(mx[1], fmaxf(acc[nt][2], acc[nt][3]));
+    }
+    float alpha[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
+        const float mn = fmaxf(s.m2[hh], mx[hh]);
+        alpha[hh] = (mn == -INFINITY) ? 1.f : ex2(s.m2[hh] - mn);
+        s.m2[hh] = mn;
+    }
+    float pr[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int hh = e >> 1;
+            pr[nt][e] = (s.m2[hh] == -INFINITY) ? 0.f : ex2(acc[nt][e] - s.m2[hh]);
+        }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh)
+        s.l2[hh] = s.l2[hh] * alpha[hh] + pr[0][2 * hh] + pr[0][2 * hh + 1] + pr[1][2 * hh] + pr[1][2 * hh + 1];
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        s.o[n][0] *= alpha[0]; s.o[n][1] *= alpha[0];
+        s.o[n][2] *= alpha[1]; s.o[n][3] *= alpha[1];
+    }
+    uint32_t pa[4];
+    pa[0] = pack_bf16(pr[0][0] * vf[0][0], pr[0][1] * vf[0][1]);
+    pa[1] = pack_bf16(pr[0][2] * vf[0][0], pr[0][3] * vf[0][1]);
+    pa[2] = pack_bf16(pr[1][0] * vf[1][0], pr[1][1] * vf[1][1]);
+    pa[3] = pack_bf16(pr[1][2] * vf[1][0], pr[1][3] * vf[1][1]);
+    const uint32_t vb = smem_u32(vt);
+    const int vr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc) {
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + swz_off<SUB>(vr, 2 * cc + (lane >> 4)), b0, b1, b2, b3);
+        mma_bf16(s.o[2 * cc], pa, b0, b1);
+        mma_bf16(s.o[2 * cc + 1], pa, b2, b3);
+    }
+}
+
+// Reduces the four warps' states to this CTA's per-head (max, sum) in cm/cl and its
+// unnormalized O (rescaled to that max) in red_o[H][D].  `slabs` (Layout::SLABS bytes)
+// must be free shared memory (the drained stages); wm/wl are [4][H] scratch.
+__device__ __forceinline__ void cta_reduce(const State& s, float* slabs, float* red_o, float (*wm)[H],
+                                           float (*wl)[H], float* cm, float* cl, int tid, int warp, int lane) {
+    const int g = lane >> 2, t = lane & 3;
+    float l2[2] = {s.l2[0], s.l2[1]};
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        l2[hh] += __shfl_xor_sync(0xffffffffu, l2[hh], 1);
+        l2[hh] += __shfl_xor_sync(0xffffffffu, l2[hh], 2);
+    }
+    if (t == 0) {
+        wm[warp][g] = s.m2[0]; wl[warp][g] = l2[0];
+        wm[warp][g + 8] = s.m2[1]; wl[warp][g + 8] = l2[1];
+    }
+    __syncthreads();
+    float f[2];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        const int h = g + 8 * hh;
+        const float M = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
+        f[hh] = (M == -INFINITY) ? 0.f : ex2(s.m2[hh] - M);
+    }
+    // each warp's rescaled O goes to its own padded slab, then the four are summed
+    float* slab = slabs + warp * H * RP;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        const int d = 8 * n + 2 * t;
+        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(s.o[n][0] * f[0], s.o[n][1] * f[0]);
+        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(s.o[n][2] * f[1], s.o[n][3] * f[1]);
+    }
+    __syncthreads();
+    for (int i = tid; i < H * D; i += NT) {
+        const int h = i / D, d = i % D;
+        red_o[i] = slabs[h * RP + d] + slabs[H * RP + h * RP + d] + slabs[2 * H * RP + h * RP + d] +
+                   slabs[3 * H * RP + h * RP + d];
+    }
+    if (tid < H) {
+        const float Mh = fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid]));
+        float Lh = 0.f;
+        if (Mh != -INFINITY)
+            for (int w = 0; w < 4; ++w) Lh += wl[w][tid] * ex2(wm[w][tid] - Mh);
+        cm[tid] = Mh; cl[tid] = Lh;
+    }
+    __syncthreads();
+}
+
+}  // namespace sparse
+}  // namespace hs2

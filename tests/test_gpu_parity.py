@@ -91,7 +91,7 @@ def test_select_all_equal_scores_picks_lowest():
 
 # ------------------------------------------------------------------ sparse attention on given indices
 @pytest.mark.parametrize("kv", ["bf16", "e4m3"])
-@pytest.mark.parametrize("rows_shape", [(4, 1), (2, 300)])
+@pytest.mark.parametrize("rows_shape", [(4, 1), (1, 200), (2, 300)])   # cluster, 2-way split, one CTA per row
 def test_sparse_attn_random_indices(kv, rows_shape):
     B, n_q = rows_shape
     T, H, D = 3000, 16, 128
