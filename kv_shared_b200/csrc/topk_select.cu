@@ -61,10 +61,12 @@ struct Smem {
     int counts[2];              // published to the cluster: #above, #equal (fallback paths)
     int dec[8];                 // rank 0's decisions: first-digit bin, count above, bin size,
                                 // candidate mode; threshold key and equal keys to take
-    int pub[2];                 // this CTA's candidate count (read by rank 0)
+    int pub[2];                 // this CTA's candidate count and bin-b1 key count (read by rank 0)
     int table[kMaxCluster][2];  // rank 0: output offset and equal-key rank base per CTA
     int cnt_gt[kMaxCluster], cnt_eq[kMaxCluster];
-    int ncand, ncand2;
+    int ncand2, nb1;
+    uint32_t bcast[2 * kMaxCluster];   // remote values fetched once and shared with the CTA
+    int lhist[256];             // rank 0's digits over the gathered bin-b1 keys
 };
 
 // Block-wide exclusive scan of one int per thread; sm.total receives the sum.
@@ -265,29 +267,124 @@ __device__ __forceinline__ void for_keys_fast(const Slice& sl, F f) {
     for (int i = sl.begin + 4 * n4 + threadIdx.x; i < sl.end; i += NT) f(i, sl.key(i));
 }
 
-// Bitonic sort of n (<= cap, cap a power of two) (a, b) pairs in shared memory,
-// ascending by a when `ascending`, else descending; entries [n, N) are padding.
-__device__ __forceinline__ void bitonic_sort(uint32_t* a, uint32_t* bvals, int n, bool ascending) {
-    int N = 1;
-    while (N < n) N <<= 1;
-    const uint32_t pad = ascending ? 0xffffffffu : 0u;
-    for (int i = n + threadIdx.x; i < N; i += NT) { a[i] = pad; if (bvals) bvals[i] = 0u; }
-    __syncthreads();
-    for (int k = 2; k <= N; k <<= 1) {
-        for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int t = threadIdx.x; t < N / 2; t += NT) {
-                const int i = (t / j) * 2 * j + (t % j);
-                const int l = i + j;
-                const bool up = ((i & k) == 0) == ascending;
-                const uint32_t x = a[i], y = a[l];
-                if ((x > y) == up && x != y) {
-                    a[i] = y; a[l] = x;
-                    if (bvals) { const uint32_t t2 = bvals[i]; bvals[i] = bvals[l]; bvals[l] = t2; }
-                }
-            }
-            __syncthreads();
+// Compacts, in position order, the slice's keys >= thr into (ck, cp); returns their
+// number.  Rounds of 4 consecutive keys per thread, one block scan per round.
+__device__ __forceinline__ int compact_ordered(const Slice& sl, uint32_t thr, uint32_t* ck, uint32_t* cp, Smem& sm) {
+    int n = 0;
+    const bool vec = sl.cache != nullptr;                  // cache rows start 16-byte aligned
+    for (int base = sl.begin; base < sl.end; base += 4 * NT) {
+        const int i0 = base + 4 * threadIdx.x;
+        uint32_t k[4];
+        if (vec && i0 + 3 < sl.end) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sl.cache + (i0 - sl.begin));
+            k[0] = v.x; k[1] = v.y; k[2] = v.z; k[3] = v.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) k[u] = i0 + u < sl.end ? sl.key(i0 + u) : 0u;
         }
+        int c = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) c += (i0 + u < sl.end) && k[u] >= thr;
+        const int at = block_excl_scan(c, sm);
+        const int tot = sm.total;
+        int o = n + at;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (i0 + u < sl.end && k[u] >= thr) { ck[o] = k[u]; cp[o] = static_cast<uint32_t>(i0 + u); ++o; }
+        n += tot;
     }
+    return n;
+}
+
+// As compact_ordered for a slice cached in shared memory: each warp owns a contiguous
+// segment (chunks of 128 keys, 4 per lane), counts its matches, one block scan of
+// the warp counts, then a second read writes them in order (warp-level scans only).
+__device__ __forceinline__ int compact_cached(const Slice& sl, uint32_t thr, uint32_t* ck, uint32_t* cp, Smem& sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = sl.end - sl.begin;
+    const int seg = ((n + NW * 128 - 1) / (NW * 128)) * 128;
+    const int s0 = min(warp * seg, n), s1 = min(s0 + seg, n);
+    auto load4 = [&](int e, uint32_t (&k)[4]) {              // keys e .. e+3 of the slice (e % 4 == 0)
+        if (e + 3 < n) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sl.cache + e);
+            k[0] = v.x; k[1] = v.y; k[2] = v.z; k[3] = v.w;
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) k[u] = e + u < n ? sl.cache[e + u] : 0u;
+        }
+    };
+    int mine = 0;
+    for (int c0 = s0; c0 < s1; c0 += 128) {
+        const int e = c0 + 4 * lane;
+        uint32_t k[4];
+        load4(e, k);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) mine += (e + u < s1) && k[u] >= thr;
+    }
+    mine = __reduce_add_sync(0xffffffffu, mine);
+    const int wbase = block_excl_scan(lane == 0 ? mine : 0, sm);
+    const int total = sm.total;
+    int o = __shfl_sync(0xffffffffu, wbase, 0);
+    for (int c0 = s0; c0 < s1; c0 += 128) {
+        const int e = c0 + 4 * lane;
+        uint32_t k[4];
+        load4(e, k);
+        int c = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) c += (e + u < s1) && k[u] >= thr;
+        int x = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, d);
+            if (lane >= d) x += y;
+        }
+        int w = o + x - c;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if ((e + u < s1) && k[u] >= thr) { ck[w] = k[u]; cp[w] = static_cast<uint32_t>(sl.begin + e + u); ++w; }
+        o += __shfl_sync(0xffffffffu, x, 31);
+    }
+    __syncthreads();
+    return total;
+}
+
+// The k-th largest (k >= 1) of the n keys g[] that match prefix under mask, resolved
+// 8 bits at a time (bits below `shift`) with the histogram sm.lhist; whole CTA.
+__device__ __forceinline__ uint32_t local_kth(const uint32_t* g, int n, uint32_t prefix, uint32_t mask, int shift,
+                                              int k, Smem& sm) {
+    int* hist = sm.lhist;
+#pragma unroll 1
+    for (int top = shift - 1; top >= 0;) {
+        const int width = min(8, top + 1);
+        const int sh = top - width + 1;
+        const int nb = 1 << width;
+        for (int i = threadIdx.x; i < nb; i += NT) hist[i] = 0;
+        __syncthreads();
+        // keys sharing a prefix crowd few bins: lanes with the same bin add once together
+        for (int e0 = 0; e0 < n; e0 += NT) {
+            const int e = e0 + threadIdx.x;
+            const uint32_t key = e < n ? g[e] : 0u;
+            const bool in = e < n && (key & mask) == prefix;
+            const int bn = in ? static_cast<int>((key >> sh) & (nb - 1)) : -1;
+            const uint32_t peers = __match_any_sync(0xffffffffu, bn);
+            if (in && (__ffs(peers) - 1) == (threadIdx.x & 31)) atomicAdd(&hist[bn], __popc(peers));
+        }
+        __syncthreads();
+        const int bin = nb - 1 - static_cast<int>(threadIdx.x);        // one bin per thread, descending
+        const int c = bin >= 0 ? hist[bin] : 0;
+        const int above = block_excl_scan(c, sm);
+        if (c > 0 && above < k && above + c >= k) {
+            sm.found_bin = bin;
+            sm.found_above = above;
+        }
+        __syncthreads();
+        prefix |= static_cast<uint32_t>(sm.found_bin) << sh;
+        mask |= static_cast<uint32_t>(nb - 1) << sh;
+        k -= sm.found_above;
+        __syncthreads();                                   // found_bin is rewritten next digit
+        top = sh - 1;
+    }
+    return prefix;
 }
 
 template <int CS>
@@ -358,13 +455,16 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
             sm.range[0] = l; sm.range[1] = h;
         }
         cluster.sync();                            // [barrier 1] ranges written once
+        // one thread per remote word, then shared: not every thread reading every peer
+        if (threadIdx.x < 2 * cs) sm.bcast[threadIdx.x] = remote(sm.range, threadIdx.x >> 1)[threadIdx.x & 1];
+        __syncthreads();
         lo = 0xffffffffu; hi = 0u;
 #pragma unroll
         for (int rr = 0; rr < cs; ++rr) {
-            const uint32_t* rg = remote(sm.range, rr);
-            lo = min(lo, rg[0]);
-            hi = max(hi, rg[1]);
+            lo = min(lo, sm.bcast[2 * rr]);
+            hi = max(hi, sm.bcast[2 * rr + 1]);
         }
+        __syncthreads();                           // bcast is reused
     }
 
     uint32_t tau = 0;
@@ -395,17 +495,27 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
                 const int bins_per = (nb + NT - 1) / NT;
                 int local[NBINS / NT];
                 int tot = 0;
-#pragma unroll
-                for (int q = 0; q < NBINS / NT; ++q) {
-                    const int bin = nb - 1 - (threadIdx.x * bins_per + q);
-                    int c = 0;
-                    if (q < bins_per && bin >= 0) {
+                // the cluster's histogram summed into hist[1] with coalesced remote reads
+                // (consecutive threads, consecutive bins), then scanned from there
+                int* hsum = sm.hist[1];
+                if (CS == 1) {
+                    hsum = hist;
+                } else {
+                    for (int bin = threadIdx.x; bin < nb; bin += NT) {
                         int v[CS];
 #pragma unroll
                         for (int rr = 0; rr < CS; ++rr) v[rr] = remote(hist, rr)[bin];
+                        int c = 0;
 #pragma unroll
                         for (int rr = 0; rr < CS; ++rr) c += v[rr];
+                        hsum[bin] = c;
                     }
+                    __syncthreads();
+                }
+#pragma unroll
+                for (int q = 0; q < NBINS / NT; ++q) {
+                    const int bin = nb - 1 - (threadIdx.x * bins_per + q);
+                    const int c = (q < bins_per && bin >= 0) ? hsum[bin] : 0;
                     local[q] = c;
                     tot += c;
                 }
@@ -428,56 +538,72 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
                 if (threadIdx.x == 0) sm.dec[3] = (K + sm.dec[2] <= kCandCap && sm.dec[2] <= 2 * NBINS) ? 1 : 0;
             }
             cluster.sync();                        // [barrier 3] decision published
-            const int* d0 = remote(sm.dec, 0);
-            const int b1 = d0[0], above1 = d0[1];
-            use_cands = d0[3] != 0;
+            if (threadIdx.x < 4) sm.bcast[threadIdx.x] = static_cast<uint32_t>(remote(sm.dec, 0)[threadIdx.x]);
+            __syncthreads();
+            const int b1 = static_cast<int>(sm.bcast[0]), above1 = static_cast<int>(sm.bcast[1]);
+            use_cands = sm.bcast[3] != 0;
+            __syncthreads();
             prefix |= static_cast<uint32_t>(b1) << shift;
             mask |= static_cast<uint32_t>(nb - 1) << shift;
             k_rem -= above1;
             if (use_cands) {
-                // ---- 3. candidates: this CTA's keys at or above bin b1, sorted by position
-                if (threadIdx.x == 0) { sm.ncand = 0; sm.ncand2 = 0; }
+                // ---- 3. candidates: this CTA's keys at or above bin b1, in position order;
+                // its bin-b1 keys (fewer than kCandCap - K on this path) copied to hist[1]
+                if (threadIdx.x == 0) { sm.ncand2 = 0; sm.nb1 = 0; }
+                n_my = sl.cache ? compact_cached(sl, prefix, cand_key, cand_pos, sm)
+                                : compact_ordered(sl, prefix, cand_key, cand_pos, sm);
+                uint32_t* b1k = reinterpret_cast<uint32_t*>(sm.hist[1]);
+                for (int e0 = 0; e0 < n_my; e0 += NT) {              // one counter update per warp
+                    const int e = e0 + threadIdx.x;
+                    const uint32_t key = e < n_my ? cand_key[e] : 0u;
+                    const bool in = e < n_my && (key & mask) == prefix;
+                    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+                    int base = 0;
+                    if (lane == 0 && bal) base = atomicAdd(&sm.nb1, __popc(bal));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    if (in) b1k[base + __popc(bal & ((1u << lane) - 1u))] = key;
+                }
                 __syncthreads();
-                for_keys_fast(sl, [&](int i, uint32_t key) {
-                    if (key >= prefix) {
-                        const int o = atomicAdd(&sm.ncand, 1);
-                        cand_key[o] = key;
-                        cand_pos[o] = static_cast<uint32_t>(i);
-                    }
-                });
-                __syncthreads();
-                n_my = sm.ncand;
-                bitonic_sort(cand_pos, cand_key, n_my, true);
-                if (threadIdx.x == 0) sm.pub[0] = n_my;
+                if (threadIdx.x == 0) { sm.pub[0] = n_my; sm.pub[1] = sm.nb1; }
                 cluster.sync();                    // [barrier 4] candidate lists complete
                 // ---- 4. rank 0: the bin-b1 keys of the whole cluster, sorted descending, give
                 // tau exactly; then every CTA's counts and output offsets
                 if (rank == 0) {
-                    uint32_t* g = reinterpret_cast<uint32_t*>(&sm.hist[0][0]);    // 2 * NBINS keys
-                    for (int rr = 0; rr < cs; ++rr) {
-                        const int n_rr = remote(sm.pub, rr)[0];
-                        const uint32_t* ck = remote(cand_key, rr);
-                        for (int e = threadIdx.x; e < n_rr; e += NT) {
-                            const uint32_t key = ck[e];
-                            if ((key & mask) == prefix) g[atomicAdd(&sm.ncand2, 1)] = key;
-                        }
+                    uint32_t* g = reinterpret_cast<uint32_t*>(&sm.hist[0][0]);    // the cluster's bin-b1 keys
+                    // every CTA's counts in one batch, then one flat copy of all bin-b1 keys
+                    int nb1[kMaxCluster], na[kMaxCluster], off[kMaxCluster + 1];
+#pragma unroll
+                    for (int rr = 0; rr < CS; ++rr) {
+                        const int* pb = remote(sm.pub, rr);
+                        na[rr] = pb[0];
+                        nb1[rr] = pb[1];
                     }
+                    off[0] = 0;
+#pragma unroll
+                    for (int rr = 0; rr < CS; ++rr) off[rr + 1] = off[rr] + nb1[rr];
+#pragma unroll
+                    for (int rr = 0; rr < CS; ++rr) {
+                        const uint32_t* bk = remote(b1k, rr);
+                        for (int e = threadIdx.x; e < nb1[rr]; e += NT) g[off[rr] + e] = bk[e];
+                    }
+                    if (threadIdx.x == 0) sm.ncand2 = off[CS];
                     if (threadIdx.x < kMaxCluster) { sm.cnt_gt[threadIdx.x] = 0; sm.cnt_eq[threadIdx.x] = 0; }
                     __syncthreads();
                     const int n1 = sm.ncand2;
-                    bitonic_sort(g, nullptr, n1, false);
-                    const uint32_t t = g[k_rem - 1];
-                    for (int rr = 0; rr < cs; ++rr) {
-                        const int n_rr = remote(sm.pub, rr)[0];
-                        const uint32_t* ck = remote(cand_key, rr);
+                    const uint32_t t = local_kth(g, n1, prefix, mask, shift, k_rem, sm);
+                    // per CTA: its candidates above bin b1, plus its bin-b1 keys (its segment
+                    // of g) above / equal to t
+#pragma unroll
+                    for (int rr = 0; rr < CS; ++rr) {
                         int cg_ = 0, ce = 0;
-                        for (int e = threadIdx.x; e < n_rr; e += NT) {
-                            const uint32_t key = ck[e];
+                        for (int e = off[rr] + threadIdx.x; e < off[rr + 1]; e += NT) {
+                            const uint32_t key = g[e];
                             cg_ += key > t;
                             ce += key == t;
                         }
                         cg_ = __reduce_add_sync(0xffffffffu, cg_);
                         ce = __reduce_add_sync(0xffffffffu, ce);
+                        if (threadIdx.x == 0) cg_ += na[rr] - nb1[rr];
                         if (lane == 0) {
                             if (cg_) atomicAdd(&sm.cnt_gt[rr], cg_);
                             if (ce) atomicAdd(&sm.cnt_eq[rr], ce);
@@ -500,12 +626,14 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
                     }
                 }
                 cluster.sync();                    // [barrier 5] threshold and offsets published
-                const int* d1 = remote(sm.dec, 0);
-                tau = static_cast<uint32_t>(d1[4]);
-                need_eq = d1[5];
-                const int* tb = remote(&sm.table[0][0], 0);
-                out_base = tb[2 * rank];
-                eq_base = tb[2 * rank + 1];
+                if (threadIdx.x < 2) sm.bcast[threadIdx.x] = static_cast<uint32_t>(remote(sm.dec, 0)[4 + threadIdx.x]);
+                else if (threadIdx.x < 4)
+                    sm.bcast[threadIdx.x] = static_cast<uint32_t>(remote(&sm.table[0][0], 0)[2 * rank + threadIdx.x - 2]);
+                __syncthreads();
+                tau = sm.bcast[0];
+                need_eq = static_cast<int>(sm.bcast[1]);
+                out_base = static_cast<int>(sm.bcast[2]);
+                eq_base = static_cast<int>(sm.bcast[3]);
                 offsets_known = true;
             } else {
                 // ---- 4'. candidate lists would not fit: remaining digits over every key
