@@ -48,6 +48,7 @@ struct Params {
     int B, n_q;
     int64_t cap, max_ctx;
     const int32_t* q_pos0;
+    const void* q;                              // [B][n_q][H][D] bf16 (pass 2 reads it directly)
     float sc2;                                  // scale * log2(e), > 0
     float* lse2;                                // [B][n_q][H] log2 units (pass 1 out, pass 2 in)
     float* lse_user;                            // [B][n_q][H] natural log or null
@@ -126,6 +127,34 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
 }
+
+// 2^x for a pair on the FMA pipe (the exponential unit is the bottleneck of pass 1, so a
+// share of the exponentials moves here): x = j + r with j the nearest integer (added to
+// and taken back from 1.5 * 2^23, whose ulp is 1) and r in [-1/2, 1/2]; 2^r by a degree-5
+// polynomial fitted here to the relative error of 2^r on that interval (weighted least
+// squares iterated to near-minimax: max relative error 2.1e-7 in fp32 Horner form, like
+// the exponential unit's); 2^j enters through the exponent bits.  x is clamped at -125 so
+// that the result stays a normal number (it is then below 2^-124, nothing beside the
+// row maximum's 1).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+    constexpr float kMagic = 12582912.f;                       // 1.5 * 2^23
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const float2 t = add2(x, make_float2(kMagic, kMagic));
+    const float2 j = add2(t, make_float2(-kMagic, -kMagic));
+    const float2 r = add2(x, make_float2(-j.x, -j.y));
+    float2 p = make_float2(1.3276455e-3f, 1.3276455e-3f);
+    p = fma2(p, r, make_float2(9.6755400e-3f, 9.6755400e-3f));
+    p = fma2(p, r, make_float2(5.5507135e-2f, 5.5507135e-2f));
+    p = fma2(p, r, make_float2(2.4022120e-1f, 2.4022120e-1f));
+    p = fma2(p, r, make_float2(6.9314694e-1f, 6.9314694e-1f));
+    p = fma2(p, r, make_float2(1.0000001f, 1.0000001f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Which groups of 4 of a 32-value chunk take exp2_poly2 in pass 1 (bit g: group g).
+constexpr uint32_t kPass1PolyGroups = 0x11;                    // groups 0, 4: 8 of 32 (measured best)
 
 // ------------------------------------------------------------------ pass 1: LSE
 constexpr int P1_STAGES = 4;
@@ -244,8 +273,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
                 for (int j = 0; j < 32; j += 4) {
                     const float2 x0 = fma2(make_float2(v[j], v[j + 1]), s2, nm);
                     const float2 x1 = fma2(make_float2(v[j + 2], v[j + 3]), s2, nm);
-                    acc0 = add2(acc0, make_float2(ex2(x0.x), ex2(x0.y)));
-                    acc1 = add2(acc1, make_float2(ex2(x1.x), ex2(x1.y)));
+                    if ((kPass1PolyGroups >> (j / 4)) & 1u) {
+                        acc0 = add2(acc0, exp2_poly2(x0));
+                        acc1 = add2(acc1, exp2_poly2(x1));
+                    } else {
+                        acc0 = add2(acc0, make_float2(ex2(x0.x), ex2(x0.y)));
+                        acc1 = add2(acc1, make_float2(ex2(x1.x), ex2(x1.y)));
+                    }
                 }
                 const float2 acc = add2(acc0, acc1);
                 run_l = run_l * ex2(run_m - mn) + (acc.x + acc.y);
@@ -289,7 +323,6 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
 }
 
 // ------------------------------------------------------------------ pass 2: P, importance, O
-constexpr int P2_STAGES = 2;                    // K and V tiles each double-buffered
 
 // Sum over the 8 lanes that share t % 4 (lane bits 2..4) of eight float2 values, one
 // per 16x256b repetition j; afterwards lane t holds in v[0] the sum for repetition t / 4.
@@ -354,38 +387,51 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
     }
 }
 
+// Pass 2 runs 8 query rows (128 (row, head) pairs) per CTA, with the queries in tensor
+// memory: both MMAs then read only K or V from shared memory (the tensor core and TMA
+// together draw about 77 bytes per cycle from shared memory, which bounds these
+// kernels), and tensor memory holds Q, O and two S buffers.  P(i) is written as packed
+// bf16 into the S(i) buffer, each softmax warp into the 32 columns at the start of the
+// 64 it read, and PV(i) takes it from there as its A operand.  S(i + 2), into the same
+// buffer, is issued right after PV(i) by the same thread: the tensor pipe executes one
+// thread's MMAs in issue order, so PV(i) has read P before S overwrites it, and the
+// softmax writes P(i + 2) only after S(i + 2) has completed, hence after PV(i).
+constexpr int ROWS2 = 8;
+constexpr int P2S = 3;                          // K and V stages of pass 2
+constexpr int NSB2 = 2;                         // S/P buffers at columns 0, 128
+constexpr uint32_t kQcol = 256;                 // Q (packed bf16 pairs) at columns 256 .. 319
+constexpr uint32_t kOcol = 384;                 // O at columns 384 .. 511
+
 __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constant__ CUtensorMap qmap,
                                                            const __grid_constant__ CUtensorMap kmap,
                                                            const __grid_constant__ CUtensorMap vmap, Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* qs = smem;                                       // Q halves 0, 1
-    uint8_t* kst = smem + 2 * TILE_BYTES;                     // K stages
-    uint8_t* vst = kst + P2_STAGES * TILE_BYTES;              // V stages
-    __shared__ uint64_t q_full, k_full[P2_STAGES], k_empty[P2_STAGES], v_full[P2_STAGES], v_empty[P2_STAGES];
-    __shared__ uint64_t s_full[2], p_full[2], o_full;
+    uint8_t* kst = smem;                                      // K stages
+    uint8_t* vst = kst + P2S * TILE_BYTES;                    // V stages
+    __shared__ uint64_t k_full[P2S], k_empty[P2S], v_full[P2S], v_empty[P2S];
+    __shared__ uint64_t s_full[NSB2], p_full[NSB2], q_tm, o_full;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int blocks_per_seq = (a.n_q + ROWS - 1) / ROWS;
+    const int blocks_per_seq = (a.n_q + ROWS2 - 1) / ROWS2;
     const int b = blockIdx.x / blocks_per_seq;
-    const int r0 = (blockIdx.x % blocks_per_seq) * ROWS;
+    const int r0 = (blockIdx.x % blocks_per_seq) * ROWS2;
     const int pos_base = a.q_pos0[b] + r0;
-    const int last_row = min(r0 + ROWS, a.n_q) - 1;
+    const int last_row = min(r0 + ROWS2, a.n_q) - 1;
     const int p_max = checked_pos(a.q_pos0[b] + last_row, a.max_ctx, a.status);
     const int n_kt = (p_max + KT) / KT;
 
     if (threadIdx.x == 0) {
-        prefetch_tmap(&qmap);
         prefetch_tmap(&kmap);
         prefetch_tmap(&vmap);
-        mbar_init(&q_full, 1);
-        for (int s = 0; s < P2_STAGES; ++s) {
+        for (int s = 0; s < P2S; ++s) {
             mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
             mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
         }
-        for (int h = 0; h < 2; ++h) { mbar_init(&s_full[h], 1); mbar_init(&p_full[h], 8); }
+        for (int u = 0; u < NSB2; ++u) { mbar_init(&s_full[u], 1); mbar_init(&p_full[u], 16); }
+        mbar_init(&q_tm, 16);
         mbar_init(&o_full, 1);
         fence_mbar_init();
         abort_flag = 0;
@@ -394,30 +440,23 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     umma::fence_before();
     __syncthreads();
     umma::fence_after();
-    const uint32_t tmem = tmem_base;            // S/P of half h at column 128 h, O of half h at 256 + 128 h
-    constexpr uint32_t kOcol = 256;
+    const uint32_t tmem = tmem_base;            // S/P buffers at 0, 128; Q at 256; O at 384
 
     if (warp == 0) {
         if (lane == 0) {
-            const int qrow = (b * a.n_q + r0) * H;
-            mbar_arrive_expect_tx(&q_full, 2 * TILE_BYTES);
-            for (int h = 0; h < 2; ++h) {
-                tma_load_2d(qs + h * TILE_BYTES, &qmap, &q_full, 0, qrow + h * 128);
-                tma_load_2d(qs + h * TILE_BYTES + BOX_BYTES, &qmap, &q_full, 64, qrow + h * 128);
-            }
             // K runs one tile ahead of V: K(t) is needed by S(t), V(t) only after P(t)
             for (int t = 0; t <= n_kt; ++t) {
                 if (t < n_kt) {
-                    const int s = t % P2_STAGES;
-                    if (t >= P2_STAGES && !wait_or_abort(&k_empty[s], ((t / P2_STAGES) - 1) & 1, &abort_flag, a.status)) break;
+                    const int s = t % P2S;
+                    if (t >= P2S && !wait_or_abort(&k_empty[s], ((t / P2S) - 1) & 1, &abort_flag, a.status)) break;
                     const int krow = static_cast<int>(b * a.cap) + t * KT;
                     mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
                     tma_load_2d(kst + s * TILE_BYTES, &kmap, &k_full[s], 0, krow);
                     tma_load_2d(kst + s * TILE_BYTES + BOX_BYTES, &kmap, &k_full[s], 64, krow);
                 }
                 if (t >= 1) {
-                    const int j = t - 1, s = j % P2_STAGES;
-                    if (j >= P2_STAGES && !wait_or_abort(&v_empty[s], ((j / P2_STAGES) - 1) & 1, &abort_flag, a.status)) break;
+                    const int j = t - 1, s = j % P2S;
+                    if (j >= P2S && !wait_or_abort(&v_empty[s], ((j / P2S) - 1) & 1, &abort_flag, a.status)) break;
                     const int vrow = static_cast<int>(b * a.cap) + j * KT;
                     mbar_arrive_expect_tx(&v_full[s], TILE_BYTES);
                     tma_load_2d(vst + s * TILE_BYTES, &vmap, &v_full[s], 0, vrow);
@@ -429,55 +468,51 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         if (lane == 0) {
             constexpr uint32_t idesc_s = umma::idesc_bf16(128, 128, false, false);
             constexpr uint32_t idesc_o = umma::idesc_bf16(128, 128, false, true);
-            const uint32_t qb = smem_u32(qs);
-            auto issue_s = [&](int h, int s) {          // S_h = Q_h K^T from K stage s
+            auto issue_s = [&](int t) {                 // S(t) = Q K(t)^T into buffer t % NSB2, Q from tensor memory
+                const int s = t % P2S;
                 const uint32_t kb = smem_u32(kst + s * TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
-                    umma::mma_bf16_ss(tmem + h * 128, kmajor_desc(qb + h * TILE_BYTES, kk), kmajor_desc(kb, kk),
-                                      idesc_s, kk > 0);
-                umma::commit(&s_full[h]);
+                    umma::mma_bf16_ts(tmem + (t % NSB2) * 128, tmem + kQcol + kk * 8, kmajor_desc(kb, kk), idesc_s,
+                                      kk > 0);
+                umma::commit(&s_full[t % NSB2]);
+                umma::commit(&k_empty[s]);
             };
-            bool ok = spin_or_abort(&q_full, 0, &abort_flag, a.status) &&
-                      spin_or_abort(&k_full[0], 0, &abort_flag, a.status);
-            if (ok) {
+            bool ok = spin_or_abort(&q_tm, 0, &abort_flag, a.status);
+            for (int t = 0; ok && t < NSB2 && t < n_kt; ++t) {
+                if (!(ok = spin_or_abort(&k_full[t % P2S], (t / P2S) & 1, &abort_flag, a.status))) break;
                 umma::fence_after();
-                issue_s(0, 0);
-                issue_s(1, 0);
-                umma::commit(&k_empty[0]);
+                issue_s(t);
             }
-            // per tile i and half h: O_h += P_h(i) V(i), then at once S_h(i + 1) into the
-            // columns that this PV MMA reads P_h from.  The tensor pipe executes one thread's
-            // MMAs in issue order, so the PV read of P_h precedes the S write; waiting for the
-            // PV to complete instead would drain the pipe twice per tile.
             for (int i = 0; ok && i < n_kt; ++i) {
-                const int vs = i % P2_STAGES, ks1 = (i + 1) % P2_STAGES;
+                // O += P(i) V(i); P(i) sits in the first 32 columns of each 64-column half of
+                // buffer i % NSB2 (keys 0..63, then 64..127)
+                const int vs = i % P2S, u = i % NSB2;
+                if (!(ok = spin_or_abort(&p_full[u], (i / NSB2) & 1, &abort_flag, a.status))) break;
+                if (!(ok = spin_or_abort(&v_full[vs], (i / P2S) & 1, &abort_flag, a.status))) break;
+                umma::fence_after();
                 const uint32_t vb = smem_u32(vst + vs * TILE_BYTES);
-                for (int h = 0; h < 2; ++h) {
-                    if (!(ok = spin_or_abort(&p_full[h], i & 1, &abort_flag, a.status))) break;
-                    if (h == 0 && !(ok = spin_or_abort(&v_full[vs], (i / P2_STAGES) & 1, &abort_flag, a.status))) break;
-                    umma::fence_after();
 #pragma unroll
-                    for (int kk = 0; kk < KT / 16; ++kk)
-                        umma::mma_bf16_ts(tmem + kOcol + h * 128, tmem + h * 128 + kk * 8, mnmajor_desc(vb, kk),
-                                          idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
-                    if (h == 1) umma::commit(&v_empty[vs]);
-                    if (i + 1 < n_kt) {
-                        if (h == 0 && !(ok = spin_or_abort(&k_full[ks1], ((i + 1) / P2_STAGES) & 1, &abort_flag, a.status))) break;
-                        issue_s(h, ks1);
-                        if (h == 1) umma::commit(&k_empty[ks1]);
-                    }
+                for (int kk = 0; kk < KT / 16; ++kk)
+                    umma::mma_bf16_ts(tmem + kOcol, tmem + u * 128 + (kk >> 2) * 64 + (kk & 3) * 8, mnmajor_desc(vb, kk),
+                                      idesc_o, (i > 0 || kk > 0) ? 1u : 0u);
+                umma::commit(&v_empty[vs]);
+                // S(i + 2) into the same buffer, after PV(i) in issue order
+                if (i + NSB2 < n_kt) {
+                    if (!(ok = spin_or_abort(&k_full[(i + NSB2) % P2S], ((i + NSB2) / P2S) & 1, &abort_flag, a.status)))
+                        break;
+                    umma::fence_after();
+                    issue_s(i + NSB2);
                 }
             }
             umma::commit(&o_full);
         }
     } else {
-        // half h, row s of lane quarter `quarter`: local row h*8 + 2*quarter + s, TMEM
-        // lanes 32 quarter + 16 s (the row's 16 heads)
+        // 16 warps: warp (quarter, s, kh) owns row 2 quarter + s (TMEM lanes 32 quarter + 16 s,
+        // the row's 16 heads) and keys 64 kh .. 64 kh + 63 of every tile
         const int sw = warp - 2, quarter = warp & 3;
-        const int h = sw >> 3, s = (sw >> 2) & 1;
-        const int wt = (sw & 7) * 32 + lane;                  // thread index within the half
-        const int lrow = h * HALF_ROWS + 2 * quarter + s;
+        const int s = (sw >> 2) & 1, kh = (sw >> 3) & 1;
+        const int lrow = 2 * quarter + s;
         const int row = r0 + lrow;
         const int p = pos_base + lrow;
         const bool row_ok = row < a.n_q;
@@ -487,17 +522,43 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         float* srow = row_ok ? a.scores + (static_cast<size_t>(b) * a.n_q + row) * a.score_ld : nullptr;
         const bool vec2 = (a.score_ld & 1) == 0;
         const float sc2 = a.sc2;
-        const uint32_t tbase = tmem + h * 128 + (static_cast<uint32_t>(32 * quarter + 16 * s) << 16);
+        const uint32_t lanes = static_cast<uint32_t>(32 * quarter + 16 * s) << 16;
+        const int vt = sw * 32 + lane;                        // V row this thread clears in the last tile
+        // the queries into tensor memory: this thread writes lane m = 32 quarter + lane (pair
+        // (row m / 16, head m % 16)), columns kQcol + 16 cg .. + 15 (dims 32 cg .. 32 cg + 31)
+        {
+            const int m = 32 * quarter + lane, cg = sw >> 2;
+            const int qr = r0 + (m >> 4);
+            uint32_t qv[16];
+            if (qr < a.n_q) {
+                const uint4* src = reinterpret_cast<const uint4*>(
+                    static_cast<const uint8_t*>(a.q) + ((static_cast<size_t>(b) * a.n_q + qr) * H + (m & 15)) * D * 2 +
+                    cg * 64);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = __ldg(src + j);
+                    qv[4 * j] = v.x; qv[4 * j + 1] = v.y; qv[4 * j + 2] = v.z; qv[4 * j + 3] = v.w;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) qv[j] = 0u;
+            }
+            umma::tmem_st32x16(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + kQcol + 16 * cg, qv);
+            umma::tmem_st_wait();
+            warp_arrive(&q_tm);
+        }
         for (int i = 0; i < n_kt; ++i) {
-            if (!wait_or_abort(&s_full[h], i & 1, &abort_flag, a.status)) break;
+            const int u = i % NSB2;
+            // warp-uniform decision: the tensor-memory accesses below are warp-collective
+            if (!__all_sync(0xffffffffu, wait_or_abort(&s_full[u], (i / NSB2) & 1, &abort_flag, a.status))) break;
             umma::fence_after();
             // last tile: cache rows past the last query position may hold anything, and
             // 0 * NaN would poison O, so those V rows are zeroed before P(i) is released
-            // (the K rows only feed probabilities that are forced to 0)
-            // (no early exit here: every lane must reach the warp's arrival below)
-            if (h == 0 && i == n_kt - 1 && wt < KT && i * KT + wt > p_max &&
-                wait_or_abort(&v_full[i % P2_STAGES], (i / P2_STAGES) & 1, &abort_flag, a.status)) {
-                uint8_t* vrow = vst + (i % P2_STAGES) * TILE_BYTES + wt * 128;
+            // (the K rows only feed probabilities that are forced to 0); no early exit, so
+            // that every lane reaches the warp's arrival
+            if (i == n_kt - 1 && vt < KT && i * KT + vt > p_max &&
+                wait_or_abort(&v_full[i % P2S], (i / P2S) & 1, &abort_flag, a.status)) {
+                uint8_t* vrow = vst + (i % P2S) * TILE_BYTES + vt * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
@@ -505,40 +566,34 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
                 }
                 umma::fence_proxy_async();
             }
-            const int kb = i * KT;
             uint32_t r[32];
-            umma::tmem_ld16x256_x8(tbase, r);                  // keys kb .. kb + 63
+            const uint32_t ta = tmem + u * 128 + lanes + 64 * kh;     // this warp's 64 S columns
+            umma::tmem_ld16x256_x8(ta, r);
             umma::tmem_ld_wait();
-            p2_chunk(r, tbase, kb, p, sc2, lse_a, lse_b, srow, vec2, lane);
-            umma::tmem_ld16x256_x8(tbase + 64, r);             // keys kb + 64 .. kb + 127
-            umma::tmem_ld_wait();
-            p2_chunk(r, tbase + 32, kb + 64, p, sc2, lse_a, lse_b, srow, vec2, lane);
+            p2_chunk(r, ta, i * KT + 64 * kh, p, sc2, lse_a, lse_b, srow, vec2, lane);    // P into the first 32
             umma::tmem_st_wait();
-            warp_arrive(&p_full[h]);
+            warp_arrive(&p_full[u]);
         }
-        // O epilogue: this thread owns TMEM lane m = (row, head) of O_h, columns 64 s .. 64 s + 63
-        // warp-uniform decision: the tensor-memory loads below are warp-collective
+        // O epilogue: 4 warps per lane quarter; this thread owns TMEM lane m = (row, head)
+        // and columns 32 cc .. 32 cc + 31
         if (__all_sync(0xffffffffu, wait_or_abort(&o_full, 0, &abort_flag, a.status))) {
             umma::fence_after();
             const int m = quarter * 32 + lane;
-            const int orow_i = r0 + h * HALF_ROWS + (m >> 4);
-            __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + orow_i) * H + (m & 15)) * D + 64 * s;
-            const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-#pragma unroll 1
-            for (int c = 0; c < 64; c += 32) {
-                uint32_t r[32];
-                umma::tmem_ld32(tmem + lane_base + kOcol + h * 128 + 64 * s + c, r);
-                umma::tmem_ld_wait();
-                if (orow_i < a.n_q) {
+            const int cc = sw >> 2;
+            const int orow_i = r0 + (m >> 4);
+            uint32_t r[32];
+            umma::tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + kOcol + 32 * cc, r);
+            umma::tmem_ld_wait();
+            if (orow_i < a.n_q) {
+                __nv_bfloat16* orow = a.o + ((static_cast<size_t>(b) * a.n_q + orow_i) * H + (m & 15)) * D + 32 * cc;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 8) {
-                        uint4 w;
-                        w.x = pack_bf16(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
-                        w.y = pack_bf16(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-                        w.z = pack_bf16(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
-                        w.w = pack_bf16(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
-                        *reinterpret_cast<uint4*>(orow + c + j) = w;
-                    }
+                for (int j = 0; j < 32; j += 8) {
+                    uint4 w;
+                    w.x = pack_bf16(__uint_as_float(r[j]), __uint_as_float(r[j + 1]));
+                    w.y = pack_bf16(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                    w.z = pack_bf16(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+                    w.w = pack_bf16(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+                    *reinterpret_cast<uint4*>(orow + j) = w;
                 }
             }
         }
@@ -567,7 +622,7 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
         !make_tmap_2d(&vmap, pa.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, kv_rows, D * 2, 64, KT, true))
         return cudaErrorInvalidValue;
     Params a{};
-    a.B = pa.batch; a.n_q = pa.n_q; a.cap = pa.cap; a.max_ctx = pa.max_ctx; a.q_pos0 = pa.q_pos0;
+    a.B = pa.batch; a.n_q = pa.n_q; a.cap = pa.cap; a.max_ctx = pa.max_ctx; a.q_pos0 = pa.q_pos0; a.q = pa.q;
     a.sc2 = pa.scale * kLog2e;
     a.lse2 = static_cast<float*>(pa.ws);
     a.lse_user = pa.lse;
@@ -575,14 +630,15 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     a.o = static_cast<__nv_bfloat16*>(pa.o);
     a.status = pa.status;
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
+    const int blocks2 = pa.batch * ((pa.n_q + ROWS2 - 1) / ROWS2);
     const size_t s1 = 1024 + 2 * TILE_BYTES + P1_STAGES * TILE_BYTES;
-    const size_t s2 = 1024 + 2 * TILE_BYTES + 2 * P2_STAGES * TILE_BYTES;
+    const size_t s2 = 1024 + 2 * P2S * TILE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(prefill_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(prefill_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));
     if (e != cudaSuccess) return e;
     prefill_lse_kernel<<<blocks, NT, s1, st>>>(qmap, kmap, a);
-    prefill_out_kernel<<<blocks, NT, s2, st>>>(qmap, kmap, vmap, a);
+    prefill_out_kernel<<<blocks2, NT, s2, st>>>(qmap, kmap, vmap, a);
     return cudaGetLastError();
 }
 
