@@ -34,9 +34,9 @@ import synth  # noqa: E402
 METRIC = "sparse-attn decode queries/s @128K ctx + prefill tokens/s; % HBM & TC roofline"
 FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum of one hs2_full_attn_select call on the
-# decode workload: 664.4 MB measured at 32768 keys per sequence (ncu capture summarised in
+# decode workload: 665.4 MB measured at 32768 keys per sequence (ncu capture summarised in
 # profiles/decode_kernels_b32_ctx32768.md), times 4 for 131072 keys (linear in keys).
-FULL_CALL_TRAFFIC_BYTES = 4 * 664.4e6
+FULL_CALL_TRAFFIC_BYTES = 4 * 665.4e6
 
 
 def _peaks():
@@ -444,32 +444,41 @@ def _oracle_block(wl, inp, b):
         oracle.sparse_attn(inp.q_sparse[l][b].double().numpy(), k, v, idx, cnt)
 
 
-def cpu_baseline(wl, seed, sample_seqs):
-    """The CPU oracle, as it stands, on a bounded sample of the same workload."""
+def cpu_baseline(wl, seed, sample_seqs, min_seconds=10.0):
+    """The CPU oracle, as it stands, on a bounded sample of the same workload: the sample
+    is run again until at least min_seconds of CPU time have been measured."""
     from concurrent.futures import ThreadPoolExecutor
     sub = synth.shrink(wl, batch=sample_seqs)
     inp = synth.make_inputs(sub, seed=seed, device="cuda")
     inp.q_full, inp.k, inp.v = inp.q_full.cpu(), inp.k.cpu(), inp.v.cpu()
     inp.q_sparse = [x.cpu() for x in inp.q_sparse]
     cores = min(sample_seqs, os.cpu_count() or 1)
-    t0 = time.perf_counter()
+    reps, dt = 0, 0.0
     with ThreadPoolExecutor(max_workers=cores) as ex:
-        list(ex.map(lambda b: _oracle_block(sub, inp, b), range(sample_seqs)))
-    dt = time.perf_counter() - t0
-    return {"value": sample_seqs * wl.n_sparse / dt, "unit": "sparse-attn queries/s", "cores": cores,
+        while reps == 0 or (dt < min_seconds and reps < 100):
+            t0 = time.perf_counter()
+            list(ex.map(lambda b: _oracle_block(sub, inp, b), range(sample_seqs)))
+            dt += time.perf_counter() - t0
+            reps += 1
+    return {"value": reps * sample_seqs * wl.n_sparse / dt, "unit": "sparse-attn queries/s", "cores": cores,
             "kind": "oracle", "seconds": dt,
             "sample": f"{sample_seqs} of the {wl.batch} sequences of {wl.name}, whole hybrid block "
-                      f"(full attention + selection + {wl.n_sparse} sparse layers), fp64, one thread per sequence"}
+                      f"(full attention + selection + {wl.n_sparse} sparse layers), fp64, one thread per "
+                      f"sequence, run {reps} times ({dt:.1f} s)"}
 
 
 def run_reference(args, ws_, rank):
     """Reference arm: the CPU oracle timed on the host, each step a bounded sample."""
     wl = synth.DECODE_128K
-    sample = args.cpu_sample
+    # per-step sample sized so that the whole run stays within a few minutes (a 16-sequence
+    # sample takes about a second on 16 host threads)
+    sample = max(1, min(args.cpu_sample, (16 * 150) // max(1, args.steps + args.warmup)))
+    for _ in range(min(args.warmup, 1)):
+        cpu_baseline(wl, seed=1002, sample_seqs=sample, min_seconds=0.0)
     times = []
     res = None
     for _ in range(args.steps):
-        res = cpu_baseline(wl, seed=1002, sample_seqs=sample)
+        res = cpu_baseline(wl, seed=1002, sample_seqs=sample, min_seconds=0.0)
         times.append(res["seconds"])
     per_step = statistics.mean(times)
     value = sample * wl.n_sparse / per_step

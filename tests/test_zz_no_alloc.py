@@ -52,7 +52,9 @@ def _case(batch, n_q, kv, seed, T=4000):
 
 
 @pytest.mark.parametrize("kv", ["bf16", "e4m3"])
-@pytest.mark.parametrize("shape", [(32, 1), (3, 1), (2, 200)])
+# (32, 1), (3, 1): one CTA cluster per row (no split partials); (1, 200): rows split in two,
+# partials and counters in the fixed array; (2, 200): one CTA per row
+@pytest.mark.parametrize("shape", [(32, 1), (3, 1), (1, 200), (2, 200)])
 def test_noalloc_matches_workspace_entry_point_twice(kv, shape):
     batch, n_q = shape
     ws = None
