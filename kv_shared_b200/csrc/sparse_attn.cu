@@ -408,30 +408,22 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
     sparse::State st;
     attend_warp_tile(kt, vt, qs, ok, fk, fv, a.sc2, st, lane);
 
-    // ---- fold the warps: per-head CTA max; each warp writes its rescaled O to its own
-    // padded slab (the gather area is free once every warp has computed)
+    // ---- fold the warps into the push: each warp writes its own (max, sum) and its O
+    // (relative to its own max) to a padded slab in the gather area (free once every
+    // warp has computed: the barrier below); the push then weights and sums the slabs.
     if (t == 0) {
         wm[warp][g] = st.m2[0]; wl[warp][g] = st.l2[0];
         wm[warp][g + 8] = st.m2[1]; wl[warp][g + 8] = st.l2[1];
     }
-    __syncthreads();
-    float f[2];
-#pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-        const int h = g + 8 * hh;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kCW; ++w) M = fmaxf(M, wm[w][h]);
-        f[hh] = (st.m2[hh] == -INFINITY) ? 0.f : ex2(st.m2[hh] - M);
-    }
     constexpr int RP = sparse::RP;
     float* slabs = reinterpret_cast<float*>(csm);
+    __syncthreads();                                     // every warp is done with the gather area
     float* slab = slabs + warp * H * RP;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
         const int d = 8 * n + 2 * t;
-        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(st.o[n][0] * f[0], st.o[n][1] * f[0]);
-        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(st.o[n][2] * f[1], st.o[n][3] * f[1]);
+        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(st.o[n][0], st.o[n][1]);
+        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(st.o[n][2], st.o[n][3]);
     }
     if (tid < H) {
         float M = -INFINITY;
@@ -443,14 +435,20 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
     }
     __syncthreads();
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    // ---- push heads 2p, 2p + 1 of this CTA's partial (the slab sum) to CTA p
+    // ---- push heads 2p, 2p + 1 of this CTA's partial (weighted slab sum) to CTA p
     for (int i = tid; i < H * D / 4; i += kCNT) {
         const int h = (4 * i) / D, d = (4 * i) % D;
-        float4 v = *reinterpret_cast<const float4*>(slabs + h * RP + d);
+        const float M = cmx[h];
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (M != -INFINITY) {
 #pragma unroll
-        for (int w = 1; w < kCW; ++w) {
-            const float4 u = *reinterpret_cast<const float4*>(slabs + w * H * RP + h * RP + d);
-            v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+            for (int w = 0; w < kCW; ++w) {
+                const float mw = wm[w][h];
+                if (mw == -INFINITY) continue;
+                const float wt = ex2(mw - M);
+                const float4 u = *reinterpret_cast<const float4*>(slabs + w * H * RP + h * RP + d);
+                v.x += wt * u.x; v.y += wt * u.y; v.z += wt * u.z; v.w += wt * u.w;
+            }
         }
         float* dst = cluster.map_shared_rank(recv_o, h >> 1) + (rank * 2 + (h & 1)) * D + d;
         *reinterpret_cast<float4*>(dst) = v;
