@@ -397,7 +397,8 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
 // thread's MMAs in issue order, so PV(i) has read P before S overwrites it, and the
 // softmax writes P(i + 2) only after S(i + 2) has completed, hence after PV(i).
 constexpr int ROWS2 = 8;
-constexpr int P2S = 3;                          // K and V stages of pass 2
+constexpr int KS2 = 4;                          // K stages of pass 2
+constexpr int VS2 = 3;                          // V stages of pass 2
 constexpr int NSB2 = 2;                         // S/P buffers at columns 0, 128
 constexpr uint32_t kQcol = 256;                 // Q (packed bf16 pairs) at columns 256 .. 319
 constexpr uint32_t kOcol = 384;                 // O at columns 384 .. 511
@@ -408,8 +409,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* kst = smem;                                      // K stages
-    uint8_t* vst = kst + P2S * TILE_BYTES;                    // V stages
-    __shared__ uint64_t k_full[P2S], k_empty[P2S], v_full[P2S], v_empty[P2S];
+    uint8_t* vst = kst + KS2 * TILE_BYTES;                    // V stages
+    __shared__ uint64_t k_full[KS2], k_empty[KS2], v_full[VS2], v_empty[VS2];
     __shared__ uint64_t s_full[NSB2], p_full[NSB2], q_tm, o_full;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
@@ -426,10 +427,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     if (threadIdx.x == 0) {
         prefetch_tmap(&kmap);
         prefetch_tmap(&vmap);
-        for (int s = 0; s < P2S; ++s) {
-            mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1);
-            mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1);
-        }
+        for (int s = 0; s < KS2; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+        for (int s = 0; s < VS2; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
         for (int u = 0; u < NSB2; ++u) { mbar_init(&s_full[u], 1); mbar_init(&p_full[u], 16); }
         mbar_init(&q_tm, 16);
         mbar_init(&o_full, 1);
@@ -447,16 +446,16 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             // K runs one tile ahead of V: K(t) is needed by S(t), V(t) only after P(t)
             for (int t = 0; t <= n_kt; ++t) {
                 if (t < n_kt) {
-                    const int s = t % P2S;
-                    if (t >= P2S && !wait_or_abort(&k_empty[s], ((t / P2S) - 1) & 1, &abort_flag, a.status)) break;
+                    const int s = t % KS2;
+                    if (t >= KS2 && !wait_or_abort(&k_empty[s], ((t / KS2) - 1) & 1, &abort_flag, a.status)) break;
                     const int krow = static_cast<int>(b * a.cap) + t * KT;
                     mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
                     tma_load_2d(kst + s * TILE_BYTES, &kmap, &k_full[s], 0, krow);
                     tma_load_2d(kst + s * TILE_BYTES + BOX_BYTES, &kmap, &k_full[s], 64, krow);
                 }
                 if (t >= 1) {
-                    const int j = t - 1, s = j % P2S;
-                    if (j >= P2S && !wait_or_abort(&v_empty[s], ((j / P2S) - 1) & 1, &abort_flag, a.status)) break;
+                    const int j = t - 1, s = j % VS2;
+                    if (j >= VS2 && !wait_or_abort(&v_empty[s], ((j / VS2) - 1) & 1, &abort_flag, a.status)) break;
                     const int vrow = static_cast<int>(b * a.cap) + j * KT;
                     mbar_arrive_expect_tx(&v_full[s], TILE_BYTES);
                     tma_load_2d(vst + s * TILE_BYTES, &vmap, &v_full[s], 0, vrow);
@@ -469,7 +468,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             constexpr uint32_t idesc_s = umma::idesc_bf16(128, 128, false, false);
             constexpr uint32_t idesc_o = umma::idesc_bf16(128, 128, false, true);
             auto issue_s = [&](int t) {                 // S(t) = Q K(t)^T into buffer t % NSB2, Q from tensor memory
-                const int s = t % P2S;
+                const int s = t % KS2;
                 const uint32_t kb = smem_u32(kst + s * TILE_BYTES);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk)
@@ -480,16 +479,16 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             };
             bool ok = spin_or_abort(&q_tm, 0, &abort_flag, a.status);
             for (int t = 0; ok && t < NSB2 && t < n_kt; ++t) {
-                if (!(ok = spin_or_abort(&k_full[t % P2S], (t / P2S) & 1, &abort_flag, a.status))) break;
+                if (!(ok = spin_or_abort(&k_full[t % KS2], (t / KS2) & 1, &abort_flag, a.status))) break;
                 umma::fence_after();
                 issue_s(t);
             }
             for (int i = 0; ok && i < n_kt; ++i) {
                 // O += P(i) V(i); P(i) sits in the first 32 columns of each 64-column half of
                 // buffer i % NSB2 (keys 0..63, then 64..127)
-                const int vs = i % P2S, u = i % NSB2;
+                const int vs = i % VS2, u = i % NSB2;
                 if (!(ok = spin_or_abort(&p_full[u], (i / NSB2) & 1, &abort_flag, a.status))) break;
-                if (!(ok = spin_or_abort(&v_full[vs], (i / P2S) & 1, &abort_flag, a.status))) break;
+                if (!(ok = spin_or_abort(&v_full[vs], (i / VS2) & 1, &abort_flag, a.status))) break;
                 umma::fence_after();
                 const uint32_t vb = smem_u32(vst + vs * TILE_BYTES);
 #pragma unroll
@@ -499,7 +498,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
                 umma::commit(&v_empty[vs]);
                 // S(i + 2) into the same buffer, after PV(i) in issue order
                 if (i + NSB2 < n_kt) {
-                    if (!(ok = spin_or_abort(&k_full[(i + NSB2) % P2S], ((i + NSB2) / P2S) & 1, &abort_flag, a.status)))
+                    if (!(ok = spin_or_abort(&k_full[(i + NSB2) % KS2], ((i + NSB2) / KS2) & 1, &abort_flag, a.status)))
                         break;
                     umma::fence_after();
                     issue_s(i + NSB2);
@@ -557,8 +556,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             // (the K rows only feed probabilities that are forced to 0); no early exit, so
             // that every lane reaches the warp's arrival
             if (i == n_kt - 1 && vt < KT && i * KT + vt > p_max &&
-                wait_or_abort(&v_full[i % P2S], (i / P2S) & 1, &abort_flag, a.status)) {
-                uint8_t* vrow = vst + (i % P2S) * TILE_BYTES + vt * 128;
+                wait_or_abort(&v_full[i % VS2], (i / VS2) & 1, &abort_flag, a.status)) {
+                uint8_t* vrow = vst + (i % VS2) * TILE_BYTES + vt * 128;
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     *reinterpret_cast<uint4*>(vrow + c * 16) = make_uint4(0, 0, 0, 0);
@@ -632,7 +631,7 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
     const int blocks2 = pa.batch * ((pa.n_q + ROWS2 - 1) / ROWS2);
     const size_t s1 = 1024 + 2 * TILE_BYTES + P1_STAGES * TILE_BYTES;
-    const size_t s2 = 1024 + 2 * P2S * TILE_BYTES;
+    const size_t s2 = 1024 + (KS2 + VS2) * TILE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(prefill_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(prefill_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));
