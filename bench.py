@@ -34,9 +34,8 @@ import synth  # noqa: E402
 METRIC = "sparse-attn decode queries/s @128K ctx + prefill tokens/s; % HBM & TC roofline"
 FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum of one hs2_full_attn_select call on the
-# decode workload: 665.4 MB measured at 32768 keys per sequence (ncu capture summarised in
-# profiles/decode_kernels_b32_ctx32768.md), times 4 for 131072 keys (linear in keys).
-FULL_CALL_TRAFFIC_BYTES = 4 * 665.4e6
+# decode workload, from an ncu capture of the current kernels (None until one is taken).
+FULL_CALL_TRAFFIC_BYTES = None
 
 
 def _peaks():
@@ -154,7 +153,8 @@ class DecodeBlock:
         self.o_sp = [torch.empty_like(self.q) for _ in self.qs]
         self.idx = torch.empty(B, 1, self.desc.idx_stride, dtype=torch.int32, device="cuda")
         self.cnt = torch.empty(B, 1, dtype=torch.int32, device="cuda")
-        self.launches_per_step = 3 + len(self.qs)       # qk, pv, select, one per sparse layer
+        # attention kernel(s) + select, one per sparse layer
+        self.launches_per_step = hs.hs2_full_attn_launches(self.desc) + len(self.qs)
 
     def full(self):
         self.hs.hs2_full_attn_select(self.desc, self.q, self.k, self.v, None, None, self.q_pos0, self.o,
@@ -204,7 +204,8 @@ class PrefillBlock:
         self.o_sp = [torch.empty_like(self.q) for _ in self.qs]
         self.idx = torch.empty(B, wl.n_q, self.desc.idx_stride, dtype=torch.int32, device="cuda")
         self.cnt = torch.empty(B, wl.n_q, dtype=torch.int32, device="cuda")
-        self.launches_per_step = 1 + 3 + len(self.qs)   # bridge, lse, out, select, sparse layers
+        # bridge, attention kernels + select, one per sparse layer
+        self.launches_per_step = 1 + hs.hs2_full_attn_launches(self.desc) + len(self.qs)
 
     def bridge(self):
         wl = self.wl
@@ -414,7 +415,7 @@ def run_ours(args, ws_, rank, local):
         },
         "roofline": {"bound": "hbm", "achieved": full_gbs, "peak": hbm, "unit": "GB/s",
                      "frac": full_gbs / hbm, "peak_source": peak_kind,
-                     "kernel": "hs2_full_attn_select (decode: QK pass, PV+importance pass, select)",
+                     "kernel": "hs2_full_attn_select (decode: fused QK / PV+importance pass, select)",
                      "traffic": FULL_CALL_TRAFFIC_BYTES},
         "e2e": {"value": e2e_value, "unit": "sparse-attn queries/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

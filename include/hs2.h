@@ -147,6 +147,14 @@ HS2_API hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q
                                 hs2_stream_t stream);
 
 /*
+ * Number of kernels one hs2_full_attn_select call with `desc` enqueues on its
+ * stream (the attention kernels plus the selection; the count depends on the
+ * shapes and on the current device's SM count).  0 for an invalid description.
+ * Host only: nothing is launched.
+ */
+HS2_API int32_t hs2_full_attn_launches(const hs2_attn_desc* desc);
+
+/*
  * Selection alone, from a caller-given importance array.
  *
  * block_size 1: token level as above ([LB] "Token-Level Sparse Selection").

@@ -18,7 +18,8 @@ HS2_F32, HS2_BF16, HS2_E4M3 = 0, 1, 2
 HS2_OK, HS2_ERR_INVALID_ARG, HS2_ERR_UNSUPPORTED, HS2_ERR_WORKSPACE, HS2_ERR_CUDA, \
     HS2_ERR_TIMEOUT, HS2_ERR_INDEX = range(7)
 
-EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_topk_select",
+EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_full_attn_launches",
+           "hs2_topk_select",
            "hs2_sparse_attn", "hs2_sparse_attn_noalloc", "hs2_kv_bridge_proj", "hs2_kv_quantize_fp8", "hs2_last_status",
            "hs2_status_string")
 
@@ -53,6 +54,7 @@ def lib():
         L.hs2_workspace_size.restype = sz
         L.hs2_workspace_init.argtypes = [vp, vp]
         L.hs2_full_attn_select.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.hs2_full_attn_launches.argtypes = [dp]
         L.hs2_topk_select.argtypes = [dp, vp, i64, vp, i32, vp, vp, vp, sz, vp]
         L.hs2_sparse_attn.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.hs2_sparse_attn_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -101,6 +103,11 @@ def make_desc(batch, n_q, heads, head_dim, window=128, budget=1024, q_dtype=HS2_
 # ------------------------------------------------------------------ C-ABI calls
 def hs2_workspace_size(desc, scores_in_workspace=True):
     return int(lib().hs2_workspace_size(ctypes.byref(desc), int(bool(scores_in_workspace))))
+
+
+def hs2_full_attn_launches(desc):
+    """Kernels one hs2_full_attn_select call with `desc` enqueues (host query)."""
+    return int(lib().hs2_full_attn_launches(ctypes.byref(desc)))
 
 
 def hs2_workspace_init(workspace, stream=None):

@@ -20,6 +20,7 @@
 // (exact) and the per-token scales are folded into the logits and into P.
 #include "common.cuh"
 #include "internal.h"
+#include "tcgen05.cuh"
 
 namespace hs2 {
 namespace {
@@ -421,6 +422,437 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     }
 }
 
+// ------------------------------------------------------------------ fused passes (one launch)
+// When a split's logits fit in tensor memory (64 tiles of 64 keys: 16 heads x 4096 keys of
+// fp32 = 256 KB), both passes run in one cooperative launch and the logits never leave the
+// SM: the 64-byte-per-key round trip through HBM disappears.  One CTA per SM; the sequences
+// are taken in waves of `wb` (CTA = group * splits + split, sequence = wave * wb + group).
+//
+// Warp 8 streams the K tiles then the V tiles of every wave through a ring of TMA stages
+// (full/empty mbarriers); warps 0-3 and 4-7 are two consumer groups taking the even and the
+// odd tiles.  Per wave a CTA runs pass A over its keys with the logits stored to tensor
+// memory (tile i, warp quarter q: lanes 32 q + 16 (i / 32), columns 16 (i % 32); the 16x256b
+// store shape is the mma.sync accumulator layout of the warp's 16 keys), publishes its
+// (max, sum) per head, waits -- bounded -- until every split of the sequence has (the first
+// V tiles are in flight meanwhile), and runs pass B with the logits read back from tensor
+// memory.  Each split leaves its O partial in the workspace and counts itself in (second
+// counter); after its waves every CTA sums the partials of a few (sequence, head) rows, each
+// once its sequence is complete, and the last row of a sequence (third counter) returns the
+// sequence's three counters to zero.
+constexpr int kFusedMaxTiles = 64;
+constexpr int FNT = 288;                       // 2 x 4 consumer warps + 1 producer warp
+constexpr int FCONS = 256;
+constexpr size_t kFusedMinSmem = 120 * 1024;   // more than half an SM: one CTA per SM
+
+template <bool KV8>
+struct FusedLayout {
+    static constexpr int FS = KV8 ? 12 : 8;    // stages of the K/V stream
+    static constexpr size_t BYTES =
+        1024 + FS * Layout<KV8>::RAW + 2 * Layout<KV8>::CVT + 2 * FS * 8 + 8 * H * D * 4;
+};
+
+__device__ __forceinline__ void bar_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Bounded wait until *p >= target; false (status set) on timeout.
+__device__ __forceinline__ bool wait_count(const int* p, int target, uint32_t* status) {
+    const uint64_t t0 = global_ns();
+#pragma unroll 1
+    for (uint32_t i = 0; i < kWaitPolls; ++i) {
+        if (ld_acquire(p) >= target) return true;
+        if ((i & 15) == 15) {
+            if (global_ns() - t0 > kWaitNs) break;
+            __nanosleep(64);
+        }
+    }
+    set_status(status, HS2_ERR_TIMEOUT);
+    return false;
+}
+
+template <bool KV8>
+__global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant__ CUtensorMap kmap,
+                                                           const __grid_constant__ CUtensorMap vmap, Params a,
+                                                           int wb) {
+    using L = Layout<KV8>;
+    constexpr int FS = FusedLayout<KV8>::FS;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = align1024(smem_raw);
+    uint8_t* cvt_base = smem + FS * L::RAW;                           // [2][CVT] (e4m3 only)
+    uint64_t* full = reinterpret_cast<uint64_t*>(cvt_base + 2 * L::CVT);
+    uint64_t* empty = full + FS;
+    float4* red_o4 = reinterpret_cast<float4*>(empty + FS);          // [8][16][32] O partials
+    __shared__ float red_m[8][H], red_l[8][H];
+    __shared__ float2 lse_part[FCONS / H][H];
+    __shared__ float lse_s[H];
+    __shared__ uint32_t tmem_base;
+    __shared__ volatile int s_abort;
+    __shared__ int s_ok[4];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
+    const int group = blockIdx.x / a.splits, split = blockIdx.x % a.splits;
+    const int nw = (a.B - group + wb - 1) / wb;                       // waves with a sequence for this group
+    const int k_begin = split * a.chunk;
+    int* cnt_ml = a.counter;                                          // [B]: splits done with pass A
+    int* cnt_o = a.counter + a.B;                                     // [B]: splits done with pass B
+    int* cnt_m = a.counter + 2 * a.B;                                 // [B]: rows of O merged
+
+    if (warp == 0) umma::tmem_alloc(&tmem_base, 512);
+    if (tid == 32) {
+        prefetch_tmap(&kmap);
+        prefetch_tmap(&vmap);
+        for (int s = 0; s < FS; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 4);
+        }
+        fence_mbar_init();
+        s_abort = 0;
+    }
+    umma::fence_before();
+    __syncthreads();
+    umma::fence_after();
+    const uint32_t tmem = tmem_base;
+
+    auto tiles_of = [&](int w, int& k_end) {
+        const int p = checked_pos(a.q_pos0[w * wb + group], a.max_ctx, a.status);
+        k_end = min(p + 1, k_begin + a.chunk);
+        return k_end > k_begin ? (k_end - k_begin + TILE - 1) / TILE : 0;
+    };
+
+    if (warp == 8) {
+        // ---------------- producer: K tiles then V tiles of each wave, one TMA stream
+        if (lane == 0) {
+            uint32_t n_issued = 0;
+            bool run = true;
+            for (int w = 0; w < nw && run; ++w) {
+                int k_end;
+                const int n = tiles_of(w, k_end);
+                const int row0 = static_cast<int>((w * wb + group) * a.cap) + k_begin;
+                for (int j = 0; j < 2 * n; ++j) {
+                    const uint32_t ld = n_issued;
+                    const int s = ld % FS;
+                    if (ld >= FS && !mbar_wait(&empty[s], ((ld / FS) & 1u) ^ 1u, a.status)) s_abort = 1;
+                    if (s_abort) {
+                        run = false;
+                        break;
+                    }
+                    const bool is_v = j >= n;
+                    const int row = row0 + (is_v ? j - n : j) * TILE;
+                    const CUtensorMap* m = is_v ? &vmap : &kmap;
+                    uint8_t* dst = smem + s * L::RAW;
+                    mbar_arrive_expect_tx(&full[s], L::RAW);
+                    tma_load_2d(dst, m, &full[s], 0, row);
+                    if (!KV8) tma_load_2d(dst + TILE * 128, m, &full[s], 64, row);
+                    ++n_issued;
+                }
+            }
+            // after an abort, let the copies in flight land before the CTA exits (bounded)
+            if (!run)
+                for (uint32_t ld = n_issued > FS ? n_issued - FS : 0; ld < n_issued; ++ld)
+                    mbar_wait(&full[ld % FS], (ld / FS) & 1u, nullptr, 100000000ull);
+        }
+        __syncwarp();
+    } else {
+        // ---------------- consumers: group c takes tiles c, c + 2, ...; q = warp quarter
+        const int c = warp >> 2, q = warp & 3, gtid = tid & 127;
+        uint8_t* cvt = cvt_base + c * L::CVT;
+        auto take = [&](uint32_t ld) -> bool {    // warp-uniform; false once the CTA aborts
+            if (__any_sync(0xffffffffu, s_abort != 0)) return false;
+            const bool okw = __all_sync(0xffffffffu, mbar_wait(&full[ld % FS], (ld / FS) & 1u, a.status));
+            if (!okw && lane == 0) s_abort = 1;
+            return okw;
+        };
+        auto release = [&](uint32_t ld) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[ld % FS]);
+        };
+        uint32_t wbase = 0;                       // loads of the earlier waves
+        for (int w = 0; w < nw; ++w) {
+            const int b = w * wb + group;
+            int k_end;
+            const int n_tiles = tiles_of(w, k_end);
+
+            // ---- pass A: logits to tensor memory, running (max, sum) per head
+            uint32_t qa[8][4];
+            load_q_frags(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
+            float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
+            const float* ksc = KV8 ? a.k_scale + b * a.cap : nullptr;
+            for (int i = c; i < n_tiles; i += 2) {
+                const uint32_t ld = wbase + i;
+                const bool okt = take(ld);
+                const int tile_key0 = k_begin + i * TILE;
+                const uint8_t* tile = smem + (ld % FS) * L::RAW;
+                if (KV8) {
+                    if (okt) convert_tile(tile, cvt, tile_key0, k_end - 1, gtid);
+                    bar_sync(1 + c, 128);
+                    tile = cvt;
+                }
+                if (okt) {
+                    const uint32_t tbase = smem_u32(tile);
+                    float acc[2][4];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+                        const int r = q * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4(tbase + swz_off<TILE>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+                            mma_bf16(acc[nt], qa[2 * kk], b0, b1);
+                            mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+                        }
+                    }
+                    const int key0 = tile_key0 + q * 16 + 2 * t;
+                    float mx[2] = {-INFINITY, -INFINITY};
+                    uint32_t sv[8];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        const int key = key0 + nt * 8;
+                        float f0 = a.sc2, f1 = a.sc2;
+                        if (KV8) {
+                            f0 *= (key < k_end) ? ksc[key] : 0.f;
+                            f1 *= (key + 1 < k_end) ? ksc[key + 1] : 0.f;
+                        }
+                        acc[nt][0] = (key < k_end) ? acc[nt][0] * f0 : -INFINITY;
+                        acc[nt][1] = (key + 1 < k_end) ? acc[nt][1] * f1 : -INFINITY;
+                        acc[nt][2] = (key < k_end) ? acc[nt][2] * f0 : -INFINITY;
+                        acc[nt][3] = (key + 1 < k_end) ? acc[nt][3] * f1 : -INFINITY;
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sv[4 * nt + e] = __float_as_uint(acc[nt][e]);
+                        mx[0] = fmaxf(mx[0], fmaxf(acc[nt][0], acc[nt][1]));
+                        mx[1] = fmaxf(mx[1], fmaxf(acc[nt][2], acc[nt][3]));
+                    }
+                    umma::tmem_st16x256_x2(
+                        tmem + (static_cast<uint32_t>(32 * q + 16 * (i >> 5)) << 16) + 16 * (i & 31), sv);
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const float mn = fmaxf(m2[hh], mx[hh]);
+                        if (mn != -INFINITY) {
+                            float sum = l2[hh] * ex2(m2[hh] - mn);
+#pragma unroll
+                            for (int nt = 0; nt < 2; ++nt)
+                                sum += ex2(acc[nt][2 * hh] - mn) + ex2(acc[nt][2 * hh + 1] - mn);
+                            l2[hh] = sum;
+                            m2[hh] = mn;
+                        }
+                    }
+                }
+                if (KV8) bar_sync(1 + c, 128);    // the group's converted tile is reused next
+                release(ld);
+            }
+            umma::tmem_st_wait();
+            // ---- exchange: publish this split's (max, sum), wait for the other splits
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+                for (int off = 1; off <= 2; off <<= 1) {
+                    const float om = __shfl_xor_sync(0xffffffffu, m2[hh], off);
+                    const float ol = __shfl_xor_sync(0xffffffffu, l2[hh], off);
+                    merge_ml(m2[hh], l2[hh], om, ol);
+                }
+            }
+            if (t == 0) {
+                red_m[warp][g] = m2[0]; red_l[warp][g] = l2[0];
+                red_m[warp][g + 8] = m2[1]; red_l[warp][g + 8] = l2[1];
+            }
+            bar_sync(3, FCONS);
+            if (tid < H) {
+                float m = red_m[0][tid], l = red_l[0][tid];
+                for (int k = 1; k < 8; ++k) merge_ml(m, l, red_m[k][tid], red_l[k][tid]);
+                a.part_ml[(static_cast<size_t>(b) * a.splits + split) * H + tid] = make_float2(m, l);
+                __threadfence();
+            }
+            bar_sync(3, FCONS);
+            if (tid == 0) {
+                bool arrived = false;
+                if (!s_abort) {
+                    atomicAdd(&cnt_ml[b], 1);
+                    arrived = wait_count(&cnt_ml[b], a.splits, a.status);
+                    __threadfence();
+                }
+                if (!arrived) s_abort = 1;
+            }
+            bar_sync(3, FCONS);
+            {
+                const int h = tid & (H - 1), grp = tid >> 4;
+                float m = -INFINITY, l = 0.f;
+                const float2* pml = a.part_ml + static_cast<size_t>(b) * a.splits * H;
+                if (!s_abort)
+                    for (int s = grp; s < a.splits; s += FCONS / H) {
+                        const float2 ml = __ldcg(pml + s * H + h);
+                        merge_ml(m, l, ml.x, ml.y);
+                    }
+                lse_part[grp][h] = make_float2(m, l);
+                bar_sync(3, FCONS);
+                if (tid < H) {
+                    float mm = -INFINITY, ll = 0.f;
+                    for (int k = 0; k < FCONS / H; ++k) merge_ml(mm, ll, lse_part[k][tid].x, lse_part[k][tid].y);
+                    lse_s[tid] = mm + log2f(ll);
+                    if (split == 0 && a.lse && !s_abort) a.lse[static_cast<size_t>(b) * H + tid] = lse_s[tid] * kLn2;
+                }
+                bar_sync(3, FCONS);
+            }
+            const float lse2[2] = {lse_s[g], lse_s[g + 8]};
+
+            // ---- pass B: P from the logits in tensor memory, importance, O = P V
+            float o[16][4];
+#pragma unroll
+            for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
+            float* score_row = a.scores + b * a.score_ld;
+            for (int i = c; i < n_tiles; i += 2) {
+                const uint32_t ld = wbase + n_tiles + i;
+                uint32_t sr[8];
+                umma::tmem_ld16x256_x2(tmem + (static_cast<uint32_t>(32 * q + 16 * (i >> 5)) << 16) + 16 * (i & 31),
+                                       sr);
+                const bool okt = take(ld);
+                const int tile_key0 = k_begin + i * TILE;
+                uint8_t* vt = smem + (ld % FS) * L::RAW;
+                if (KV8) {
+                    if (okt) convert_tile(vt, cvt, tile_key0, k_end - 1, gtid);
+                    bar_sync(1 + c, 128);
+                    vt = cvt;
+                } else if (tile_key0 + TILE > k_end) {
+                    // tail tile: zero the V rows past the last key (0 * NaN would poison O); the
+                    // stage is refilled by TMA later, so order these writes before the async proxy
+                    if (okt)
+                        for (int it = gtid; it < TILE * 16; it += 128) {
+                            const int r = it >> 4, cc = it & 15;
+                            if (tile_key0 + r >= k_end)
+                                *reinterpret_cast<uint4*>(vt + swz_off<TILE>(r, cc)) = make_uint4(0, 0, 0, 0);
+                        }
+                    umma::fence_proxy_async();
+                    bar_sync(1 + c, 128);
+                }
+                umma::tmem_ld_wait();
+                if (okt) {
+                    const float2 sgl = make_float2(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
+                    const float2 sg8l = make_float2(__uint_as_float(sr[2]), __uint_as_float(sr[3]));
+                    const float2 sgh = make_float2(__uint_as_float(sr[4]), __uint_as_float(sr[5]));
+                    const float2 sg8h = make_float2(__uint_as_float(sr[6]), __uint_as_float(sr[7]));
+                    const int kl = tile_key0 + q * 16 + 2 * t, kh = kl + 8;
+                    const bool v0 = kl < k_end, v1 = kl + 1 < k_end, v2 = kh < k_end, v3 = kh + 1 < k_end;
+                    const float p00 = v0 ? ex2(sgl.x - lse2[0]) : 0.f, p01 = v1 ? ex2(sgl.y - lse2[0]) : 0.f;
+                    const float p10 = v0 ? ex2(sg8l.x - lse2[1]) : 0.f, p11 = v1 ? ex2(sg8l.y - lse2[1]) : 0.f;
+                    const float p02 = v2 ? ex2(sgh.x - lse2[0]) : 0.f, p03 = v3 ? ex2(sgh.y - lse2[0]) : 0.f;
+                    const float p12 = v2 ? ex2(sg8h.x - lse2[1]) : 0.f, p13 = v3 ? ex2(sg8h.y - lse2[1]) : 0.f;
+                    float sc[4] = {p00 + p10, p01 + p11, p02 + p12, p03 + p13};
+#pragma unroll
+                    for (int off = 4; off <= 16; off <<= 1)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) sc[e] += __shfl_xor_sync(0xffffffffu, sc[e], off);
+                    if (g == 0) {
+                        if (v0) score_row[kl] = sc[0];
+                        if (v1) score_row[kl + 1] = sc[1];
+                        if (v2) score_row[kh] = sc[2];
+                        if (v3) score_row[kh + 1] = sc[3];
+                    }
+                    float f0 = 1.f, f1 = 1.f, f2 = 1.f, f3 = 1.f;
+                    if (KV8) {
+                        f0 = v0 ? vsc[kl] : 0.f; f1 = v1 ? vsc[kl + 1] : 0.f;
+                        f2 = v2 ? vsc[kh] : 0.f; f3 = v3 ? vsc[kh + 1] : 0.f;
+                    }
+                    uint32_t pa[4];
+                    pa[0] = pack_bf16(p00 * f0, p01 * f1);
+                    pa[1] = pack_bf16(p10 * f0, p11 * f1);
+                    pa[2] = pack_bf16(p02 * f2, p03 * f3);
+                    pa[3] = pack_bf16(p12 * f2, p13 * f3);
+                    const uint32_t vbase = smem_u32(vt);
+                    const int vr = q * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+                    for (int cv = 0; cv < 8; ++cv) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(vbase + swz_off<TILE>(vr, 2 * cv + (lane >> 4)), b0, b1, b2, b3);
+                        mma_bf16(o[2 * cv], pa, b0, b1);
+                        mma_bf16(o[2 * cv + 1], pa, b2, b3);
+                    }
+                }
+                if (KV8) bar_sync(1 + c, 128);
+                release(ld);
+            }
+
+            // ---- this split's O partial: the 8 warps' accumulators go to shared memory as
+            // [warp][n][lane] float4 (conflict-free), then each (n, lane) slot is summed over the
+            // warps in a fixed order; the last split of the sequence merges the partials at the end
+#pragma unroll
+            for (int n = 0; n < 16; ++n)
+                red_o4[(warp * 16 + n) * 32 + lane] = make_float4(o[n][0], o[n][1], o[n][2], o[n][3]);
+            bar_sync(3, FCONS);
+            float* my = a.part_o + (static_cast<size_t>(b) * a.splits + split) * H * D;
+#pragma unroll
+            for (int k = 0; k < 512 / FCONS; ++k) {
+                const int e = tid + k * FCONS, n = e >> 5, ln = e & 31;
+                float4 sum = red_o4[e];
+#pragma unroll
+                for (int w8 = 1; w8 < 8; ++w8) {
+                    const float4 v = red_o4[w8 * 512 + e];
+                    sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
+                }
+                const int d = 8 * n + 2 * (ln & 3), h = ln >> 2;
+                *reinterpret_cast<float2*>(my + h * D + d) = make_float2(sum.x, sum.y);
+                *reinterpret_cast<float2*>(my + (h + 8) * D + d) = make_float2(sum.z, sum.w);
+            }
+            bar_sync(3, FCONS);
+            if (tid == 0 && !s_abort) {
+                __threadfence();                  // the CTA's partial, ordered by the barrier
+                atomicAdd(&cnt_o[b], 1);
+            }
+            wbase += 2 * n_tiles;
+        }
+
+        // ---- O = sum of the split partials, spread over all CTAs: rows (sequence, head) in
+        // sequence order, four per pass (64 threads each: 32 float4 columns x 2 split lanes)
+        const int k4 = tid >> 6, c4 = tid & 31, sl = (tid >> 5) & 1;
+        for (int base = blockIdx.x; base < a.B * H; base += 4 * gridDim.x) {
+            const int item = base + k4 * gridDim.x;
+            const bool have = item < a.B * H;
+            const int b = have ? item / H : 0, h = item % H;
+            bar_sync(3, FCONS);               // s_ok and red_o4 of the previous pass are free
+            if ((tid & 63) == 0) s_ok[k4] = (have && !s_abort) ? wait_count(&cnt_o[b], a.splits, a.status) : 0;
+            bar_sync(3, FCONS);
+            const bool go = have && s_ok[k4] != 0;
+            if (have && !go) s_abort = 1;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (go) {
+                const float4* src =
+                    reinterpret_cast<const float4*>(a.part_o + static_cast<size_t>(b) * a.splits * H * D + h * D) + c4;
+#pragma unroll 4
+                for (int sp = sl; sp < a.splits; sp += 2) {
+                    const float4 v = __ldcg(src + static_cast<size_t>(sp) * (H * D / 4));
+                    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+                }
+            }
+            if (sl == 1) red_o4[k4 * 32 + c4] = acc;
+            bar_sync(3, FCONS);
+            if (go && sl == 0) {
+                const float4 v = red_o4[k4 * 32 + c4];
+                uint2 packed;
+                packed.x = pack_bf16(acc.x + v.x, acc.y + v.y);
+                packed.y = pack_bf16(acc.z + v.z, acc.w + v.w);
+                *reinterpret_cast<uint2*>(a.o + (static_cast<size_t>(b) * H + h) * D + 4 * c4) = packed;
+                // the last of the 16 rows of b returns the sequence's counters to zero (every
+                // row's CTA has passed its wait on cnt_o by then)
+                if (c4 == 0 && atomicAdd(&cnt_m[b], 1) == H - 1) {
+                    cnt_ml[b] = 0;
+                    cnt_o[b] = 0;
+                    cnt_m[b] = 0;
+                }
+            }
+        }
+    }
+    umma::fence_before();
+    __syncthreads();
+    umma::fence_after();
+    if (warp == 0) umma::tmem_dealloc(tmem, 512);
+}
+
 template <bool KV8>
 size_t smem_a() { return 1024 + STAGES * Layout<KV8>::RAW + Layout<KV8>::CVT + STAGES * 8; }
 template <bool KV8>
@@ -440,13 +872,15 @@ cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
     a.k_scale = da.k_scale; a.v_scale = da.v_scale;
     a.sc2 = da.scale * kLog2e;
     uint8_t* ws = static_cast<uint8_t*>(da.ws);
-    a.S = reinterpret_cast<float*>(ws);
+    a.S = pl.fused ? nullptr : reinterpret_cast<float*>(ws);
     ws += align256(sizeof(float) * da.batch * H * static_cast<size_t>(pl.s_ld));
     a.part_ml = reinterpret_cast<float2*>(ws);
     ws += align256(sizeof(float2) * da.batch * pl.splits * H);
     a.part_o = reinterpret_cast<float*>(ws);
     ws += align256(sizeof(float) * da.batch * pl.splits * H * D);
-    a.counter = reinterpret_cast<int*>(ws);
+    // two-kernel path: per-sequence semaphores in the workspace, reset by pass A;
+    // fused path: three [B] counters in the status block (zero when idle)
+    a.counter = pl.fused ? reinterpret_cast<int*>(da.status) + kCounterOffsetInts : reinterpret_cast<int*>(ws);
     a.o = static_cast<__nv_bfloat16*>(da.o);
     a.lse = da.lse;
     a.scores = da.scores; a.score_ld = da.score_ld;
@@ -459,6 +893,24 @@ cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
     const uint32_t box_cols = KV8 ? 128 : 64;
     if (!make_tmap_2d(&kmap, da.k, dt, eb, D, rows, D * eb, box_cols, TILE, true)) return cudaErrorInvalidValue;
     if (!make_tmap_2d(&vmap, da.v, dt, eb, D, rows, D * eb, box_cols, TILE, true)) return cudaErrorInvalidValue;
+    if (pl.fused) {
+        size_t sm = FusedLayout<KV8>::BYTES;
+        if (sm < kFusedMinSmem) sm = kFusedMinSmem;
+        cudaError_t e = cudaFuncSetAttribute(dec_fused_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(sm));
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3(pl.wb * pl.splits);
+        cfg.blockDim = dim3(FNT);
+        cfg.dynamicSmemBytes = sm;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;     // all CTAs resident: the splits wait on one another
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, dec_fused_kernel<KV8>, kmap, vmap, a, pl.wb);
+    }
     if (!make_tmap_2d(&smap, a.S, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, pl.s_ld,
                       static_cast<uint64_t>(da.batch) * H, static_cast<uint64_t>(pl.s_ld) * 4, 32, 16, true))
         return cudaErrorInvalidValue;
@@ -478,6 +930,29 @@ cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
 
 DecodePlan plan_decode(int batch, int64_t max_ctx) {
     DecodePlan pl;
+    // fused: enough splits that each fits tensor memory, as many sequences per wave as
+    // the SMs allow, waves balanced, then as many splits as the SMs allow
+    const int sms = num_sms();
+    const int64_t cap_keys = static_cast<int64_t>(kFusedMaxTiles) * TILE;
+    const int64_t min_splits = (max_ctx + cap_keys - 1) / cap_keys;
+    if (batch >= 1 && min_splits <= sms && 3 * batch <= kMaxCounters) {
+        int wb = static_cast<int>(sms / min_splits);
+        if (wb > batch) wb = batch;
+        const int waves = (batch + wb - 1) / wb;
+        {
+            wb = (batch + waves - 1) / waves;
+            int64_t chunk = (max_ctx + sms / wb - 1) / (sms / wb);
+            chunk = (chunk + TILE - 1) / TILE * TILE;
+            pl.fused = true;
+            pl.wb = wb;
+            pl.chunk = static_cast<int>(chunk);
+            pl.splits = static_cast<int>((max_ctx + chunk - 1) / chunk);
+            pl.s_ld = 0;
+            return pl;
+        }
+    }
+    pl.fused = false;
+    pl.wb = 0;
     int splits = (2 * num_sms()) / (batch > 0 ? batch : 1);
     if (splits < 1) splits = 1;
     int64_t chunk = (max_ctx + splits - 1) / splits;

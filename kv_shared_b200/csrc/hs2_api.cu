@@ -197,6 +197,16 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     return from_cuda(launch_select(sa, st));
 }
 
+int32_t hs2_full_attn_launches(const hs2_attn_desc* desc) {
+    Path path;
+    if (check_desc(desc, &path) != HS2_OK) return 0;
+    int32_t n = 1;                                      // the selection
+    if (path == Path::F32) n += 1;
+    else if (desc->n_q > 1) n += 2;                     // prefill: log-sum-exp pass, output pass
+    else n += plan_decode(desc->batch, desc->max_ctx).fused ? 1 : 2;
+    return n;
+}
+
 hs2_status hs2_topk_select(const hs2_attn_desc* desc, const float* scores, int64_t score_row_stride,
                            const int32_t* q_pos0, int32_t block_size, int32_t* idx, int32_t* cnt,
                            void* workspace, size_t ws_bytes, hs2_stream_t stream) {

@@ -21,9 +21,11 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
 
 // ---------------------------------------------------------------- decode (n_q == 1)
 struct DecodePlan {
+    bool fused;          // one cooperative launch, logits in tensor memory
+    int wb;              // fused: sequences per wave (CTAs = wb * splits <= SMs)
     int splits;          // key splits per sequence
     int chunk;           // keys per split (multiple of 64)
-    int s_ld;            // row pitch of the logit buffer (multiple of 64)
+    int s_ld;            // row pitch of the logit buffer (multiple of 64; 0 when fused)
 };
 DecodePlan plan_decode(int batch, int64_t max_ctx);
 size_t decode_ws_bytes(int batch, int64_t max_ctx);   // logits + partials + counters

@@ -176,12 +176,15 @@ Dev.bridge = _dev_bridge
 Dev.oracle_bridged_kv = _oracle_bridged_kv
 
 
-def block_parity(wl, seed, seqs=None, device="cpu", rows=None):
+def block_parity(wl, seed, seqs=None, device="cpu", rows=None, pos0=None):
     """Runs the hybrid block through the C ABI and checks it against the oracle on the
-    given sequences and query rows (all by default)."""
+    given sequences and query rows (all by default).  `pos0` gives each sequence its own
+    first query position (ragged batch); by default every sequence ends at the context."""
     import synth
     inp = synth.make_inputs(wl, seed=seed, device=device)
     dev = Dev(inp)
+    if pos0 is not None:
+        dev.q_pos0 = torch.tensor(pos0, dtype=torch.int32, device="cuda")
     if wl.n_new:
         dev.hidden_in, dev.w_in = inp.hidden, inp.w_kv
         dev.hidden = inp.hidden.to("cuda").contiguous()
@@ -193,9 +196,9 @@ def block_parity(wl, seed, seqs=None, device="cpu", rows=None):
     assert dev.status() == hs.HS2_OK
     seqs = range(wl.batch) if seqs is None else seqs
     rows = np.arange(wl.n_q) if rows is None else np.asarray(rows)
-    pos = wl.q_pos0 + rows
     report = {"differing_rows": 0, "rows": 0}
     for b in seqs:
+        pos = (wl.q_pos0 if pos0 is None else int(pos0[b])) + rows
         k, v = dev.kv_f64(b)
         if wl.n_new:
             k, v = dev.oracle_bridged_kv(b, k, v)
@@ -210,7 +213,7 @@ def block_parity(wl, seed, seqs=None, device="cpu", rows=None):
         g_cnt = dev.cnt[b].cpu().numpy()[rows]
         report["differing_rows"] += check_selection(g_idx, g_cnt, o_idx, o_cnt, sc_ref, pos, wl.window)
         report["rows"] += len(rows)
-        if inp.needle_pos is not None and wl.block_size == 1:
+        if inp.needle_pos is not None and wl.block_size == 1 and pos0 is None:
             sel = set(g_idx[-1, :g_cnt[-1]].tolist())
             assert set(inp.needle_pos[b].tolist()) <= sel, "planted key not selected"
         same = np.array([np.array_equal(g_idx[r], o_idx[r]) for r in range(len(rows))])

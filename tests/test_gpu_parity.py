@@ -147,6 +147,24 @@ def test_decode_bf16_small(ctx):
     _block_parity(wl, seed=1002)
 
 
+@pytest.mark.parametrize("batch,ctx", [(40, 20000), (200, 4096 + 77)])
+def test_decode_bf16_several_waves(batch, ctx):
+    # more sequences than one wave of the single-launch path holds (2 and 3 waves)
+    wl = synth.shrink(synth.DECODE_128K, batch=batch, ctx=ctx, needles=16)
+    _block_parity(wl, seed=1003)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "e4m3"])
+def test_decode_ragged_positions(kv):
+    # every sequence at its own position: splits past a short sequence's end hold no keys
+    base = synth.DECODE_128K if kv == "bf16" else synth.DECODE_1M_FP8
+    wl = synth.shrink(base, batch=40, ctx=20000, needles=16)
+    rng = np.random.default_rng(7)
+    pos0 = rng.integers(0, wl.ctx, size=wl.batch)
+    pos0[:8] = [0, 1, 63, 64, 1151, 1152, 2879, wl.ctx - 1]
+    _block_parity(wl, seed=1006, pos0=pos0)
+
+
 def test_decode_fp8_small():
     wl = synth.shrink(synth.DECODE_1M_FP8, batch=2, ctx=16384 + 5)
     _block_parity(wl, seed=1004)
