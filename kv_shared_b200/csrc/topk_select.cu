@@ -14,11 +14,15 @@
 // is handled by a cluster of CS CTAs (CS = 1..8), CTA r owning a contiguous
 // slice of the keys, cached in shared memory when it fits.
 //   1. the row's key range (reduced over the cluster) gives the bits all keys
-//      share; the first radix digit (<= 11 bits) is taken right below them
+//      share; the first radix digit (<= 11 bits) is taken right below them.  Slices
+//      too long for shared memory skip this pass (one read of the row saved) and take
+//      the top 11 bits as the first digit
 //   2. one histogram of that digit over every key (summed over the cluster by
 //      distributed shared memory) locates the bin b1 holding the K-th best key
 //   3. every CTA compacts, in position order, its keys in bins >= b1 into a
-//      short candidate list (about K plus the few keys of bin b1 per row)
+//      short candidate list (about K plus the few keys of bin b1 per row); slices
+//      read from global memory in one streaming pass, each warp buffering the
+//      matches of its own segment
 //   4. the remaining digits are resolved on the candidate lists only -> the exact
 //      threshold key tau and how many keys equal to it are taken (need_eq)
 //   5. each CTA writes its candidates above tau and its share of the first
@@ -43,6 +47,7 @@ constexpr int NBINS = 2048;
 constexpr int kMaxCluster = 8;
 constexpr int kSmemKeys = 24576;          // keys cached per CTA (96 KB)
 constexpr int kCandCap = 2048;            // candidates per CTA (16 KB), a power of two
+constexpr int kWarpCap = 512;             // streamed compaction: matches buffered per warp
 
 __device__ __forceinline__ uint32_t ord_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -293,6 +298,7 @@ __device__ __forceinline__ int compact_ordered(const Slice& sl, uint32_t thr, ui
             if (i0 + u < sl.end && k[u] >= thr) { ck[o] = k[u]; cp[o] = static_cast<uint32_t>(i0 + u); ++o; }
         n += tot;
     }
+    __syncthreads();                                      // the last round's entries are read next
     return n;
 }
 
@@ -348,6 +354,80 @@ __device__ __forceinline__ int compact_cached(const Slice& sl, uint32_t thr, uin
     return total;
 }
 
+// As compact_ordered for a slice read from global memory (token keys, 16-byte aligned
+// start): one streaming pass, 16-byte loads, 4 in flight per lane.  Warp w takes a
+// contiguous segment of the slice and appends its matches, in order, to its own buffer
+// (wk, wp: kWarpCap entries per warp) with warp scans only; the buffers are then
+// concatenated in warp order.  Returns -1, having written nothing to (ck, cp), if a warp's
+// matches would overflow its buffer.
+__device__ __forceinline__ int compact_stream(const Slice& sl, uint32_t thr, uint32_t* ck, uint32_t* cp,
+                                              uint32_t* wk, uint32_t* wp, Smem& sm) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n = sl.end - sl.begin, n4 = n >> 2;
+    const int seg4 = (n4 + NW - 1) / NW;                     // 16-byte groups per warp
+    const int q_begin = min(warp * seg4, n4), q_end = min(q_begin + seg4, n4);
+    const float4* src = reinterpret_cast<const float4*>(sl.s + sl.begin);
+    uint32_t* mk = wk + warp * kWarpCap;
+    uint32_t* mp = wp + warp * kWarpCap;
+    int cnt = 0;
+    bool over = false;
+    auto append = [&](const uint32_t (&k)[4], int first, int valid) {   // keys first .. first+3, in order
+        int c = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c += (e < valid) && k[e] >= thr;
+        int incl = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        const int tot = __shfl_sync(0xffffffffu, incl, 31);
+        if (cnt + tot > kWarpCap) {
+            over = true;
+        } else if (c) {
+            int o = cnt + incl - c;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if ((e < valid) && k[e] >= thr) { mk[o] = k[e]; mp[o] = static_cast<uint32_t>(first + e); ++o; }
+        }
+        cnt += tot;
+    };
+    for (int q0 = q_begin; q0 < q_end && !over; q0 += 4 * 32) {
+        float4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int q = q0 + u * 32 + lane;
+            x[u] = q < q_end ? __ldg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int q = q0 + u * 32 + lane;
+            const uint32_t k[4] = {ord_key(x[u].x), ord_key(x[u].y), ord_key(x[u].z), ord_key(x[u].w)};
+            append(k, sl.begin + 4 * q, q < q_end ? 4 : 0);
+        }
+    }
+    if (warp == NW - 1 && !over && 4 * n4 < n) {               // the last 1..3 keys, after every segment
+        uint32_t k[4] = {0u, 0u, 0u, 0u};
+        const int rest = n - 4 * n4;
+        if (lane == 0)
+            for (int e = 0; e < rest; ++e) k[e] = sl.key(sl.begin + 4 * n4 + e);
+        append(k, sl.begin + 4 * n4, lane == 0 ? rest : 0);
+    }
+    if (threadIdx.x == 0) sm.found_above = 0;                // overflow flag
+    __syncthreads();
+    if (over && lane == 0) sm.found_above = 1;
+    const int wbase = block_excl_scan(lane == 0 ? cnt : 0, sm);
+    const int total = sm.total;
+    if (sm.found_above) return -1;
+    const int base = __shfl_sync(0xffffffffu, wbase, 0);
+    for (int e = lane; e < cnt; e += 32) {
+        ck[base + e] = mk[e];
+        cp[base + e] = mp[e];
+    }
+    __syncthreads();
+    return total;
+}
+
 // The k-th largest (k >= 1) of the n keys g[] that match prefix under mask, resolved
 // 8 bits at a time (bits below `shift`) with the histogram sm.lhist; whole CTA.
 __device__ __forceinline__ uint32_t local_kth(const uint32_t* g, int n, uint32_t prefix, uint32_t mask, int shift,
@@ -394,6 +474,7 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
     uint32_t* key_cache = dsm;                                 // [cache_keys]
     uint32_t* cand_key = dsm + cache_keys;                     // [kCandCap]
     uint32_t* cand_pos = cand_key + kCandCap;                  // [kCandCap]
+    uint32_t* warp_buf = cand_pos + kCandCap;                  // [2][NW][kWarpCap] when cache_keys == 0
     __shared__ Smem sm;
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
@@ -421,10 +502,15 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
     sl.end = min(sl.begin + per, n_keys);
     sl.cache = nullptr;
 
-    // ---- 1. cache the slice's keys (when they fit) and find the row's key range
+    // ---- 1. cache the slice's keys (when they fit) and find the row's key range; a slice
+    // read from global memory skips this pass and takes the first digit at the top bits
     uint32_t lo = 0xffffffffu, hi = 0u;
     const bool cached = per <= cache_keys;
-    if (!take_all && !take_none) {
+    if (!take_all && !take_none && !cached) {
+        lo = 0u;
+        hi = 0xffffffffu;
+    }
+    if (!take_all && !take_none && cached) {
         if (cached && bs > 1) {
             // block keys: one warp per block, max over its tokens by shuffles
             for (int bb = sl.begin + warp; bb < sl.end; bb += NW) {
@@ -550,8 +636,14 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
                 // ---- 3. candidates: this CTA's keys at or above bin b1, in position order;
                 // its bin-b1 keys (fewer than kCandCap - K on this path) copied to hist[1]
                 if (threadIdx.x == 0) { sm.ncand2 = 0; sm.nb1 = 0; }
-                n_my = sl.cache ? compact_cached(sl, prefix, cand_key, cand_pos, sm)
-                                : compact_ordered(sl, prefix, cand_key, cand_pos, sm);
+                if (sl.cache) {
+                    n_my = compact_cached(sl, prefix, cand_key, cand_pos, sm);
+                } else {
+                    n_my = -1;
+                    if (cache_keys == 0 && bs == 1 && (reinterpret_cast<uintptr_t>(sl.s + sl.begin) & 15u) == 0)
+                        n_my = compact_stream(sl, prefix, cand_key, cand_pos, warp_buf, warp_buf + NW * kWarpCap, sm);
+                    if (n_my < 0) n_my = compact_ordered(sl, prefix, cand_key, cand_pos, sm);
+                }
                 uint32_t* b1k = reinterpret_cast<uint32_t*>(sm.hist[1]);
                 for (int e0 = 0; e0 < n_my; e0 += NT) {              // one counter update per warp
                     const int e = e0 + threadIdx.x;
@@ -738,7 +830,8 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
     const int cs = pick_cluster(a.rows, max_keys);
     const int64_t per = ((max_keys + cs - 1) / cs + 3) & ~int64_t(3);
     const int cache_keys = per <= kSmemKeys ? static_cast<int>(per) : 0;
-    const size_t smem = (static_cast<size_t>(cache_keys) + 2 * kCandCap) * sizeof(uint32_t);
+    const size_t smem = (static_cast<size_t>(cache_keys) + 2 * kCandCap + (cache_keys == 0 ? 2 * NW * kWarpCap : 0)) *
+                        sizeof(uint32_t);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(a.rows) * cs);
     cfg.blockDim = dim3(NT);

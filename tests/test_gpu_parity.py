@@ -45,6 +45,10 @@ def _select_case(n_rows, T, pos, W, K, bs, values, seed):
         s = (rng.integers(0, 8, size=(n_rows, T)) / 8.0).astype(np.float32)
     elif values == "signed":
         s = rng.standard_normal((n_rows, T)).astype(np.float32)
+    elif values == "increasing":
+        s = np.broadcast_to(np.arange(T, dtype=np.float32), (n_rows, T)).copy()
+    elif values == "equal":
+        s = np.ones((n_rows, T), dtype=np.float32)
     else:
         s = (rng.random((n_rows, T)) * 1e-3).astype(np.float32)
     desc = hs.make_desc(1, n_rows, 16, 128, window=W, budget=K, max_ctx=T,
@@ -74,6 +78,15 @@ def test_select_bit_exact_long_rows(values):
     # 128 + 1024 at contexts that span many rounds of the compaction and a ragged tail
     _select_case(6, 50000, 50000 - 6, 128, 1024, 1, values, seed=7)
     _select_case(3, 70001, 70001 - 3, 128, 1024, 64, values, seed=8)
+
+
+@pytest.mark.parametrize("values", ["uniform", "coarse", "signed", "increasing", "equal"])
+def test_select_bit_exact_streamed_rows(values):
+    # enough rows for one CTA per row and more keys than shared memory holds: the keys are
+    # streamed from global memory (first digit at the top bits, compaction by warp
+    # segments); increasing scores put every pick in the last warp's segment (its buffer
+    # overflows: ordered compaction), equal scores crowd one bin (radix over every key)
+    _select_case(300, 30001, 30001 - 300, 128, 1024, 1, values, seed=9)
 
 
 def test_select_all_equal_scores_picks_lowest():
