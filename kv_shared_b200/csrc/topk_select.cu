@@ -16,7 +16,7 @@
 //   1. the row's key range (reduced over the cluster) gives the bits all keys
 //      share; the first radix digit (<= 11 bits) is taken right below them.  Slices
 //      too long for shared memory skip this pass (one read of the row saved) and take
-//      the top 11 bits as the first digit
+//      the top 13 bits as the first digit
 //   2. one histogram of that digit over every key (summed over the cluster by
 //      distributed shared memory) locates the bin b1 holding the K-th best key
 //   3. every CTA compacts, in position order, its keys in bins >= b1 into a
@@ -48,6 +48,9 @@ constexpr int kMaxCluster = 8;
 constexpr int kSmemKeys = 24576;          // keys cached per CTA (96 KB)
 constexpr int kCandCap = 2048;            // candidates per CTA (16 KB), a power of two
 constexpr int kWarpCap = 512;             // streamed compaction: matches buffered per warp
+constexpr int kStreamBits = 13;           // first digit of a streamed slice (fixed: top 13 bits)
+constexpr int kMaxBins = 1 << kStreamBits;
+static_assert(2 * kMaxBins <= 2 * NW * kWarpCap, "a streamed slice's histograms live in the warp buffers");
 
 __device__ __forceinline__ uint32_t ord_key(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -428,6 +431,47 @@ __device__ __forceinline__ int compact_stream(const Slice& sl, uint32_t thr, uin
     return total;
 }
 
+// Bin of h[0..nb) (bins ascending in key) holding the k-th largest key: out[0] = bin,
+// out[1] = keys in the bins above it, out[2] = keys in it.  Chunks of 32 bins are summed by
+// warps (conflict-free reads), the chunk sums scanned by the block, the chunk found scanned
+// by one warp.  Whole CTA; nb a power of two <= kMaxBins; uses sm.lhist as chunk sums.
+__device__ __forceinline__ void find_bin(const int* h, int nb, int k, Smem& sm, int* out) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nch = (nb + 31) / 32;                          // chunk c: bins nb-1-32c-31 .. nb-1-32c
+    int* csum = sm.lhist;
+    for (int c = warp; c < nch; c += NW) {
+        const int bin = nb - 1 - (c * 32 + lane);
+        const int v = __reduce_add_sync(0xffffffffu, bin >= 0 ? h[bin] : 0);
+        if (lane == 0) csum[c] = v;
+    }
+    __syncthreads();
+    const int cv = static_cast<int>(threadIdx.x) < nch ? csum[threadIdx.x] : 0;
+    const int above = block_excl_scan(cv, sm);
+    if (static_cast<int>(threadIdx.x) < nch && above < k && above + cv >= k) {
+        sm.found_bin = threadIdx.x;
+        sm.found_above = above;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const int c = sm.found_bin;
+        const int bin = nb - 1 - (c * 32 + lane);
+        const int v = bin >= 0 ? h[bin] : 0;
+        int incl = v;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += y;
+        }
+        const int ab = sm.found_above + incl - v;
+        if (v > 0 && ab < k && ab + v >= k) {
+            out[0] = bin;
+            out[1] = ab;
+            out[2] = v;
+        }
+    }
+    __syncthreads();
+}
+
 // The k-th largest (k >= 1) of the n keys g[] that match prefix under mask, resolved
 // 8 bits at a time (bits below `shift`) with the histogram sm.lhist; whole CTA.
 __device__ __forceinline__ uint32_t local_kth(const uint32_t* g, int n, uint32_t prefix, uint32_t mask, int shift,
@@ -568,22 +612,22 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
             uint32_t mask = ~((2u << hb) - 1u);    // (hb == 31 gives 0: nothing shared)
             uint32_t prefix = hi & mask;
             int k_rem = K;
-            int width = min(11, hb + 1);
+            // streamed slices (no range pass) take the top 13 bits: importance values span few
+            // octaves, so bins of an eighth of an octave keep bin b1 short; the histogram and
+            // rank 0's sum live in the warp buffers, which are free until the compaction
+            int width = cached ? min(11, hb + 1) : kStreamBits;
             int shift = hb - width + 1;
             const int nb = 1 << width;
             // ---- 2. first digit over every key; rank 0 sums the cluster's histograms
-            int* hist = sm.hist[0];
+            int* hist = cached ? sm.hist[0] : reinterpret_cast<int*>(warp_buf);
             for (int i = threadIdx.x; i < nb; i += NT) hist[i] = 0;
             __syncthreads();
             for_keys_fast(sl, [&](int, uint32_t key) { atomicAdd(&hist[(key >> shift) & (nb - 1)], 1); });
             cluster.sync();                        // [barrier 2] histograms complete
             if (rank == 0) {
-                const int bins_per = (nb + NT - 1) / NT;
-                int local[NBINS / NT];
-                int tot = 0;
                 // the cluster's histogram summed into hist[1] with coalesced remote reads
                 // (consecutive threads, consecutive bins), then scanned from there
-                int* hsum = sm.hist[1];
+                int* hsum = cached ? sm.hist[1] : reinterpret_cast<int*>(warp_buf) + kMaxBins;
                 if (CS == 1) {
                     hsum = hist;
                 } else {
@@ -598,27 +642,7 @@ __global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys
                     }
                     __syncthreads();
                 }
-#pragma unroll
-                for (int q = 0; q < NBINS / NT; ++q) {
-                    const int bin = nb - 1 - (threadIdx.x * bins_per + q);
-                    const int c = (q < bins_per && bin >= 0) ? hsum[bin] : 0;
-                    local[q] = c;
-                    tot += c;
-                }
-                const int above = block_excl_scan(tot, sm);
-                if (above < k_rem && above + tot >= k_rem) {
-                    int acc = above;
-                    for (int q = 0; q < bins_per; ++q) {
-                        if (acc + local[q] >= k_rem) {
-                            sm.dec[0] = nb - 1 - (threadIdx.x * bins_per + q);
-                            sm.dec[1] = acc;
-                            sm.dec[2] = local[q];
-                            break;
-                        }
-                        acc += local[q];
-                    }
-                }
-                __syncthreads();
+                find_bin(hsum, nb, k_rem, sm, sm.dec);
                 // candidate lists fit when K + |bin b1| <= kCandCap (a CTA holds at most the
                 // row's keys above b1 (< K) plus those in b1); the gather buffer holds |b1|
                 if (threadIdx.x == 0) sm.dec[3] = (K + sm.dec[2] <= kCandCap && sm.dec[2] <= 2 * NBINS) ? 1 : 0;
