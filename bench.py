@@ -428,8 +428,167 @@ def run_ours(args, ws_, rank, local):
     if not args.no_prefill and args.workload == "all":
         out["prefill"] = run_prefill(args, ws_)
         out["gpu_launches"] += out["prefill"]["gpu_launches"]
+    if not args.no_configs and args.workload == "all" and not args.small:
+        out["other_configs"] = run_configs(args)
     if ws_ == 1 and rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, seed=1002, sample_seqs=args.cpu_sample)
+    return out
+
+
+# ------------------------------------------------------------------ the other workloads
+class ConfigBlock:
+    """Device buffers of one hybrid-block call pattern for any workload (f32, bf16 or e4m3
+    cache; e4m3 caches are quantized from the generator's fp32 values by the library)."""
+
+    def __init__(self, wl, seed):
+        import kv_shared_b200 as hs
+        self.hs, self.wl = hs, wl
+        inp = synth.make_inputs(wl, seed=seed, device="cuda")
+        self.q = inp.q_full.contiguous()
+        self.qs = [x.contiguous() for x in inp.q_sparse]
+        self.k_scale = self.v_scale = None
+        if wl.kv_dtype == "e4m3":
+            B, T, D = inp.k_src.shape
+            self.k = torch.empty(B, T, D, dtype=torch.uint8, device="cuda")
+            self.v = torch.empty_like(self.k)
+            self.k_scale = torch.empty(B, T, dtype=torch.float32, device="cuda")
+            self.v_scale = torch.empty_like(self.k_scale)
+            hs.hs2_kv_quantize_fp8(inp.k_src, B * T, D, self.k, self.k_scale)
+            hs.hs2_kv_quantize_fp8(inp.v_src, B * T, D, self.v, self.v_scale)
+        else:
+            self.k, self.v = inp.k.contiguous(), inp.v.contiguous()
+        self.needle_pos = inp.needle_pos
+        del inp
+        code = {"f32": hs.HS2_F32, "bf16": hs.HS2_BF16, "e4m3": hs.HS2_E4M3}
+        B = wl.batch
+        self.q_pos0 = torch.full((B,), wl.q_pos0, dtype=torch.int32, device="cuda")
+        self.desc = hs.make_desc(B, wl.n_q, wl.heads, wl.head_dim, wl.window, wl.budget,
+                                 q_dtype=code[wl.q_dtype], kv_dtype=code[wl.kv_dtype], max_ctx=wl.ctx)
+        self.ws = hs.alloc_workspace(self.desc, scores_in_workspace=False)
+        self.o = torch.empty_like(self.q)
+        self.o_sp = torch.empty_like(self.q)
+        self.scores = torch.empty(B, wl.n_q, wl.ctx, dtype=torch.float32, device="cuda")
+        self.idx = torch.empty(B, wl.n_q, self.desc.idx_stride, dtype=torch.int32, device="cuda")
+        self.cnt = torch.empty(B, wl.n_q, dtype=torch.int32, device="cuda")
+        self.bidx = torch.empty_like(self.idx)
+        self.bcnt = torch.empty_like(self.cnt)
+
+    def full(self):
+        self.hs.hs2_full_attn_select(self.desc, self.q, self.k, self.v, self.k_scale, self.v_scale, self.q_pos0,
+                                     self.o, None, self.idx, self.cnt, self.scores, self.ws)
+
+    def sparse(self):
+        self.hs.hs2_sparse_attn(self.desc, self.qs[0], self.k, self.v, self.k_scale, self.v_scale, self.idx,
+                                self.cnt, self.o_sp, None, self.ws)
+
+    def block_select(self):
+        wl = self.wl
+        self.hs.hs2_topk_select(self.desc, self.scores.view(-1, wl.ctx), wl.ctx, self.q_pos0, 64, self.bidx,
+                                self.bcnt, self.ws)
+
+    def recall(self, idx, cnt):
+        """Share of the planted keys that the last query row of each sequence selected."""
+        if self.needle_pos is None:
+            return None
+        found = total = 0
+        for b in range(self.wl.batch):
+            sel = set(idx[b, -1, :int(cnt[b, -1])].tolist())
+            pos = self.needle_pos[b].tolist()
+            found += sum(p in sel for p in pos)
+            total += len(pos)
+        return found / total
+
+    def cache_bytes(self):
+        """K + V (+ e4m3 scales) read and importance written per call, Q/O included."""
+        wl = self.wl
+        row = {"f32": 2 * wl.head_dim * 4, "bf16": 2 * wl.head_dim * 2, "e4m3": 2 * wl.head_dim + 8}[wl.kv_dtype]
+        qo = 2 * wl.heads * wl.head_dim * (4 if wl.q_dtype == "f32" else 2)
+        return wl.batch * (wl.ctx * (row + 4) + wl.n_q * qo)
+
+    def sparse_bytes(self):
+        wl = self.wl
+        row = {"f32": 2 * wl.head_dim * 4, "bf16": 2 * wl.head_dim * 2, "e4m3": 2 * wl.head_dim + 8}[wl.kv_dtype]
+        qo = 2 * wl.heads * wl.head_dim * (4 if wl.q_dtype == "f32" else 2)
+        per_row = min(wl.q_pos0 + 1, wl.window + wl.budget) * (row + 4) + qo
+        return wl.batch * wl.n_q * per_row
+
+
+def _time_graph(fn, stream, reps):
+    """Device time of one replay of fn captured in a CUDA graph (events around reps replays)."""
+    (g,) = _capture([fn], stream)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    del g
+    return ms
+
+
+def run_configs(args):
+    """The parity workloads other than the two headline ones, each timed on its own: the
+    1M-token e4m3 decode, the selection-granularity sweep (token arm vs the 64-token block
+    arm on the same importance) and the tiny fp32 prefill."""
+    import kv_shared_b200 as hs
+    stream = torch.cuda.current_stream()
+    hbm, _, _ = _peaks()
+    out = {}
+
+    wl = synth.DECODE_1M_FP8
+    blk = ConfigBlock(wl, seed=1004)
+    blk.full(); blk.sparse()
+    torch.cuda.synchronize()
+    if hs.hs2_last_status(blk.ws) != hs.HS2_OK:
+        raise RuntimeError("1M e4m3 decode: device status " + hs.status_string(hs.hs2_last_status(blk.ws)))
+    full_ms = _time_graph(blk.full, stream, 20)
+    sparse_ms = _time_graph(blk.sparse, stream, 50)
+    out["decode_1m_e4m3"] = {
+        "workload": wl.name,
+        "full_attn_select": {"ms": full_ms, "bytes_per_call": blk.cache_bytes(),
+                             "hbm_frac": blk.cache_bytes() / (full_ms / 1e3) / 1e9 / hbm,
+                             "launches": hs.hs2_full_attn_launches(blk.desc)},
+        "sparse_attn": {"ms": sparse_ms, "queries/s": wl.batch / (sparse_ms / 1e3),
+                        "bytes_per_call": blk.sparse_bytes(),
+                        "hbm_frac": blk.sparse_bytes() / (sparse_ms / 1e3) / 1e9 / hbm,
+                        "note": "4 query rows: latency-bound"},
+        "needle_recall": blk.recall(blk.idx.cpu(), blk.cnt.cpu()),
+    }
+    del blk
+    torch.cuda.empty_cache()
+
+    sweep = []
+    for ctx in synth.SWEEP_CTX:
+        wl = synth.sweep(ctx)
+        blk = ConfigBlock(wl, seed=1005)
+        blk.full(); blk.block_select(); blk.sparse()
+        torch.cuda.synchronize()
+        reps = 50 if ctx <= 262144 else 20
+        full_ms = _time_graph(blk.full, stream, reps)
+        block_ms = _time_graph(blk.block_select, stream, reps)
+        sparse_ms = _time_graph(blk.sparse, stream, reps)
+        sweep.append({"ctx": ctx, "full_attn_select_us": full_ms * 1e3, "block_select_us": block_ms * 1e3,
+                      "sparse_attn_us": sparse_ms * 1e3, "end_to_end_us": (full_ms + sparse_ms) * 1e3,
+                      "recall_token": blk.recall(blk.idx.cpu(), blk.cnt.cpu()),
+                      "recall_block64": blk.recall(blk.bidx.cpu(), blk.bcnt.cpu())})
+        del blk
+        torch.cuda.empty_cache()
+    out["granularity_sweep"] = {"workload": "sweep_ctx{4096,32768,262144,1048576}, 64 planted tokens, "
+                                            "one per 64-token block", "points": sweep}
+
+    wl = synth.TINY
+    blk = ConfigBlock(wl, seed=1001)
+    blk.full(); blk.sparse()
+    torch.cuda.synchronize()
+    out["tiny_f32"] = {"workload": wl.name, "full_attn_select_ms": _time_graph(blk.full, stream, 20),
+                       "sparse_attn_ms": _time_graph(blk.sparse, stream, 20),
+                       "note": "fp32 CUDA-core path; parity workload, timing informational"}
+    del blk
+    torch.cuda.empty_cache()
     return out
 
 
@@ -505,6 +664,7 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the 1M e4m3, sweep and tiny workloads")
     ap.add_argument("--workload", choices=["all", "decode", "prefill"], default="all",
                     help="all: decode headline + prefill leg")
     ap.add_argument("--small", action="store_true",
