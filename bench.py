@@ -366,29 +366,70 @@ def run_ours(args, ws_, rank, local):
     value = ws_ * queries_per_step / (ms_per_step / 1e3)
 
     # end to end through the C ABI: per-step inputs (the 4 layers' queries and the new
-    # token's K/V row) come from pinned host memory, the last layer's output goes back
-    host_q = [torch.empty_like(x, device="cpu").pin_memory() for x in [blk.q] + blk.qs]
-    for h, d in zip(host_q, [blk.q] + blk.qs):
+    # token's K/V row) come from pinned host memory, the last layer's output goes back.  Two
+    # sets of device inputs and outputs (a second step graph over the second set) let one
+    # step's copies run on a copy stream while the neighbouring step computes; every copy of
+    # every step is inside the timed region, which ends when the last output is on the host.
+    outs = [blk.o_sp[-1]]
+    ins = [[blk.q] + blk.qs]
+    alt_in = [torch.empty_like(x) for x in ins[0]]
+    alt_out = torch.empty_like(outs[0])
+    ins.append(alt_in)
+    outs.append(alt_out)
+    dev_kv = [torch.empty(2, wl.batch, wl.head_dim, dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+
+    def step_with_row(u):
+        # the new token's K/V row into the cache, then the step (both in the graph)
+        blk.k[:, wl.ctx - 1].copy_(dev_kv[u][0])
+        blk.v[:, wl.ctx - 1].copy_(dev_kv[u][1])
+        blk.step()
+
+    saved = (blk.q, blk.qs, blk.o_sp[-1])
+    graphs = []
+    for u in range(2):
+        blk.q, blk.qs, blk.o_sp[-1] = ins[u][0], ins[u][1:], outs[u]
+        graphs += _capture([lambda u=u: step_with_row(u)], stream)
+    blk.q, blk.qs, blk.o_sp[-1] = saved
+    host_q = [torch.empty_like(x, device="cpu").pin_memory() for x in ins[0]]
+    for h, d in zip(host_q, ins[0]):
         h.copy_(d)
     host_kv = torch.empty(2, wl.batch, wl.head_dim, dtype=torch.bfloat16).pin_memory()
     host_kv[0].copy_(blk.k[:, wl.ctx - 1])
     host_kv[1].copy_(blk.v[:, wl.ctx - 1])
-    dev_kv = torch.empty(2, wl.batch, wl.head_dim, dtype=torch.bfloat16, device="cuda")
-    host_out = torch.empty_like(blk.o_sp[-1], device="cpu").pin_memory()
+    host_out = [torch.empty_like(outs[0], device="cpu").pin_memory() for _ in range(2)]
     h2d = sum(h.numel() * h.element_size() for h in host_q) + host_kv.numel() * host_kv.element_size()
-    d2h = host_out.numel() * host_out.element_size()
+    d2h = host_out[0].numel() * host_out[0].element_size()
+    # inputs and outputs on streams of their own: a step's input copies never queue
+    # behind the previous step's output copy
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
     _barrier(ws_)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    s_in.wait_stream(stream)
+    s_out.wait_stream(stream)
     for i in range(K):
-        for h, d in zip(host_q, [blk.q] + blk.qs):
-            d.copy_(h, non_blocking=True)
-        dev_kv.copy_(host_kv, non_blocking=True)
-        blk.k[:, wl.ctx - 1].copy_(dev_kv[0])
-        blk.v[:, wl.ctx - 1].copy_(dev_kv[1])
-        step_graph.replay()
-        host_out.copy_(blk.o_sp[-1], non_blocking=True)
+        u = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(ev_comp[u])         # step i - 2 has consumed this input set
+            for h, d in zip(host_q, ins[u]):
+                d.copy_(h, non_blocking=True)
+            dev_kv[u].copy_(host_kv, non_blocking=True)
+            ev_in[u].record(s_in)
+        stream.wait_event(ev_in[u])
+        if i >= 2:
+            stream.wait_event(ev_out[u])            # step i - 2's output has left this buffer
+        graphs[u].replay()
+        ev_comp[u].record(stream)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_comp[u])
+            host_out[u].copy_(outs[u], non_blocking=True)
+            ev_out[u].record(s_out)
+    stream.wait_stream(s_out)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = _max_over_ranks(ws_, e0.elapsed_time(e1)) / K
@@ -423,7 +464,7 @@ def run_ours(args, ws_, rank, local):
         "gpu_launches": K * blk.launches_per_step,
         "clocks": clk.summary(),
     }
-    del blk, step_graph, full_graph
+    del blk, step_graph, graphs, full_graph
     torch.cuda.empty_cache()
     if not args.no_prefill and args.workload == "all":
         out["prefill"] = run_prefill(args, ws_)
