@@ -11,8 +11,8 @@
 //           each CTA keeps a running (max, sum) per head -> per-split partials.
 //   pass B  every CTA merges the partials into LSE, re-reads its logits, forms
 //           P exactly normalized, writes importance = sum_h P and accumulates
-//           O = P V (no online rescaling is needed: LSE is final).  The last CTA
-//           of a sequence sums the split partials into O (semaphore, no spin).
+//           O = P V (no online rescaling is needed: LSE is final); a third small
+//           kernel sums the split partials of O per (sequence, head).
 //
 // K is read once (pass A) and V once (pass B): 512 B of cache per key plus the
 // 64-B logit round trip.  Tiles of 64 keys stream through a 4-stage TMA pipeline
@@ -122,7 +122,6 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
     const int k_end = min(p + 1, k_begin + a.chunk);
     const int n_tiles = k_end > k_begin ? (k_end - k_begin + TILE - 1) / TILE : 0;
 
-    if (split == 0 && tid == 0) a.counter[b] = 0;     // consumed by pass B (stream order)
     if (tid == 0) {
         prefetch_tmap(&kmap);
         for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
@@ -246,8 +245,7 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     uint8_t* smem = align1024(smem_raw);
     uint8_t* cvt = smem + STAGES * STAGE;
     uint64_t* full = reinterpret_cast<uint64_t*>(cvt + L::CVT);
-    float* red_o = reinterpret_cast<float*>(full + STAGES);          // [H][D]
-    __shared__ int s_last;
+    float4* red_o4 = reinterpret_cast<float4*>(smem);              // [4][16][32] after the tiles
 
     const int b = blockIdx.y, split = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
@@ -262,7 +260,6 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
         for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
-    for (int i = tid; i < H * D; i += NT) red_o[i] = 0.f;
     __syncthreads();
 
     auto issue = [&](int i, int s) {
@@ -378,47 +375,59 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
         if (tid == 0 && i + STAGES < n_tiles) issue(i + STAGES, s);
     }
 
-    // CTA partial O = sum over warps
+    // this split's O partial: the 4 warps' accumulators through shared memory (the stage
+    // area, free once every tile is consumed) as [warp][n][lane] float4 (conflict-free),
+    // each (n, lane) slot summed over the warps in a fixed order; the partials of all splits
+    // are summed by dec_merge_kernel
+    __syncthreads();
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-        const int d = 8 * n + 2 * t;
-        atomicAdd(&red_o[g * D + d], o[n][0]);
-        atomicAdd(&red_o[g * D + d + 1], o[n][1]);
-        atomicAdd(&red_o[(g + 8) * D + d], o[n][2]);
-        atomicAdd(&red_o[(g + 8) * D + d + 1], o[n][3]);
-    }
+    for (int n = 0; n < 16; ++n) red_o4[(warp * 16 + n) * 32 + lane] = make_float4(o[n][0], o[n][1], o[n][2], o[n][3]);
     __syncthreads();
     float* my = a.part_o + (static_cast<size_t>(b) * a.splits + split) * H * D;
-    for (int i = tid; i < H * D; i += NT) my[i] = red_o[i];
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = (atomicAdd(&a.counter[b], 1) == a.splits - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    // sum of the split partials with independent 16-byte loads (4 per thread per split)
-    const float4* base4 = reinterpret_cast<const float4*>(a.part_o + static_cast<size_t>(b) * a.splits * H * D);
-    constexpr int F4 = H * D / 4;
-    constexpr int PER = F4 / NT;
-    float4 acc[PER];
 #pragma unroll
-    for (int k = 0; k < PER; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
-    for (int s = 0; s < a.splits; ++s) {
-        float4 v[PER];
+    for (int k = 0; k < 512 / NT; ++k) {
+        const int e = tid + k * NT, n = e >> 5, ln = e & 31;
+        float4 sum = red_o4[e];
 #pragma unroll
-        for (int k = 0; k < PER; ++k) v[k] = __ldcg(base4 + static_cast<size_t>(s) * F4 + tid + k * NT);
-#pragma unroll
-        for (int k = 0; k < PER; ++k) {
-            acc[k].x += v[k].x; acc[k].y += v[k].y; acc[k].z += v[k].z; acc[k].w += v[k].w;
+        for (int w4 = 1; w4 < 4; ++w4) {
+            const float4 v = red_o4[w4 * 512 + e];
+            sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
         }
+        const int d = 8 * n + 2 * (ln & 3), h = ln >> 2;
+        *reinterpret_cast<float2*>(my + h * D + d) = make_float2(sum.x, sum.y);
+        *reinterpret_cast<float2*>(my + (h + 8) * D + d) = make_float2(sum.z, sum.w);
     }
-#pragma unroll
-    for (int k = 0; k < PER; ++k) {
+}
+
+// O = sum of the split partials: CTA (row, group) = (blockIdx.x / 8, blockIdx.x % 8) takes
+// dims 16 group .. + 15 of row (sequence, head): 4 float4 columns x 32 split lanes, the
+// lanes combined in a fixed order.
+constexpr int kMergeGroups = 8;
+__global__ void __launch_bounds__(NT) dec_merge_kernel(Params a) {
+    __shared__ float4 part[32][4];
+    const int row = blockIdx.x / kMergeGroups, grp = blockIdx.x % kMergeGroups;
+    const int b = row / H, h = row % H;
+    const int c4 = threadIdx.x & 3, sl = threadIdx.x >> 2;
+    const float4* src = reinterpret_cast<const float4*>(a.part_o + static_cast<size_t>(b) * a.splits * H * D + h * D) +
+                        4 * grp + c4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int sp = sl; sp < a.splits; sp += 32) {
+        const float4 v = __ldg(src + static_cast<size_t>(sp) * (H * D / 4));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    }
+    part[sl][c4] = acc;
+    __syncthreads();
+    if (threadIdx.x < 4) {
+        float4 t = part[0][c4];
+        for (int q = 1; q < 32; ++q) {
+            const float4 v = part[q][c4];
+            t.x += v.x; t.y += v.y; t.z += v.z; t.w += v.w;
+        }
         uint2 packed;
-        packed.x = pack_bf16(acc[k].x, acc[k].y);
-        packed.y = pack_bf16(acc[k].z, acc[k].w);
-        *reinterpret_cast<uint2*>(a.o + static_cast<size_t>(b) * H * D + 4 * (tid + k * NT)) = packed;
+        packed.x = pack_bf16(t.x, t.y);
+        packed.y = pack_bf16(t.z, t.w);
+        *reinterpret_cast<uint2*>(a.o + (static_cast<size_t>(b) * H + h) * D + 16 * grp + 4 * c4) = packed;
     }
 }
 
@@ -857,14 +866,15 @@ template <bool KV8>
 size_t smem_a() { return 1024 + STAGES * Layout<KV8>::RAW + Layout<KV8>::CVT + STAGES * 8; }
 template <bool KV8>
 size_t smem_b() {
-    return 1024 + STAGES * (Layout<KV8>::RAW + Layout<KV8>::STILE) + Layout<KV8>::CVT + STAGES * 8 + H * D * 4;
+    static_assert(STAGES * (Layout<KV8>::RAW + Layout<KV8>::STILE) >= 4 * H * D * 4, "O partials reuse the stages");
+    return 1024 + STAGES * (Layout<KV8>::RAW + Layout<KV8>::STILE) + Layout<KV8>::CVT + STAGES * 8;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 template <bool KV8>
 cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
-    const DecodePlan pl = plan_decode(da.batch, da.max_ctx);
+    const DecodePlan pl = plan_decode(da.batch, da.max_ctx, KV8);
     Params a{};
     a.B = da.batch; a.cap = da.cap; a.max_ctx = da.max_ctx; a.splits = pl.splits; a.chunk = pl.chunk; a.s_ld = pl.s_ld;
     a.q_pos0 = da.q_pos0;
@@ -923,12 +933,13 @@ cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     dec_qk_kernel<KV8><<<grid, NT, sa, st>>>(kmap, a);
     dec_pv_kernel<KV8><<<grid, NT, sb, st>>>(vmap, smap, a);
+    dec_merge_kernel<<<da.batch * H * kMergeGroups, NT, 0, st>>>(a);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-DecodePlan plan_decode(int batch, int64_t max_ctx) {
+DecodePlan plan_decode(int batch, int64_t max_ctx, bool kv8) {
     DecodePlan pl;
     // fused: enough splits that each fits tensor memory, as many sequences per wave as
     // the SMs allow, waves balanced, then as many splits as the SMs allow
@@ -953,7 +964,9 @@ DecodePlan plan_decode(int batch, int64_t max_ctx) {
     }
     pl.fused = false;
     pl.wb = 0;
-    int splits = (2 * num_sms()) / (batch > 0 ? batch : 1);
+    // two-kernel path: two CTAs per SM suffice to stream a bf16 cache; e4m3 tiles are
+    // converted in shared memory, which takes three (as many as pass B fits per SM)
+    int splits = ((kv8 ? 3 : 2) * num_sms()) / (batch > 0 ? batch : 1);
     if (splits < 1) splits = 1;
     int64_t chunk = (max_ctx + splits - 1) / splits;
     chunk = (chunk + TILE - 1) / TILE * TILE;
@@ -965,8 +978,8 @@ DecodePlan plan_decode(int batch, int64_t max_ctx) {
     return pl;
 }
 
-size_t decode_ws_bytes(int batch, int64_t max_ctx) {
-    const DecodePlan pl = plan_decode(batch, max_ctx);
+size_t decode_ws_bytes(int batch, int64_t max_ctx, bool kv8) {
+    const DecodePlan pl = plan_decode(batch, max_ctx, kv8);
     return align256(sizeof(float) * batch * H * static_cast<size_t>(pl.s_ld)) +
            align256(sizeof(float2) * batch * pl.splits * H) +
            align256(sizeof(float) * batch * pl.splits * H * D) + align256(sizeof(int) * batch);

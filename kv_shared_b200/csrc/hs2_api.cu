@@ -102,7 +102,7 @@ int64_t score_pitch(const hs2_attn_desc* d) { return (d->max_ctx + 63) / 64 * 64
 size_t full_region(const hs2_attn_desc* d, Path path, bool scores_in_ws) {
     const size_t rows = static_cast<size_t>(d->batch) * d->n_q;
     size_t n = 0;
-    if (path == Path::TC && d->n_q == 1) n += a256(decode_ws_bytes(d->batch, d->max_ctx));
+    if (path == Path::TC && d->n_q == 1) n += a256(decode_ws_bytes(d->batch, d->max_ctx, d->kv_dtype == HS2_E4M3));
     if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q));
     if (scores_in_ws) n += a256(sizeof(float) * rows * static_cast<size_t>(score_pitch(d)));
     return n;
@@ -158,7 +158,7 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     int64_t score_ld = desc->max_ctx;
     size_t used = 0;
     if (path == Path::TC)
-        used = desc->n_q == 1 ? a256(decode_ws_bytes(desc->batch, desc->max_ctx))
+        used = desc->n_q == 1 ? a256(decode_ws_bytes(desc->batch, desc->max_ctx, desc->kv_dtype == HS2_E4M3))
                               : a256(prefill_ws_bytes(desc->batch, desc->n_q));
     if (!score_buf) {
         score_buf = reinterpret_cast<float*>(region + used);
@@ -203,7 +203,7 @@ int32_t hs2_full_attn_launches(const hs2_attn_desc* desc) {
     int32_t n = 1;                                      // the selection
     if (path == Path::F32) n += 1;
     else if (desc->n_q > 1) n += 2;                     // prefill: log-sum-exp pass, output pass
-    else n += plan_decode(desc->batch, desc->max_ctx).fused ? 1 : 2;
+    else n += plan_decode(desc->batch, desc->max_ctx, desc->kv_dtype == HS2_E4M3).fused ? 1 : 3;  // or: 2 passes + merge
     return n;
 }
 

@@ -27,8 +27,8 @@ struct DecodePlan {
     int chunk;           // keys per split (multiple of 64)
     int s_ld;            // row pitch of the logit buffer (multiple of 64; 0 when fused)
 };
-DecodePlan plan_decode(int batch, int64_t max_ctx);
-size_t decode_ws_bytes(int batch, int64_t max_ctx);   // logits + partials + counters
+DecodePlan plan_decode(int batch, int64_t max_ctx, bool kv8);
+size_t decode_ws_bytes(int batch, int64_t max_ctx, bool kv8);   // logits + partials + counters
 
 struct DecodeArgs {
     int batch;

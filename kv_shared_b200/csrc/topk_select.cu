@@ -239,7 +239,7 @@ __device__ __forceinline__ int ordered_write(Smem& sm, const Slice& sl, int n, P
 }
 
 // Visits every key of the slice as f(i, key) (any order).  Token keys go through
-// 16-byte loads, 4 keys each and 4 loads in flight per thread, whenever the slice
+// 16-byte loads, 4 keys each and 8 loads in flight per thread, whenever the slice
 // start is 16-byte aligned (shared-memory cache or score row); otherwise for_keys.
 template <typename F>
 __device__ __forceinline__ void for_keys_fast(const Slice& sl, F f) {
@@ -249,10 +249,10 @@ __device__ __forceinline__ void for_keys_fast(const Slice& sl, F f) {
         return;
     }
     const int n = sl.end - sl.begin, n4 = n >> 2;
-    for (int base = 0; base < n4; base += NT * 4) {
-        uint4 v[4];
+    for (int base = 0; base < n4; base += NT * 8) {
+        uint4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int q = base + u * NT + threadIdx.x;
             if (q < n4) {
                 if (sl.cache) {
@@ -264,7 +264,7 @@ __device__ __forceinline__ void for_keys_fast(const Slice& sl, F f) {
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int q = base + u * NT + threadIdx.x;
             if (q < n4) {
                 const int i = sl.begin + 4 * q;
@@ -358,7 +358,7 @@ __device__ __forceinline__ int compact_cached(const Slice& sl, uint32_t thr, uin
 }
 
 // As compact_ordered for a slice read from global memory (token keys, 16-byte aligned
-// start): one streaming pass, 16-byte loads, 4 in flight per lane.  Warp w takes a
+// start): one streaming pass, 16-byte loads, 8 in flight per lane.  Warp w takes a
 // contiguous segment of the slice and appends its matches, in order, to its own buffer
 // (wk, wp: kWarpCap entries per warp) with warp scans only; the buffers are then
 // concatenated in warp order.  Returns -1, having written nothing to (ck, cp), if a warp's
@@ -395,15 +395,15 @@ __device__ __forceinline__ int compact_stream(const Slice& sl, uint32_t thr, uin
         }
         cnt += tot;
     };
-    for (int q0 = q_begin; q0 < q_end && !over; q0 += 4 * 32) {
-        float4 x[4];
+    for (int q0 = q_begin; q0 < q_end && !over; q0 += 8 * 32) {
+        float4 x[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int q = q0 + u * 32 + lane;
             x[u] = q < q_end ? __ldg(src + q) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int q = q0 + u * 32 + lane;
             const uint32_t k[4] = {ord_key(x[u].x), ord_key(x[u].y), ord_key(x[u].z), ord_key(x[u].w)};
             append(k, sl.begin + 4 * q, q < q_end ? 4 : 0);
@@ -512,7 +512,7 @@ __device__ __forceinline__ uint32_t local_kth(const uint32_t* g, int n, uint32_t
 }
 
 template <int CS>
-__global__ void __launch_bounds__(NT) select_kernel(SelectArgs a, int cache_keys) {
+__global__ void __launch_bounds__(NT, 2) select_kernel(SelectArgs a, int cache_keys) {
     constexpr int cs = CS;
     extern __shared__ uint32_t dsm[];
     uint32_t* key_cache = dsm;                                 // [cache_keys]
