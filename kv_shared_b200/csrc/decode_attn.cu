@@ -43,8 +43,9 @@ struct Params {
     float sc2;                      // softmax scale * log2(e)
     float* S;                       // [B][H][s_ld] logits, log2 units
     float2* part_ml;                // [B][splits][H]: (max, sum) in log2 units
+    float* part_vmax;               // [B][splits]: largest V scale of the split (e4m3)
     float* part_o;                  // [B][splits][H][D]
-    int* counter;                   // [B]
+    int* counter;                   // fused path: [3][B] in the status block
     __nv_bfloat16* o;               // [B][H][D]
     float* lse;                     // [B][H] natural log, or null
     float* scores;                  // [B][score_ld]
@@ -97,6 +98,104 @@ __device__ __forceinline__ void convert_tile(const uint8_t* raw, uint8_t* cvt, i
     }
 }
 
+// ---- e4m3 tiles without a conversion pass (the two-kernel path): f16 MMAs fed straight
+// from the tile as TMA wrote it (64 rows of 128 B, 128-byte swizzle); e4m3 -> f16 is exact.
+
+// f16 A-fragments of Q for keys from e4m3 tiles.  Within each 16-dim step the k order is
+// permuted so that the 4 consecutive dims 4t .. 4t+3 that ldmatrix gives a thread of a key
+// (two b16 units = four e4m3 bytes) form its B registers: k = 2t, 2t+1 <-> dims 4t, 4t+1 and
+// k = 2t+8, 2t+9 <-> dims 4t+2, 4t+3.  Q is scaled by 2^-e (e > 0 only if max |q| >= 2^14)
+// to fit f16; returns 2^e.  Every warp loads all of Q, so all warps find the same e.
+__device__ __forceinline__ float load_q_frags_e4m3(const __nv_bfloat16* qb, int g, int t, uint32_t (&qa)[8][4]) {
+    uint2 raw[8][2];
+    float mx = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        raw[ks][0] = __ldg(reinterpret_cast<const uint2*>(qb + g * D + 16 * ks + 4 * t));
+        raw[ks][1] = __ldg(reinterpret_cast<const uint2*>(qb + (g + 8) * D + 16 * ks + 4 * t));
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[ks][r].x));
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[ks][r].y));
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x.x), fabsf(x.y)), fmaxf(fabsf(y.x), fabsf(y.y))));
+        }
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    int e = 0;
+    if (mx >= 16384.f) {
+        int ex;
+        frexpf(mx, &ex);                        // mx < 2^ex
+        e = ex - 14;
+    }
+    const float s = ldexpf(1.f, -e);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+        uint32_t v[2][2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[ks][r].x));
+            const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[ks][r].y));
+            v[r][0] = pack_f16(x.x * s, x.y * s);    // dims 4t, 4t+1
+            v[r][1] = pack_f16(y.x * s, y.y * s);    // dims 4t+2, 4t+3
+        }
+        qa[ks][0] = v[0][0];        // row g,     k = 2t, 2t+1
+        qa[ks][1] = v[1][0];        // row g + 8
+        qa[ks][2] = v[0][1];        // row g,     k = 2t+8, 2t+9
+        qa[ks][3] = v[1][1];        // row g + 8
+    }
+    return ldexpf(1.f, e);
+}
+
+// S for 16 heads x this warp's 16 keys (rows row0 .. row0 + 15 of the tile at shared address
+// tbase): two n-tiles of 8 keys, 8 k-steps each, K fragments by ldmatrix of the raw tile.
+__device__ __forceinline__ void qk_e4m3(uint32_t tbase, int row0, const uint32_t (&qa)[8][4], float (&acc)[2][4],
+                                        int lane) {
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+        const int r = row0 + nt * 8 + (lane & 7);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int chunk = 4 * half + (lane >> 3);
+            uint32_t k[4];
+            ldsm_x4(tbase + r * 128 + ((chunk ^ (r & 7)) << 4), k[0], k[1], k[2], k[3]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                uint32_t b0, b1;
+                e4m3x4_to_f16x2x2(k[j], b0, b1);
+                mma_f16(acc[nt], qa[4 * half + j], b0, b1);
+            }
+        }
+    }
+}
+
+// O += P V for this warp's 16 keys (rows row0 .. row0 + 15 of the tile at tbase).  ldmatrix
+// .trans on b16 units (two dims) gives a thread keys 2t, 2t+1 (and 2t+8, 2t+9) of dims 2g,
+// 2g+1 of a 16-dim chunk; a byte permute regroups them into one f16 pair of keys per dim.
+// Accumulator o[4 G + 2 h + p] then holds dims 32 G + 16 h + 4 t + p (c0, c2) and that + 2
+// (c1, c3), rows g and g + 8.
+__device__ __forceinline__ void pv_e4m3(uint32_t tbase, int row0, const uint32_t (&pa)[4], float (&o)[16][4],
+                                        int lane) {
+    const int j = lane >> 3;
+    const int r = row0 + (j & 1) * 8 + (lane & 7);
+#pragma unroll
+    for (int G = 0; G < 4; ++G) {
+        const int chunk = 2 * G + (j >> 1);
+        uint32_t v[4];
+        ldsm_x4_t(tbase + r * 128 + ((chunk ^ (r & 7)) << 4), v[0], v[1], v[2], v[3]);
+#pragma unroll
+        for (int hs = 0; hs < 2; ++hs) {
+            uint32_t e0, o0, e1, o1;
+            e4m3x4_to_f16x2x2(prmt(v[2 * hs], 0u, 0x3120u), e0, o0);        // keys 2t, 2t+1
+            e4m3x4_to_f16x2x2(prmt(v[2 * hs + 1], 0u, 0x3120u), e1, o1);    // keys 2t+8, 2t+9
+            mma_f16(o[4 * G + 2 * hs], pa, e0, e1);
+            mma_f16(o[4 * G + 2 * hs + 1], pa, o0, o1);
+        }
+    }
+}
+
 __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
     const float mn = fmaxf(m, m2);
     if (mn == -INFINITY) return;
@@ -111,9 +210,8 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* raw = smem;
-    uint8_t* cvt = smem + STAGES * L::RAW;
-    uint64_t* full = reinterpret_cast<uint64_t*>(cvt + L::CVT);
-    __shared__ float red_m[4][H], red_l[4][H];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::RAW);
+    __shared__ float red_m[4][H], red_l[4][H], red_v[4];
 
     const int b = blockIdx.y, split = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
@@ -142,37 +240,60 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
     if (tid == 0)
         for (int s = 0; s < STAGES && s < n_tiles; ++s) issue(s, s);
 
+    // e4m3 keys: f16 MMAs straight from the raw tile (Q in f16, k order permuted, scaled
+    // by 1 / qscale); the largest V scale of the split is kept for pass B's f16 P
     uint32_t qa[8][4];
-    load_q_frags(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
+    float qscale = 1.f, vmax = 0.f;
+    if (KV8) qscale = load_q_frags_e4m3(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
+    else load_q_frags(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
 
     float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
     float* Sg = a.S + (static_cast<size_t>(b) * H + g) * a.s_ld;
     float* Sg8 = Sg + static_cast<size_t>(8) * a.s_ld;
     const float* ksc = KV8 ? a.k_scale + b * a.cap : nullptr;
+    const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
+    const float sc2 = a.sc2 * qscale;
+    // e4m3: this thread's four key scales (and V scales) of the next tile, loaded one tile
+    // ahead so that their latency stays off the tile's path
+    auto load_scales = [&](int i, float (&ks)[4], float (&vs)[4]) {
+        const int key0 = k_begin + i * TILE + warp * 16 + 2 * t;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int key = key0 + (e >> 1) * 8 + (e & 1);
+            const bool in = key < k_end && i < n_tiles;
+            ks[e] = in ? __ldg(ksc + key) : 0.f;
+            vs[e] = in ? __ldg(vsc + key) : 0.f;
+        }
+    };
+    float ks_next[4] = {0.f, 0.f, 0.f, 0.f}, vs_next[4] = {0.f, 0.f, 0.f, 0.f};
+    if (KV8) load_scales(0, ks_next, vs_next);
 
     for (int i = 0; i < n_tiles; ++i) {
         const int s = i % STAGES;
         bool ok = mbar_wait(&full[s], (i / STAGES) & 1, a.status);
         const int tile_key0 = k_begin + i * TILE;
         const uint8_t* tile = raw + s * L::RAW;
-        if (KV8) {
-            convert_tile(tile, cvt, tile_key0, k_end - 1, tid);
-            __syncthreads();
-            tile = cvt;
-        }
+        float ks_cur[4], vs_cur[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { ks_cur[e] = ks_next[e]; vs_cur[e] = vs_next[e]; }
+        if (KV8) load_scales(i + 1, ks_next, vs_next);
         const uint32_t tbase = smem_u32(tile);
         float acc[2][4];
+        if (KV8) {
+            qk_e4m3(tbase, warp * 16, qa, acc, lane);
+        } else {
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
+            for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-            const int r = warp * 16 + nt * 8 + (lane & 7);
+                for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+                const int r = warp * 16 + nt * 8 + (lane & 7);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(tbase + swz_off<TILE>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
-                mma_bf16(acc[nt], qa[2 * kk], b0, b1);
-                mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+                for (int kk = 0; kk < 4; ++kk) {
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(tbase + swz_off<TILE>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+                    mma_bf16(acc[nt], qa[2 * kk], b0, b1);
+                    mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+                }
             }
         }
         // logits (log2 units), masked past the last key
@@ -181,10 +302,11 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
             const int key = key0 + nt * 8;
-            float f0 = a.sc2, f1 = a.sc2;
+            float f0 = sc2, f1 = sc2;
             if (KV8) {
-                f0 *= (key < k_end) ? ksc[key] : 0.f;
-                f1 *= (key + 1 < k_end) ? ksc[key + 1] : 0.f;
+                f0 *= ks_cur[2 * nt];
+                f1 *= ks_cur[2 * nt + 1];
+                vmax = fmaxf(vmax, fmaxf(vs_cur[2 * nt], vs_cur[2 * nt + 1]));
             }
             acc[nt][0] = (key < k_end) ? acc[nt][0] * f0 : -INFINITY;
             acc[nt][1] = (key + 1 < k_end) ? acc[nt][1] * f1 : -INFINITY;
@@ -227,12 +349,20 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
         red_m[warp][g] = m2[0]; red_l[warp][g] = l2[0];
         red_m[warp][g + 8] = m2[1]; red_l[warp][g + 8] = l2[1];
     }
+    if (KV8) {
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+        if (lane == 0) red_v[warp] = vmax;
+    }
     __syncthreads();
     if (tid < H) {
         float m = red_m[0][tid], l = red_l[0][tid];
         for (int w = 1; w < 4; ++w) merge_ml(m, l, red_m[w][tid], red_l[w][tid]);
         a.part_ml[(static_cast<size_t>(b) * a.splits + split) * H + tid] = make_float2(m, l);
     }
+    if (KV8 && tid == 0)
+        a.part_vmax[static_cast<size_t>(b) * a.splits + split] =
+            fmaxf(fmaxf(red_v[0], red_v[1]), fmaxf(red_v[2], red_v[3]));
 }
 
 // ------------------------------------------------------------------ pass B
@@ -243,8 +373,7 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     constexpr int STAGE = L::RAW + L::STILE;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* cvt = smem + STAGES * STAGE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(cvt + L::CVT);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE);
     float4* red_o4 = reinterpret_cast<float4*>(smem);              // [4][16][32] after the tiles
 
     const int b = blockIdx.y, split = blockIdx.x;
@@ -305,6 +434,16 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
     const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
     float* score_row = a.scores + b * a.score_ld;
+    // e4m3 values: P V in f16 with P * v_scale * 2^pe, the largest product of the split
+    // (at most its largest V scale, P <= 1) scaled to 2^14 or below; O is scaled back
+    float pscale = 1.f, pinv = 1.f;
+    if (KV8) {
+        const float vm = a.part_vmax[static_cast<size_t>(b) * a.splits + split];
+        int ex = 0;
+        if (vm > 0.f) frexpf(vm, &ex);          // vm < 2^ex
+        pscale = ldexpf(1.f, 14 - ex);
+        pinv = ldexpf(1.f, ex - 14);
+    }
 
     for (int i = 0; i < n_tiles; ++i) {
         const int s = i % STAGES;
@@ -313,9 +452,14 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
         const int tile_key0 = k_begin + i * TILE;
         uint8_t* vt = st;
         if (KV8) {
-            convert_tile(st, cvt, tile_key0, k_end - 1, tid);
-            vt = cvt;
-            __syncthreads();
+            if (tile_key0 + TILE > k_end) {
+                // tail tile: zero the e4m3 rows past the last key (codes there may be NaN)
+                for (int it = tid; it < TILE * 8; it += NT) {
+                    const int r = it >> 3, c = it & 7;
+                    if (tile_key0 + r >= k_end) *reinterpret_cast<uint4*>(vt + r * 128 + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+                __syncthreads();
+            }
         } else if (tile_key0 + TILE > k_end) {
             // tail tile: zero the V rows past the last key (cache rows there may hold
             // anything, and 0 * NaN would poison the accumulators)
@@ -352,24 +496,30 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
             if (v2) score_row[kh] = sc[2];
             if (v3) score_row[kh + 1] = sc[3];
         }
-        float f0 = 1.f, f1 = 1.f, f2 = 1.f, f3 = 1.f;
-        if (KV8) {
-            f0 = v0 ? vsc[kl] : 0.f; f1 = v1 ? vsc[kl + 1] : 0.f;
-            f2 = v2 ? vsc[kh] : 0.f; f3 = v3 ? vsc[kh + 1] : 0.f;
-        }
-        uint32_t pa[4];
-        pa[0] = pack_bf16(p00 * f0, p01 * f1);
-        pa[1] = pack_bf16(p10 * f0, p11 * f1);
-        pa[2] = pack_bf16(p02 * f2, p03 * f3);
-        pa[3] = pack_bf16(p12 * f2, p13 * f3);
         const uint32_t vbase = smem_u32(vt);
-        const int vr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        if (KV8) {
+            const float f0 = v0 ? vsc[kl] * pscale : 0.f, f1 = v1 ? vsc[kl + 1] * pscale : 0.f;
+            const float f2 = v2 ? vsc[kh] * pscale : 0.f, f3 = v3 ? vsc[kh + 1] * pscale : 0.f;
+            uint32_t pa[4];
+            pa[0] = pack_f16(p00 * f0, p01 * f1);
+            pa[1] = pack_f16(p10 * f0, p11 * f1);
+            pa[2] = pack_f16(p02 * f2, p03 * f3);
+            pa[3] = pack_f16(p12 * f2, p13 * f3);
+            pv_e4m3(vbase, warp * 16, pa, o, lane);
+        } else {
+            uint32_t pa[4];
+            pa[0] = pack_bf16(p00, p01);
+            pa[1] = pack_bf16(p10, p11);
+            pa[2] = pack_bf16(p02, p03);
+            pa[3] = pack_bf16(p12, p13);
+            const int vr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vbase + swz_off<TILE>(vr, 2 * c + (lane >> 4)), b0, b1, b2, b3);
-            mma_bf16(o[2 * c], pa, b0, b1);
-            mma_bf16(o[2 * c + 1], pa, b2, b3);
+            for (int c = 0; c < 8; ++c) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vbase + swz_off<TILE>(vr, 2 * c + (lane >> 4)), b0, b1, b2, b3);
+                mma_bf16(o[2 * c], pa, b0, b1);
+                mma_bf16(o[2 * c + 1], pa, b2, b3);
+            }
         }
         if (__syncthreads_or(!ok)) break;
         if (tid == 0 && i + STAGES < n_tiles) issue(i + STAGES, s);
@@ -378,10 +528,12 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     // this split's O partial: the 4 warps' accumulators through shared memory (the stage
     // area, free once every tile is consumed) as [warp][n][lane] float4 (conflict-free),
     // each (n, lane) slot summed over the warps in a fixed order; the partials of all splits
-    // are summed by dec_merge_kernel
+    // are summed by dec_merge_kernel.  e4m3: accumulator n holds dims 32 (n / 4) + 16 ((n / 2)
+    // % 2) + 4 t + n % 2 and that + 2 (see pv_e4m3), scaled by pscale.
     __syncthreads();
 #pragma unroll
-    for (int n = 0; n < 16; ++n) red_o4[(warp * 16 + n) * 32 + lane] = make_float4(o[n][0], o[n][1], o[n][2], o[n][3]);
+    for (int n = 0; n < 16; ++n)
+        red_o4[(warp * 16 + n) * 32 + lane] = make_float4(o[n][0] * pinv, o[n][1] * pinv, o[n][2] * pinv, o[n][3] * pinv);
     __syncthreads();
     float* my = a.part_o + (static_cast<size_t>(b) * a.splits + split) * H * D;
 #pragma unroll
@@ -393,9 +545,18 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
             const float4 v = red_o4[w4 * 512 + e];
             sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
         }
-        const int d = 8 * n + 2 * (ln & 3), h = ln >> 2;
-        *reinterpret_cast<float2*>(my + h * D + d) = make_float2(sum.x, sum.y);
-        *reinterpret_cast<float2*>(my + (h + 8) * D + d) = make_float2(sum.z, sum.w);
+        const int h = ln >> 2, tq = ln & 3;
+        if (KV8) {
+            const int d = 32 * (n >> 2) + 16 * ((n >> 1) & 1) + 4 * tq + (n & 1);
+            my[h * D + d] = sum.x;
+            my[h * D + d + 2] = sum.y;
+            my[(h + 8) * D + d] = sum.z;
+            my[(h + 8) * D + d + 2] = sum.w;
+        } else {
+            const int d = 8 * n + 2 * tq;
+            *reinterpret_cast<float2*>(my + h * D + d) = make_float2(sum.x, sum.y);
+            *reinterpret_cast<float2*>(my + (h + 8) * D + d) = make_float2(sum.z, sum.w);
+        }
     }
 }
 
@@ -863,11 +1024,11 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
 }
 
 template <bool KV8>
-size_t smem_a() { return 1024 + STAGES * Layout<KV8>::RAW + Layout<KV8>::CVT + STAGES * 8; }
+size_t smem_a() { return 1024 + STAGES * Layout<KV8>::RAW + STAGES * 8; }
 template <bool KV8>
 size_t smem_b() {
     static_assert(STAGES * (Layout<KV8>::RAW + Layout<KV8>::STILE) >= 4 * H * D * 4, "O partials reuse the stages");
-    return 1024 + STAGES * (Layout<KV8>::RAW + Layout<KV8>::STILE) + Layout<KV8>::CVT + STAGES * 8;
+    return 1024 + STAGES * (Layout<KV8>::RAW + Layout<KV8>::STILE) + STAGES * 8;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -888,9 +1049,9 @@ cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
     ws += align256(sizeof(float2) * da.batch * pl.splits * H);
     a.part_o = reinterpret_cast<float*>(ws);
     ws += align256(sizeof(float) * da.batch * pl.splits * H * D);
-    // two-kernel path: per-sequence semaphores in the workspace, reset by pass A;
+    a.part_vmax = reinterpret_cast<float*>(ws);                      // two-kernel path, e4m3
     // fused path: three [B] counters in the status block (zero when idle)
-    a.counter = pl.fused ? reinterpret_cast<int*>(da.status) + kCounterOffsetInts : reinterpret_cast<int*>(ws);
+    a.counter = reinterpret_cast<int*>(da.status) + kCounterOffsetInts;
     a.o = static_cast<__nv_bfloat16*>(da.o);
     a.lse = da.lse;
     a.scores = da.scores; a.score_ld = da.score_ld;
@@ -965,8 +1126,8 @@ DecodePlan plan_decode(int batch, int64_t max_ctx, bool kv8) {
     pl.fused = false;
     pl.wb = 0;
     // two-kernel path: two CTAs per SM suffice to stream a bf16 cache; e4m3 tiles are
-    // converted in shared memory, which takes three (as many as pass B fits per SM)
-    int splits = ((kv8 ? 3 : 2) * num_sms()) / (batch > 0 ? batch : 1);
+    // decoded in registers with per-key scales, which takes four
+    int splits = ((kv8 ? 4 : 2) * num_sms()) / (batch > 0 ? batch : 1);
     if (splits < 1) splits = 1;
     int64_t chunk = (max_ctx + splits - 1) / splits;
     chunk = (chunk + TILE - 1) / TILE * TILE;
@@ -982,7 +1143,7 @@ size_t decode_ws_bytes(int batch, int64_t max_ctx, bool kv8) {
     const DecodePlan pl = plan_decode(batch, max_ctx, kv8);
     return align256(sizeof(float) * batch * H * static_cast<size_t>(pl.s_ld)) +
            align256(sizeof(float2) * batch * pl.splits * H) +
-           align256(sizeof(float) * batch * pl.splits * H * D) + align256(sizeof(int) * batch);
+           align256(sizeof(float) * batch * pl.splits * H * D) + align256(sizeof(float) * batch * pl.splits);
 }
 
 cudaError_t launch_decode_full(const DecodeArgs& a, cudaStream_t st) {
