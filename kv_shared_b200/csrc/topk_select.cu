@@ -44,7 +44,7 @@ namespace {
 constexpr int NT = 512;
 constexpr int NW = NT / 32;
 constexpr int NBINS = 2048;
-constexpr int kMaxCluster = 8;
+constexpr int kMaxCluster = 16;           // 16 is a non-portable cluster size (few long rows)
 constexpr int kSmemKeys = 24576;          // keys cached per CTA (96 KB)
 constexpr int kCandCap = 2048;            // candidates per CTA (16 KB), a power of two
 constexpr int kWarpCap = 512;             // streamed compaction: matches buffered per warp
@@ -838,10 +838,12 @@ int pick_cluster(int rows, int64_t max_keys) {
     // enough rows to fill the GPU: one CTA per row (keys streamed when they do not fit)
     if (rows >= 2 * num_sms()) return 1;
     int cs = 1;
-    while (cs < kMaxCluster && (max_keys + cs - 1) / cs > kSmemKeys) cs *= 2;
+    while (cs < 8 && (max_keys + cs - 1) / cs > kSmemKeys) cs *= 2;
     const int target = 2 * num_sms();
-    while (cs < kMaxCluster && static_cast<int64_t>(rows) * cs * 2 <= target && max_keys / (cs * 2) >= 1024)
+    while (cs < 8 && static_cast<int64_t>(rows) * cs * 2 <= target && max_keys / (cs * 2) >= 1024)
         cs *= 2;
+    // a few rows still streamed from global memory by 8 CTAs each: 16 per row
+    if (cs == 8 && (max_keys + 7) / 8 > kSmemKeys && rows * 16 <= num_sms()) cs = 16;
     return cs;
 }
 
@@ -851,33 +853,51 @@ cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
     if (a.rows <= 0) return cudaSuccess;
     const int bs = a.block_size < 1 ? 1 : a.block_size;
     const int64_t max_keys = (a.max_ctx + bs - 1) / bs;
-    const int cs = pick_cluster(a.rows, max_keys);
-    const int64_t per = ((max_keys + cs - 1) / cs + 3) & ~int64_t(3);
-    const int cache_keys = per <= kSmemKeys ? static_cast<int>(per) : 0;
-    const size_t smem = (static_cast<size_t>(cache_keys) + 2 * kCandCap + (cache_keys == 0 ? 2 * NW * kWarpCap : 0)) *
-                        sizeof(uint32_t);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(a.rows) * cs);
-    cfg.blockDim = dim3(NT);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cs;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    auto launch = [&](auto kern) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        return cudaLaunchKernelEx(&cfg, kern, a, cache_keys);
-    };
-    switch (cs) {
-        case 1: return launch(select_kernel<1>);
-        case 2: return launch(select_kernel<2>);
-        case 4: return launch(select_kernel<4>);
-        default: return launch(select_kernel<8>);
+    int cs = pick_cluster(a.rows, max_keys);
+    for (;;) {
+        const int64_t per = ((max_keys + cs - 1) / cs + 3) & ~int64_t(3);
+        const int cache_keys = per <= kSmemKeys ? static_cast<int>(per) : 0;
+        const size_t smem = (static_cast<size_t>(cache_keys) + 2 * kCandCap + (cache_keys == 0 ? 2 * NW * kWarpCap : 0)) *
+                            sizeof(uint32_t);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(a.rows) * cs);
+        cfg.blockDim = dim3(NT);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = cs;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        auto prepare = [&](auto kern) {
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            if (e == cudaSuccess && cs > 8) e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+            return e;
+        };
+        auto launch = [&](auto kern) {
+            cudaError_t e = prepare(kern);
+            if (e != cudaSuccess) return e;
+            return cudaLaunchKernelEx(&cfg, kern, a, cache_keys);
+        };
+        if (cs == 16) {
+            // a 16-CTA cluster must fit a GPC with this shared memory; otherwise 8
+            int n = 0;
+            if (prepare(select_kernel<16>) != cudaSuccess ||
+                cudaOccupancyMaxActiveClusters(&n, select_kernel<16>, &cfg) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                cs = 8;
+                continue;
+            }
+            return launch(select_kernel<16>);
+        }
+        switch (cs) {
+            case 1: return launch(select_kernel<1>);
+            case 2: return launch(select_kernel<2>);
+            case 4: return launch(select_kernel<4>);
+            default: return launch(select_kernel<8>);
+        }
     }
 }
 
