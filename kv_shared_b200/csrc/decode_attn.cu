@@ -16,8 +16,9 @@
 //
 // K is read once (pass A) and V once (pass B): 512 B of cache per key plus the
 // 64-B logit round trip.  Tiles of 64 keys stream through a 4-stage TMA pipeline
-// with 128-byte swizzle; e4m3 caches are converted to bf16 in shared memory
-// (exact) and the per-token scales are folded into the logits and into P.
+// with 128-byte swizzle; e4m3 tiles feed f16 MMAs straight from shared memory
+// (e4m3 -> f16 is exact) and the per-token scales are folded into the logits and
+// into P.
 #include "common.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -56,7 +57,6 @@ struct Params {
 template <bool KV8>
 struct Layout {
     static constexpr int RAW = KV8 ? TILE * 128 : TILE * 256;   // one cache tile as loaded
-    static constexpr int CVT = KV8 ? TILE * 256 : 0;            // bf16 copy (e4m3 only)
     static constexpr int STILE = 16 * 32 * 4 * 2;               // logits tile: 2 boxes 16x32 fp32
 };
 
@@ -76,29 +76,7 @@ __device__ __forceinline__ void load_q_frags(const __nv_bfloat16* qb, int g, int
     }
 }
 
-// e4m3 tile (64 rows x 128 B, 128-byte swizzle) -> bf16 tile (swz_off layout),
-// rows whose key is past `last` are zeroed.
-__device__ __forceinline__ void convert_tile(const uint8_t* raw, uint8_t* cvt, int key0, int last, int tid) {
-#pragma unroll
-    for (int it = tid; it < TILE * 8; it += NT) {
-        const int r = it >> 3, c8 = it & 7;
-        uint4 in = *reinterpret_cast<const uint4*>(raw + r * 128 + ((c8 ^ (r & 7)) << 4));
-        uint4 lo, hi;
-        if (key0 + r <= last) {
-            const uint16_t* b = reinterpret_cast<const uint16_t*>(&in);
-            lo.x = e4m3x2_to_bf16x2(b[0]); lo.y = e4m3x2_to_bf16x2(b[1]);
-            lo.z = e4m3x2_to_bf16x2(b[2]); lo.w = e4m3x2_to_bf16x2(b[3]);
-            hi.x = e4m3x2_to_bf16x2(b[4]); hi.y = e4m3x2_to_bf16x2(b[5]);
-            hi.z = e4m3x2_to_bf16x2(b[6]); hi.w = e4m3x2_to_bf16x2(b[7]);
-        } else {
-            lo = make_uint4(0, 0, 0, 0); hi = lo;
-        }
-        *reinterpret_cast<uint4*>(cvt + swz_off<TILE>(r, 2 * c8)) = lo;
-        *reinterpret_cast<uint4*>(cvt + swz_off<TILE>(r, 2 * c8 + 1)) = hi;
-    }
-}
-
-// ---- e4m3 tiles without a conversion pass (the two-kernel path): f16 MMAs fed straight
+// ---- e4m3 tiles without a conversion pass: f16 MMAs fed straight
 // from the tile as TMA wrote it (64 rows of 128 B, 128-byte swizzle); e4m3 -> f16 is exact.
 
 // f16 A-fragments of Q for keys from e4m3 tiles.  Within each 16-dim step the k order is
@@ -616,9 +594,9 @@ constexpr size_t kFusedMinSmem = 120 * 1024;   // more than half an SM: one CTA 
 
 template <bool KV8>
 struct FusedLayout {
-    static constexpr int FS = KV8 ? 12 : 8;    // stages of the K/V stream
-    static constexpr size_t BYTES =
-        1024 + FS * Layout<KV8>::RAW + 2 * Layout<KV8>::CVT + 2 * FS * 8 + 8 * H * D * 4;
+    static constexpr int FS = KV8 ? 16 : 8;    // stages of the K/V stream (128 KB)
+    static constexpr size_t VSC = KV8 ? kFusedMaxTiles * TILE * 4 : 0;   // V scales of the split
+    static constexpr size_t BYTES = 1024 + FS * Layout<KV8>::RAW + 2 * FS * 8 + 8 * H * D * 4 + VSC;
 };
 
 __device__ __forceinline__ void bar_sync(int id, int n) {
@@ -654,11 +632,11 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
     constexpr int FS = FusedLayout<KV8>::FS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
-    uint8_t* cvt_base = smem + FS * L::RAW;                           // [2][CVT] (e4m3 only)
-    uint64_t* full = reinterpret_cast<uint64_t*>(cvt_base + 2 * L::CVT);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + FS * L::RAW);
     uint64_t* empty = full + FS;
     float4* red_o4 = reinterpret_cast<float4*>(empty + FS);          // [8][16][32] O partials
-    __shared__ float red_m[8][H], red_l[8][H];
+    float* vsm = reinterpret_cast<float*>(red_o4 + 8 * 16 * 32);      // [64 tiles][64] (e4m3)
+    __shared__ float red_m[8][H], red_l[8][H], red_v[8];
     __shared__ float2 lse_part[FCONS / H][H];
     __shared__ float lse_s[H];
     __shared__ uint32_t tmem_base;
@@ -731,7 +709,6 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
     } else {
         // ---------------- consumers: group c takes tiles c, c + 2, ...; q = warp quarter
         const int c = warp >> 2, q = warp & 3, gtid = tid & 127;
-        uint8_t* cvt = cvt_base + c * L::CVT;
         auto take = [&](uint32_t ld) -> bool {    // warp-uniform; false once the CTA aborts
             if (__any_sync(0xffffffffu, s_abort != 0)) return false;
             const bool okw = __all_sync(0xffffffffu, mbar_wait(&full[ld % FS], (ld / FS) & 1u, a.status));
@@ -748,35 +725,60 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
             int k_end;
             const int n_tiles = tiles_of(w, k_end);
 
-            // ---- pass A: logits to tensor memory, running (max, sum) per head
+            // ---- pass A: logits to tensor memory, running (max, sum) per head.  e4m3 keys:
+            // f16 MMAs straight from the raw tile (Q in f16, k order permuted, scaled by
+            // 1 / qscale); the largest V scale of the split is kept for pass B's f16 P
             uint32_t qa[8][4];
-            load_q_frags(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
+            float qscale = 1.f, vmax = 0.f;
+            if (KV8) qscale = load_q_frags_e4m3(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
+            else load_q_frags(a.q + static_cast<size_t>(b) * H * D, g, t, qa);
+            const float sc2 = a.sc2 * qscale;
             float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.f, 0.f};
             const float* ksc = KV8 ? a.k_scale + b * a.cap : nullptr;
+            const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
+            // e4m3: lane l of a warp holds the key scale (l < 16) or the V scale (l >= 16) of
+            // key l % 16 of its 16 keys of a tile: one coalesced load per tile, issued four of the
+            // group's tiles ahead so that the memory latency stays off the tile's path.  The V
+            // scales also go to shared memory for pass B (the same warp reads them back).
+            auto load_sc = [&](int i) -> float {
+                const int key = k_begin + i * TILE + q * 16 + (lane & 15);
+                return (i < n_tiles && key < k_end) ? __ldg((lane < 16 ? ksc : vsc) + key) : 0.f;
+            };
+            float sc_p[4] = {0.f, 0.f, 0.f, 0.f};
+            if (KV8)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) sc_p[j] = load_sc(c + 2 * j);
             for (int i = c; i < n_tiles; i += 2) {
                 const uint32_t ld = wbase + i;
+                const float sc_cur = sc_p[0];
+                if (KV8) {
+                    sc_p[0] = sc_p[1]; sc_p[1] = sc_p[2]; sc_p[2] = sc_p[3];
+                    sc_p[3] = load_sc(i + 8);
+                    if (lane >= 16) {
+                        vmax = fmaxf(vmax, sc_cur);
+                        vsm[i * TILE + q * 16 + (lane & 15)] = sc_cur;
+                    }
+                }
                 const bool okt = take(ld);
                 const int tile_key0 = k_begin + i * TILE;
-                const uint8_t* tile = smem + (ld % FS) * L::RAW;
-                if (KV8) {
-                    if (okt) convert_tile(tile, cvt, tile_key0, k_end - 1, gtid);
-                    bar_sync(1 + c, 128);
-                    tile = cvt;
-                }
+                const uint32_t tbase = smem_u32(smem + (ld % FS) * L::RAW);
                 if (okt) {
-                    const uint32_t tbase = smem_u32(tile);
                     float acc[2][4];
+                    if (KV8) {
+                        qk_e4m3(tbase, q * 16, qa, acc, lane);
+                    } else {
 #pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
+                        for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-                        const int r = q * 16 + nt * 8 + (lane & 7);
+                            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+                            const int r = q * 16 + nt * 8 + (lane & 7);
 #pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            uint32_t b0, b1, b2, b3;
-                            ldsm_x4(tbase + swz_off<TILE>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
-                            mma_bf16(acc[nt], qa[2 * kk], b0, b1);
-                            mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                uint32_t b0, b1, b2, b3;
+                                ldsm_x4(tbase + swz_off<TILE>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+                                mma_bf16(acc[nt], qa[2 * kk], b0, b1);
+                                mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+                            }
                         }
                     }
                     const int key0 = tile_key0 + q * 16 + 2 * t;
@@ -785,10 +787,10 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt) {
                         const int key = key0 + nt * 8;
-                        float f0 = a.sc2, f1 = a.sc2;
+                        float f0 = sc2, f1 = sc2;
                         if (KV8) {
-                            f0 *= (key < k_end) ? ksc[key] : 0.f;
-                            f1 *= (key + 1 < k_end) ? ksc[key + 1] : 0.f;
+                            f0 *= __shfl_sync(0xffffffffu, sc_cur, nt * 8 + 2 * t);
+                            f1 *= __shfl_sync(0xffffffffu, sc_cur, nt * 8 + 2 * t + 1);
                         }
                         acc[nt][0] = (key < k_end) ? acc[nt][0] * f0 : -INFINITY;
                         acc[nt][1] = (key + 1 < k_end) ? acc[nt][1] * f1 : -INFINITY;
@@ -814,7 +816,6 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                         }
                     }
                 }
-                if (KV8) bar_sync(1 + c, 128);    // the group's converted tile is reused next
                 release(ld);
             }
             umma::tmem_st_wait();
@@ -832,7 +833,24 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                 red_m[warp][g] = m2[0]; red_l[warp][g] = l2[0];
                 red_m[warp][g + 8] = m2[1]; red_l[warp][g + 8] = l2[1];
             }
+            if (KV8) {
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+                if (lane == 0) red_v[warp] = vmax;
+            }
             bar_sync(3, FCONS);
+            // e4m3 values: P V in f16 with P * v_scale * 2^pe, the largest product of the split
+            // (at most its largest V scale, P <= 1) scaled to 2^14 or below; O is scaled back
+            float pscale = 1.f, pinv = 1.f;
+            if (KV8) {
+                float vm = red_v[0];
+#pragma unroll
+                for (int k = 1; k < 8; ++k) vm = fmaxf(vm, red_v[k]);
+                int ex = 0;
+                if (vm > 0.f) frexpf(vm, &ex);      // vm < 2^ex
+                pscale = ldexpf(1.f, 14 - ex);
+                pinv = ldexpf(1.f, ex - 14);
+            }
             if (tid < H) {
                 float m = red_m[0][tid], l = red_l[0][tid];
                 for (int k = 1; k < 8; ++k) merge_ml(m, l, red_m[k][tid], red_l[k][tid]);
@@ -875,29 +893,41 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
             float o[16][4];
 #pragma unroll
             for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-            const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
             float* score_row = a.scores + b * a.score_ld;
             for (int i = c; i < n_tiles; i += 2) {
                 const uint32_t ld = wbase + n_tiles + i;
                 uint32_t sr[8];
                 umma::tmem_ld16x256_x2(tmem + (static_cast<uint32_t>(32 * q + 16 * (i >> 5)) << 16) + 16 * (i & 31),
                                        sr);
-                const bool okt = take(ld);
                 const int tile_key0 = k_begin + i * TILE;
+                const int kl = tile_key0 + q * 16 + 2 * t, kh = kl + 8;
+                const bool v0 = kl < k_end, v1 = kl + 1 < k_end, v2 = kh < k_end, v3 = kh + 1 < k_end;
+                float f0 = 1.f, f1 = 1.f, f2 = 1.f, f3 = 1.f;
+                if (KV8) {                        // V scales kept by pass A (zero past the end)
+                    const float* vs = vsm + (kl - k_begin);
+                    f0 = vs[0] * pscale; f1 = vs[1] * pscale; f2 = vs[8] * pscale; f3 = vs[9] * pscale;
+                }
+                const bool okt = take(ld);
                 uint8_t* vt = smem + (ld % FS) * L::RAW;
-                if (KV8) {
-                    if (okt) convert_tile(vt, cvt, tile_key0, k_end - 1, gtid);
-                    bar_sync(1 + c, 128);
-                    vt = cvt;
-                } else if (tile_key0 + TILE > k_end) {
-                    // tail tile: zero the V rows past the last key (0 * NaN would poison O); the
-                    // stage is refilled by TMA later, so order these writes before the async proxy
-                    if (okt)
-                        for (int it = gtid; it < TILE * 16; it += 128) {
-                            const int r = it >> 4, cc = it & 15;
-                            if (tile_key0 + r >= k_end)
-                                *reinterpret_cast<uint4*>(vt + swz_off<TILE>(r, cc)) = make_uint4(0, 0, 0, 0);
+                if (tile_key0 + TILE > k_end) {
+                    // tail tile: zero the V rows past the last key (cache rows there may hold
+                    // anything, and 0 * NaN would poison O); the stage is refilled by TMA later,
+                    // so order these writes before the async proxy
+                    if (okt) {
+                        if (KV8) {
+                            for (int it = gtid; it < TILE * 8; it += 128) {
+                                const int r = it >> 3, cc = it & 7;
+                                if (tile_key0 + r >= k_end)
+                                    *reinterpret_cast<uint4*>(vt + r * 128 + cc * 16) = make_uint4(0, 0, 0, 0);
+                            }
+                        } else {
+                            for (int it = gtid; it < TILE * 16; it += 128) {
+                                const int r = it >> 4, cc = it & 15;
+                                if (tile_key0 + r >= k_end)
+                                    *reinterpret_cast<uint4*>(vt + swz_off<TILE>(r, cc)) = make_uint4(0, 0, 0, 0);
+                            }
                         }
+                    }
                     umma::fence_proxy_async();
                     bar_sync(1 + c, 128);
                 }
@@ -907,8 +937,6 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                     const float2 sg8l = make_float2(__uint_as_float(sr[2]), __uint_as_float(sr[3]));
                     const float2 sgh = make_float2(__uint_as_float(sr[4]), __uint_as_float(sr[5]));
                     const float2 sg8h = make_float2(__uint_as_float(sr[6]), __uint_as_float(sr[7]));
-                    const int kl = tile_key0 + q * 16 + 2 * t, kh = kl + 8;
-                    const bool v0 = kl < k_end, v1 = kl + 1 < k_end, v2 = kh < k_end, v3 = kh + 1 < k_end;
                     const float p00 = v0 ? ex2(sgl.x - lse2[0]) : 0.f, p01 = v1 ? ex2(sgl.y - lse2[0]) : 0.f;
                     const float p10 = v0 ? ex2(sg8l.x - lse2[1]) : 0.f, p11 = v1 ? ex2(sg8l.y - lse2[1]) : 0.f;
                     const float p02 = v2 ? ex2(sgh.x - lse2[0]) : 0.f, p03 = v3 ? ex2(sgh.y - lse2[0]) : 0.f;
@@ -924,36 +952,41 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                         if (v2) score_row[kh] = sc[2];
                         if (v3) score_row[kh + 1] = sc[3];
                     }
-                    float f0 = 1.f, f1 = 1.f, f2 = 1.f, f3 = 1.f;
-                    if (KV8) {
-                        f0 = v0 ? vsc[kl] : 0.f; f1 = v1 ? vsc[kl + 1] : 0.f;
-                        f2 = v2 ? vsc[kh] : 0.f; f3 = v3 ? vsc[kh + 1] : 0.f;
-                    }
-                    uint32_t pa[4];
-                    pa[0] = pack_bf16(p00 * f0, p01 * f1);
-                    pa[1] = pack_bf16(p10 * f0, p11 * f1);
-                    pa[2] = pack_bf16(p02 * f2, p03 * f3);
-                    pa[3] = pack_bf16(p12 * f2, p13 * f3);
                     const uint32_t vbase = smem_u32(vt);
-                    const int vr = q * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+                    uint32_t pa[4];
+                    if (KV8) {
+                        pa[0] = pack_f16(p00 * f0, p01 * f1);
+                        pa[1] = pack_f16(p10 * f0, p11 * f1);
+                        pa[2] = pack_f16(p02 * f2, p03 * f3);
+                        pa[3] = pack_f16(p12 * f2, p13 * f3);
+                        pv_e4m3(vbase, q * 16, pa, o, lane);
+                    } else {
+                        pa[0] = pack_bf16(p00, p01);
+                        pa[1] = pack_bf16(p10, p11);
+                        pa[2] = pack_bf16(p02, p03);
+                        pa[3] = pack_bf16(p12, p13);
+                        const int vr = q * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-                    for (int cv = 0; cv < 8; ++cv) {
-                        uint32_t b0, b1, b2, b3;
-                        ldsm_x4_t(vbase + swz_off<TILE>(vr, 2 * cv + (lane >> 4)), b0, b1, b2, b3);
-                        mma_bf16(o[2 * cv], pa, b0, b1);
-                        mma_bf16(o[2 * cv + 1], pa, b2, b3);
+                        for (int cv = 0; cv < 8; ++cv) {
+                            uint32_t b0, b1, b2, b3;
+                            ldsm_x4_t(vbase + swz_off<TILE>(vr, 2 * cv + (lane >> 4)), b0, b1, b2, b3);
+                            mma_bf16(o[2 * cv], pa, b0, b1);
+                            mma_bf16(o[2 * cv + 1], pa, b2, b3);
+                        }
                     }
                 }
-                if (KV8) bar_sync(1 + c, 128);
                 release(ld);
             }
 
             // ---- this split's O partial: the 8 warps' accumulators go to shared memory as
             // [warp][n][lane] float4 (conflict-free), then each (n, lane) slot is summed over the
-            // warps in a fixed order; the last split of the sequence merges the partials at the end
+            // warps in a fixed order; the partials are merged at the end.  e4m3: accumulator n
+            // holds dims 32 (n / 4) + 16 ((n / 2) % 2) + 4 t + n % 2 and that + 2 (see pv_e4m3),
+            // scaled by pscale
 #pragma unroll
             for (int n = 0; n < 16; ++n)
-                red_o4[(warp * 16 + n) * 32 + lane] = make_float4(o[n][0], o[n][1], o[n][2], o[n][3]);
+                red_o4[(warp * 16 + n) * 32 + lane] =
+                    make_float4(o[n][0] * pinv, o[n][1] * pinv, o[n][2] * pinv, o[n][3] * pinv);
             bar_sync(3, FCONS);
             float* my = a.part_o + (static_cast<size_t>(b) * a.splits + split) * H * D;
 #pragma unroll
@@ -965,9 +998,18 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                     const float4 v = red_o4[w8 * 512 + e];
                     sum.x += v.x; sum.y += v.y; sum.z += v.z; sum.w += v.w;
                 }
-                const int d = 8 * n + 2 * (ln & 3), h = ln >> 2;
-                *reinterpret_cast<float2*>(my + h * D + d) = make_float2(sum.x, sum.y);
-                *reinterpret_cast<float2*>(my + (h + 8) * D + d) = make_float2(sum.z, sum.w);
+                const int h = ln >> 2, tq = ln & 3;
+                if (KV8) {
+                    const int d = 32 * (n >> 2) + 16 * ((n >> 1) & 1) + 4 * tq + (n & 1);
+                    my[h * D + d] = sum.x;
+                    my[h * D + d + 2] = sum.y;
+                    my[(h + 8) * D + d] = sum.z;
+                    my[(h + 8) * D + d + 2] = sum.w;
+                } else {
+                    const int d = 8 * n + 2 * tq;
+                    *reinterpret_cast<float2*>(my + h * D + d) = make_float2(sum.x, sum.y);
+                    *reinterpret_cast<float2*>(my + (h + 8) * D + d) = make_float2(sum.z, sum.w);
+                }
             }
             bar_sync(3, FCONS);
             if (tid == 0 && !s_abort) {
