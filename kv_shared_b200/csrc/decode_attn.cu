@@ -231,30 +231,29 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
     const float* ksc = KV8 ? a.k_scale + b * a.cap : nullptr;
     const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
     const float sc2 = a.sc2 * qscale;
-    // e4m3: this thread's four key scales (and V scales) of the next tile, loaded one tile
-    // ahead so that their latency stays off the tile's path
-    auto load_scales = [&](int i, float (&ks)[4], float (&vs)[4]) {
-        const int key0 = k_begin + i * TILE + warp * 16 + 2 * t;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int key = key0 + (e >> 1) * 8 + (e & 1);
-            const bool in = key < k_end && i < n_tiles;
-            ks[e] = in ? __ldg(ksc + key) : 0.f;
-            vs[e] = in ? __ldg(vsc + key) : 0.f;
-        }
+    // e4m3: lane l of a warp holds the key scale (l < 16) or the V scale (l >= 16) of key
+    // l % 16 of its 16 keys of a tile: one coalesced load per tile, issued four tiles ahead
+    // so that the memory latency stays off the tile's path
+    auto load_sc = [&](int i) -> float {
+        const int key = k_begin + i * TILE + warp * 16 + (lane & 15);
+        return (i < n_tiles && key < k_end) ? __ldg((lane < 16 ? ksc : vsc) + key) : 0.f;
     };
-    float ks_next[4] = {0.f, 0.f, 0.f, 0.f}, vs_next[4] = {0.f, 0.f, 0.f, 0.f};
-    if (KV8) load_scales(0, ks_next, vs_next);
+    float sc_p[4] = {0.f, 0.f, 0.f, 0.f};
+    if (KV8)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sc_p[j] = load_sc(j);
 
     for (int i = 0; i < n_tiles; ++i) {
         const int s = i % STAGES;
+        const float sc_cur = sc_p[0];
+        if (KV8) {
+            sc_p[0] = sc_p[1]; sc_p[1] = sc_p[2]; sc_p[2] = sc_p[3];
+            sc_p[3] = load_sc(i + 4);
+            if (lane >= 16) vmax = fmaxf(vmax, sc_cur);
+        }
         bool ok = mbar_wait(&full[s], (i / STAGES) & 1, a.status);
         const int tile_key0 = k_begin + i * TILE;
         const uint8_t* tile = raw + s * L::RAW;
-        float ks_cur[4], vs_cur[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) { ks_cur[e] = ks_next[e]; vs_cur[e] = vs_next[e]; }
-        if (KV8) load_scales(i + 1, ks_next, vs_next);
         const uint32_t tbase = smem_u32(tile);
         float acc[2][4];
         if (KV8) {
@@ -282,9 +281,8 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
             const int key = key0 + nt * 8;
             float f0 = sc2, f1 = sc2;
             if (KV8) {
-                f0 *= ks_cur[2 * nt];
-                f1 *= ks_cur[2 * nt + 1];
-                vmax = fmaxf(vmax, fmaxf(vs_cur[2 * nt], vs_cur[2 * nt + 1]));
+                f0 *= __shfl_sync(0xffffffffu, sc_cur, nt * 8 + 2 * t);
+                f1 *= __shfl_sync(0xffffffffu, sc_cur, nt * 8 + 2 * t + 1);
             }
             acc[nt][0] = (key < k_end) ? acc[nt][0] * f0 : -INFINITY;
             acc[nt][1] = (key + 1 < k_end) ? acc[nt][1] * f1 : -INFINITY;
@@ -422,9 +420,24 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
         pscale = ldexpf(1.f, 14 - ex);
         pinv = ldexpf(1.f, ex - 14);
     }
+    // e4m3: lane l holds the V scale of key l % 16 of the warp's 16 keys of a tile, loaded
+    // four tiles ahead (one coalesced load per tile)
+    auto load_vs = [&](int i) -> float {
+        const int key = k_begin + i * TILE + warp * 16 + (lane & 15);
+        return (i < n_tiles && key < k_end) ? __ldg(vsc + key) : 0.f;
+    };
+    float vs_p[4] = {0.f, 0.f, 0.f, 0.f};
+    if (KV8)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) vs_p[j] = load_vs(j);
 
     for (int i = 0; i < n_tiles; ++i) {
         const int s = i % STAGES;
+        const float vs_cur = vs_p[0];
+        if (KV8) {
+            vs_p[0] = vs_p[1]; vs_p[1] = vs_p[2]; vs_p[2] = vs_p[3];
+            vs_p[3] = load_vs(i + 4);
+        }
         bool ok = mbar_wait(&full[s], (i / STAGES) & 1, a.status);
         uint8_t* st = smem + s * STAGE;
         const int tile_key0 = k_begin + i * TILE;
@@ -476,8 +489,10 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
         }
         const uint32_t vbase = smem_u32(vt);
         if (KV8) {
-            const float f0 = v0 ? vsc[kl] * pscale : 0.f, f1 = v1 ? vsc[kl + 1] * pscale : 0.f;
-            const float f2 = v2 ? vsc[kh] * pscale : 0.f, f3 = v3 ? vsc[kh + 1] * pscale : 0.f;
+            const float f0 = __shfl_sync(0xffffffffu, vs_cur, 2 * t) * pscale;
+            const float f1 = __shfl_sync(0xffffffffu, vs_cur, 2 * t + 1) * pscale;
+            const float f2 = __shfl_sync(0xffffffffu, vs_cur, 2 * t + 8) * pscale;
+            const float f3 = __shfl_sync(0xffffffffu, vs_cur, 2 * t + 9) * pscale;
             uint32_t pa[4];
             pa[0] = pack_f16(p00 * f0, p01 * f1);
             pa[1] = pack_f16(p10 * f0, p11 * f1);
