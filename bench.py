@@ -68,8 +68,9 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, interval_ms=200):
         self.dev = device_index
+        self.interval_ms = interval_ms
         self.proc = None
         self.lines = []
 
@@ -77,7 +78,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -290,12 +291,13 @@ def run_prefill(args, ws_):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(graphs) + 1)] for _ in range(K)]
     _barrier(ws_)
     torch.cuda.synchronize()
-    for i in range(K):
-        ev[i][0].record(stream)
-        for j, g in enumerate(graphs):
-            g.replay()
-            ev[i][j + 1].record(stream)
-    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device(), interval_ms=50) as clk:
+        for i in range(K):
+            ev[i][0].record(stream)
+            for j, g in enumerate(graphs):
+                g.replay()
+                ev[i][j + 1].record(stream)
+        torch.cuda.synchronize()
     step_ms = _max_over_ranks(ws_, statistics.mean(e[0].elapsed_time(e[-1]) for e in ev))
     bridge_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     full_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
@@ -320,6 +322,7 @@ def run_prefill(args, ws_):
                       "hbm_frac": bridge_bytes / (bridge_ms / 1e3) / 1e9 / hbm},
         "sparse_attn": {"ms": sparse_ms},
         "gpu_launches": K * blk.launches_per_step,
+        "clocks": clk.summary(),
     }
 
 

@@ -90,15 +90,22 @@ __device__ __forceinline__ void load_entries(const Params& a, int row, int e_beg
 }
 
 template <bool KV8>
-__global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
+__global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) {
     using L = Layout<KV8>;
+    using sparse::STAGES;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = sparse::align1024(smem_raw);
-    uint8_t* cvt = smem + 2 * L::STAGE;                    // e4m3 only: K bf16 then V bf16
-    float* red_o = reinterpret_cast<float*>(cvt + L::CVT); // [H][D]
-    int* sidx = reinterpret_cast<int*>(red_o + H * D);     // [chunk] cache row per entry (-1 invalid)
+    uint8_t* smem = sparse::align128(smem_raw);
+    uint8_t* cvt = smem + STAGES * L::STAGE;               // e4m3 only: K bf16 then V bf16
+    int* sidx = reinterpret_cast<int*>(cvt + L::CVT);      // [chunk] cache row per entry (-1 invalid)
     float* sks = reinterpret_cast<float*>(sidx + a.chunk); // [chunk] k scales (e4m3)
     float* svs = sks + a.chunk;                            // [chunk] v scales (e4m3)
+    // after the sub-tiles the stages (and the e4m3 tiles after them) hold the warp slabs,
+    // then these:
+    float* red_o = reinterpret_cast<float*>(smem + L::SLABS);                  // [H][D]
+    float2 (*sml)[H] = reinterpret_cast<float2 (*)[H]>(red_o + H * D);        // [kMaxSplits][H]
+    float (*sw)[H] = reinterpret_cast<float (*)[H]>(sml + kMaxSplits);        // [kMaxSplits][H]
+    static_assert(L::SLABS + H * D * 4 + kMaxSplits * H * 12 <= STAGES * L::STAGE + L::CVT,
+                  "merge scratch fits the stage area");
     __shared__ float wm[4][H], wl[4][H], cm[H], cl[H];
     __shared__ int s_last;
 
@@ -117,23 +124,23 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
 
     uint32_t qa[8][4];
     sparse::load_q(a.q + static_cast<size_t>(row) * H * D, qa, lane >> 2, lane & 3);
-    auto gather = [&](int i, int st) {
-        sparse::gather_rows<KV8>(smem + st * L::STAGE, sidx + i * SUB, a.k, a.v, seq_base, tid);
+    auto gather = [&](int i) {
+        sparse::gather_rows<KV8>(smem + (i % STAGES) * L::STAGE, sidx + i * SUB, a.k, a.v, seq_base, tid);
         cp_async_commit();
     };
-    if (n_sub > 0) gather(0, 0);
-    if (n_sub > 1) gather(1, 1);
+    static_assert(STAGES == 2 || STAGES == 3, "the group waits below allow one or two gathers in flight");
+    for (int i = 0; i < STAGES - 1 && i < n_sub; ++i) gather(i);
 
     sparse::State stt;
     stt.init();
     for (int i = 0; i < n_sub; ++i) {
-        const int st = i & 1;
-        if (i + 1 < n_sub) cp_async_wait<1>(); else cp_async_wait<0>();
+        // sub-tile i landed (with three stages the gather of i + 1 could stay in flight);
+        // the barrier also ends every warp's reads of sub-tile i - 1, whose stage is refilled
+        if (i + 1 < n_sub) cp_async_wait<STAGES - 2>(); else cp_async_wait<0>();
         __syncthreads();
-        sparse::attend_subtile<KV8>(smem + st * L::STAGE, cvt, sidx + i * SUB, sks + i * SUB, svs + i * SUB, qa,
-                                    a.sc2, stt, tid, warp, lane);
-        __syncthreads();
-        if (i + 2 < n_sub) gather(i + 2, st);
+        if (i + STAGES - 1 < n_sub) gather(i + STAGES - 1);
+        sparse::attend_subtile<KV8>(smem + (i % STAGES) * L::STAGE, cvt, sidx + i * SUB, sks + i * SUB,
+                                    svs + i * SUB, qa, a.sc2, stt, tid, warp, lane);
     }
     sparse::cta_reduce(stt, reinterpret_cast<float*>(smem), red_o, wm, wl, cm, cl, tid, warp, lane);
 
@@ -160,8 +167,6 @@ __global__ void __launch_bounds__(NT) sparse_kernel(Params a) {
     // merge the splits: every split's (max, sum) is staged in shared memory by one
     // parallel round of loads, then the partial outputs are weighted and summed with
     // independent 16-byte loads (4 per thread per split)
-    __shared__ float2 sml[kMaxSplits][H];
-    __shared__ float sw[kMaxSplits][H];
     __shared__ float fm[H], finv[H];
     const float2* pml = a.part_ml + static_cast<size_t>(row) * a.splits * H;
     for (int i = tid; i < a.splits * H; i += NT) sml[i / H][i % H] = __ldcg(pml + i);
@@ -483,7 +488,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 template <bool KV8>
 size_t smem_bytes(int chunk) {
     using L = Layout<KV8>;
-    return 1024 + 2 * L::STAGE + L::CVT + H * D * 4 + static_cast<size_t>(chunk) * 4 * (KV8 ? 3 : 1);
+    return 128 + sparse::STAGES * L::STAGE + L::CVT + static_cast<size_t>(chunk) * 4 * (KV8 ? 3 : 1);
 }
 
 template <bool KV8>

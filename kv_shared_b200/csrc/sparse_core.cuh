@@ -15,17 +15,25 @@ constexpr int D = 128;
 constexpr int SUB = 64;            // gathered rows per sub-tile
 constexpr int NT = 128;            // 4 warps x 16 rows
 constexpr int RP = D + 4;          // padded slab row (floats) of the warp merge
+// Two sub-tile buffers (one gather in flight while the other is attended) and three CTAs
+// per SM: with two CTAs per SM a third buffer bought nothing, while a third CTA hides the
+// latency of the per-warp MMA chains and softmax (about a fifth less time per layer).
+constexpr int STAGES = 2;
+constexpr int MIN_CTAS = 3;        // resident CTAs per SM the register budget must allow
 
+// A stage holds SUB K rows then SUB V rows as copied, each row padded by 16 bytes so that
+// the 8 rows an ldmatrix phase reads fall on distinct banks.
 template <bool KV8>
 struct Layout {
     static constexpr int ROWB = KV8 ? 128 : 256;      // bytes per gathered cache row
-    static constexpr int STAGE = 2 * SUB * ROWB;       // K rows then V rows
+    static constexpr int ROWP = ROWB + 16;             // row pitch in a stage
+    static constexpr int STAGE = 2 * SUB * ROWP;       // K rows then V rows
     static constexpr int CVT = KV8 ? 2 * SUB * 256 : 0;
     static constexpr int SLABS = 4 * H * RP * 4;       // warp-merge slabs (bytes)
 };
 
-__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
-    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+__device__ __forceinline__ uint8_t* align128(uint8_t* p) {
+    return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 127) & ~uintptr_t(127));
 }
 
 __device__ __forceinline__ void merge_ml(float& m, float& l, float m2, float l2) {
@@ -62,44 +70,45 @@ __device__ __forceinline__ void load_q(const __nv_bfloat16* qrow, uint32_t (&qa)
 
 // Issues the 16-byte cp.async copies of the SUB gathered rows `si` (cache row per
 // entry, -1 = none: zero-filled) into stage `st` (K rows, then V rows); no commit.
+// Consecutive lanes copy consecutive chunks of a row (whole rows per instruction).
 template <bool KV8>
 __device__ __forceinline__ void gather_rows(uint8_t* st, const int* si, const uint8_t* k, const uint8_t* v,
                                             size_t seq_base, int tid) {
     using L = Layout<KV8>;
     constexpr int CH = L::ROWB / 16;                   // 16-byte chunks per row
+#pragma unroll 4
     for (int it = tid; it < SUB * CH; it += NT) {
         const int r = it / CH, ch = it % CH;
         const int j = si[r];
         const size_t off = (seq_base + (j >= 0 ? j : 0)) * L::ROWB + ch * 16;
-        uint32_t dk, dv;
-        if (KV8) {
-            dk = r * 128 + ((ch ^ (r & 7)) << 4);
-            dv = SUB * 128 + dk;
-        } else {
-            dk = swz_off<SUB>(r, ch);
-            dv = SUB * 256 + dk;
-        }
-        cp_async16_zfill(st + dk, k + off, j >= 0);
-        cp_async16_zfill(st + dv, v + off, j >= 0);
+        const uint32_t d = r * L::ROWP + ch * 16;
+        cp_async16_zfill(st + d, k + off, j >= 0);
+        cp_async16_zfill(st + SUB * L::ROWP + d, v + off, j >= 0);
     }
 }
 
 // One landed sub-tile (stage `st`): e4m3 rows are first converted to bf16 in `cvt`
-// (exact; contains a CTA barrier, so every thread calls this), then this warp's 16
-// rows are scored against the 16 heads, the online softmax advanced and P V added.
+// (exact, swizzled layout; contains a CTA barrier, so every thread calls this), then this
+// warp's 16 rows are scored against the 16 heads, the online softmax advanced and P V added.
 // `si` / `sks` / `svs`: the sub-tile's cache rows and (e4m3) per-token scales.
 template <bool KV8>
 __device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, const int* si, const float* sks,
                                                const float* svs, const uint32_t (&qa)[8][4], float sc2, State& s,
                                                int tid, int warp, int lane) {
+    using L = Layout<KV8>;
     const int t = lane & 3;
     const uint8_t* kt = st;
-    const uint8_t* vt = st + SUB * Layout<KV8>::ROWB;
+    const uint8_t* vt = st + SUB * L::ROWP;
+    // byte offset of 16-byte chunk ch of row r: padded rows as copied (bf16), the
+    // swizzled converted tile (e4m3)
+    auto off = [](int r, int ch) -> uint32_t {
+        return KV8 ? swz_off<SUB>(r, ch) : static_cast<uint32_t>(r * L::ROWP + ch * 16);
+    };
     if (KV8) {
-        // e4m3 rows (128-byte swizzle) -> bf16 tiles (swz_off layout), exact
+        // e4m3 rows -> bf16 tiles (swz_off layout), exact
         for (int it = tid; it < 2 * SUB * 8; it += NT) {
             const int half = it / (SUB * 8), rr = (it / 8) % SUB, c8 = it & 7;
-            const uint8_t* src = st + half * SUB * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4);
+            const uint8_t* src = st + half * SUB * L::ROWP + rr * L::ROWP + c8 * 16;
             uint8_t* dst = cvt + half * SUB * 256;
             const uint4 in = *reinterpret_cast<const uint4*>(src);
             const uint16_t* bb = reinterpret_cast<const uint16_t*>(&in);
@@ -126,7 +135,7 @@ __device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, 
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             uint32_t b0, b1, b2, b3;
-            ldsm_x4(kb + swz_off<SUB>(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+            ldsm_x4(kb + off(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
             mma_bf16(acc[nt], qa[2 * kk], b0, b1);
             mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
         }
@@ -186,7 +195,7 @@ __device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, 
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vb + swz_off<SUB>(vr, 2 * cc + (lane >> 4)), b0, b1, b2, b3);
+        ldsm_x4_t(vb + off(vr, 2 * cc + (lane >> 4)), b0, b1, b2, b3);
         mma_bf16(s.o[2 * cc], pa, b0, b1);
         mma_bf16(s.o[2 * cc + 1], pa, b2, b3);
     }
