@@ -167,6 +167,13 @@ def test_decode_bf16_several_waves(batch, ctx):
     _block_parity(wl, seed=1003)
 
 
+def test_decode_e4m3_several_waves():
+    # e4m3 cache through the single-launch path over three waves (per-wave V scales kept
+    # in shared memory, tail tiles of every split)
+    wl = synth.shrink(synth.DECODE_1M_FP8, batch=200, ctx=4096 + 77, needles=16)
+    _block_parity(wl, seed=1007)
+
+
 @pytest.mark.parametrize("kv", ["bf16", "e4m3"])
 def test_decode_ragged_positions(kv):
     # every sequence at its own position: splits past a short sequence's end hold no keys
