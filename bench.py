@@ -34,9 +34,9 @@ import synth  # noqa: E402
 METRIC = "sparse-attn decode queries/s @128K ctx + prefill tokens/s; % HBM & TC roofline"
 FALLBACK_HBM_GBS = 6650.0
 # dram__bytes_read.sum + dram__bytes_write.sum of one hs2_full_attn_select call on the
-# decode workload: 550.7 MB measured at 32768 keys per sequence (ncu capture summarised in
+# decode workload: 550.4 MB measured at 32768 keys per sequence (ncu capture summarised in
 # profiles/decode_kernels_b32_ctx32768.md), times 4 for 131072 keys (linear in keys).
-FULL_CALL_TRAFFIC_BYTES = 4 * 550.7e6
+FULL_CALL_TRAFFIC_BYTES = 4 * 550.4e6
 
 
 def _peaks():

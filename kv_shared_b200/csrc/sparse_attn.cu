@@ -6,13 +6,15 @@
 // cache, so a single softmax covers the whole chosen set.
 //
 // For each query row (16 heads) the selected cache rows are gathered by index
-// with 16-byte cp.async copies into shared memory (swizzled so ldmatrix reads
-// are conflict-free), all 16 heads are computed against each gathered row once
-// (mma.sync m16n8k16, M = the 16 heads), and the softmax stays online in
-// registers.  A row's selected set is split across CTAs when there are few rows
-// (decode); split partials (max, sum, O) are merged by the last CTA of the row
-// (semaphore counter, no spin).  e4m3 rows are converted to bf16 in shared
-// memory (exact) and their per-token scales folded into the logits and into P.
+// with 16-byte cp.async copies into shared memory (swizzled or padded so that
+// ldmatrix reads are conflict-free), all 16 heads are computed against each
+// gathered row once (mma.sync m16n8k16, M = the 16 heads), and the softmax stays
+// online in registers.  Few rows (decode): one 8-CTA cluster per row, the CTAs'
+// partials merged through distributed shared memory.  Many rows (prefill): one
+// CTA per row, or a few split CTAs per row whose partials (max, sum, O) the last
+// of them merges (semaphore counter, no spin).  e4m3 rows are converted to bf16
+// in shared memory (exact) and their per-token scales folded into the logits and
+// into P.
 #include <mutex>
 
 #include <cooperative_groups.h>
