@@ -591,33 +591,35 @@ def _time_graph(fn, stream, reps):
 def run_configs(args):
     """The parity workloads other than the two headline ones, each timed on its own: the
     1M-token e4m3 decode, the selection-granularity sweep (token arm vs the 64-token block
-    arm on the same importance) and the tiny fp32 prefill."""
+    arm on the same importance) and the tiny fp32 prefill; plus the 128K decode shape on an
+    e4m3 cache (informational)."""
     import kv_shared_b200 as hs
     stream = torch.cuda.current_stream()
     hbm, _, _ = _peaks()
     out = {}
 
-    wl = synth.DECODE_1M_FP8
-    blk = ConfigBlock(wl, seed=1004)
-    blk.full(); blk.sparse()
-    torch.cuda.synchronize()
-    if hs.hs2_last_status(blk.ws) != hs.HS2_OK:
-        raise RuntimeError("1M e4m3 decode: device status " + hs.status_string(hs.hs2_last_status(blk.ws)))
-    full_ms = _time_graph(blk.full, stream, 20)
-    sparse_ms = _time_graph(blk.sparse, stream, 50)
-    out["decode_1m_e4m3"] = {
-        "workload": wl.name,
-        "full_attn_select": {"ms": full_ms, "bytes_per_call": blk.cache_bytes(),
-                             "hbm_frac": blk.cache_bytes() / (full_ms / 1e3) / 1e9 / hbm,
-                             "launches": hs.hs2_full_attn_launches(blk.desc)},
-        "sparse_attn": {"ms": sparse_ms, "queries/s": wl.batch / (sparse_ms / 1e3),
-                        "bytes_per_call": blk.sparse_bytes(),
-                        "hbm_frac": blk.sparse_bytes() / (sparse_ms / 1e3) / 1e9 / hbm,
-                        "note": "4 query rows: latency-bound"},
-        "needle_recall": blk.recall(blk.idx.cpu(), blk.cnt.cpu()),
-    }
-    del blk
-    torch.cuda.empty_cache()
+    for key, wl, seed, note in (("decode_1m_e4m3", synth.DECODE_1M_FP8, 1004, "4 query rows: latency-bound"),
+                                ("decode_128k_e4m3", synth.DECODE_128K_FP8, 1008, "32 query rows")):
+        blk = ConfigBlock(wl, seed=seed)
+        blk.full(); blk.sparse()
+        torch.cuda.synchronize()
+        if hs.hs2_last_status(blk.ws) != hs.HS2_OK:
+            raise RuntimeError(wl.name + ": device status " + hs.status_string(hs.hs2_last_status(blk.ws)))
+        full_ms = _time_graph(blk.full, stream, 20)
+        sparse_ms = _time_graph(blk.sparse, stream, 50)
+        out[key] = {
+            "workload": wl.name,
+            "full_attn_select": {"ms": full_ms, "bytes_per_call": blk.cache_bytes(),
+                                 "hbm_frac": blk.cache_bytes() / (full_ms / 1e3) / 1e9 / hbm,
+                                 "launches": hs.hs2_full_attn_launches(blk.desc)},
+            "sparse_attn": {"ms": sparse_ms, "queries/s": wl.batch / (sparse_ms / 1e3),
+                            "bytes_per_call": blk.sparse_bytes(),
+                            "hbm_frac": blk.sparse_bytes() / (sparse_ms / 1e3) / 1e9 / hbm,
+                            "note": note},
+            "needle_recall": blk.recall(blk.idx.cpu(), blk.cnt.cpu()),
+        }
+        del blk
+        torch.cuda.empty_cache()
 
     sweep = []
     for ctx in synth.SWEEP_CTX:

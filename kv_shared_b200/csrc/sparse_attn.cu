@@ -20,6 +20,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "e4m3_mma.cuh"
 #include "internal.h"
 #include "sparse_core.cuh"
 
@@ -227,10 +228,9 @@ template <bool KV8>
 struct CLayout {
     static constexpr int ROWB = KV8 ? 128 : 256;          // bytes per gathered row
     static constexpr int RAW = 2 * kWT * ROWB;            // one warp's gathered K then V rows
-    static constexpr int TILE = 2 * kWT * 256;            // one warp's bf16 K then V tiles
+    static constexpr int TILE = 2 * kWT * 256;            // one warp's bf16 K then V tiles (= RAW)
     static constexpr int RAW_OFF = 0;
-    static constexpr int BF_OFF = KV8 ? kCW * RAW : 0;    // e4m3: converted copies after the raw rows
-    static constexpr int GATHER_END = BF_OFF + kCW * TILE;
+    static constexpr int GATHER_END = kCW * (KV8 ? RAW : TILE);
     static constexpr int SLAB_BYTES = kCW * H * sparse::RP * 4;   // the warps' rescaled O, after the compute
     static constexpr int Q_OFF = GATHER_END > SLAB_BYTES ? GATHER_END : SLAB_BYTES;
     static constexpr int RECV_OFF = Q_OFF + H * D * 2;    // [kCluster][2][D] f32 pushed partials
@@ -313,6 +313,65 @@ __device__ __forceinline__ void attend_warp_tile(const uint8_t* kt, const uint8_
     }
 }
 
+// The same for e4m3 rows: f16 MMAs straight from the gathered rows (128-byte swizzled, see
+// e4m3_mma.cuh); `qa` are Q's f16 fragments in the permuted k order, scaled by 1 / qscale
+// (folded into sc2q); P * v_scale is scaled by a power of two so that the warp's largest
+// product stays at or below 2^14 in f16.  s.o ends in pv_e4m3's accumulator layout (dims
+// permuted), scaled back to plain P V.
+__device__ __forceinline__ void attend_warp_tile_e4m3(uint32_t kb, uint32_t vb, const uint32_t (&qa)[8][4],
+                                                      const bool (&ok)[2][2], const float (&fk)[2][2],
+                                                      const float (&fv)[2][2], float sc2q, float vmax,
+                                                      sparse::State& s, int lane) {
+    float acc[2][4];
+    qk_e4m3(kb, 0, qa, acc, lane);
+    float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        acc[nt][0] = ok[nt][0] ? acc[nt][0] * (sc2q * fk[nt][0]) : -INFINITY;
+        acc[nt][1] = ok[nt][1] ? acc[nt][1] * (sc2q * fk[nt][1]) : -INFINITY;
+        acc[nt][2] = ok[nt][0] ? acc[nt][2] * (sc2q * fk[nt][0]) : -INFINITY;
+        acc[nt][3] = ok[nt][1] ? acc[nt][3] * (sc2q * fk[nt][1]) : -INFINITY;
+        mx[0] = fmaxf(mx[0], fmaxf(acc[nt][0], acc[nt][1]));
+        mx[1] = fmaxf(mx[1], fmaxf(acc[nt][2], acc[nt][3]));
+    }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 1));
+        mx[hh] = fmaxf(mx[hh], __shfl_xor_sync(0xffffffffu, mx[hh], 2));
+        s.m2[hh] = mx[hh];
+    }
+    float pr[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int hh = e >> 1;
+            pr[nt][e] = (mx[hh] == -INFINITY) ? 0.f : ex2(acc[nt][e] - mx[hh]);
+        }
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        float l = pr[0][2 * hh] + pr[0][2 * hh + 1] + pr[1][2 * hh] + pr[1][2 * hh + 1];
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        s.l2[hh] = l;
+    }
+    int ex = 0;
+    if (vmax > 0.f) frexpf(vmax, &ex);                  // vmax < 2^ex
+    const float pscale = ldexpf(1.f, 14 - ex), pinv = ldexpf(1.f, ex - 14);
+    uint32_t pa[4];
+    pa[0] = pack_f16(pr[0][0] * fv[0][0] * pscale, pr[0][1] * fv[0][1] * pscale);
+    pa[1] = pack_f16(pr[0][2] * fv[0][0] * pscale, pr[0][3] * fv[0][1] * pscale);
+    pa[2] = pack_f16(pr[1][0] * fv[1][0] * pscale, pr[1][1] * fv[1][1] * pscale);
+    pa[3] = pack_f16(pr[1][2] * fv[1][0] * pscale, pr[1][3] * fv[1][1] * pscale);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) s.o[n][0] = s.o[n][1] = s.o[n][2] = s.o[n][3] = 0.f;
+    pv_e4m3(vb, 0, pa, s.o, lane);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+        s.o[n][0] *= pinv; s.o[n][1] *= pinv; s.o[n][2] *= pinv; s.o[n][3] *= pinv;
+    }
+}
+
 template <bool KV8>
 __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
     using CL = CLayout<KV8>;
@@ -333,7 +392,8 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
     // just before the pushes
     asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     // the row's queries (16 heads x 128) into shared memory, one 16-byte chunk per thread
-    if (tid < H * 16) {
+    // (bf16 rows; e4m3 rows take Q's fragments straight from global memory)
+    if (!KV8 && tid < H * 16) {
         const int r = tid >> 4, ch = tid & 15;
         cp_async16(qs + swz_off<kWT>(r, ch), reinterpret_cast<const uint8_t*>(a.q + static_cast<size_t>(row) * H * D) +
                                                  r * 256 + ch * 16);
@@ -385,35 +445,25 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
             fk[nt][e] = KV8 ? __shfl_sync(0xffffffffu, ksc, r) : 1.f;
             fv[nt][e] = KV8 ? __shfl_sync(0xffffffffu, vsc, r) : 1.f;
         }
+    // e4m3: Q's f16 fragments and the warp's largest V scale while the rows land
+    uint32_t qa8[8][4];
+    float qscale = 1.f, vmax = 0.f;
+    if (KV8) {
+        qscale = load_q_frags_e4m3(a.q + static_cast<size_t>(row) * H * D, g, t, qa8);
+        vmax = vsc;                                      // 0 for lanes without a row
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, off));
+    }
     cp_async_wait<1>();                                  // the queries (committed first) have landed
     __syncthreads();
     cp_async_wait<0>();                                  // and this warp's rows
     __syncwarp();
-    const uint8_t* kt = raw;
-    const uint8_t* vt = raw + kWT * CL::ROWB;
-    if (KV8) {
-        // e4m3 rows (128-byte swizzle) -> bf16 tiles of this warp (swz_off<16> layout), exact
-        uint8_t* bf = csm + CL::BF_OFF + warp * CL::TILE;
-        for (int it = lane; it < 2 * kWT * 8; it += 32) {
-            const int half = it / (kWT * 8), rr = (it / 8) % kWT, c8 = it & 7;
-            const uint8_t* src = raw + half * kWT * 128 + rr * 128 + ((c8 ^ (rr & 7)) << 4);
-            uint8_t* dst = bf + half * kWT * 256;
-            const uint4 in = *reinterpret_cast<const uint4*>(src);
-            const uint16_t* bb = reinterpret_cast<const uint16_t*>(&in);
-            uint4 lo, hi;
-            lo.x = e4m3x2_to_bf16x2(bb[0]); lo.y = e4m3x2_to_bf16x2(bb[1]);
-            lo.z = e4m3x2_to_bf16x2(bb[2]); lo.w = e4m3x2_to_bf16x2(bb[3]);
-            hi.x = e4m3x2_to_bf16x2(bb[4]); hi.y = e4m3x2_to_bf16x2(bb[5]);
-            hi.z = e4m3x2_to_bf16x2(bb[6]); hi.w = e4m3x2_to_bf16x2(bb[7]);
-            *reinterpret_cast<uint4*>(dst + swz_off<kWT>(rr, 2 * c8)) = lo;
-            *reinterpret_cast<uint4*>(dst + swz_off<kWT>(rr, 2 * c8 + 1)) = hi;
-        }
-        __syncwarp();
-        kt = bf;
-        vt = bf + kWT * 256;
-    }
     sparse::State st;
-    attend_warp_tile(kt, vt, qs, ok, fk, fv, a.sc2, st, lane);
+    if (KV8)
+        attend_warp_tile_e4m3(smem_u32(raw), smem_u32(raw + kWT * CL::ROWB), qa8, ok, fk, fv, a.sc2 * qscale, vmax,
+                              st, lane);
+    else
+        attend_warp_tile(raw, raw + kWT * CL::ROWB, qs, ok, fk, fv, a.sc2, st, lane);
 
     // ---- fold the warps into the push: each warp writes its own (max, sum) and its O
     // (relative to its own max) to a padded slab in the gather area (free once every
@@ -428,9 +478,17 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
     float* slab = slabs + warp * H * RP;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-        const int d = 8 * n + 2 * t;
-        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(st.o[n][0], st.o[n][1]);
-        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(st.o[n][2], st.o[n][3]);
+        if (KV8) {                                       // pv_e4m3's dim order
+            const int d = 32 * (n >> 2) + 16 * ((n >> 1) & 1) + 4 * t + (n & 1);
+            slab[g * RP + d] = st.o[n][0];
+            slab[g * RP + d + 2] = st.o[n][1];
+            slab[(g + 8) * RP + d] = st.o[n][2];
+            slab[(g + 8) * RP + d + 2] = st.o[n][3];
+        } else {
+            const int d = 8 * n + 2 * t;
+            *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(st.o[n][0], st.o[n][1]);
+            *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(st.o[n][2], st.o[n][3]);
+        }
     }
     if (tid < H) {
         float M = -INFINITY;

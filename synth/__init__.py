@@ -69,6 +69,13 @@ DECODE_1M_FP8 = Workload("decode_b4_ctx1048576_h16_d128_e4m3", batch=4, n_q=1, c
                          needle_norm=4.0 * 128 ** 0.5)
 
 
+# Not one of the five: the 128K decode shape with the e4m3 cache recipe of the 1M workload
+# (the single-launch decode kernel on an e4m3 cache; informational in the bench).
+DECODE_128K_FP8 = Workload("decode_b32_ctx131072_h16_d128_e4m3", batch=32, n_q=1, ctx=131072,
+                           heads=16, head_dim=128, kv_dtype="e4m3", needles=16,
+                           needle_norm=4.0 * 128 ** 0.5)
+
+
 def sweep(ctx: int, block_size: int = 1, layout: str = "one_per_block") -> Workload:
     """Selection-granularity sweep: one sequence, decode at p = ctx - 1, 64 planted tokens."""
     return Workload(f"sweep_ctx{ctx}_{'token' if block_size == 1 else 'block%d' % block_size}",
