@@ -550,6 +550,22 @@ __global__ void __launch_bounds__(NT, 2) select_kernel(SelectArgs a, int cache_k
     // read from global memory skips this pass and takes the first digit at the top bits
     uint32_t lo = 0xffffffffu, hi = 0u;
     const bool cached = per <= cache_keys;
+    if (!take_all && !take_none && !cached && warp == 0) {
+        // a streamed slice is read twice (first digit, then compaction): ask for all of it in
+        // L2 at once (bulk prefetch, 16-byte aligned pieces inside the slice) so that the
+        // first pass is not limited by the loads this CTA keeps in flight
+        const int t0 = sl.begin * bs, t1 = min(sl.end * bs, n_cand);
+        const uintptr_t b0 = (reinterpret_cast<uintptr_t>(sl.s + t0) + 15) & ~uintptr_t(15);
+        const uintptr_t b1 = reinterpret_cast<uintptr_t>(sl.s + t1) & ~uintptr_t(15);
+        if (b1 > b0) {
+            const uintptr_t step = ((b1 - b0 + 31) / 32 + 15) & ~uintptr_t(15);
+            const uintptr_t c0 = b0 + lane * step;
+            if (c0 < b1) {
+                const uint32_t n = static_cast<uint32_t>(min(step, b1 - c0));
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(c0), "r"(n) : "memory");
+            }
+        }
+    }
     if (!take_all && !take_none && !cached) {
         lo = 0u;
         hi = 0xffffffffu;
