@@ -7,15 +7,18 @@
 //   [K | V] = hidden [rows x d_model] * W_kv [d_model x 2D],  bf16 in, fp32
 //   accumulation, rounded to bf16 and written to cache rows pos0[b] + t.
 //
-// One CTA computes a 128-row x 256-column tile (all of K and V for 128 tokens):
-//   warp 0        TMA producer: A tile [128 x 64] (K-major, 128-byte swizzle) and
-//                 B tile [64 x 256] as four [64 x 64] boxes of W_kv, which is
+// One CTA computes a 256-row x 256-column tile (all of K and V for 256 tokens) as two
+// M = 128 halves that share every W_kv tile, so that W_kv (re-read from L2 by every CTA)
+// costs half as much traffic per row and the 32768-row agent workload runs in one wave:
+//   warp 0        TMA producer: two A tiles [128 x 64] (K-major, 128-byte swizzle) and
+//                 the B tile [64 x 256] as four [64 x 64] boxes of W_kv, which is
 //                 row-major (d_model x 2D) and therefore an MN-major B operand
-//   warp 1        allocates 256 TMEM columns; one thread issues tcgen05.mma
-//                 (M=128, N=256, K=16) and commits each stage back to the producer
-//   warps 2..5    epilogue: tcgen05.ld of the fp32 accumulator rows (one TMEM lane
-//                 quarter per warp), bf16 rounding, stores into the cache
-// A 4-stage mbarrier pipeline (48 KB per stage) keeps TMA and MMA overlapped.
+//   warp 1        allocates 512 TMEM columns; one thread issues tcgen05.mma
+//                 (M=128, N=256, K=16, one per half) and commits each stage back
+//   warps 2..9    epilogue: tcgen05.ld of the fp32 accumulator rows (warp 2 + 4 h + j
+//                 takes half h, TMEM lane quarter (2 + j) % 4), bf16 rounding, stores
+//                 into the cache
+// A 3-stage mbarrier pipeline (64 KB per stage) keeps TMA and MMA overlapped.
 #include "common.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
@@ -23,14 +26,16 @@
 namespace hs2 {
 namespace {
 
-constexpr int BM = 128;
+constexpr int BM = 128;                      // rows of one MMA half
+constexpr int MH = 2;                        // halves per CTA
+constexpr int BMC = BM * MH;                 // rows per CTA
 constexpr int BN = 256;
 constexpr int BK = 64;                       // one 128-byte swizzle atom of bf16
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr int STAGES = 3;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB per half
 constexpr int B_BYTES = BK * BN * 2;         // 32 KB (four 64x64 boxes)
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NT = 192;
+constexpr int STAGE_BYTES = MH * A_BYTES + B_BYTES;
+constexpr int NT = 64 + 128 * MH;
 
 struct Params {
     int rows;                                // batch * n
@@ -56,8 +61,9 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BM;
+    const int m0 = blockIdx.x * BMC;
     const int nk = a.d_model / BK;
+    const int mh = (m0 + BM < a.rows) ? MH : 1;     // halves holding rows (a partial one is zero-filled)
 
     if (threadIdx.x == 0) {
         prefetch_tmap(&amap);
@@ -67,7 +73,7 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
         fence_mbar_init();
         abort_flag = 0;
     }
-    if (warp == 1) umma::tmem_alloc(&tmem_base, 256);
+    if (warp == 1) umma::tmem_alloc(&tmem_base, 512);
     umma::fence_before();
     __syncthreads();
     umma::fence_after();
@@ -82,11 +88,11 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
                     break;
                 }
                 uint8_t* st = smem + s * STAGE_BYTES;
-                mbar_arrive_expect_tx(&full[s], STAGE_BYTES);
-                tma_load_2d(st, &amap, &full[s], kb * BK, m0);
+                mbar_arrive_expect_tx(&full[s], mh * A_BYTES + B_BYTES);
+                for (int h = 0; h < mh; ++h) tma_load_2d(st + h * A_BYTES, &amap, &full[s], kb * BK, m0 + h * BM);
 #pragma unroll
                 for (int nb = 0; nb < BN / 64; ++nb)
-                    tma_load_2d(st + A_BYTES + nb * (BK * 128), &bmap, &full[s], nb * 64, kb * BK);
+                    tma_load_2d(st + MH * A_BYTES + nb * (BK * 128), &bmap, &full[s], nb * 64, kb * BK);
             }
         }
     } else if (warp == 1) {
@@ -99,15 +105,17 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
                 if (!ok) break;
                 umma::fence_after();
                 const uint32_t sa = smem_u32(smem + s * STAGE_BYTES);
-                const uint32_t sb = sa + A_BYTES;
+                const uint32_t sb = sa + MH * A_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk) {
-                    // A: K-major rows of 128 B; step 16 elements = 32 B inside the atom
-                    const uint64_t ad = umma::sdesc_sw128(sa + kk * 32, 16, 1024);
                     // B: MN-major; 64-column groups 8 KB apart, 8-row K groups 1 KB apart;
                     // step 16 K-rows = 2 KB
                     const uint64_t bd = umma::sdesc_sw128(sb + kk * 2048, BK * 128, 1024);
-                    umma::mma_bf16_ss(tmem, ad, bd, idesc, (kb | kk) != 0);
+                    for (int h = 0; h < mh; ++h) {
+                        // A: K-major rows of 128 B; step 16 elements = 32 B inside the atom
+                        const uint64_t ad = umma::sdesc_sw128(sa + h * A_BYTES + kk * 32, 16, 1024);
+                        umma::mma_bf16_ss(tmem + h * BN, ad, bd, idesc, (kb | kk) != 0);
+                    }
                 }
                 umma::commit(&empty[s]);
             }
@@ -115,9 +123,9 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
             umma::commit(&acc_ready);
         }
     } else {
-        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 = tile rows
-        const int q = warp & 3;
-        const int row = m0 + q * 32 + lane;
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31 of half (w - 2) / 4 = tile rows
+        const int q = warp & 3, h = (warp - 2) >> 2;
+        const int row = m0 + h * BM + q * 32 + lane;
         const bool ok = mbar_wait(&acc_ready, 0, a.status);
         umma::fence_after();
         __nv_bfloat16* dk = nullptr;
@@ -136,7 +144,7 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
             uint32_t r[32];
-            umma::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c * 32, r);
+            umma::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * BN + c * 32, r);
             umma::tmem_ld_wait();
             if (dk && ok) {
                 __nv_bfloat16* dst = (c < 4 ? dk : dv) + (c & 3) * 32;
@@ -156,7 +164,7 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
     __syncthreads();
     if (warp == 1) {
         umma::fence_after();
-        umma::tmem_dealloc(tmem, 256);
+        umma::tmem_dealloc(tmem, 512);
     }
 }
 
@@ -179,7 +187,7 @@ cudaError_t launch_bridge(const BridgeArgs& ba, cudaStream_t st) {
     const size_t smem = 1024 + STAGES * STAGE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(bridge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    bridge_kernel<<<(rows + BM - 1) / BM, NT, smem, st>>>(amap, bmap, a);
+    bridge_kernel<<<(rows + BMC - 1) / BMC, NT, smem, st>>>(amap, bmap, a);
     return cudaGetLastError();
 }
 
