@@ -148,6 +148,28 @@ def test_sparse_attn_bad_index_reports_status():
     assert dev.status() == hs.HS2_OK          # the word is cleared once read
 
 
+def test_decode_wait_timeout_reports_status():
+    # The splits of a sequence in the single-launch decode wait (bounded, 2 s) on counters in
+    # the workspace's status block.  Counters that can never reach their target make every
+    # such wait run out: the call must come back with HS2_ERR_TIMEOUT, the context must stay
+    # usable, and after hs2_workspace_init the same workspace must give the normal result.
+    wl = synth.shrink(synth.DECODE_128K, batch=2, ctx=20000, needles=4)
+    dev = Dev(synth.make_inputs(wl, seed=1009))
+    dev.full()
+    assert dev.status() == hs.HS2_OK
+    ref = [t.clone() for t in (dev.o_full, dev.idx, dev.cnt, dev.scores)]
+    status_ints = dev.ws[:4096].view(torch.int32)
+    status_ints[1:] = -(10 ** 9)                     # every counter far below any split count
+    dev.scores.zero_()
+    dev.full()
+    assert dev.status() == hs.HS2_ERR_TIMEOUT
+    hs.hs2_workspace_init(dev.ws)
+    dev.full()
+    assert dev.status() == hs.HS2_OK
+    for got, want in zip((dev.o_full, dev.idx, dev.cnt, dev.scores), ref):
+        assert torch.equal(got, want)
+
+
 # ------------------------------------------------------------------ whole hybrid block
 def test_tiny_f32_block_all_rows():
     rep = _block_parity(synth.TINY, seed=1001)
