@@ -355,7 +355,7 @@ def run_ours(args, ws_, rank, local):
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     _barrier(ws_)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, interval_ms=50) as clk:
         start.record(stream)
         for i in range(K):
             step_graph.replay()
