@@ -167,10 +167,14 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
     sparse::cta_reduce(stt, reinterpret_cast<float*>(smem), red_o, wm, wl, cm, cl, tid, warp, lane);
 
     if (a.splits == 1) {
-        for (int i = tid; i < H * D; i += NT) {
-            const int h = i / D;
-            const float val = cl[h] > 0.f ? red_o[i] / cl[h] : 0.f;
-            a.o[static_cast<size_t>(row) * H * D + i] = __float2bfloat16_rn(val);
+        for (int i = tid; i < H * D / 4; i += NT) {
+            const int h = (4 * i) / D;
+            const float inv = cl[h] > 0.f ? 1.f / cl[h] : 0.f;
+            const float4 v = *reinterpret_cast<const float4*>(&red_o[4 * i]);
+            uint2 packed;
+            packed.x = pack_bf16(v.x * inv, v.y * inv);
+            packed.y = pack_bf16(v.z * inv, v.w * inv);
+            *reinterpret_cast<uint2*>(a.o + static_cast<size_t>(row) * H * D + 4 * i) = packed;
         }
         if (a.lse && tid < H)
             a.lse[static_cast<size_t>(row) * H + tid] = cl[tid] > 0.f ? (cm[tid] + log2f(cl[tid])) * kLn2 : -INFINITY;

@@ -15,6 +15,7 @@ constexpr int D = 128;
 constexpr int SUB = 64;            // gathered rows per sub-tile
 constexpr int NT = 128;            // 4 warps x 16 rows
 constexpr int RP = D + 4;          // padded slab row (floats) of the warp merge
+static_assert((RP * 4) % 16 == 0, "slab rows stay 16-byte aligned");
 // Two sub-tile buffers (one gather in flight while the other is attended) and three CTAs
 // per SM: with two CTAs per SM a third buffer bought nothing, while a third CTA hides the
 // latency of the per-warp MMA chains and softmax (about a fifth less time per layer).
@@ -234,10 +235,15 @@ __device__ __forceinline__ void cta_reduce(const State& s, float* slabs, float* 
         *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(s.o[n][2] * f[1], s.o[n][3] * f[1]);
     }
     __syncthreads();
-    for (int i = tid; i < H * D; i += NT) {
-        const int h = i / D, d = i % D;
-        red_o[i] = slabs[h * RP + d] + slabs[H * RP + h * RP + d] + slabs[2 * H * RP + h * RP + d] +
-                   slabs[3 * H * RP + h * RP + d];
+    for (int i = tid; i < H * D / 4; i += NT) {            // 16-byte slab reads (RP * 4 B is a multiple of 16)
+        const int h = (4 * i) / D, d = (4 * i) % D;
+        float4 acc = *reinterpret_cast<const float4*>(&slabs[h * RP + d]);
+#pragma unroll
+        for (int w = 1; w < 4; ++w) {
+            const float4 u = *reinterpret_cast<const float4*>(&slabs[w * H * RP + h * RP + d]);
+            acc.x += u.x; acc.y += u.y; acc.z += u.z; acc.w += u.w;
+        }
+        *reinterpret_cast<float4*>(&red_o[4 * i]) = acc;
     }
     if (tid < H) {
         const float Mh = fmaxf(fmaxf(wm[0][tid], wm[1][tid]), fmaxf(wm[2][tid], wm[3][tid]));
