@@ -117,7 +117,9 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
     using sparse::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = sparse::align128(smem_raw);
-    uint8_t* cvt = smem + STAGES * L::STAGE;               // e4m3 only: K bf16 then V bf16
+    using WS = sparse::WarpSlot<KV8>;
+    static_assert(4 * WS::BYTES == L::STAGE && 4 * WS::CVT == L::CVT, "four warps' slots make a sub-tile");
+    uint8_t* cvt = smem + STAGES * L::STAGE;               // e4m3 only: each warp's K bf16 then V bf16
     int* sidx = reinterpret_cast<int*>(cvt + L::CVT);      // [chunk] cache row per entry (-1 invalid)
     float* sks = reinterpret_cast<float*>(sidx + a.chunk); // [chunk] k scales (e4m3)
     float* svs = sks + a.chunk;                            // [chunk] v scales (e4m3)
@@ -146,23 +148,33 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
     sparse::load_q(a.q + static_cast<size_t>(row) * H * D, qa, lane >> 2, lane & 3);
     load_entries<KV8>(a, row, e_begin, a.chunk, a.chunk, c, sidx, sks, svs, seq_base);
     __syncthreads();
+    // this warp's rows 16 warp .. 16 warp + 15 of every sub-tile, through its own STAGES slots
+    uint8_t* wslots = smem + warp * STAGES * WS::BYTES;
+    uint8_t* wcvt = cvt + warp * WS::CVT;
     auto gather = [&](int i) {
-        sparse::gather_rows<KV8>(smem + (i % STAGES) * L::STAGE, sidx + i * SUB, a.k, a.v, seq_base, tid);
+        sparse::gather_warp_rows<KV8>(wslots + (i % STAGES) * WS::BYTES, sidx + i * SUB + warp * 16, a.k, a.v,
+                                      seq_base, lane);
         cp_async_commit();
     };
-    static_assert(STAGES == 2 || STAGES == 3, "the group waits below allow one or two gathers in flight");
-    for (int i = 0; i < STAGES - 1 && i < n_sub; ++i) gather(i);
+    static_assert(STAGES == 2, "one gather in flight per warp while the other slot is attended");
+    if (n_sub > 0) gather(0);
 
     sparse::State stt;
     stt.init();
     for (int i = 0; i < n_sub; ++i) {
-        // sub-tile i landed (with three stages the gather of i + 1 could stay in flight);
-        // the barrier also ends every warp's reads of sub-tile i - 1, whose stage is refilled
-        if (i + 1 < n_sub) cp_async_wait<STAGES - 2>(); else cp_async_wait<0>();
-        __syncthreads();
-        if (i + STAGES - 1 < n_sub) gather(i + STAGES - 1);
-        sparse::attend_subtile<KV8>(smem + (i % STAGES) * L::STAGE, cvt, sidx + i * SUB, sks + i * SUB,
-                                    svs + i * SUB, qa, a.sc2, stt, tid, warp, lane);
+        // the slot of sub-tile i - 1 (read by this warp's last, completed, step) takes i + 1;
+        // then sub-tile i must have landed, every lane's copies visible to the warp
+        __syncwarp();
+        if (i + 1 < n_sub) {
+            gather(i + 1);
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncwarp();
+        const int e = i * SUB + warp * 16;
+        sparse::attend_warp_rows<KV8>(wslots + (i % STAGES) * WS::BYTES, wcvt, sidx + e, sks + e, svs + e, qa, a.sc2,
+                                      stt, lane);
     }
     sparse::cta_reduce(stt, reinterpret_cast<float*>(smem), red_o, wm, wl, cm, cl, tid, warp, lane);
 

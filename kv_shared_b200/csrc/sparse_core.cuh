@@ -1,6 +1,5 @@
-// sparse_core.cuh -- the per-CTA arithmetic of the sparse-attention layer, shared
-// by the split kernel (global-memory merge) and the cluster kernel (merge through
-// distributed shared memory): one 64-row gathered sub-tile against the 16 query
+// sparse_core.cuh -- the per-CTA arithmetic of the many-rows sparse-attention
+// kernel: each warp's 16 gathered rows of a 64-row sub-tile against the 16 query
 // heads (mma.sync m16n8k16, M = the heads, online softmax in registers), and the
 // reduction of the four warps' states to one (max, sum, O) per head.
 #pragma once
@@ -16,7 +15,7 @@ constexpr int SUB = 64;            // gathered rows per sub-tile
 constexpr int NT = 128;            // 4 warps x 16 rows
 constexpr int RP = D + 4;          // padded slab row (floats) of the warp merge
 static_assert((RP * 4) % 16 == 0, "slab rows stay 16-byte aligned");
-// Two sub-tile buffers (one gather in flight while the other is attended) and three CTAs
+// Two buffers per warp (one gather in flight while the other is attended) and three CTAs
 // per SM: with two CTAs per SM a third buffer bought nothing, while a third CTA hides the
 // latency of the per-warp MMA chains and softmax (about a fifth less time per layer).
 constexpr int STAGES = 2;
@@ -69,48 +68,60 @@ __device__ __forceinline__ void load_q(const __nv_bfloat16* qrow, uint32_t (&qa)
     }
 }
 
-// Issues the 16-byte cp.async copies of the SUB gathered rows `si` (cache row per
-// entry, -1 = none: zero-filled) into stage `st` (K rows, then V rows); no commit.
-// Consecutive lanes copy consecutive chunks of a row (whole rows per instruction).
+// Each warp gathers and attends its own 16 rows of every 64-row sub-tile, with its own
+// buffers and cp.async groups, so that no warp waits for another's rows.  A warp's slot
+// holds its 16 K rows, then its 16 V rows, each padded by 16 bytes so that the 8 rows an
+// ldmatrix phase reads fall on distinct banks.
 template <bool KV8>
-__device__ __forceinline__ void gather_rows(uint8_t* st, const int* si, const uint8_t* k, const uint8_t* v,
-                                            size_t seq_base, int tid) {
+struct WarpSlot {
+    static constexpr int BYTES = 2 * 16 * Layout<KV8>::ROWP;
+    static constexpr int CVT = KV8 ? 2 * 16 * 256 : 0;      // the warp's converted K, V (e4m3)
+};
+
+// Issues the 16-byte cp.async copies of this warp's 16 rows `si` (cache row per entry, -1 =
+// none: zero-filled) into its slot `ws`; consecutive lanes copy consecutive chunks of a row.
+// No commit.
+template <bool KV8>
+__device__ __forceinline__ void gather_warp_rows(uint8_t* ws, const int* si, const uint8_t* k, const uint8_t* v,
+                                                 size_t seq_base, int lane) {
     using L = Layout<KV8>;
     constexpr int CH = L::ROWB / 16;                   // 16-byte chunks per row
-#pragma unroll 4
-    for (int it = tid; it < SUB * CH; it += NT) {
-        const int r = it / CH, ch = it % CH;
+    constexpr int RPI = 32 / CH;                       // rows per instruction
+    const int ch = lane % CH;
+#pragma unroll
+    for (int u = 0; u < 16 / RPI; ++u) {
+        const int r = u * RPI + lane / CH;
         const int j = si[r];
         const size_t off = (seq_base + (j >= 0 ? j : 0)) * L::ROWB + ch * 16;
         const uint32_t d = r * L::ROWP + ch * 16;
-        cp_async16_zfill(st + d, k + off, j >= 0);
-        cp_async16_zfill(st + SUB * L::ROWP + d, v + off, j >= 0);
+        cp_async16_zfill(ws + d, k + off, j >= 0);
+        cp_async16_zfill(ws + 16 * L::ROWP + d, v + off, j >= 0);
     }
 }
 
-// One landed sub-tile (stage `st`): e4m3 rows are first converted to bf16 in `cvt`
-// (exact, swizzled layout; contains a CTA barrier, so every thread calls this), then this
-// warp's 16 rows are scored against the 16 heads, the online softmax advanced and P V added.
-// `si` / `sks` / `svs`: the sub-tile's cache rows and (e4m3) per-token scales.
+// This warp's landed 16 rows (slot `ws`): e4m3 rows are first converted to bf16 in the
+// warp's `cvtw` (exact, swizzled layout), then they are scored against the 16 heads, the
+// online softmax advanced and P V added.  `si` / `sks` / `svs`: the rows' cache rows and
+// (e4m3) per-token scales.
 template <bool KV8>
-__device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, const int* si, const float* sks,
-                                               const float* svs, const uint32_t (&qa)[8][4], float sc2, State& s,
-                                               int tid, int warp, int lane) {
+__device__ __forceinline__ void attend_warp_rows(const uint8_t* ws, uint8_t* cvtw, const int* si, const float* sks,
+                                                 const float* svs, const uint32_t (&qa)[8][4], float sc2, State& s,
+                                                 int lane) {
     using L = Layout<KV8>;
     const int t = lane & 3;
-    const uint8_t* kt = st;
-    const uint8_t* vt = st + SUB * L::ROWP;
+    const uint8_t* kt = ws;
+    const uint8_t* vt = ws + 16 * L::ROWP;
     // byte offset of 16-byte chunk ch of row r: padded rows as copied (bf16), the
-    // swizzled converted tile (e4m3)
+    // swizzled converted rows (e4m3)
     auto off = [](int r, int ch) -> uint32_t {
-        return KV8 ? swz_off<SUB>(r, ch) : static_cast<uint32_t>(r * L::ROWP + ch * 16);
+        return KV8 ? swz_off<16>(r, ch) : static_cast<uint32_t>(r * L::ROWP + ch * 16);
     };
     if (KV8) {
-        // e4m3 rows -> bf16 tiles (swz_off layout), exact
-        for (int it = tid; it < 2 * SUB * 8; it += NT) {
-            const int half = it / (SUB * 8), rr = (it / 8) % SUB, c8 = it & 7;
-            const uint8_t* src = st + half * SUB * L::ROWP + rr * L::ROWP + c8 * 16;
-            uint8_t* dst = cvt + half * SUB * 256;
+#pragma unroll 2
+        for (int it = lane; it < 2 * 16 * 8; it += 32) {
+            const int half = it / (16 * 8), rr = (it / 8) % 16, c8 = it & 7;
+            const uint8_t* src = ws + half * 16 * L::ROWP + rr * L::ROWP + c8 * 16;
+            uint8_t* dst = cvtw + half * 16 * 256;
             const uint4 in = *reinterpret_cast<const uint4*>(src);
             const uint16_t* bb = reinterpret_cast<const uint16_t*>(&in);
             uint4 lo, hi;
@@ -118,21 +129,21 @@ __device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, 
             lo.z = e4m3x2_to_bf16x2(bb[2]); lo.w = e4m3x2_to_bf16x2(bb[3]);
             hi.x = e4m3x2_to_bf16x2(bb[4]); hi.y = e4m3x2_to_bf16x2(bb[5]);
             hi.z = e4m3x2_to_bf16x2(bb[6]); hi.w = e4m3x2_to_bf16x2(bb[7]);
-            *reinterpret_cast<uint4*>(dst + swz_off<SUB>(rr, 2 * c8)) = lo;
-            *reinterpret_cast<uint4*>(dst + swz_off<SUB>(rr, 2 * c8 + 1)) = hi;
+            *reinterpret_cast<uint4*>(dst + swz_off<16>(rr, 2 * c8)) = lo;
+            *reinterpret_cast<uint4*>(dst + swz_off<16>(rr, 2 * c8 + 1)) = hi;
         }
-        __syncthreads();
-        kt = cvt;
-        vt = cvt + SUB * 256;
+        __syncwarp();
+        kt = cvtw;
+        vt = cvtw + 16 * 256;
     }
-    // S = Q K^T for this warp's 16 gathered rows
+    // S = Q K^T for the warp's 16 rows
     float acc[2][4];
     const uint32_t kb = smem_u32(kt);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-        const int r = warp * 16 + nt * 8 + (lane & 7);
+        const int r = nt * 8 + (lane & 7);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             uint32_t b0, b1, b2, b3;
@@ -145,7 +156,7 @@ __device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, 
     float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-        const int r0 = warp * 16 + nt * 8 + 2 * t;
+        const int r0 = nt * 8 + 2 * t;
         const bool ok0 = si[r0] >= 0, ok1 = si[r0 + 1] >= 0;
         float f0 = sc2, f1 = sc2;
         if (KV8) {
@@ -192,7 +203,7 @@ __device__ __forceinline__ void attend_subtile(const uint8_t* st, uint8_t* cvt, 
     pa[2] = pack_bf16(pr[1][0] * vf[1][0], pr[1][1] * vf[1][1]);
     pa[3] = pack_bf16(pr[1][2] * vf[1][0], pr[1][3] * vf[1][1]);
     const uint32_t vb = smem_u32(vt);
-    const int vr = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int vr = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
     for (int cc = 0; cc < 8; ++cc) {
         uint32_t b0, b1, b2, b3;
