@@ -220,7 +220,7 @@ def test_decode_1m_fp8_full_size_sampled():
     _block_parity(synth.DECODE_1M_FP8, seed=1004, seqs=[3], device="cuda")
 
 
-@pytest.mark.parametrize("ctx", [4096, 32768, 262144])
+@pytest.mark.parametrize("ctx", [4096, 32768, 262144, 1 << 20])   # 1M: two-kernel decode path
 def test_granularity_sweep_recall(ctx):
     tok = synth.sweep(ctx)
     _block_parity(tok, seed=1005, device="cuda")
