@@ -16,18 +16,19 @@ constexpr int NT = 128;            // 4 warps x 16 rows
 constexpr int RP = D + 4;          // padded slab row (floats) of the warp merge
 static_assert((RP * 4) % 16 == 0, "slab rows stay 16-byte aligned");
 // Two buffers per warp (one gather in flight while the other is attended) and three CTAs
-// per SM: with two CTAs per SM a third buffer bought nothing, while a third CTA hides the
-// latency of the per-warp MMA chains and softmax (about a fifth less time per layer).
+// per SM: a third buffer per warp, which leaves room for only two CTAs per SM, was slower,
+// while the third CTA hides the latency of the per-warp MMA chains and softmax.
 constexpr int STAGES = 2;
 constexpr int MIN_CTAS = 3;        // resident CTAs per SM the register budget must allow
 
-// A stage holds SUB K rows then SUB V rows as copied, each row padded by 16 bytes so that
-// the 8 rows an ldmatrix phase reads fall on distinct banks.
+// One stage (the four warps' buffers for one sub-tile) holds SUB K rows and SUB V rows as
+// copied, each row padded by 16 bytes so that the 8 rows an ldmatrix phase reads fall on
+// distinct banks; see WarpSlot for the layout of a warp's share.
 template <bool KV8>
 struct Layout {
     static constexpr int ROWB = KV8 ? 128 : 256;      // bytes per gathered cache row
-    static constexpr int ROWP = ROWB + 16;             // row pitch in a stage
-    static constexpr int STAGE = 2 * SUB * ROWP;       // K rows then V rows
+    static constexpr int ROWP = ROWB + 16;             // row pitch in a buffer
+    static constexpr int STAGE = 2 * SUB * ROWP;       // K and V rows of one sub-tile
     static constexpr int CVT = KV8 ? 2 * SUB * 256 : 0;
     static constexpr int SLABS = 4 * H * RP * 4;       // warp-merge slabs (bytes)
 };
