@@ -4,21 +4,25 @@
 // Importance of key j = sum over the 16 query heads of the softmax probability
 // P_h[j] = exp(s_h[j] - LSE_h) (the pages leave the rule open: "What HySparse2 is
 // actually optimizing", "What is not documented"), so every probability must be
-// normalized by the FINAL log-sum-exp.  Two streaming passes over the cache:
+// normalized by the FINAL log-sum-exp.  Two streaming passes over each split of
+// the cache:
 //
-//   pass A  S = scale * K q^T for all heads (tensor cores, M = 16 heads), the
-//           scaled logits go to a [B][16][S_ld] fp32 buffer (64 B per key) and
-//           each CTA keeps a running (max, sum) per head -> per-split partials.
-//   pass B  every CTA merges the partials into LSE, re-reads its logits, forms
-//           P exactly normalized, writes importance = sum_h P and accumulates
-//           O = P V (no online rescaling is needed: LSE is final); a third small
-//           kernel sums the split partials of O per (sequence, head).
+//   pass A  S = scale * K q^T for all heads (mma.sync, M = 16 heads), the scaled
+//           logits kept, and a running (max, sum) per head -> per-split partials.
+//   pass B  the partials of all splits merged into LSE, the logits re-read, P
+//           formed exactly normalized, importance = sum_h P written and O = P V
+//           accumulated (no online rescaling: LSE is final); the split partials
+//           of O are then summed per (sequence, head).
 //
-// K is read once (pass A) and V once (pass B): 512 B of cache per key plus the
-// 64-B logit round trip.  Tiles of 64 keys stream through a 4-stage TMA pipeline
-// with 128-byte swizzle; e4m3 tiles feed f16 MMAs straight from shared memory
-// (e4m3 -> f16 is exact) and the per-token scales are folded into the logits and
-// into P.
+// Single-launch path (dec_fused_kernel, splits of up to 4096 keys): one
+// cooperative launch, the logits kept in tensor memory between the passes, the
+// splits of a sequence exchanging (max, sum) through counters.  Two-kernel path
+// (contexts over 148 x 4096 keys): dec_qk_kernel, dec_pv_kernel and
+// dec_merge_kernel, the logits through a [B][16][S_ld] fp32 buffer (64 B per key).
+// K is read once (pass A) and V once (pass B).  Tiles of 64 keys stream through
+// TMA rings with 128-byte swizzle; e4m3 tiles feed f16 MMAs straight from shared
+// memory (e4m3 -> f16 is exact) and the per-token scales are folded into the
+// logits and into P.
 #include "common.cuh"
 #include "e4m3_mma.cuh"
 #include "internal.h"
