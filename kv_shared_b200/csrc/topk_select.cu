@@ -11,12 +11,13 @@
 // 0, block importance = max, floor(K/bs) best blocks (lower block on ties).
 //
 // Exact selection on order-preserving uint32 images of the fp32 values.  A row
-// is handled by a cluster of CS CTAs (CS = 1..8), CTA r owning a contiguous
+// is handled by a cluster of CS CTAs (CS = 1..16), CTA r owning a contiguous
 // slice of the keys, cached in shared memory when it fits.
 //   1. the row's key range (reduced over the cluster) gives the bits all keys
 //      share; the first radix digit (<= 11 bits) is taken right below them.  Slices
-//      too long for shared memory skip this pass (one read of the row saved) and take
-//      the top 13 bits as the first digit
+//      too long for shared memory skip this pass (one read of the row saved), ask
+//      for the whole slice in L2 up front (it is read twice) and take the top 13
+//      bits as the first digit
 //   2. one histogram of that digit over every key (summed over the cluster by
 //      distributed shared memory) locates the bin b1 holding the K-th best key
 //   3. every CTA compacts, in position order, its keys in bins >= b1 into a
