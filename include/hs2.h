@@ -194,15 +194,21 @@ HS2_API hs2_status hs2_sparse_attn(const hs2_attn_desc* desc, const void* q, con
  * caches (an f32 description returns HS2_ERR_UNSUPPORTED).  Its scratch (split
  * partials, semaphore counters, status word) is a fixed 4 MiB array inside the
  * library, held on every GPU that loads the library until the process exits.
- *   - A problem whose scratch would exceed 4 MiB is rejected with
- *     HS2_ERR_WORKSPACE before anything is enqueued (one 1,152-entry index row
- *     per query needs at most about 2.7 MB at any batch size).
+ *   - Every valid description is served.  When the partials of the split plan
+ *     hs2_sparse_attn would use do not fit the array (on a 148-SM B200 with
+ *     1,152-entry index rows: 252 to 295 rows), the rows run one CTA each,
+ *     which needs no partials; the output then equals hs2_sparse_attn's within
+ *     rounding, not bit for bit.  A problem whose scratch would still exceed
+ *     4 MiB would be rejected with HS2_ERR_WORKSPACE before anything is
+ *     enqueued; no supported shape reaches that limit.
  *   - The first call on each device looks up the array's device address with
  *     the device current; make that first call before any stream capture.
- *   - All calls share the array and it keeps the last call's contents; the
- *     counters that must start at zero are cleared by every call.  Calls that
- *     overlap on the GPU (different streams, or different host threads on one
- *     device) race on the array and must be ordered by the caller.
+ *   - Every call first clears the array's status word and counters on
+ *     `stream` (one memset node), so a call never depends on what an earlier
+ *     one left there; the partials are fully written before they are read.
+ *     All calls share the array: calls that overlap on the GPU (different
+ *     streams, or different host threads on one device) race on it and must
+ *     be ordered by the caller.
  *   - Conditions found on the device (an index outside the cache) are handled
  *     as in hs2_sparse_attn (the entry is skipped) but are not reported: there
  *     is no caller workspace to hold the status word.
@@ -217,18 +223,30 @@ HS2_API hs2_status hs2_sparse_attn_noalloc(const hs2_attn_desc* desc, const void
  * KV Bridging projection ([LB] "Two-Level KV Sharing": the caches of the
  * cross-decoder's full layers are projections of self-decoder activations, a
  * separate K/V weight per target layer; [AN]: the second half of the model
- * obtains its caches this way from the first half).
+ * obtains its caches this way from the first half, and the million-token caches
+ * are FP8).
  *
  * hidden [batch][n][d_model] bf16, w_kv [d_model][2*head_dim] bf16 (columns
  * 0..D-1 give K, D..2D-1 give V; no bias).  Rows t = 0..n-1 of sequence b are
- * written to cache rows pos0[b] + t of the bf16 caches k, v
- * ([batch][kv_capacity][head_dim]) with fp32 accumulation and round-to-nearest-
- * even.  pos0 is a device int32 array; pos0[b] + n <= kv_capacity.
- * d_model must be a multiple of 64, n >= 1, head_dim 128.
+ * written to cache rows pos0[b] + t of k, v ([batch][kv_capacity][head_dim]),
+ * from fp32 accumulators:
+ *   kv_dtype HS2_BF16  rounded to nearest even bf16; k_scale, v_scale unused
+ *                      (may be NULL)
+ *   kv_dtype HS2_E4M3  quantized per token exactly as hs2_kv_quantize_fp8 does
+ *                      it, separately for the K row and the V row: s = amax/448
+ *                      of the row's fp32 accumulators (s = 1 for a zero row),
+ *                      codes = e4m3(x / s) round to nearest even, saturating;
+ *                      codes to k, v (uint8) and s to k_scale, v_scale
+ *                      ([batch][kv_capacity] fp32, required)
+ * pos0 is a device int32 array; pos0[b] + n <= kv_capacity (a row outside the
+ * cache is not written).  d_model must be a multiple of 64, n >= 1, head_dim
+ * 128.  No workspace: the call allocates nothing and reports only synchronous
+ * errors.
  */
 HS2_API hs2_status hs2_kv_bridge_proj(const void* hidden, const void* w_kv, int32_t batch, int32_t n,
                               int32_t d_model, int32_t head_dim, const int32_t* pos0,
-                              int64_t kv_capacity, void* k, void* v, hs2_stream_t stream);
+                              int32_t kv_dtype, int64_t kv_capacity, void* k, void* v,
+                              float* k_scale, float* v_scale, hs2_stream_t stream);
 
 /*
  * FP8 cache quantizer ([AN]: the one-million-token analysis uses FP8 caches).

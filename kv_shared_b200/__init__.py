@@ -58,7 +58,7 @@ def lib():
         L.hs2_topk_select.argtypes = [dp, vp, i64, vp, i32, vp, vp, vp, sz, vp]
         L.hs2_sparse_attn.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.hs2_sparse_attn_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
-        L.hs2_kv_bridge_proj.argtypes = [vp, vp, i32, i32, i32, i32, vp, i64, vp, vp, vp]
+        L.hs2_kv_bridge_proj.argtypes = [vp, vp, i32, i32, i32, i32, vp, i32, i64, vp, vp, vp, vp, vp]
         L.hs2_kv_quantize_fp8.argtypes = [vp, i64, i32, vp, vp, vp]
         L.hs2_last_status.argtypes = [vp, vp]
         L.hs2_status_string.argtypes = [ctypes.c_int]
@@ -145,9 +145,11 @@ def hs2_sparse_attn_noalloc(desc, q, k, v, k_scale, v_scale, idx, cnt, o, lse, s
     _check("hs2_sparse_attn_noalloc", st)
 
 
-def hs2_kv_bridge_proj(hidden, w_kv, batch, n, d_model, head_dim, pos0, kv_capacity, k, v, stream=None):
+def hs2_kv_bridge_proj(hidden, w_kv, batch, n, d_model, head_dim, pos0, kv_capacity, k, v,
+                       kv_dtype=HS2_BF16, k_scale=None, v_scale=None, stream=None):
     st = lib().hs2_kv_bridge_proj(_p(hidden), _p(w_kv), batch, n, d_model, head_dim, _p(pos0),
-                                  int(kv_capacity), _p(k), _p(v), _stream(stream))
+                                  int(kv_dtype), int(kv_capacity), _p(k), _p(v), _p(k_scale), _p(v_scale),
+                                  _stream(stream))
     _check("hs2_kv_bridge_proj", st)
 
 

@@ -16,8 +16,13 @@
 //   warp 1        allocates 512 TMEM columns; one thread issues tcgen05.mma
 //                 (M=128, N=256, K=16, one per half) and commits each stage back
 //   warps 2..9    epilogue: tcgen05.ld of the fp32 accumulator rows (warp 2 + 4 h + j
-//                 takes half h, TMEM lane quarter (2 + j) % 4), bf16 rounding, stores
-//                 into the cache
+//                 takes half h, TMEM lane quarter (2 + j) % 4), then either bf16
+//                 rounding, or -- for an FP8 cache ("Xiaomi unveils HySparse2 ...",
+//                 AINews article: the million-token caches are FP8) -- the per-token
+//                 e4m3 quantizer of hs2_kv_quantize_fp8 applied to the fp32 row:
+//                 amax over the row's 128 K (then V) accumulators, s = amax / 448,
+//                 codes = e4m3(x / s) rounded to nearest even and saturated; stores
+//                 into the cache rows (and the row scales)
 // A 3-stage mbarrier pipeline (64 KB per stage) keeps TMA and MMA overlapped.
 #include "common.cuh"
 #include "internal.h"
@@ -43,10 +48,31 @@ struct Params {
     int d_model;
     int64_t cap;
     const int32_t* pos0;
-    __nv_bfloat16* k;
-    __nv_bfloat16* v;
+    uint8_t* k;                              // [B][cap][128] bf16 or e4m3 codes
+    uint8_t* v;
+    float* k_scale;                          // [B][cap] (e4m3 only)
+    float* v_scale;
+    bool kv8;
     uint32_t* status;                        // may be null
 };
+
+// 32 fp32 values -> 32 e4m3 codes (x / s, round to nearest even, saturating), as the
+// cache quantizer computes them
+__device__ __forceinline__ void quant32_e4m3(const uint32_t (&r)[32], float s, uint8_t* dst) {
+    uint32_t w[8];
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        const float y0 = __fdiv_rn(__uint_as_float(r[j + 0]), s), y1 = __fdiv_rn(__uint_as_float(r[j + 1]), s);
+        const float y2 = __fdiv_rn(__uint_as_float(r[j + 2]), s), y3 = __fdiv_rn(__uint_as_float(r[j + 3]), s);
+        uint16_t lo, hi;
+        // the second source operand lands in the low byte
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(y1), "f"(y0));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(y3), "f"(y2));
+        w[j / 4] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+    }
+    reinterpret_cast<uint4*>(dst)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    reinterpret_cast<uint4*>(dst)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
     return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
@@ -128,35 +154,59 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
         const int row = m0 + h * BM + q * 32 + lane;
         const bool ok = mbar_wait(&acc_ready, 0, a.status);
         umma::fence_after();
-        __nv_bfloat16* dk = nullptr;
-        __nv_bfloat16* dv = nullptr;
+        int64_t crow = -1;
         if (row < a.rows) {
             const int b = row / a.n, t = row % a.n;
             const int p0 = a.pos0[b];
-            if (p0 < 0 || static_cast<int64_t>(p0) + a.n > a.cap) {
+            if (p0 < 0 || static_cast<int64_t>(p0) + a.n > a.cap)
                 set_status(a.status, HS2_ERR_INDEX);         // destination outside the cache
-            } else {
-                const int64_t crow = static_cast<int64_t>(b) * a.cap + p0 + t;
-                dk = a.k + crow * 128;
-                dv = a.v + crow * 128;
-            }
+            else
+                crow = static_cast<int64_t>(b) * a.cap + p0 + t;
         }
+        const bool store = crow >= 0 && ok;
+        const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * BN;
+        if (!a.kv8) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-            uint32_t r[32];
-            umma::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * BN + c * 32, r);
-            umma::tmem_ld_wait();
-            if (dk && ok) {
-                __nv_bfloat16* dst = (c < 4 ? dk : dv) + (c & 3) * 32;
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                umma::tmem_ld32(trow + c * 32, r);
+                umma::tmem_ld_wait();
+                if (store) {
+                    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(c < 4 ? a.k : a.v) + crow * 128 + (c & 3) * 32;
 #pragma unroll
-                for (int j = 0; j < 32; j += 8) {
-                    uint4 pk;
-                    pk.x = pack_bf16(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]));
-                    pk.y = pack_bf16(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
-                    pk.z = pack_bf16(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
-                    pk.w = pack_bf16(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
-                    *reinterpret_cast<uint4*>(dst + j) = pk;
+                    for (int j = 0; j < 32; j += 8) {
+                        uint4 pk;
+                        pk.x = pack_bf16(__uint_as_float(r[j + 0]), __uint_as_float(r[j + 1]));
+                        pk.y = pack_bf16(__uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+                        pk.z = pack_bf16(__uint_as_float(r[j + 4]), __uint_as_float(r[j + 5]));
+                        pk.w = pack_bf16(__uint_as_float(r[j + 6]), __uint_as_float(r[j + 7]));
+                        *reinterpret_cast<uint4*>(dst + j) = pk;
+                    }
                 }
+            }
+        } else {
+            // K (columns 0..127) then V (128..255): the row's amax from a first read of its
+            // 128 accumulators, the codes from a second
+#pragma unroll 1
+            for (int part = 0; part < 2; ++part) {
+                float amax = 0.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    umma::tmem_ld32(trow + (4 * part + c) * 32, r);
+                    umma::tmem_ld_wait();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(__uint_as_float(r[j])));
+                }
+                const float sc = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    umma::tmem_ld32(trow + (4 * part + c) * 32, r);
+                    umma::tmem_ld_wait();
+                    if (store) quant32_e4m3(r, sc, (part ? a.v : a.k) + crow * 128 + c * 32);
+                }
+                if (store) (part ? a.v_scale : a.k_scale)[crow] = sc;
             }
         }
     }
@@ -181,8 +231,9 @@ cudaError_t launch_bridge(const BridgeArgs& ba, cudaStream_t st) {
         return cudaErrorInvalidValue;
     Params a{};
     a.rows = rows; a.n = ba.n; a.d_model = ba.d_model; a.cap = ba.cap; a.pos0 = ba.pos0;
-    a.k = static_cast<__nv_bfloat16*>(ba.k);
-    a.v = static_cast<__nv_bfloat16*>(ba.v);
+    a.k = static_cast<uint8_t*>(ba.k);
+    a.v = static_cast<uint8_t*>(ba.v);
+    a.k_scale = ba.k_scale; a.v_scale = ba.v_scale; a.kv8 = ba.kv8;
     a.status = ba.status;
     const size_t smem = 1024 + STAGES * STAGE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(bridge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));

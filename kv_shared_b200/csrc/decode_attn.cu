@@ -517,6 +517,11 @@ constexpr size_t kFusedMinSmem = 120 * 1024;   // more than half an SM: one CTA 
 template <bool KV8>
 struct FusedLayout {
     static constexpr int FS = KV8 ? 16 : 8;    // stages of the K/V stream (128 KB)
+    // The two consumer groups take alternate loads.  With an odd depth, load ld - FS of
+    // stage ld % FS belongs to the other group, which may lag: a group waiting for load ld
+    // before ld - FS has landed would see the phase of ld - 2 FS, whose parity equals ld's,
+    // and read a stale tile.  An even depth keeps every stage within one group.
+    static_assert(FS % 2 == 0, "the ring depth must be even (stage parity per consumer group)");
     static constexpr size_t VSC = KV8 ? kFusedMaxTiles * TILE * 4 : 0;   // V scales of the split
     static constexpr size_t BYTES = 1024 + FS * Layout<KV8>::RAW + 2 * FS * 8 + 8 * H * D * 4 + VSC;
 };

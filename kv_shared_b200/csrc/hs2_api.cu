@@ -291,19 +291,25 @@ hs2_status hs2_sparse_attn_noalloc(const hs2_attn_desc* desc, const void* q, con
 }
 
 hs2_status hs2_kv_bridge_proj(const void* hidden, const void* w_kv, int32_t batch, int32_t n, int32_t d_model,
-                              int32_t head_dim, const int32_t* pos0, int64_t kv_capacity, void* k, void* v,
-                              hs2_stream_t stream) {
+                              int32_t head_dim, const int32_t* pos0, int32_t kv_dtype, int64_t kv_capacity, void* k,
+                              void* v, float* k_scale, float* v_scale, hs2_stream_t stream) {
     if (!hidden || !w_kv || !pos0 || !k || !v || batch < 1 || n < 1 || d_model < 1 || kv_capacity < n)
         return HS2_ERR_INVALID_ARG;
+    const bool kv8 = kv_dtype == HS2_E4M3;
+    if (kv_dtype != HS2_BF16 && !kv8) return HS2_ERR_UNSUPPORTED;
+    if (kv8 && (!k_scale || !v_scale)) return HS2_ERR_INVALID_ARG;
     const void* ptrs[] = {hidden, w_kv, pos0, k, v};
     for (const void* p : ptrs)
         if (!aligned16(p)) return HS2_ERR_INVALID_ARG;
+    if (kv8 && ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u)))
+        return HS2_ERR_INVALID_ARG;
     if (head_dim != 128 || d_model % 64 != 0) return HS2_ERR_UNSUPPORTED;
     if (static_cast<int64_t>(batch) * n >= (int64_t(1) << 31) || static_cast<int64_t>(batch) * kv_capacity >= (int64_t(1) << 31))
         return HS2_ERR_UNSUPPORTED;
     BridgeArgs a{};
     a.hidden = hidden; a.w_kv = w_kv; a.batch = batch; a.n = n; a.d_model = d_model;
     a.pos0 = pos0; a.cap = kv_capacity; a.k = k; a.v = v; a.status = nullptr;
+    a.k_scale = k_scale; a.v_scale = v_scale; a.kv8 = kv8;
     return from_cuda(launch_bridge(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 

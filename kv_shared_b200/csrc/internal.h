@@ -111,12 +111,13 @@ struct SparseArgs {
     float* lse;
     void* ws;
     uint32_t* status;
+    bool one_split;           // one CTA per row whatever the row count (no split partials)
 };
 cudaError_t launch_sparse(const SparseArgs& a, cudaStream_t st);
 
-// Same kernel with its scratch in a fixed device array (no caller workspace);
-// *too_large is set, and nothing launched, when the problem needs more scratch
-// than sparse_noalloc_capacity() bytes.
+// Same kernel with its scratch in a fixed device array (no caller workspace).  When
+// the split plan's partials would not fit the array, the rows run one CTA each, which
+// needs none; *too_large is set, and nothing launched, only if even that does not fit.
 cudaError_t launch_sparse_noalloc(const SparseArgs& a, cudaStream_t st, bool* too_large);
 size_t sparse_noalloc_capacity();
 
@@ -150,8 +151,11 @@ struct BridgeArgs {
     int batch, n, d_model;
     const int32_t* pos0;     // [batch] device
     int64_t cap;
-    void* k;                 // [batch][cap][128] bf16
+    void* k;                 // [batch][cap][128] bf16, or e4m3 codes when kv8
     void* v;
+    float* k_scale;          // [batch][cap] per-row scales (kv8 only)
+    float* v_scale;
+    bool kv8;
     uint32_t* status;        // may be null
 };
 cudaError_t launch_bridge(const BridgeArgs& a, cudaStream_t st);

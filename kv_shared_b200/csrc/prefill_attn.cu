@@ -131,9 +131,10 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // 2^x for a pair on the FMA pipe (the exponential unit is the bottleneck of pass 1, so a
 // share of the exponentials moves here): x = j + r with j the nearest integer (added to
 // and taken back from 1.5 * 2^23, whose ulp is 1) and r in [-1/2, 1/2]; 2^r by a degree-5
-// polynomial fitted here to the relative error of 2^r on that interval (weighted least
-// squares iterated to near-minimax: max relative error 2.1e-7 in fp32 Horner form, like
-// the exponential unit's); 2^j enters through the exponent bits.  x is clamped at -125 so
+// polynomial, the minimax relative-error fit of 2^r on that interval by Lawson's algorithm
+// (least squares reweighted by the error until it equioscillates; exp2_poly_fit.py beside
+// this package prints the coefficients): max relative error 2.1e-7 in fp32 Horner form,
+// like the exponential unit's; 2^j enters through the exponent bits.  x is clamped at -125 so
 // that the result stays a normal number (it is then below 2^-124, nothing beside the
 // row maximum's 1).
 __device__ __forceinline__ float2 exp2_poly2(float2 x) {

@@ -580,6 +580,15 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// One CTA per row over the whole index row: no split partials, no counters.
+SparsePlan plan_sparse_single(int idx_stride) {
+    SparsePlan pl;
+    pl.cluster = false;
+    pl.splits = 1;
+    pl.chunk = (idx_stride + SUB - 1) / SUB * SUB;
+    return pl;
+}
+
 template <bool KV8>
 size_t smem_bytes(int chunk) {
     using L = Layout<KV8>;
@@ -588,7 +597,7 @@ size_t smem_bytes(int chunk) {
 
 template <bool KV8>
 cudaError_t launch_impl(const SparseArgs& sa, cudaStream_t st) {
-    const SparsePlan pl = plan_sparse(sa.rows, sa.idx_stride);
+    const SparsePlan pl = sa.one_split ? plan_sparse_single(sa.idx_stride) : plan_sparse(sa.rows, sa.idx_stride);
     Params a{};
     a.rows = sa.rows; a.n_q = sa.n_q; a.idx_stride = sa.idx_stride;
     a.splits = pl.splits; a.chunk = pl.chunk; a.cap = sa.cap;
@@ -704,10 +713,6 @@ cudaError_t scratch_address(void** out) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_sparse_scratch);
         if (e != cudaSuccess) return e;
-        // status word and semaphore counters start at zero (the counters return to
-        // zero at the end of every call)
-        e = cudaMemset(p, 0, kStatusBytes);
-        if (e != cudaSuccess) return e;
         g_scratch_addr[dev] = p;
     }
     *out = g_scratch_addr[dev];
@@ -721,14 +726,20 @@ size_t sparse_noalloc_capacity() { return kNoAllocScratchBytes; }
 cudaError_t launch_sparse_noalloc(const SparseArgs& in, cudaStream_t st, bool* too_large) {
     *too_large = false;
     if (in.rows <= 0) return cudaSuccess;
-    if (kStatusBytes + sparse_ws_bytes(in.rows, in.idx_stride) > kNoAllocScratchBytes) {
+    SparseArgs a = in;
+    // the split plan when its partials fit the array, else one CTA per row (no partials)
+    a.one_split = kStatusBytes + sparse_ws_bytes(in.rows, in.idx_stride) > kNoAllocScratchBytes;
+    if (a.one_split && kStatusBytes > kNoAllocScratchBytes) {
         *too_large = true;
         return cudaSuccess;
     }
     void* base = nullptr;
-    const cudaError_t e = scratch_address(&base);
+    cudaError_t e = scratch_address(&base);
     if (e != cudaSuccess) return e;
-    SparseArgs a = in;
+    // status word and split counters start every call at zero, in stream order (a call
+    // that ended early, e.g. after a failed launch, may have left a counter set)
+    e = cudaMemsetAsync(base, 0, kStatusBytes, st);
+    if (e != cudaSuccess) return e;
     a.status = static_cast<uint32_t*>(base);
     a.ws = static_cast<uint8_t*>(base) + kStatusBytes;
     return launch_sparse(a, st);

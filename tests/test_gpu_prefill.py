@@ -71,6 +71,98 @@ def test_bridge_full_size_sampled():
         assert (np.abs(got_v - vv) <= bound[:, 128:]).all()
 
 
+def _e4m3_ordinal(codes):
+    """Signed rank of e4m3 codes in value order (sign-magnitude: the low 7 bits rank the
+    magnitude); neighbouring values differ by one."""
+    c = np.asarray(codes).astype(np.int64)
+    mag = c & 0x7F
+    return np.where(c & 0x80, -mag, mag)
+
+
+def _check_bridge_e4m3(x64, w64, got_codes, got_scales, what):
+    """GPU e4m3 bridge rows against the oracle's exact rows.
+
+    The GPU quantizes its fp32-accumulated rows, which differ from the exact ones by at
+    most E = 2 K 2^-24 sum_m |x_m w_m| per element (the bound the bf16 test uses).  So:
+      - scales: within the range the quantizer gives for row maxima amax_exact -+ E;
+      - codes: each GPU code lies between the codes of (x_exact -+ E) / s_gpu, with
+        s_gpu checked first;
+      - and the codes equal the oracle quantizer applied to the exact rows (fp32
+        division and rounding, as both sides compute it), except where the exact value
+        sits near a rounding midpoint: at most 1% of the elements, each one code away.
+    Returns the number of codes that differ from the oracle's."""
+    K = x64.shape[1]
+    ref_k, ref_v = oracle.bridge(x64, w64, 128)
+    A = np.abs(x64) @ np.abs(w64)
+    mism = 0
+    for part, ref in enumerate((ref_k, ref_v)):
+        E = 2.0 * K * 2.0 ** -24 * A[:, part * 128:(part + 1) * 128]
+        codes, s_gpu = got_codes[part], got_scales[part].astype(np.float64)
+        amax_lo = np.maximum(np.abs(ref) - E, 0).max(axis=1)
+        amax_hi = (np.abs(ref) + E).max(axis=1)
+        s_lo = (amax_lo.astype(np.float32) / np.float32(448)).astype(np.float64)
+        s_hi = (amax_hi.astype(np.float32) / np.float32(448)).astype(np.float64)
+        assert ((s_gpu >= s_lo * (1 - 2 ** -23)) & (s_gpu <= s_hi * (1 + 2 ** -23))).all(), what + ": scale"
+        lo = oracle.e4m3_encode(np.clip((ref - E) / s_gpu[:, None], -448, 448))
+        hi = oracle.e4m3_encode(np.clip((ref + E) / s_gpu[:, None], -448, 448))
+        og = _e4m3_ordinal(codes)
+        assert ((og >= _e4m3_ordinal(lo)) & (og <= _e4m3_ordinal(hi))).all(), what + ": code outside its interval"
+        o_codes, o_scales = oracle.fp8_quantize(ref.astype(np.float32))
+        diff = codes != o_codes
+        assert (np.abs(og - _e4m3_ordinal(o_codes)) <= 1).all(), what + ": code more than one step away"
+        assert diff.mean() <= 0.01, f"{what}: {diff.mean():.4f} of the codes differ from the oracle's"
+        assert (np.abs(s_gpu / o_scales - 1) <= 1e-5).all(), what + ": scale differs from the oracle's"
+        mism += int(diff.sum())
+    return mism
+
+
+@pytest.mark.parametrize("batch,n,d_model,cap", [(2, 300, 256, 1300), (3, 257, 2048, 600)])
+def test_bridge_projection_e4m3(batch, n, d_model, cap):
+    g = torch.Generator().manual_seed(n + d_model + 1)
+    x = torch.randn(batch, n, d_model, generator=g).to(torch.bfloat16)
+    w = (torch.randn(d_model, 256, generator=g) * d_model ** -0.5).to(torch.bfloat16)
+    pos0 = torch.tensor([(5 * b + 3) % (cap - n + 1) for b in range(batch)], dtype=torch.int32)
+    k = torch.full((batch, cap, 128), 0x5A, dtype=torch.uint8, device="cuda")
+    v = torch.full_like(k, 0x5A)
+    ks = torch.full((batch, cap), -1.0, device="cuda")
+    vs = torch.full_like(ks, -1.0)
+    hs.hs2_kv_bridge_proj(x.cuda(), w.cuda(), batch, n, d_model, 128, pos0.cuda(), cap, k, v,
+                          kv_dtype=hs.HS2_E4M3, k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    kc, vc, ksc, vsc = k.cpu().numpy(), v.cpu().numpy(), ks.cpu().numpy(), vs.cpu().numpy()
+    total = 0
+    for b in range(batch):
+        p0 = int(pos0[b])
+        rows = slice(p0, p0 + n)
+        total += _check_bridge_e4m3(f64(x[b]), f64(w), (kc[b, rows], vc[b, rows]), (ksc[b, rows], vsc[b, rows]),
+                                    f"seq {b}")
+        untouched = np.ones(cap, bool)
+        untouched[p0:p0 + n] = False
+        assert (kc[b, untouched] == 0x5A).all() and (vc[b, untouched] == 0x5A).all()
+        assert (ksc[b, untouched] == -1).all() and (vsc[b, untouched] == -1).all()
+    print(f"codes differing from the oracle's (near midpoints): {total} of {2 * batch * n * 128}")
+
+
+def test_bridge_e4m3_full_size_sampled():
+    wl = synth.PREFILL_AGENT
+    inp = synth.make_inputs(synth.shrink(wl, n_sparse=0), seed=1003, device="cuda")
+    B, T = wl.batch, wl.ctx
+    k = torch.empty(B, T, 128, dtype=torch.uint8, device="cuda")
+    v = torch.empty_like(k)
+    ks = torch.empty(B, T, device="cuda")
+    vs = torch.empty_like(ks)
+    pos0 = torch.full((B,), T - wl.n_new, dtype=torch.int32, device="cuda")
+    hs.hs2_kv_bridge_proj(inp.hidden, inp.w_kv, B, wl.n_new, wl.d_model, 128, pos0, T, k, v,
+                          kv_dtype=hs.HS2_E4M3, k_scale=ks, v_scale=vs)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(2).choice(wl.n_new, 96, replace=False))
+    sel = T - wl.n_new + torch.from_numpy(rows).cuda()
+    for b in (0, B - 1):
+        _check_bridge_e4m3(f64(inp.hidden[b])[rows], f64(inp.w_kv),
+                           (k[b, sel].cpu().numpy(), v[b, sel].cpu().numpy()),
+                           (ks[b, sel].cpu().numpy(), vs[b, sel].cpu().numpy()), f"seq {b}")
+
+
 @pytest.mark.parametrize("n_q,ctx", [(300, 300), (300, 1000), (8, 129), (77, 2048 + 5)])
 def test_prefill_small_all_rows(n_q, ctx):
     # rows below the window and below the budget, a partial row block, ragged key tiles
