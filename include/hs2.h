@@ -105,9 +105,13 @@ typedef struct {
 
 /*
  * Workspace bytes the three attention calls need for `desc` (the largest of the
- * three).  If `scores_in_workspace` is non-zero the full-attention scores are
- * kept in the workspace ([batch][n_q][max_ctx] fp32) when the caller passes no
- * scores buffer.  Returns 0 for an invalid description.
+ * three).  Decode (n_q = 1) and f32 descriptions select from importance rows: if
+ * `scores_in_workspace` is non-zero they are kept in the workspace
+ * ([batch][n_q][max_ctx] fp32) when the caller passes no scores buffer.  Prefill
+ * on the tensor-core path (n_q > 1, budget <= 4096) selects from candidate lists
+ * that its second pass streams into the workspace (up to max_ctx (importance,
+ * position) pairs of 8 bytes per query row; in practice a few thousand are
+ * written) and needs no importance rows.  Returns 0 for an invalid description.
  */
 HS2_API size_t hs2_workspace_size(const hs2_attn_desc* desc, int32_t scores_in_workspace);
 
@@ -137,8 +141,9 @@ HS2_API hs2_status hs2_workspace_init(void* workspace, hs2_stream_t stream);
  * lse         optional (NULL) [batch][n_q][heads]
  * idx, cnt    selection output
  * scores      optional [batch][n_q][max_ctx] fp32 importance (entries beyond p
- *             are unspecified); NULL keeps them in the workspace (see
- *             hs2_workspace_size)
+ *             are unspecified); NULL keeps them in the workspace where the
+ *             selection needs them (see hs2_workspace_size).  The selection does
+ *             not depend on whether they are requested.
  */
 HS2_API hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const void* k,
                                 const void* v, const float* k_scale, const float* v_scale,

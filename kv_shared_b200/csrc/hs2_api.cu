@@ -98,13 +98,20 @@ float eff_scale(const hs2_attn_desc* d) {
 
 int64_t score_pitch(const hs2_attn_desc* d) { return (d->max_ctx + 63) / 64 * 64; }
 
+// prefill on tensor cores selects from candidates streamed out of its second pass, so it
+// needs no importance rows (budgets up to kFusedSelectMaxBudget)
+bool fused_prefill_select(const hs2_attn_desc* d, Path path) {
+    return path == Path::TC && d->n_q > 1 && d->budget <= kFusedSelectMaxBudget;
+}
+
 // bytes after the status block needed by hs2_full_attn_select
 size_t full_region(const hs2_attn_desc* d, Path path, bool scores_in_ws) {
     const size_t rows = static_cast<size_t>(d->batch) * d->n_q;
+    const bool fused = fused_prefill_select(d, path);
     size_t n = 0;
     if (path == Path::TC && d->n_q == 1) n += a256(decode_ws_bytes(d->batch, d->max_ctx, d->kv_dtype == HS2_E4M3));
-    if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q));
-    if (scores_in_ws) n += a256(sizeof(float) * rows * static_cast<size_t>(score_pitch(d)));
+    if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q, d->max_ctx, fused));
+    if (scores_in_ws && !fused) n += a256(sizeof(float) * rows * static_cast<size_t>(score_pitch(d)));
     return n;
 }
 
@@ -157,10 +164,11 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     float* score_buf = scores;
     int64_t score_ld = desc->max_ctx;
     size_t used = 0;
+    const bool fused = fused_prefill_select(desc, path);
     if (path == Path::TC)
         used = desc->n_q == 1 ? a256(decode_ws_bytes(desc->batch, desc->max_ctx, desc->kv_dtype == HS2_E4M3))
-                              : a256(prefill_ws_bytes(desc->batch, desc->n_q));
-    if (!score_buf) {
+                              : a256(prefill_ws_bytes(desc->batch, desc->n_q, desc->max_ctx, fused));
+    if (!score_buf && !fused) {
         score_buf = reinterpret_cast<float*>(region + used);
         score_ld = score_pitch(desc);
     }
@@ -180,7 +188,10 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
         a.batch = desc->batch; a.n_q = desc->n_q; a.cap = desc->kv_capacity; a.max_ctx = desc->max_ctx;
         a.q_pos0 = q_pos0; a.q = q; a.k = k; a.v = v; a.scale = scale; a.o = o; a.lse = lse;
         a.scores = score_buf; a.score_ld = score_ld; a.ws = region; a.status = status;
+        a.fused_select = fused; a.window = desc->window; a.budget = desc->budget;
+        a.idx_stride = desc->idx_stride; a.idx = idx; a.cnt = cnt;
         e = launch_prefill_full(a, st);
+        if (fused) return from_cuda(e);
     } else {
         DecodeArgs a{};
         a.batch = desc->batch; a.cap = desc->kv_capacity; a.max_ctx = desc->max_ctx; a.q_pos0 = q_pos0;

@@ -52,6 +52,27 @@ struct DecodeArgs {
 cudaError_t launch_decode_full(const DecodeArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- prefill (n_q > 1), tcgen05
+// Token-level selection of a prefill call runs fused: pass 2 streams each row's
+// candidates (keys whose importance reaches the row's running cutoff bound) into the
+// workspace, and launch_cand_select picks the top K from them.  Budgets above
+// kFusedSelectMaxBudget use the importance rows and launch_select instead.
+constexpr int kFusedSelectMaxBudget = 4096;
+
+struct CandSelectArgs {
+    int rows, n_q;
+    const int32_t* q_pos0;
+    int64_t max_ctx;
+    int window, budget, idx_stride;
+    const uint32_t* hist;     // [rows][kImpBins] candidates per importance bin
+    const int* cand_cnt;      // [rows]
+    const uint2* cand;        // [rows][cand_ld] (importance bits, position)
+    int64_t cand_ld;
+    int32_t* idx;
+    int32_t* cnt;
+    uint32_t* status;
+};
+cudaError_t launch_cand_select(const CandSelectArgs& a, cudaStream_t st);
+
 struct PrefillArgs {
     int batch, n_q;
     int64_t cap, max_ctx;
@@ -62,12 +83,16 @@ struct PrefillArgs {
     float scale;
     void* o;                  // [B][n_q][16][128] bf16
     float* lse;               // [B][n_q][16] natural log, or null
-    float* scores;            // [B][n_q][score_ld]
+    float* scores;            // [B][n_q][score_ld] importance rows, or null
     int64_t score_ld;
-    void* ws;                 // prefill_ws_bytes: per-(row, head) log-sum-exp
+    void* ws;                 // prefill_ws_bytes
     uint32_t* status;
+    bool fused_select;        // selection fused into pass 2 (then idx/cnt are written here)
+    int window, budget, idx_stride;
+    int32_t* idx;
+    int32_t* cnt;
 };
-size_t prefill_ws_bytes(int batch, int n_q);
+size_t prefill_ws_bytes(int batch, int n_q, int64_t max_ctx, bool fused_select);
 cudaError_t launch_prefill_full(const PrefillArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- selection

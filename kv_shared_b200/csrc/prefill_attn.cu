@@ -52,10 +52,17 @@ struct Params {
     float sc2;                                  // scale * log2(e), > 0
     float* lse2;                                // [B][n_q][H] log2 units (pass 1 out, pass 2 in)
     float* lse_user;                            // [B][n_q][H] natural log or null
-    float* scores;                              // [B][n_q][score_ld]
+    float* scores;                              // [B][n_q][score_ld] or null (no importance rows)
     int64_t score_ld;
     __nv_bfloat16* o;                           // [B][n_q][H][D]
     uint32_t* status;
+    // streaming selection (pass 2): keys of [0, p - window] whose importance reaches the
+    // row's running cutoff bound are appended to the row's candidate list
+    int window, budget;
+    uint2* cand;                                // [B*n_q][cand_ld] (importance bits, position) or null
+    int64_t cand_ld;
+    int* cand_cnt;                              // [B*n_q] entries appended
+    uint32_t* hist;                             // [B*n_q][kImpBins] candidates per importance bin
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -352,15 +359,15 @@ __device__ __forceinline__ float2 transpose_reduce8(float2 (&v)[8], int t) {
 // One 64-key chunk of one row (16 lanes = the row's 16 heads) of S_h, read with the
 // 16x256b shape: thread t holds heads t/4 (A) and t/4 + 8 (B) at keys
 // key_base + 8j + 2(t%4) + {0, 1}.  Forms P, writes it back as packed bf16 (16x128b
-// shape, key pair -> one column) and stores the row's importance for its keys
-// key_base + 2t, key_base + 2t + 1.
+// shape, key pair -> one column) and leaves in imp[j] the pair's sum over its two heads;
+// transpose_reduce8(imp) then gives lane t the row's importance of keys key_base + 2t,
+// key_base + 2t + 1.
 __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_taddr, int key_base, int p, float sc2,
-                                         float lse_a, float lse_b, float* srow, bool vec2, int t) {
+                                         float lse_a, float lse_b, float2 (&imp)[8], int t) {
     const float2 s2 = make_float2(sc2, sc2);
     const float2 na = make_float2(-lse_a, -lse_a), nb = make_float2(-lse_b, -lse_b);
     const bool need_mask = key_base + 63 > p;
     uint32_t pk[16];
-    float2 imp[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
         const float2 xa = fma2(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s2, na);
@@ -376,15 +383,69 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
         imp[j] = add2(pa, pb);
     }
     umma::tmem_st16x128_x8(p_taddr, pk);
-    const float2 s = transpose_reduce8(imp, t);
-    if (srow) {
-        const int k = key_base + 2 * t;
-        if (vec2 && k + 1 <= p) {
-            *reinterpret_cast<float2*>(srow + k) = s;
-        } else {
-            if (k <= p) srow[k] = s.x;
-            if (k + 1 <= p) srow[k + 1] = s.y;
-        }
+}
+
+// Streaming selection state of one query row, in shared memory.  Candidates are the keys
+// of [0, p - W] whose importance is at least thr when they appear; thr only rises, and
+// only to the floor of a bin at or above which K candidates have already been counted,
+// so every key of the row's final top K is a candidate (a key below thr has K better
+// ones before it, and the lower position wins ties).  The bins count candidates only:
+// every key at or above the current thr is a candidate, so the counts from thr's bin
+// up are those of all keys seen.
+struct RowSel {
+    uint32_t hist[kImpBins];
+    int count;
+    float thr;
+};
+
+// Appends this warp's candidates among its two keys per lane (positions k, k + 1).
+__device__ __forceinline__ void p2_candidates(float2 v, int k, int last_cand, RowSel& rs, uint2* crow, int lane) {
+    const float th = *reinterpret_cast<volatile float*>(&rs.thr);
+    const bool a0 = k <= last_cand && v.x >= th;
+    const bool a1 = k + 1 <= last_cand && v.y >= th;
+    const uint32_t m0 = __ballot_sync(0xffffffffu, a0), m1 = __ballot_sync(0xffffffffu, a1);
+    if ((m0 | m1) == 0u) return;
+    int base = 0;
+    if (lane == 0) base = atomicAdd(&rs.count, __popc(m0) + __popc(m1));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const uint32_t lt = (1u << lane) - 1u;
+    int off = base + __popc(m0 & lt) + __popc(m1 & lt);
+    if (a0) {
+        atomicAdd(&rs.hist[imp_bin(v.x)], 1u);
+        crow[off++] = make_uint2(__float_as_uint(v.x), static_cast<uint32_t>(k));
+    }
+    if (a1) {
+        atomicAdd(&rs.hist[imp_bin(v.y)], 1u);
+        crow[off] = make_uint2(__float_as_uint(v.y), static_cast<uint32_t>(k + 1));
+    }
+}
+
+// Raises rs.thr to the floor of the highest bin b with at least K candidates in bins >= b
+// (a warp reads the bins while others may still add to them: a stale count is smaller,
+// which only lowers the bound).
+__device__ __forceinline__ void p2_raise_threshold(RowSel& rs, int K, int lane) {
+    uint32_t h[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) h[j] = *reinterpret_cast<volatile uint32_t*>(&rs.hist[4 * lane + j]);
+    const uint32_t mine = h[0] + h[1] + h[2] + h[3];
+    uint32_t above = mine;                                     // suffix sum over lanes >= lane
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, above, o);
+        if (lane + o < 32) above += y;
+    }
+    uint32_t cum = above - mine;                               // counts of the lanes above
+    int best = -1;
+#pragma unroll
+    for (int j = 3; j >= 0; --j) {
+        cum += h[j];
+        if (best < 0 && cum >= static_cast<uint32_t>(K)) best = 4 * lane + j;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+    if (lane == 0 && best > 0) {
+        const float f = imp_bin_floor(best);
+        if (f > rs.thr) *reinterpret_cast<volatile float*>(&rs.thr) = f;
     }
 }
 
@@ -398,7 +459,7 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
 // thread's MMAs in issue order, so PV(i) has read P before S overwrites it, and the
 // softmax writes P(i + 2) only after S(i + 2) has completed, hence after PV(i).
 constexpr int ROWS2 = 8;
-constexpr int KS2 = 4;                          // K stages of pass 2
+constexpr int KS2 = 3;                          // K stages of pass 2
 constexpr int VS2 = 3;                          // V stages of pass 2
 constexpr int NSB2 = 2;                         // S/P buffers at columns 0, 128
 constexpr uint32_t kQcol = 256;                 // Q (packed bf16 pairs) at columns 256 .. 319
@@ -415,6 +476,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     __shared__ uint64_t s_full[NSB2], p_full[NSB2], q_tm, o_full;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
+    __shared__ RowSel rsel[ROWS2];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int blocks_per_seq = (a.n_q + ROWS2 - 1) / ROWS2;
@@ -435,6 +497,11 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         mbar_init(&o_full, 1);
         fence_mbar_init();
         abort_flag = 0;
+    }
+    for (int i = threadIdx.x; i < ROWS2 * kImpBins; i += NT) rsel[i / kImpBins].hist[i % kImpBins] = 0u;
+    if (threadIdx.x < ROWS2) {
+        rsel[threadIdx.x].count = 0;
+        rsel[threadIdx.x].thr = a.budget > 0 ? 0.f : INFINITY;
     }
     if (warp == 1) umma::tmem_alloc(&tmem_base, 512);
     umma::fence_before();
@@ -519,8 +586,12 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         const size_t li = (static_cast<size_t>(b) * a.n_q + row) * H;
         const float lse_a = row_ok ? a.lse2[li + (lane >> 2)] : INFINITY;      // P = 0 for rows past n_q
         const float lse_b = row_ok ? a.lse2[li + (lane >> 2) + 8] : INFINITY;
-        float* srow = row_ok ? a.scores + (static_cast<size_t>(b) * a.n_q + row) * a.score_ld : nullptr;
+        float* srow = (row_ok && a.scores) ? a.scores + (static_cast<size_t>(b) * a.n_q + row) * a.score_ld : nullptr;
         const bool vec2 = (a.score_ld & 1) == 0;
+        const size_t grow = static_cast<size_t>(b) * a.n_q + row;
+        uint2* crow = (row_ok && a.cand) ? a.cand + grow * a.cand_ld : nullptr;
+        const int last_cand = p - a.window;                  // candidates: positions 0 .. p - W
+        RowSel& rs = rsel[lrow];
         const float sc2 = a.sc2;
         const uint32_t lanes = static_cast<uint32_t>(32 * quarter + 16 * s) << 16;
         const int vt = sw * 32 + lane;                        // V row this thread clears in the last tile
@@ -567,12 +638,38 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
                 umma::fence_proxy_async();
             }
             uint32_t r[32];
+            float2 imp[8];
+            const int key0 = i * KT + 64 * kh;
             const uint32_t ta = tmem + u * 128 + lanes + 64 * kh;     // this warp's 64 S columns
             umma::tmem_ld16x256_x8(ta, r);
             umma::tmem_ld_wait();
-            p2_chunk(r, ta, i * KT + 64 * kh, p, sc2, lse_a, lse_b, srow, vec2, lane);    // P into the first 32
+            p2_chunk(r, ta, key0, p, sc2, lse_a, lse_b, imp, lane);    // P into the first 32
             umma::tmem_st_wait();
             warp_arrive(&p_full[u]);
+            // importance of the row's keys key0 + 2 lane, + 1: reduced and stored after P has
+            // been handed to the MMA issuer, off the S -> P -> PV path
+            const float2 sv = transpose_reduce8(imp, lane);
+            const int k = key0 + 2 * lane;
+            if (srow) {
+                if (vec2 && k + 1 <= p) {
+                    *reinterpret_cast<float2*>(srow + k) = sv;
+                } else {
+                    if (k <= p) srow[k] = sv.x;
+                    if (k + 1 <= p) srow[k + 1] = sv.y;
+                }
+            }
+            if (crow && key0 <= last_cand) {
+                p2_candidates(sv, k, last_cand, rs, crow, lane);
+                if (kh == 0 && (i & 3) == 3) p2_raise_threshold(rs, a.budget, lane);
+            }
+        }
+        // the row's candidate count and bins, for the selection kernel
+        named_sync(2, NSOFT);
+        if (crow && kh == 0) {
+            uint4 h;
+            h.x = rs.hist[4 * lane]; h.y = rs.hist[4 * lane + 1]; h.z = rs.hist[4 * lane + 2]; h.w = rs.hist[4 * lane + 3];
+            reinterpret_cast<uint4*>(a.hist + grow * kImpBins)[lane] = h;
+            if (lane == 0) a.cand_cnt[grow] = rs.count;
         }
         // O epilogue: 4 warps per lane quarter; this thread owns TMEM lane m = (row, head)
         // and columns 32 cc .. 32 cc + 31
@@ -608,8 +705,17 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
 
 }  // namespace
 
-size_t prefill_ws_bytes(int batch, int n_q) {
-    return (sizeof(float) * static_cast<size_t>(batch) * n_q * H + 255) & ~size_t(255);
+namespace {
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+}  // namespace
+
+size_t prefill_ws_bytes(int batch, int n_q, int64_t max_ctx, bool fused_select) {
+    const size_t rows = static_cast<size_t>(batch) * n_q;
+    size_t n = al256(sizeof(float) * rows * H);                               // log-sum-exp (log2)
+    if (fused_select)
+        n += al256(sizeof(uint32_t) * rows * kImpBins) + al256(sizeof(int) * rows) +
+             al256(sizeof(uint2) * rows * static_cast<size_t>(max_ctx));    // bins, counts, candidates
+    return n;
 }
 
 cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
@@ -621,14 +727,30 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
         !make_tmap_2d(&kmap, pa.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, kv_rows, D * 2, 64, KT, true) ||
         !make_tmap_2d(&vmap, pa.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, kv_rows, D * 2, 64, KT, true))
         return cudaErrorInvalidValue;
+    uint8_t* ws = static_cast<uint8_t*>(pa.ws);
     Params a{};
     a.B = pa.batch; a.n_q = pa.n_q; a.cap = pa.cap; a.max_ctx = pa.max_ctx; a.q_pos0 = pa.q_pos0; a.q = pa.q;
     a.sc2 = pa.scale * kLog2e;
-    a.lse2 = static_cast<float*>(pa.ws);
+    a.lse2 = reinterpret_cast<float*>(ws);
+    ws += al256(sizeof(float) * static_cast<size_t>(rows) * H);
     a.lse_user = pa.lse;
     a.scores = pa.scores; a.score_ld = pa.score_ld;
     a.o = static_cast<__nv_bfloat16*>(pa.o);
     a.status = pa.status;
+    a.window = pa.window; a.budget = pa.budget;
+    CandSelectArgs cs{};
+    if (pa.fused_select) {
+        a.hist = reinterpret_cast<uint32_t*>(ws);
+        ws += al256(sizeof(uint32_t) * static_cast<size_t>(rows) * kImpBins);
+        a.cand_cnt = reinterpret_cast<int*>(ws);
+        ws += al256(sizeof(int) * static_cast<size_t>(rows));
+        a.cand = reinterpret_cast<uint2*>(ws);
+        a.cand_ld = pa.max_ctx;
+        cs.rows = rows; cs.n_q = pa.n_q; cs.q_pos0 = pa.q_pos0; cs.max_ctx = pa.max_ctx;
+        cs.window = pa.window; cs.budget = pa.budget; cs.idx_stride = pa.idx_stride;
+        cs.hist = a.hist; cs.cand_cnt = a.cand_cnt; cs.cand = a.cand; cs.cand_ld = a.cand_ld;
+        cs.idx = pa.idx; cs.cnt = pa.cnt; cs.status = pa.status;
+    }
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
     const int blocks2 = pa.batch * ((pa.n_q + ROWS2 - 1) / ROWS2);
     const size_t s1 = 1024 + 2 * TILE_BYTES + P1_STAGES * TILE_BYTES;
@@ -639,7 +761,9 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     prefill_lse_kernel<<<blocks, NT, s1, st>>>(qmap, kmap, a);
     prefill_out_kernel<<<blocks2, NT, s2, st>>>(qmap, kmap, vmap, a);
-    return cudaGetLastError();
+    e = cudaGetLastError();
+    if (e != cudaSuccess || !pa.fused_select) return e;
+    return launch_cand_select(cs, st);
 }
 
 }  // namespace hs2

@@ -185,3 +185,72 @@ def test_prefill_agent_full_size_sampled():
                                      rng.choice(wl.n_q, 23, replace=False)]))
     rep = block_parity(wl, seed=1003, seqs=[0, 3], device="cuda", rows=rows)
     assert rep["differing_rows"] <= max(2, rep["rows"] // 20)
+
+
+def _select_case(q, k, v, n_q, ctx, budget=1024, window=128):
+    """Runs the prefill call on one sequence (rows at positions ctx-n_q .. ctx-1) with and
+    without the importance rows and checks the selection against the oracle's."""
+    from hs2_check import check_selection
+    B, H, D = 1, 16, 128
+    desc = hs.make_desc(B, n_q, H, D, window, budget, max_ctx=ctx)
+    qd = q.to(torch.bfloat16).cuda().contiguous().view(1, n_q, H, D)
+    kd = k.to(torch.bfloat16).cuda().contiguous().view(1, ctx, D)
+    vd = v.to(torch.bfloat16).cuda().contiguous().view(1, ctx, D)
+    q_pos0 = torch.tensor([ctx - n_q], dtype=torch.int32, device="cuda")
+    pos = np.arange(ctx - n_q, ctx)
+    o_ref, _, sc_ref = oracle.full_attn(f64(qd[0]), f64(kd[0]), f64(vd[0]), pos)
+    o_idx, o_cnt = oracle.select_rows(sc_ref, pos, window, budget)
+    results = []
+    for with_scores in (True, False):
+        ws = hs.alloc_workspace(desc, scores_in_workspace=False)
+        o = torch.empty_like(qd)
+        idx = torch.empty(1, n_q, desc.idx_stride, dtype=torch.int32, device="cuda")
+        cnt = torch.empty(1, n_q, dtype=torch.int32, device="cuda")
+        scores = torch.zeros(1, n_q, ctx, device="cuda") if with_scores else None
+        hs.hs2_full_attn_select(desc, qd, kd, vd, None, None, q_pos0, o, None, idx, cnt, scores, ws)
+        assert hs.hs2_last_status(ws) == hs.HS2_OK
+        if with_scores:
+            from hs2_check import compare_scores
+            compare_scores(scores[0].cpu().numpy(), sc_ref, pos)
+        g_idx, g_cnt = idx[0].cpu().numpy(), cnt[0].cpu().numpy()
+        check_selection(g_idx, g_cnt, o_idx, o_cnt, sc_ref, pos, window)
+        results.append(g_idx)
+    # the importance rows are an extra output: the selection does not depend on them
+    np.testing.assert_array_equal(results[0], results[1])
+    return o_idx, results[0]
+
+
+def test_fused_select_increasing_importance():
+    # every key more important than all earlier ones: each key is a candidate when it
+    # appears, so the candidate lists hold whole rows
+    g = torch.Generator().manual_seed(11)
+    n_q, ctx = 48, 5000
+    u = torch.randn(128, generator=g)
+    u = u / u.norm()
+    q = (6.0 * u).expand(n_q, 16, 128).clone()
+    c = torch.linspace(0.2, 3.0, ctx)
+    k = c[:, None] * u[None, :] + 0.01 * torch.randn(ctx, 128, generator=g)
+    v = torch.randn(ctx, 128, generator=g)
+    _select_case(q, k, v, n_q, ctx)
+
+
+def test_fused_select_all_equal_importance():
+    # zero keys: every logit 0, every importance equal -> the lowest positions win; the
+    # cutoff bin holds all ~5800 candidates, more than the selection sorts in shared memory
+    g = torch.Generator().manual_seed(12)
+    n_q, ctx = 40, 6000
+    q = torch.randn(n_q, 16, 128, generator=g)
+    k = torch.zeros(ctx, 128)
+    v = torch.randn(ctx, 128, generator=g)
+    o_idx, g_idx = _select_case(q, k, v, n_q, ctx)
+    np.testing.assert_array_equal(o_idx, g_idx)
+
+
+@pytest.mark.parametrize("budget", [0, 1, 64, 4096])
+def test_fused_select_budgets(budget):
+    g = torch.Generator().manual_seed(13 + budget)
+    n_q, ctx = 64, 4500
+    q = torch.randn(n_q, 16, 128, generator=g)
+    k = torch.randn(ctx, 128, generator=g)
+    v = torch.randn(ctx, 128, generator=g)
+    _select_case(q, k, v, n_q, ctx, budget=budget)
