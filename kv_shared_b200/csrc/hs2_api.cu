@@ -110,7 +110,7 @@ size_t full_region(const hs2_attn_desc* d, Path path, bool scores_in_ws) {
     const bool fused = fused_prefill_select(d, path);
     size_t n = 0;
     if (path == Path::TC && d->n_q == 1) n += a256(decode_ws_bytes(d->batch, d->max_ctx, d->kv_dtype == HS2_E4M3));
-    if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q, d->max_ctx, fused));
+    if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q, d->max_ctx, fused, d->kv_dtype == HS2_E4M3));
     if (scores_in_ws && !fused) n += a256(sizeof(float) * rows * static_cast<size_t>(score_pitch(d)));
     return n;
 }
@@ -153,7 +153,6 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     for (const void* p : ptrs)
         if (!aligned16(p)) return HS2_ERR_INVALID_ARG;
     if ((lse && !aligned16(lse)) || (scores && !aligned16(scores)) || !aligned16(q_pos0)) return HS2_ERR_INVALID_ARG;
-    if (path == Path::TC && desc->n_q > 1 && desc->kv_dtype != HS2_BF16) return HS2_ERR_UNSUPPORTED;
     if (ws_bytes < hs2_workspace_size(desc, scores == nullptr)) return HS2_ERR_WORKSPACE;
 
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -167,7 +166,7 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     const bool fused = fused_prefill_select(desc, path);
     if (path == Path::TC)
         used = desc->n_q == 1 ? a256(decode_ws_bytes(desc->batch, desc->max_ctx, desc->kv_dtype == HS2_E4M3))
-                              : a256(prefill_ws_bytes(desc->batch, desc->n_q, desc->max_ctx, fused));
+                              : a256(prefill_ws_bytes(desc->batch, desc->n_q, desc->max_ctx, fused, kv8));
     if (!score_buf && !fused) {
         score_buf = reinterpret_cast<float*>(region + used);
         score_ld = score_pitch(desc);
@@ -187,6 +186,7 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
         PrefillArgs a{};
         a.batch = desc->batch; a.n_q = desc->n_q; a.cap = desc->kv_capacity; a.max_ctx = desc->max_ctx;
         a.q_pos0 = q_pos0; a.q = q; a.k = k; a.v = v; a.scale = scale; a.o = o; a.lse = lse;
+        a.k_scale = k_scale; a.v_scale = v_scale; a.kv8 = kv8;
         a.scores = score_buf; a.score_ld = score_ld; a.ws = region; a.status = status;
         a.fused_select = fused; a.window = desc->window; a.budget = desc->budget;
         a.idx_stride = desc->idx_stride; a.idx = idx; a.cnt = cnt;

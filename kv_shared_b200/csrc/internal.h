@@ -78,8 +78,11 @@ struct PrefillArgs {
     int64_t cap, max_ctx;
     const int32_t* q_pos0;
     const void* q;            // [B][n_q][16][128] bf16
-    const void* k;            // [B][cap][128] bf16
+    const void* k;            // [B][cap][128] bf16, or e4m3 codes when kv8
     const void* v;
+    const float* k_scale;     // [B][cap] (kv8)
+    const float* v_scale;
+    bool kv8;
     float scale;
     void* o;                  // [B][n_q][16][128] bf16
     float* lse;               // [B][n_q][16] natural log, or null
@@ -92,7 +95,7 @@ struct PrefillArgs {
     int32_t* idx;
     int32_t* cnt;
 };
-size_t prefill_ws_bytes(int batch, int n_q, int64_t max_ctx, bool fused_select);
+size_t prefill_ws_bytes(int batch, int n_q, int64_t max_ctx, bool fused_select, bool kv8);
 cudaError_t launch_prefill_full(const PrefillArgs& a, cudaStream_t st);
 
 // ---------------------------------------------------------------- selection

@@ -59,6 +59,10 @@ struct Params {
     // streaming selection (pass 2): keys of [0, p - window] whose importance reaches the
     // row's running cutoff bound are appended to the row's candidate list
     int window, budget;
+    // e4m3 caches: the kernels read exact bf16 copies of the codes (cap = their padded row
+    // count per sequence) and apply these per-token scales in fp32
+    const float* ksc;                           // [B][cap] K row scales (0 past max_ctx)
+    const float* vsc;                           // [B][cap] V row scales
     uint2* cand;                                // [B*n_q][cand_ld] (importance bits, position) or null
     int64_t cand_ld;
     int* cand_cnt;                              // [B*n_q] entries appended
@@ -164,16 +168,27 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
 // Which groups of 4 of a 32-value chunk take exp2_poly2 in pass 1 (bit g: group g).
 constexpr uint32_t kPass1PolyGroups = 0x11;                    // groups 0, 4: 8 of 32 (measured best)
 
+// e4m3 caches: the scales of a tile's 128 keys (K, then V in pass 2) travel through a
+// ring of shared-memory slots, written by the producer warp when it issues the tile's
+// loads and read by the softmax warps when they process its S.  The producer is at most
+// (K stages + 2 S buffers) tiles ahead of the oldest tile still being read, so 8 slots
+// never overwrite one in use.
+constexpr int SC_SLOTS = 8;
+
 // ------------------------------------------------------------------ pass 1: LSE
 constexpr int P1_STAGES = 4;
+static_assert(P1_STAGES + 2 < SC_SLOTS, "scale ring shorter than the pass-1 lookahead");
 
+template <bool KV8>
 __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constant__ CUtensorMap qmap,
                                                            const __grid_constant__ CUtensorMap kmap, Params a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = align1024(smem_raw);
     uint8_t* qs = smem;                                       // Q halves 0, 1
     uint8_t* ks = smem + 2 * TILE_BYTES;
+    float* ring = reinterpret_cast<float*>(ks + P1_STAGES * TILE_BYTES);   // [SC_SLOTS][KT] (e4m3)
     __shared__ uint64_t q_full, k_full[P1_STAGES], k_empty[P1_STAGES], s_full[2][2], s_empty[2][2];
+    __shared__ uint64_t sc_full[SC_SLOTS];
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
     __shared__ float2 part[NSOFT];
@@ -194,6 +209,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         for (int s = 0; s < P1_STAGES; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
         for (int s = 0; s < 2; ++s)
             for (int h = 0; h < 2; ++h) { mbar_init(&s_full[s][h], 1); mbar_init(&s_empty[s][h], 8); }
+        for (int s = 0; s < SC_SLOTS; ++s) mbar_init(&sc_full[s], 1);
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -204,21 +220,35 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
     const uint32_t tmem = tmem_base;            // S of (buffer u, half h) at column (2u + h) * 128
 
     if (warp == 0) {
-        if (lane == 0) {
-            const int qrow = (b * a.n_q + r0) * H;
-            mbar_arrive_expect_tx(&q_full, 2 * TILE_BYTES);
-            for (int h = 0; h < 2; ++h) {
-                tma_load_2d(qs + h * TILE_BYTES, &qmap, &q_full, 0, qrow + h * 128);
-                tma_load_2d(qs + h * TILE_BYTES + BOX_BYTES, &qmap, &q_full, 64, qrow + h * 128);
+        if (KV8 || lane == 0) {
+            if (lane == 0) {
+                const int qrow = (b * a.n_q + r0) * H;
+                mbar_arrive_expect_tx(&q_full, 2 * TILE_BYTES);
+                for (int h = 0; h < 2; ++h) {
+                    tma_load_2d(qs + h * TILE_BYTES, &qmap, &q_full, 0, qrow + h * 128);
+                    tma_load_2d(qs + h * TILE_BYTES + BOX_BYTES, &qmap, &q_full, 64, qrow + h * 128);
+                }
             }
             for (int i = 0; i < n_kt; ++i) {
                 const int s = i % P1_STAGES;
-                if (i >= P1_STAGES && !wait_or_abort(&k_empty[s], ((i / P1_STAGES) - 1) & 1, &abort_flag, a.status)) break;
-                uint8_t* dst = ks + s * TILE_BYTES;
+                bool ok = true;
+                if (lane == 0 && i >= P1_STAGES)
+                    ok = wait_or_abort(&k_empty[s], ((i / P1_STAGES) - 1) & 1, &abort_flag, a.status);
+                if (KV8) ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
                 const int krow = static_cast<int>(b * a.cap) + i * KT;
-                mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
-                tma_load_2d(dst, &kmap, &k_full[s], 0, krow);
-                tma_load_2d(dst + BOX_BYTES, &kmap, &k_full[s], 64, krow);
+                if (lane == 0) {
+                    uint8_t* dst = ks + s * TILE_BYTES;
+                    mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
+                    tma_load_2d(dst, &kmap, &k_full[s], 0, krow);
+                    tma_load_2d(dst + BOX_BYTES, &kmap, &k_full[s], 64, krow);
+                }
+                if (KV8) {      // the tile's 128 key scales into ring slot i % SC_SLOTS
+                    reinterpret_cast<float4*>(ring + (i % SC_SLOTS) * KT)[lane] =
+                        __ldg(reinterpret_cast<const float4*>(a.ksc + krow) + lane);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&sc_full[i % SC_SLOTS]);
+                }
             }
         }
     } else if (warp == 1) {
@@ -257,10 +287,17 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
         float run_m = -INFINITY, run_l = 0.f;
         // scale > 0, so the row maximum of S sc2 is sc2 times the maximum of S
-        auto reduce_chunk = [&](const uint32_t (&r)[32], int key0) {
+        auto reduce_chunk = [&](const uint32_t (&r)[32], int key0, const float* kscale) {
             float v[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (KV8) {          // logit = (q . code) * key scale, exact in the oracle's terms
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    const float4 c = *reinterpret_cast<const float4*>(kscale + j);
+                    v[j] *= c.x; v[j + 1] *= c.y; v[j + 2] *= c.z; v[j + 3] *= c.w;
+                }
+            }
             if (key0 + 31 > p) {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
@@ -297,17 +334,21 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         for (int i = 0; i < n_kt; ++i) {
             const int u = i & 1;
             if (!wait_or_abort(&s_full[u][h], (i >> 1) & 1, &abort_flag, a.status)) break;
+            if (KV8 && !__all_sync(0xffffffffu, wait_or_abort(&sc_full[i % SC_SLOTS], (i / SC_SLOTS) & 1, &abort_flag,
+                                                              a.status)))
+                break;
             umma::fence_after();
             const uint32_t ta = tmem + lane_base + (2 * u + h) * 128 + 64 * c;
             const int key0 = i * KT + 64 * c;
+            const float* kscale = ring + (i % SC_SLOTS) * KT + 64 * c;
             uint32_t ra[32], rb[32];
             umma::tmem_ld32(ta, ra);
             umma::tmem_ld_wait();
             umma::tmem_ld32(ta + 32, rb);
-            reduce_chunk(ra, key0);
+            reduce_chunk(ra, key0, kscale);
             umma::tmem_ld_wait();
             warp_arrive(&s_empty[u][h]);
-            reduce_chunk(rb, key0 + 32);
+            reduce_chunk(rb, key0 + 32, kscale + 32);
         }
         part[sw * 32 + lane] = make_float2(run_m, run_l);
         named_sync(1, NSOFT);
@@ -362,24 +403,40 @@ __device__ __forceinline__ float2 transpose_reduce8(float2 (&v)[8], int t) {
 // shape, key pair -> one column) and leaves in imp[j] the pair's sum over its two heads;
 // transpose_reduce8(imp) then gives lane t the row's importance of keys key_base + 2t,
 // key_base + 2t + 1.
+// e4m3 caches (KV8): S holds q . code; the key pair's scales come from `sc` (K scales of
+// the tile at sc[0 .. 127], V scales at sc[128 .. 255], chunk-relative key index), the K
+// scale multiplies the logit and the V scale multiplies P before its bf16 rounding for
+// O += P V (the importance uses P itself).
+template <bool KV8>
 __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_taddr, int key_base, int p, float sc2,
-                                         float lse_a, float lse_b, float2 (&imp)[8], int t) {
+                                         float lse_a, float lse_b, float2 (&imp)[8], int t, const float* sc) {
     const float2 s2 = make_float2(sc2, sc2);
     const float2 na = make_float2(-lse_a, -lse_a), nb = make_float2(-lse_b, -lse_b);
     const bool need_mask = key_base + 63 > p;
     uint32_t pk[16];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-        const float2 xa = fma2(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), s2, na);
-        const float2 xb = fma2(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), s2, nb);
+        float2 c2 = s2, vs = make_float2(1.f, 1.f);
+        if (KV8) {
+            const float2 k2 = *reinterpret_cast<const float2*>(sc + 8 * j + 2 * (t & 3));
+            vs = *reinterpret_cast<const float2*>(sc + KT + 8 * j + 2 * (t & 3));
+            c2 = make_float2(sc2 * k2.x, sc2 * k2.y);
+        }
+        const float2 xa = fma2(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), c2, na);
+        const float2 xb = fma2(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), c2, nb);
         float2 pa = make_float2(ex2(xa.x), ex2(xa.y)), pb = make_float2(ex2(xb.x), ex2(xb.y));
         if (need_mask) {
             const int k0 = key_base + 8 * j + 2 * (t & 3);
             if (k0 > p) { pa.x = 0.f; pb.x = 0.f; }
             if (k0 + 1 > p) { pa.y = 0.f; pb.y = 0.f; }
         }
-        pk[2 * j] = pack_bf16(pa.x, pa.y);
-        pk[2 * j + 1] = pack_bf16(pb.x, pb.y);
+        if (KV8) {
+            pk[2 * j] = pack_bf16(pa.x * vs.x, pa.y * vs.y);
+            pk[2 * j + 1] = pack_bf16(pb.x * vs.x, pb.y * vs.y);
+        } else {
+            pk[2 * j] = pack_bf16(pa.x, pa.y);
+            pk[2 * j + 1] = pack_bf16(pb.x, pb.y);
+        }
         imp[j] = add2(pa, pb);
     }
     umma::tmem_st16x128_x8(p_taddr, pk);
@@ -464,7 +521,9 @@ constexpr int VS2 = 3;                          // V stages of pass 2
 constexpr int NSB2 = 2;                         // S/P buffers at columns 0, 128
 constexpr uint32_t kQcol = 256;                 // Q (packed bf16 pairs) at columns 256 .. 319
 constexpr uint32_t kOcol = 384;                 // O at columns 384 .. 511
+static_assert(KS2 + 2 < SC_SLOTS, "scale ring shorter than the pass-2 lookahead");
 
+template <bool KV8>
 __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constant__ CUtensorMap qmap,
                                                            const __grid_constant__ CUtensorMap kmap,
                                                            const __grid_constant__ CUtensorMap vmap, Params a) {
@@ -472,7 +531,9 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     uint8_t* smem = align1024(smem_raw);
     uint8_t* kst = smem;                                      // K stages
     uint8_t* vst = kst + KS2 * TILE_BYTES;                    // V stages
+    float* ring = reinterpret_cast<float*>(vst + VS2 * TILE_BYTES);   // [SC_SLOTS][2][KT] (e4m3)
     __shared__ uint64_t k_full[KS2], k_empty[KS2], v_full[VS2], v_empty[VS2];
+    __shared__ uint64_t sc_full[SC_SLOTS];
     __shared__ uint64_t s_full[NSB2], p_full[NSB2], q_tm, o_full;
     __shared__ uint32_t tmem_base;
     __shared__ volatile int abort_flag;
@@ -495,6 +556,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         for (int u = 0; u < NSB2; ++u) { mbar_init(&s_full[u], 1); mbar_init(&p_full[u], 16); }
         mbar_init(&q_tm, 16);
         mbar_init(&o_full, 1);
+        for (int s = 0; s < SC_SLOTS; ++s) mbar_init(&sc_full[s], 1);
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -510,24 +572,41 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     const uint32_t tmem = tmem_base;            // S/P buffers at 0, 128; Q at 256; O at 384
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (KV8 || lane == 0) {
             // K runs one tile ahead of V: K(t) is needed by S(t), V(t) only after P(t)
             for (int t = 0; t <= n_kt; ++t) {
                 if (t < n_kt) {
                     const int s = t % KS2;
-                    if (t >= KS2 && !wait_or_abort(&k_empty[s], ((t / KS2) - 1) & 1, &abort_flag, a.status)) break;
+                    bool ok = true;
+                    if (lane == 0 && t >= KS2) ok = wait_or_abort(&k_empty[s], ((t / KS2) - 1) & 1, &abort_flag, a.status);
+                    if (KV8) ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
                     const int krow = static_cast<int>(b * a.cap) + t * KT;
-                    mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
-                    tma_load_2d(kst + s * TILE_BYTES, &kmap, &k_full[s], 0, krow);
-                    tma_load_2d(kst + s * TILE_BYTES + BOX_BYTES, &kmap, &k_full[s], 64, krow);
+                    if (lane == 0) {
+                        mbar_arrive_expect_tx(&k_full[s], TILE_BYTES);
+                        tma_load_2d(kst + s * TILE_BYTES, &kmap, &k_full[s], 0, krow);
+                        tma_load_2d(kst + s * TILE_BYTES + BOX_BYTES, &kmap, &k_full[s], 64, krow);
+                    }
+                    if (KV8) {  // the tile's 128 K and 128 V scales into ring slot t % SC_SLOTS
+                        float4* slot = reinterpret_cast<float4*>(ring + (t % SC_SLOTS) * 2 * KT);
+                        slot[lane] = __ldg(reinterpret_cast<const float4*>(a.ksc + krow) + lane);
+                        slot[32 + lane] = __ldg(reinterpret_cast<const float4*>(a.vsc + krow) + lane);
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&sc_full[t % SC_SLOTS]);
+                    }
                 }
                 if (t >= 1) {
                     const int j = t - 1, s = j % VS2;
-                    if (j >= VS2 && !wait_or_abort(&v_empty[s], ((j / VS2) - 1) & 1, &abort_flag, a.status)) break;
-                    const int vrow = static_cast<int>(b * a.cap) + j * KT;
-                    mbar_arrive_expect_tx(&v_full[s], TILE_BYTES);
-                    tma_load_2d(vst + s * TILE_BYTES, &vmap, &v_full[s], 0, vrow);
-                    tma_load_2d(vst + s * TILE_BYTES + BOX_BYTES, &vmap, &v_full[s], 64, vrow);
+                    bool ok = true;
+                    if (lane == 0 && j >= VS2) ok = wait_or_abort(&v_empty[s], ((j / VS2) - 1) & 1, &abort_flag, a.status);
+                    if (KV8) ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
+                    if (lane == 0) {
+                        const int vrow = static_cast<int>(b * a.cap) + j * KT;
+                        mbar_arrive_expect_tx(&v_full[s], TILE_BYTES);
+                        tma_load_2d(vst + s * TILE_BYTES, &vmap, &v_full[s], 0, vrow);
+                        tma_load_2d(vst + s * TILE_BYTES + BOX_BYTES, &vmap, &v_full[s], 64, vrow);
+                    }
                 }
             }
         }
@@ -641,9 +720,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             float2 imp[8];
             const int key0 = i * KT + 64 * kh;
             const uint32_t ta = tmem + u * 128 + lanes + 64 * kh;     // this warp's 64 S columns
+            const float* sc = ring + (i % SC_SLOTS) * 2 * KT + 64 * kh;
+            if (KV8 && !__all_sync(0xffffffffu, wait_or_abort(&sc_full[i % SC_SLOTS], (i / SC_SLOTS) & 1, &abort_flag,
+                                                              a.status)))
+                break;
             umma::tmem_ld16x256_x8(ta, r);
             umma::tmem_ld_wait();
-            p2_chunk(r, ta, key0, p, sc2, lse_a, lse_b, imp, lane);    // P into the first 32
+            p2_chunk<KV8>(r, ta, key0, p, sc2, lse_a, lse_b, imp, lane, sc);    // P into the first 32
             umma::tmem_st_wait();
             warp_arrive(&p_full[u]);
             // importance of the row's keys key0 + 2 lane, + 1: reduced and stored after P has
@@ -703,33 +786,100 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
     }
 }
 
+// e4m3 cache rows 0 .. max_ctx - 1 of every sequence -> exact bf16 copies of their codes,
+// [B][capw][128] with capw = max_ctx rounded up to the 128-key tile, zero rows after
+// max_ctx; and the row scales copied to [B][capw] (0 after max_ctx), 16-byte aligned per
+// tile.  Each thread converts 8 codes.
+__global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint8_t* __restrict__ k8, const uint8_t* __restrict__ v8,
+                                                         const float* __restrict__ ks, const float* __restrict__ vs,
+                                                         int B, int64_t cap, int64_t max_ctx, int64_t capw,
+                                                         __nv_bfloat16* __restrict__ kw, __nv_bfloat16* __restrict__ vw,
+                                                         float* __restrict__ ksw, float* __restrict__ vsw) {
+    const int64_t n = static_cast<int64_t>(B) * capw * 16;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t row = i >> 4;
+        const int c = static_cast<int>(i & 15);
+        const int64_t b = row / capw, t = row % capw;
+        uint4 ko = make_uint4(0, 0, 0, 0), vo = ko;
+        float kscale = 0.f, vscale = 0.f;
+        if (t < max_ctx) {
+            const int64_t src = (b * cap + t) * D + c * 8;
+            const uint2 kc = *reinterpret_cast<const uint2*>(k8 + src);
+            const uint2 vc = *reinterpret_cast<const uint2*>(v8 + src);
+            ko = make_uint4(e4m3x2_to_bf16x2(kc.x & 0xffff), e4m3x2_to_bf16x2(kc.x >> 16),
+                            e4m3x2_to_bf16x2(kc.y & 0xffff), e4m3x2_to_bf16x2(kc.y >> 16));
+            vo = make_uint4(e4m3x2_to_bf16x2(vc.x & 0xffff), e4m3x2_to_bf16x2(vc.x >> 16),
+                            e4m3x2_to_bf16x2(vc.y & 0xffff), e4m3x2_to_bf16x2(vc.y >> 16));
+            if (c == 0) { kscale = ks[b * cap + t]; vscale = vs[b * cap + t]; }
+        }
+        reinterpret_cast<uint4*>(kw + row * D)[c] = ko;
+        reinterpret_cast<uint4*>(vw + row * D)[c] = vo;
+        if (c == 0) { ksw[row] = kscale; vsw[row] = vscale; }
+    }
+}
+
 }  // namespace
 
 namespace {
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+int64_t widened_rows(int64_t max_ctx) { return (max_ctx + KT - 1) / KT * KT; }
 }  // namespace
 
-size_t prefill_ws_bytes(int batch, int n_q, int64_t max_ctx, bool fused_select) {
+size_t prefill_ws_bytes(int batch, int n_q, int64_t max_ctx, bool fused_select, bool kv8) {
     const size_t rows = static_cast<size_t>(batch) * n_q;
     size_t n = al256(sizeof(float) * rows * H);                               // log-sum-exp (log2)
     if (fused_select)
         n += al256(sizeof(uint32_t) * rows * kImpBins) + al256(sizeof(int) * rows) +
              al256(sizeof(uint2) * rows * static_cast<size_t>(max_ctx));    // bins, counts, candidates
+    if (kv8) {                                                                // widened K, V and scales
+        const size_t wr = static_cast<size_t>(batch) * widened_rows(max_ctx);
+        n += 2 * al256(wr * D * 2) + 2 * al256(wr * 4);
+    }
     return n;
 }
 
 cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     const int rows = pa.batch * pa.n_q;
     if (rows <= 0) return cudaSuccess;
-    CUtensorMap qmap, kmap, vmap;
-    const uint64_t kv_rows = static_cast<uint64_t>(pa.batch) * pa.cap;
-    if (!make_tmap_2d(&qmap, pa.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, static_cast<uint64_t>(rows) * H, D * 2, 64, 128, true) ||
-        !make_tmap_2d(&kmap, pa.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, kv_rows, D * 2, 64, KT, true) ||
-        !make_tmap_2d(&vmap, pa.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, kv_rows, D * 2, 64, KT, true))
-        return cudaErrorInvalidValue;
     uint8_t* ws = static_cast<uint8_t*>(pa.ws);
+    // e4m3 cache: the tiles come from exact bf16 copies of the codes in the workspace (the
+    // end of the prefill region), the scales are applied in the kernels
+    const void* kb = pa.k;
+    const void* vb = pa.v;
+    int64_t cap = pa.cap;
+    const float* ksw = nullptr;
+    const float* vsw = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (pa.kv8) {
+        const int64_t capw = widened_rows(pa.max_ctx);
+        const size_t wr = static_cast<size_t>(pa.batch) * capw;
+        uint8_t* w = ws + prefill_ws_bytes(pa.batch, pa.n_q, pa.max_ctx, pa.fused_select, false);
+        __nv_bfloat16* kw = reinterpret_cast<__nv_bfloat16*>(w);
+        w += al256(wr * D * 2);
+        __nv_bfloat16* vw = reinterpret_cast<__nv_bfloat16*>(w);
+        w += al256(wr * D * 2);
+        float* kscw = reinterpret_cast<float*>(w);
+        w += al256(wr * 4);
+        float* vscw = reinterpret_cast<float*>(w);
+        const int64_t work = static_cast<int64_t>(wr) * 16;
+        const int grid = static_cast<int>(work / 256 + 1 < 8 * 148 ? work / 256 + 1 : 8 * 148);
+        widen_e4m3_kernel<<<grid, 256, 0, st>>>(static_cast<const uint8_t*>(pa.k), static_cast<const uint8_t*>(pa.v),
+                                                pa.k_scale, pa.v_scale, pa.batch, pa.cap, pa.max_ctx, capw, kw, vw,
+                                                kscw, vscw);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        kb = kw; vb = vw; cap = capw; ksw = kscw; vsw = vscw;
+    }
+    CUtensorMap qmap, kmap, vmap;
+    const uint64_t kv_rows = static_cast<uint64_t>(pa.batch) * cap;
+    if (!make_tmap_2d(&qmap, pa.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, static_cast<uint64_t>(rows) * H, D * 2, 64, 128, true) ||
+        !make_tmap_2d(&kmap, kb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, kv_rows, D * 2, 64, KT, true) ||
+        !make_tmap_2d(&vmap, vb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, D, kv_rows, D * 2, 64, KT, true))
+        return cudaErrorInvalidValue;
     Params a{};
-    a.B = pa.batch; a.n_q = pa.n_q; a.cap = pa.cap; a.max_ctx = pa.max_ctx; a.q_pos0 = pa.q_pos0; a.q = pa.q;
+    a.B = pa.batch; a.n_q = pa.n_q; a.cap = cap; a.max_ctx = pa.max_ctx; a.q_pos0 = pa.q_pos0; a.q = pa.q;
+    a.ksc = ksw; a.vsc = vsw;
     a.sc2 = pa.scale * kLog2e;
     a.lse2 = reinterpret_cast<float*>(ws);
     ws += al256(sizeof(float) * static_cast<size_t>(rows) * H);
@@ -753,14 +903,16 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
     }
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
     const int blocks2 = pa.batch * ((pa.n_q + ROWS2 - 1) / ROWS2);
-    const size_t s1 = 1024 + 2 * TILE_BYTES + P1_STAGES * TILE_BYTES;
-    const size_t s2 = 1024 + (KS2 + VS2) * TILE_BYTES;
-    cudaError_t e = cudaFuncSetAttribute(prefill_lse_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
+    const size_t s1 = 1024 + 2 * TILE_BYTES + P1_STAGES * TILE_BYTES + (pa.kv8 ? SC_SLOTS * KT * 4 : 0);
+    const size_t s2 = 1024 + (KS2 + VS2) * TILE_BYTES + (pa.kv8 ? SC_SLOTS * 2 * KT * 4 : 0);
+    auto k1 = pa.kv8 ? prefill_lse_kernel<true> : prefill_lse_kernel<false>;
+    auto k2 = pa.kv8 ? prefill_out_kernel<true> : prefill_out_kernel<false>;
+    e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s1));
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(prefill_out_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));
+    e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(s2));
     if (e != cudaSuccess) return e;
-    prefill_lse_kernel<<<blocks, NT, s1, st>>>(qmap, kmap, a);
-    prefill_out_kernel<<<blocks2, NT, s2, st>>>(qmap, kmap, vmap, a);
+    k1<<<blocks, NT, s1, st>>>(qmap, kmap, a);
+    k2<<<blocks2, NT, s2, st>>>(qmap, kmap, vmap, a);
     e = cudaGetLastError();
     if (e != cudaSuccess || !pa.fused_select) return e;
     return launch_cand_select(cs, st);

@@ -76,6 +76,12 @@ DECODE_128K_FP8 = Workload("decode_b32_ctx131072_h16_d128_e4m3", batch=32, n_q=1
                            needle_norm=4.0 * 128 ** 0.5)
 
 
+# Not one of the five: the agent-round prefill shape against an e4m3 cache (all rows of
+# the N(0,1) source quantized per token; the bridge's e4m3 output is timed on its own).
+PREFILL_AGENT_FP8 = Workload("prefill_b4_ctx65536+8192_h16_d128_e4m3", batch=4, n_q=8192,
+                             ctx=65536 + 8192, heads=16, head_dim=128, kv_dtype="e4m3")
+
+
 def sweep(ctx: int, block_size: int = 1, layout: str = "one_per_block") -> Workload:
     """Selection-granularity sweep: one sequence, decode at p = ctx - 1, 64 planted tokens."""
     return Workload(f"sweep_ctx{ctx}_{'token' if block_size == 1 else 'block%d' % block_size}",
@@ -186,4 +192,4 @@ def bf16_bits(t: torch.Tensor):
 
 
 __all__ = ["Workload", "Inputs", "make_inputs", "shrink", "sweep", "TINY", "DECODE_128K",
-           "PREFILL_AGENT", "DECODE_1M_FP8", "SWEEP_CTX", "WINDOW", "BUDGET", "bf16_bits"]
+           "PREFILL_AGENT", "PREFILL_AGENT_FP8", "DECODE_1M_FP8", "SWEEP_CTX", "WINDOW", "BUDGET", "bf16_bits"]

@@ -172,6 +172,24 @@ def test_prefill_small_all_rows(n_q, ctx):
     assert rep["differing_rows"] <= max(2, rep["rows"] // 50)
 
 
+@pytest.mark.parametrize("n_q,ctx", [(300, 1000), (8, 129), (77, 2048 + 5)])
+def test_prefill_e4m3_small_all_rows(n_q, ctx):
+    # FP8 cache ("Xiaomi unveils HySparse2 ...", AINews article: million-token caches in FP8):
+    # codes widened exactly to bf16 for the tensor cores, scales applied in fp32
+    wl = synth.Workload("prefill_e4m3_case", batch=2, n_q=n_q, ctx=ctx, heads=16, head_dim=128,
+                        kv_dtype="e4m3", n_sparse=1)
+    rep = block_parity(wl, seed=n_q + ctx + 5)
+    assert rep["differing_rows"] <= max(2, rep["rows"] // 50)
+
+
+def test_prefill_e4m3_agent_full_size_sampled():
+    wl = synth.PREFILL_AGENT_FP8
+    rng = np.random.default_rng(4)
+    rows = np.unique(np.concatenate([[0, 127, 128, 1151, 1152, 8191], rng.choice(wl.n_q, 14, replace=False)]))
+    rep = block_parity(wl, seed=1009, seqs=[0, 3], device="cuda", rows=rows)
+    assert rep["differing_rows"] <= max(2, rep["rows"] // 20)
+
+
 def test_prefill_with_bridge_small():
     wl = synth.shrink(synth.PREFILL_AGENT, batch=2, n_q=200, ctx=1500 + 200, n_new=200, d_model=256,
                       n_sparse=1)
