@@ -400,6 +400,9 @@ def run_ours(args, ws_, rank, local):
     st = hs.hs2_last_status(blk.ws)
     if st != hs.HS2_OK:
         raise RuntimeError("device status after timing: " + hs.status_string(st))
+    sparse_direct = sparse_layer_timing(blk, stream)
+    if hs.hs2_last_status(blk.ws) != hs.HS2_OK:
+        raise RuntimeError("device status after the sparse-layer timing")
 
     ms_per_step = total_ms / K
     queries_per_step = wl.batch * len(blk.qs)
@@ -490,6 +493,7 @@ def run_ours(args, ws_, rank, local):
         "layers": {
             "full_attn_select": {"ms": full_ms, "GB/s": full_gbs, "hbm_frac": full_gbs / hbm,
                                  "bytes_per_call": blk.full_bytes()},
+            "sparse_attn_direct": sparse_direct,
             "sparse_attn": {"ms": sparse_ms, "timing": "(step - full call) / sparse layers, back-to-back graph replays",
                             "queries/s": wl.batch / (sparse_ms / 1e3),
                             "GB/s": sparse_gbs, "hbm_frac": sparse_gbs / hbm,
@@ -513,6 +517,9 @@ def run_ours(args, ws_, rank, local):
         out["other_configs"] = run_configs(args)
     if ws_ == 1 and rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(wl, seed=1002, sample_seqs=args.cpu_sample)
+        out["cpu_baseline"].update(_cpu_info())
+        if not args.no_configs and args.workload == "all" and not args.small:
+            out["cpu_baseline_configs"] = cpu_baseline_configs()
     return out
 
 
@@ -592,6 +599,59 @@ class ConfigBlock:
         qo = 2 * wl.heads * wl.head_dim * (4 if wl.q_dtype == "f32" else 2)
         per_row = min(wl.q_pos0 + 1, wl.window + wl.budget) * (row + 4) + qo
         return wl.batch * wl.n_q * per_row
+
+
+def sparse_layer_timing(blk, stream, n_sets=14, reps=50):
+    """One decode sparse layer timed directly.  Cold: a graph of n_sets layers, each over a
+    different index set (the step's own selection, then sets of seeded distinct positions,
+    disjoint from one another), so that the rows a layer gathers were last touched
+    n_sets - 1 layers earlier -- 14 x 18.9 MB, over twice the 126 MB L2.  Warm: the same
+    graph over the step's own selection every time (layers 2 and 3 of a real step)."""
+    wl = blk.wl
+    B, S = wl.batch, blk.desc.idx_stride
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234)
+    perms = torch.stack([torch.randperm(wl.ctx - 1, generator=g, device="cuda") for _ in range(B)])
+    sets = [blk.idx]
+    for k in range(1, n_sets):
+        sel = perms[:, (k - 1) * S:k * S].sort(dim=1).values.to(torch.int32)
+        sets.append(sel.view(B, 1, S).contiguous())
+    cnt = torch.full_like(blk.cnt, S)
+    out = torch.empty_like(blk.q)
+    hs = blk.hs
+
+    def run(idx_sets):
+        def f():
+            for i, idx in enumerate(idx_sets):
+                hs.hs2_sparse_attn(blk.desc, blk.qs[i % len(blk.qs)], blk.k, blk.v, None, None, idx,
+                                   cnt if i else blk.cnt, out, None, blk.ws)
+        (graph,) = _capture([f], stream)
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(reps + 1)]
+        ev[0].record(stream)
+        for i in range(reps):
+            graph.replay()
+            ev[i + 1].record(stream)
+        torch.cuda.synchronize()
+        t = sorted(ev[i].elapsed_time(ev[i + 1]) / len(idx_sets) for i in range(reps))
+        del graph
+        return t
+
+    hbm, _, _ = _peaks()
+    res = {}
+    for key, idx_sets in (("cold", sets), ("warm", [blk.idx] * n_sets)):
+        t = run(idx_sets)
+        med = statistics.median(t)
+        gbs = blk.sparse_bytes() / (med / 1e3) / 1e9
+        res[key] = {"ms_median": med, "ms_p10": t[len(t) // 10], "ms_p90": t[(9 * len(t)) // 10],
+                    "queries/s": wl.batch / (med / 1e3), "GB/s": gbs, "hbm_frac": gbs / hbm,
+                    "replays": reps, "layers_per_replay": n_sets}
+    res["cold"]["l2"] = (f"{n_sets} index sets rotated, {n_sets} x {blk.sparse_bytes() / 1e6:.1f} MB gathered "
+                         "per replay (> 2 x L2)")
+    res["warm"]["l2"] = "the step's own selection every layer: rows L2-resident after the first (warm, labelled)"
+    return res
 
 
 def _time_graph(fn, stream, reps):
@@ -709,6 +769,115 @@ def cpu_baseline(wl, seed, sample_seqs, min_seconds=10.0):
             "sample": f"{sample_seqs} of the {wl.batch} sequences of {wl.name}, whole hybrid block "
                       f"(full attention + selection + {wl.n_sparse} sparse layers), fp64, one thread per "
                       f"sequence, run {reps} times ({dt:.1f} s)"}
+
+
+def _cpu_info():
+    model = ""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    model = ln.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_cores": os.cpu_count(), "cpu_model": model}
+
+
+def _host_inputs(wl, seed):
+    """The workload's inputs drawn on the GPU (host draws of ~1e9 normals take minutes) and
+    copied to the host; e4m3 caches are quantized by the oracle from the fp32 source."""
+    import numpy as np
+    import oracle
+    inp = synth.make_inputs(wl, seed=seed, device="cuda")
+    q = inp.q_full.double().cpu().numpy()
+    qs = [x.double().cpu().numpy() for x in inp.q_sparse]
+    kv = []
+    for b in range(wl.batch):
+        if wl.kv_dtype == "e4m3":
+            pair = []
+            for src in (inp.k_src, inp.v_src):
+                codes, scales = oracle.fp8_quantize(src[b].cpu().numpy())
+                pair.append(oracle.fp8_dequantize(codes, scales))
+            kv.append(tuple(pair))
+        else:
+            kv.append((inp.k[b].double().cpu().numpy(), inp.v[b].double().cpu().numpy()))
+    del inp
+    torch.cuda.empty_cache()
+    return q, qs, kv, np
+
+
+def cpu_baseline_configs():
+    """The CPU oracle, as it stands, on each of the other workloads: the tiny prefill, the
+    1M-token e4m3 decode and the granularity sweep on their complete inputs, the agent
+    prefill on a fixed 256-row subset of one sequence (its full oracle is ~19 TFLOP of fp64
+    work).  The oracle parallelises a call over its query rows with OpenMP on every host
+    core; decode calls (one row) run one sequence per host thread."""
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    out = {"host": _cpu_info()}
+
+    def block(wl, q, qs, k, v, pos, block_size=1):
+        _, _, sc = oracle.full_attn(q, k, v, pos)
+        idx, cnt = oracle.select_rows(sc, pos, wl.window, wl.budget, block_size=block_size)
+        for ql in qs:
+            oracle.sparse_attn(ql, k, v, idx, cnt)
+        return sc
+
+    # tiny fp32 prefill: all 2048 rows, 1 sparse layer
+    wl = synth.TINY
+    q, qs, kv, np = _host_inputs(wl, 1001)
+    t0 = time.perf_counter()
+    block(wl, q[0], [x[0] for x in qs], kv[0][0], kv[0][1], np.arange(wl.n_q))
+    dt = time.perf_counter() - t0
+    out["tiny_f32"] = {"value": wl.n_q / dt, "unit": "query rows/s (whole block)", "seconds": dt,
+                       "cores": os.cpu_count(), "kind": "oracle",
+                       "sample": f"complete {wl.name}: full attention + selection + 1 sparse layer, all rows"}
+
+    # agent prefill: 256 fixed rows of sequence 0 (the first 65536 rows are the cached context)
+    wl = synth.shrink(synth.PREFILL_AGENT, batch=1, n_new=0, n_sparse=3)
+    q, qs, kv, np = _host_inputs(wl, 1003)
+    rng = np.random.default_rng(0)
+    fixed = np.array([0, 127, 128, 1151, 1152, 8191])
+    rest = rng.choice(np.setdiff1d(np.arange(wl.n_q), fixed), 256 - fixed.size, replace=False)
+    rows = np.sort(np.concatenate([fixed, rest]))
+    t0 = time.perf_counter()
+    block(wl, q[0][rows], [x[0][rows] for x in qs], kv[0][0], kv[0][1], wl.q_pos0 + rows)
+    dt = time.perf_counter() - t0
+    out["prefill_agent"] = {"value": rows.size / dt, "unit": "query rows/s (whole block, 3 sparse layers)",
+                            "seconds": dt, "cores": os.cpu_count(), "kind": "oracle",
+                            "sample": "256 fixed rows (0, 127, 128, 1151, 1152, 8191 and 250 seeded others) of one "
+                                      "sequence of " + synth.PREFILL_AGENT.name + " (bridge rows drawn directly)",
+                            "extrapolated_full_config_s": dt / rows.size * synth.PREFILL_AGENT.batch * wl.n_q,
+                            "extrapolation": "linear in rows; labelled, not measured"}
+
+    # 1M-token e4m3 decode: the 4 sequences on 4 host threads, whole block
+    wl = synth.DECODE_1M_FP8
+    q, qs, kv, np = _host_inputs(wl, 1004)
+    pos = np.array([wl.ctx - 1])
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=wl.batch) as ex:
+        list(ex.map(lambda b: block(wl, q[b], [x[b] for x in qs], kv[b][0], kv[b][1], pos), range(wl.batch)))
+    dt = time.perf_counter() - t0
+    out["decode_1m_e4m3"] = {"value": wl.batch * wl.n_sparse / dt, "unit": "sparse-attn queries/s (whole block)",
+                             "seconds": dt, "cores": wl.batch, "kind": "oracle",
+                             "sample": f"complete {wl.name} (dequantized cache), one sequence per thread"}
+    del q, qs, kv
+
+    # granularity sweep: each context, token arm and block arm on the same importance
+    pts = []
+    for ctx in synth.SWEEP_CTX:
+        wl = synth.sweep(ctx)
+        q, qs, kv, np = _host_inputs(wl, 1005)
+        pos = np.array([ctx - 1])
+        t0 = time.perf_counter()
+        sc = block(wl, q[0], [x[0] for x in qs], kv[0][0], kv[0][1], pos)
+        oracle.select_rows(sc, pos, wl.window, wl.budget, block_size=64)
+        pts.append({"ctx": ctx, "seconds": time.perf_counter() - t0})
+    out["granularity_sweep"] = {"points": pts, "unit": "seconds per point (full attention, both selections, "
+                                "1 sparse layer)", "cores": 1, "kind": "oracle",
+                                "sample": "complete sweep workloads (one sequence each)"}
+    return out
 
 
 def run_reference(args, ws_, rank):
