@@ -109,9 +109,10 @@ typedef struct {
  * `scores_in_workspace` is non-zero they are kept in the workspace
  * ([batch][n_q][max_ctx] fp32) when the caller passes no scores buffer.  Prefill
  * on the tensor-core path (n_q > 1, budget <= 4096) selects from candidate lists
- * that its second pass streams into the workspace (up to max_ctx (importance,
- * position) pairs of 8 bytes per query row; in practice a few thousand are
- * written) and needs no importance rows.  Returns 0 for an invalid description.
+ * that its second pass streams into the workspace (room for max_ctx + 128
+ * (importance, position) pairs of 8 bytes per query row; in practice a few
+ * thousand are written) and needs no importance rows.  Returns 0 for an invalid
+ * description.
  */
 HS2_API size_t hs2_workspace_size(const hs2_attn_desc* desc, int32_t scores_in_workspace);
 

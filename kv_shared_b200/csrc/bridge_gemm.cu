@@ -7,9 +7,10 @@
 //   [K | V] = hidden [rows x d_model] * W_kv [d_model x 2D],  bf16 in, fp32
 //   accumulation, rounded to bf16 and written to cache rows pos0[b] + t.
 //
-// One CTA computes a 256-row x 256-column tile (all of K and V for 256 tokens) as two
+// One CTA computes up to 256 rows x 256 columns (all of K and V for its tokens) as two
 // M = 128 halves that share every W_kv tile, so that W_kv (re-read from L2 by every CTA)
-// costs half as much traffic per row and the 32768-row agent workload runs in one wave:
+// costs half as much traffic per row; the rows are spread evenly over one CTA per SM
+// (221 or 222 rows each for the 32768-row agent workload: one wave on every SM):
 //   warp 0        TMA producer: two A tiles [128 x 64] (K-major, 128-byte swizzle) and
 //                 the B tile [64 x 256] as four [64 x 64] boxes of W_kv, which is
 //                 row-major (d_model x 2D) and therefore an MN-major B operand
@@ -87,9 +88,13 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
     __shared__ int abort_flag;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.x * BMC;
+    // this CTA's rows [m0, m1): the rows spread evenly over the grid (between BM and BMC
+    // rows per CTA); a half past m1 still loads and multiplies rows of the next CTA (or
+    // zero-filled ones past the end) and stores nothing
+    const int m0 = static_cast<int>(static_cast<int64_t>(blockIdx.x) * a.rows / gridDim.x);
+    const int m1 = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * a.rows / gridDim.x);
     const int nk = a.d_model / BK;
-    const int mh = (m0 + BM < a.rows) ? MH : 1;     // halves holding rows (a partial one is zero-filled)
+    const int mh = (m0 + BM < m1) ? MH : 1;         // halves holding rows of this CTA
 
     if (threadIdx.x == 0) {
         prefetch_tmap(&amap);
@@ -155,7 +160,7 @@ __global__ void __launch_bounds__(NT, 1) bridge_kernel(const __grid_constant__ C
         const bool ok = mbar_wait(&acc_ready, 0, a.status);
         umma::fence_after();
         int64_t crow = -1;
-        if (row < a.rows) {
+        if (row < m1) {
             const int b = row / a.n, t = row % a.n;
             const int p0 = a.pos0[b];
             if (p0 < 0 || static_cast<int64_t>(p0) + a.n > a.cap)
@@ -238,7 +243,12 @@ cudaError_t launch_bridge(const BridgeArgs& ba, cudaStream_t st) {
     const size_t smem = 1024 + STAGES * STAGE_BYTES;
     cudaError_t e = cudaFuncSetAttribute(bridge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    bridge_kernel<<<(rows + BMC - 1) / BMC, NT, smem, st>>>(amap, bmap, a);
+    // one CTA per SM when that gives each CTA BM .. BMC rows (the arithmetic intensity sits
+    // just under the HBM ridge, so idle SMs cost bandwidth); fewer, fuller CTAs otherwise
+    int grid = num_sms();
+    if (grid * BMC < rows) grid = (rows + BMC - 1) / BMC;
+    if (grid * BM > rows) grid = (rows + BM - 1) / BM;
+    bridge_kernel<<<grid, NT, smem, st>>>(amap, bmap, a);
     return cudaGetLastError();
 }
 

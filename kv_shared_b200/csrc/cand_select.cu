@@ -112,9 +112,14 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
     const int words = (n_cand + 31) >> 5;
 
     if (kg > 0) {
-        const uint2* list = a.cand + static_cast<size_t>(row) * a.cand_ld;
-        const int cap = a.cand_ld < n_cand ? static_cast<int>(a.cand_ld) : n_cand;
-        const int c = min(a.cand_cnt[row], cap);
+        // the row's two segments (one per key half of the tiles), read as one list
+        const uint2* seg0 = a.cand + static_cast<size_t>(row) * 2 * a.cand_seg;
+        const uint2* seg1 = seg0 + a.cand_seg;
+        const int segcap = a.cand_seg < n_cand ? static_cast<int>(a.cand_seg) : n_cand;
+        const int c0 = max(0, min(a.cand_cnt[2 * row], segcap));
+        const int c = c0 + max(0, min(a.cand_cnt[2 * row + 1], segcap));
+        auto entry = [&](int i) -> uint2 { return i < c0 ? seg0[i] : seg1[i - c0]; };
+        auto entry_cs = [&](int i) -> uint2 { return i < c0 ? __ldcs(seg0 + i) : __ldcs(seg1 + (i - c0)); };
         if (tid < kImpBins) sm.hist[tid] = a.hist[static_cast<size_t>(row) * kImpBins + tid];
         if (use_map)
             for (int i = tid; i < words; i += CNT) sm.map[i] = 0u;
@@ -161,7 +166,7 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
 #pragma unroll
             for (int u = 0; u < kLd; ++u) {
                 const int i = base + u * CNT + tid;
-                e[u] = i < c ? __ldcs(list + i) : make_uint2(0u, 0x7fffffffu);
+                e[u] = i < c ? entry_cs(i) : make_uint2(0u, 0x7fffffffu);
             }
 #pragma unroll
             for (int u = 0; u < kLd; ++u) {
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
                 sm.dh[tid] = 0;
                 __syncthreads();
                 for (int i = tid; i < c; i += CNT) {
-                    const uint2 e = list[i];
+                    const uint2 e = entry(i);
                     const unsigned long long k = sel_key(e);
                     if (imp_bin(__uint_as_float(e.x)) == bs && (k & msk) == pre) atomicAdd(&sm.dh[(k >> shift) & 255u], 1);
                 }
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
                 __syncthreads();
                 const int d = sm.digit;
                 for (int i = tid; i < c; i += CNT) {                  // keys of higher digits are in
-                    const uint2 e = list[i];
+                    const uint2 e = entry(i);
                     const unsigned long long k = sel_key(e);
                     if (imp_bin(__uint_as_float(e.x)) == bs && (k & msk) == pre &&
                         static_cast<int>((k >> shift) & 255u) > d)
@@ -231,7 +236,7 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
             }
             for (int base = 0; base < c; base += CNT) {
                 const int i = base + tid;
-                const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
+                const uint2 e = i < c ? entry(i) : make_uint2(0u, 0u);
                 const unsigned long long k = sel_key(e);
                 warp_append(i < c && imp_bin(__uint_as_float(e.x)) == bs && (k & msk) == pre, k, sm.bnd[0],
                             &sm.nbnd[0], kBndCap);

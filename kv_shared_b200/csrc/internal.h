@@ -64,9 +64,9 @@ struct CandSelectArgs {
     int64_t max_ctx;
     int window, budget, idx_stride;
     const uint32_t* hist;     // [rows][kImpBins] candidates per importance bin
-    const int* cand_cnt;      // [rows]
-    const uint2* cand;        // [rows][cand_ld] (importance bits, position)
-    int64_t cand_ld;
+    const int* cand_cnt;      // [rows][2] entries per segment
+    const uint2* cand;        // [rows][2][cand_seg] (importance bits, position)
+    int64_t cand_seg;
     int32_t* idx;
     int32_t* cnt;
     uint32_t* status;

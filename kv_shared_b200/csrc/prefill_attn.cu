@@ -63,9 +63,9 @@ struct Params {
     // count per sequence) and apply these per-token scales in fp32
     const float* ksc;                           // [B][cap] K row scales (0 past max_ctx)
     const float* vsc;                           // [B][cap] V row scales
-    uint2* cand;                                // [B*n_q][cand_ld] (importance bits, position) or null
-    int64_t cand_ld;
-    int* cand_cnt;                              // [B*n_q] entries appended
+    uint2* cand;                                // [B*n_q][2][cand_seg] (importance bits, position) or null:
+    int64_t cand_seg;                           // one segment per key half of the tiles
+    int* cand_cnt;                              // [B*n_q][2] entries appended per segment
     uint32_t* hist;                             // [B*n_q][kImpBins] candidates per importance bin
 };
 
@@ -451,29 +451,28 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
 // up are those of all keys seen.
 struct RowSel {
     uint32_t hist[kImpBins];
-    int count;
     float thr;
 };
 
-// Appends this warp's candidates among its two keys per lane (positions k, k + 1).
-__device__ __forceinline__ void p2_candidates(float2 v, int k, int last_cand, RowSel& rs, uint2* crow, int lane) {
+// Appends this warp's candidates among its two keys per lane (positions k, k + 1) to its
+// own segment `seg` of the row's list, `count` entries long so far (the same in every lane).
+__device__ __forceinline__ void p2_candidates(float2 v, int k, int last_cand, RowSel& rs, uint2* seg, int& count,
+                                              int lane) {
     const float th = *reinterpret_cast<volatile float*>(&rs.thr);
     const bool a0 = k <= last_cand && v.x >= th;
     const bool a1 = k + 1 <= last_cand && v.y >= th;
     const uint32_t m0 = __ballot_sync(0xffffffffu, a0), m1 = __ballot_sync(0xffffffffu, a1);
     if ((m0 | m1) == 0u) return;
-    int base = 0;
-    if (lane == 0) base = atomicAdd(&rs.count, __popc(m0) + __popc(m1));
-    base = __shfl_sync(0xffffffffu, base, 0);
     const uint32_t lt = (1u << lane) - 1u;
-    int off = base + __popc(m0 & lt) + __popc(m1 & lt);
+    int off = count + __popc(m0 & lt) + __popc(m1 & lt);
+    count += __popc(m0) + __popc(m1);
     if (a0) {
         atomicAdd(&rs.hist[imp_bin(v.x)], 1u);
-        crow[off++] = make_uint2(__float_as_uint(v.x), static_cast<uint32_t>(k));
+        seg[off++] = make_uint2(__float_as_uint(v.x), static_cast<uint32_t>(k));
     }
     if (a1) {
         atomicAdd(&rs.hist[imp_bin(v.y)], 1u);
-        crow[off] = make_uint2(__float_as_uint(v.y), static_cast<uint32_t>(k + 1));
+        seg[off] = make_uint2(__float_as_uint(v.y), static_cast<uint32_t>(k + 1));
     }
 }
 
@@ -561,10 +560,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         abort_flag = 0;
     }
     for (int i = threadIdx.x; i < ROWS2 * kImpBins; i += NT) rsel[i / kImpBins].hist[i % kImpBins] = 0u;
-    if (threadIdx.x < ROWS2) {
-        rsel[threadIdx.x].count = 0;
-        rsel[threadIdx.x].thr = a.budget > 0 ? 0.f : INFINITY;
-    }
+    if (threadIdx.x < ROWS2) rsel[threadIdx.x].thr = a.budget > 0 ? 0.f : INFINITY;
     if (warp == 1) umma::tmem_alloc(&tmem_base, 512);
     umma::fence_before();
     __syncthreads();
@@ -668,7 +664,8 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         float* srow = (row_ok && a.scores) ? a.scores + (static_cast<size_t>(b) * a.n_q + row) * a.score_ld : nullptr;
         const bool vec2 = (a.score_ld & 1) == 0;
         const size_t grow = static_cast<size_t>(b) * a.n_q + row;
-        uint2* crow = (row_ok && a.cand) ? a.cand + grow * a.cand_ld : nullptr;
+        uint2* crow = (row_ok && a.cand) ? a.cand + (2 * grow + kh) * a.cand_seg : nullptr;   // this warp's segment
+        int ccount = 0;
         const int last_cand = p - a.window;                  // candidates: positions 0 .. p - W
         RowSel& rs = rsel[lrow];
         const float sc2 = a.sc2;
@@ -742,17 +739,19 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
                 }
             }
             if (crow && key0 <= last_cand) {
-                p2_candidates(sv, k, last_cand, rs, crow, lane);
+                p2_candidates(sv, k, last_cand, rs, crow, ccount, lane);
                 if (kh == 0 && (i & 3) == 3) p2_raise_threshold(rs, a.budget, lane);
             }
         }
         // the row's candidate count and bins, for the selection kernel
         named_sync(2, NSOFT);
-        if (crow && kh == 0) {
-            uint4 h;
-            h.x = rs.hist[4 * lane]; h.y = rs.hist[4 * lane + 1]; h.z = rs.hist[4 * lane + 2]; h.w = rs.hist[4 * lane + 3];
-            reinterpret_cast<uint4*>(a.hist + grow * kImpBins)[lane] = h;
-            if (lane == 0) a.cand_cnt[grow] = rs.count;
+        if (crow) {
+            if (kh == 0) {
+                uint4 h;
+                h.x = rs.hist[4 * lane]; h.y = rs.hist[4 * lane + 1]; h.z = rs.hist[4 * lane + 2]; h.w = rs.hist[4 * lane + 3];
+                reinterpret_cast<uint4*>(a.hist + grow * kImpBins)[lane] = h;
+            }
+            if (lane == 0) a.cand_cnt[2 * grow + kh] = ccount;
         }
         // O epilogue: 4 warps per lane quarter; this thread owns TMEM lane m = (row, head)
         // and columns 32 cc .. 32 cc + 31
@@ -824,14 +823,16 @@ __global__ void __launch_bounds__(256) widen_e4m3_kernel(const uint8_t* __restri
 namespace {
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 int64_t widened_rows(int64_t max_ctx) { return (max_ctx + KT - 1) / KT * KT; }
+// entries of one warp's candidate segment: the keys of its 64-key half of every tile
+int64_t cand_segment(int64_t max_ctx) { return (max_ctx + 1) / 2 + KT / 2; }
 }  // namespace
 
 size_t prefill_ws_bytes(int batch, int n_q, int64_t max_ctx, bool fused_select, bool kv8) {
     const size_t rows = static_cast<size_t>(batch) * n_q;
     size_t n = al256(sizeof(float) * rows * H);                               // log-sum-exp (log2)
     if (fused_select)
-        n += al256(sizeof(uint32_t) * rows * kImpBins) + al256(sizeof(int) * rows) +
-             al256(sizeof(uint2) * rows * static_cast<size_t>(max_ctx));    // bins, counts, candidates
+        n += al256(sizeof(uint32_t) * rows * kImpBins) + al256(sizeof(int) * 2 * rows) +
+             al256(sizeof(uint2) * rows * 2 * static_cast<size_t>(cand_segment(max_ctx)));   // bins, counts, lists
     if (kv8) {                                                                // widened K, V and scales
         const size_t wr = static_cast<size_t>(batch) * widened_rows(max_ctx);
         n += 2 * al256(wr * D * 2) + 2 * al256(wr * 4);
@@ -893,12 +894,12 @@ cudaError_t launch_prefill_full(const PrefillArgs& pa, cudaStream_t st) {
         a.hist = reinterpret_cast<uint32_t*>(ws);
         ws += al256(sizeof(uint32_t) * static_cast<size_t>(rows) * kImpBins);
         a.cand_cnt = reinterpret_cast<int*>(ws);
-        ws += al256(sizeof(int) * static_cast<size_t>(rows));
+        ws += al256(sizeof(int) * 2 * static_cast<size_t>(rows));
         a.cand = reinterpret_cast<uint2*>(ws);
-        a.cand_ld = pa.max_ctx;
+        a.cand_seg = cand_segment(pa.max_ctx);
         cs.rows = rows; cs.n_q = pa.n_q; cs.q_pos0 = pa.q_pos0; cs.max_ctx = pa.max_ctx;
         cs.window = pa.window; cs.budget = pa.budget; cs.idx_stride = pa.idx_stride;
-        cs.hist = a.hist; cs.cand_cnt = a.cand_cnt; cs.cand = a.cand; cs.cand_ld = a.cand_ld;
+        cs.hist = a.hist; cs.cand_cnt = a.cand_cnt; cs.cand = a.cand; cs.cand_seg = a.cand_seg;
         cs.idx = pa.idx; cs.cnt = pa.cnt; cs.status = pa.status;
     }
     const int blocks = pa.batch * ((pa.n_q + ROWS - 1) / ROWS);
