@@ -483,6 +483,7 @@ def run_ours(args, ws_, rank, local):
     sparse_gbs = blk.sparse_bytes() / (sparse_ms / 1e3) / 1e9
     out = {
         "metric": METRIC, "value": value, "unit": "sparse-attn queries/s", "n_gpus": ws_,
+        "block_steps/s": ws_ * 1e3 / ms_per_step,
         "steps": K, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx, "heads": wl.heads,
@@ -555,7 +556,10 @@ class ConfigBlock:
         self.ws = hs.alloc_workspace(self.desc, scores_in_workspace=False)
         self.o = torch.empty_like(self.q)
         self.o_sp = torch.empty_like(self.q)
-        self.scores = torch.empty(B, wl.n_q, wl.ctx, dtype=torch.float32, device="cuda")
+        # importance rows returned to the caller (decode workloads: the block arm reads them)
+        # (the tensor-core prefill selects from its own candidate lists and returns none)
+        self.scores = (torch.empty(B, wl.n_q, wl.ctx, dtype=torch.float32, device="cuda")
+                       if wl.n_q == 1 or wl.kv_dtype == "f32" else None)
         self.idx = torch.empty(B, wl.n_q, self.desc.idx_stride, dtype=torch.int32, device="cuda")
         self.cnt = torch.empty(B, wl.n_q, dtype=torch.int32, device="cuda")
         self.bidx = torch.empty_like(self.idx)
@@ -722,6 +726,28 @@ def run_configs(args):
         torch.cuda.empty_cache()
     out["granularity_sweep"] = {"workload": "sweep_ctx{4096,32768,262144,1048576}, 64 planted tokens, "
                                             "one per 64-token block", "points": sweep}
+
+    # the agent-round prefill shape against an e4m3 cache: the full-attention call (widening of
+    # the codes, both passes with the scales applied, selection) and one sparse layer
+    wl = synth.PREFILL_AGENT_FP8
+    blk = ConfigBlock(wl, seed=1009)
+    blk.full(); blk.sparse()
+    torch.cuda.synchronize()
+    if hs.hs2_last_status(blk.ws) != hs.HS2_OK:
+        raise RuntimeError(wl.name + ": device status " + hs.status_string(hs.hs2_last_status(blk.ws)))
+    full_ms = _time_graph(blk.full, stream, 3)
+    sparse_ms = _time_graph(blk.sparse, stream, 3)
+    flops = wl.batch * sum(wl.q_pos0 + r + 1 for r in range(wl.n_q)) * wl.heads * wl.head_dim * 4
+    tf_sus, _ = _sustained_tflops()
+    _, tf_burst, _ = _peaks()
+    out["prefill_agent_e4m3"] = {"workload": wl.name, "full_attn_select_ms": full_ms,
+                                 "TFLOP/s": flops / (full_ms / 1e3) / 1e12,
+                                 "tc_frac": flops / (full_ms / 1e3) / 1e12 / tf_sus,
+                                 "tc_frac_of_burst": flops / (full_ms / 1e3) / 1e12 / tf_burst,
+                                 "sparse_attn_ms": sparse_ms,
+                                 "tokens/s (full call + 1 sparse layer)": wl.batch * wl.n_q / ((full_ms + sparse_ms) / 1e3)}
+    del blk
+    torch.cuda.empty_cache()
 
     wl = synth.TINY
     blk = ConfigBlock(wl, seed=1001)

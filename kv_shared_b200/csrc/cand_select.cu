@@ -32,11 +32,10 @@ constexpr int kBndCap = 2048;                  // cutoff-bin keys held in shared
 constexpr int kMapWords = 8192;                // bitmap of candidate positions (262144 bits)
 constexpr int kFinal = 32;                     // keys ranked by one warp at the end
 
+// Shared memory: this struct, then the bitmap of the longest candidate range of the launch
+// (or the position list when that range is too long for a bitmap), sized at launch so that
+// more CTAs fit on an SM.
 struct Smem {
-    union {
-        uint32_t map[kMapWords];               // selected candidate positions (bitmap mode)
-        int sel[kFusedSelectMaxBudget];        // selected positions (list mode)
-    };
     unsigned long long bnd[2][kBndCap];        // cutoff keys (ping-pong while narrowing)
     uint32_t hist[kImpBins];
     int dh[256];                               // digit counts
@@ -100,15 +99,17 @@ __device__ __forceinline__ int block_excl_scan(int x, Smem& sm) {
 }
 
 __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
-    extern __shared__ uint8_t smem_raw[];
+    extern __shared__ __align__(16) uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+    uint32_t* map = reinterpret_cast<uint32_t*>(smem_raw + sizeof(Smem));     // bitmap mode
+    int* sel = reinterpret_cast<int*>(smem_raw + sizeof(Smem));               // list mode
     const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int b = row / a.n_q, r = row % a.n_q;
     const int p = checked_pos(a.q_pos0[b] + r, a.max_ctx, a.status);
     const int n_cand = max(0, p - a.window + 1);
     const int kg = min(a.budget, n_cand);              // global picks of this row
     const int nwin = min(p + 1, a.window);
-    const bool use_map = n_cand <= kMapWords * 32;
+    const bool use_map = a.map_words > 0;                  // launch-wide: n_cand <= 32 * map_words
     const int words = (n_cand + 31) >> 5;
 
     if (kg > 0) {
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
         auto entry_cs = [&](int i) -> uint2 { return i < c0 ? __ldcs(seg0 + i) : __ldcs(seg1 + (i - c0)); };
         if (tid < kImpBins) sm.hist[tid] = a.hist[static_cast<size_t>(row) * kImpBins + tid];
         if (use_map)
-            for (int i = tid; i < words; i += CNT) sm.map[i] = 0u;
+            for (int i = tid; i < words; i += CNT) map[i] = 0u;
         if (tid == 0) { sm.nsel = 0; sm.nbnd[0] = 0; sm.nbnd[1] = 0; sm.cur = 0; sm.kand = ~0ull; sm.kor = 0ull; }
         __syncthreads();
         if (warp == 0) {                               // 1. the cutoff bin
@@ -175,9 +176,9 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
                 const int pos = static_cast<int>(e[u].y);
                 const bool hi = bin > bs;
                 if (use_map) {
-                    if (hi && pos < n_cand) atomicOr(&sm.map[pos >> 5], 1u << (pos & 31));
+                    if (hi && pos < n_cand) atomicOr(&map[pos >> 5], 1u << (pos & 31));
                 } else {
-                    warp_append(hi, pos, sm.sel, &sm.nsel, kFusedSelectMaxBudget);
+                    warp_append(hi, pos, sel, &sm.nsel, kFusedSelectMaxBudget);
                 }
                 warp_append(bin == bs && bnd_smem, sel_key(e[u]), sm.bnd[0], &sm.nbnd[0], kBndCap);
                 if (bin == bs) { kand &= sel_key(e[u]); kor |= sel_key(e[u]); }
@@ -190,10 +191,10 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
         auto take = [&](unsigned long long k) {
             const int pos = key_pos(k);
             if (use_map) {
-                if (pos >= 0 && pos < n_cand) atomicOr(&sm.map[pos >> 5], 1u << (pos & 31));
+                if (pos >= 0 && pos < n_cand) atomicOr(&map[pos >> 5], 1u << (pos & 31));
             } else {
                 const int s = atomicAdd(&sm.nsel, 1);
-                if (s < kFusedSelectMaxBudget) sm.sel[s] = pos;
+                if (s < kFusedSelectMaxBudget) sel[s] = pos;
             }
         };
         if (!bnd_smem) {
@@ -315,10 +316,10 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
         const int per = (words + CNT - 1) / CNT;
         const int w0 = min(tid * per, words), w1 = min(w0 + per, words);
         int cnt_bits = 0;
-        for (int w = w0; w < w1; ++w) cnt_bits += __popc(sm.map[w]);
+        for (int w = w0; w < w1; ++w) cnt_bits += __popc(map[w]);
         int o = block_excl_scan(cnt_bits, sm);
         for (int w = w0; w < w1; ++w) {
-            uint32_t m = sm.map[w];
+            uint32_t m = map[w];
             while (m) {
                 const int bit = __ffs(m) - 1;
                 m &= m - 1;
@@ -332,10 +333,10 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
         while (np < kg) np <<= 1;
         const int ns = min(sm.nsel, kg);
         if (tid == 0 && sm.nsel != kg) set_status(a.status, HS2_ERR_INDEX);
-        for (int i = ns + tid; i < np; i += CNT) sm.sel[i] = 0x7fffffff;
+        for (int i = ns + tid; i < np; i += CNT) sel[i] = 0x7fffffff;
         __syncthreads();
-        bitonic_asc(sm.sel, np);
-        for (int j = tid; j < kg; j += CNT) out[j] = sm.sel[j];
+        bitonic_asc(sel, np);
+        for (int j = tid; j < kg; j += CNT) out[j] = sel[j];
     }
     for (int j = kg + tid; j < a.idx_stride; j += CNT) out[j] = j < kg + nwin ? win0 + (j - kg) : -1;
     if (tid == 0) a.cnt[row] = kg + nwin;
@@ -343,10 +344,16 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
 
 }  // namespace
 
-cudaError_t launch_cand_select(const CandSelectArgs& a, cudaStream_t st) {
-    if (a.rows <= 0) return cudaSuccess;
-    if (a.budget > kFusedSelectMaxBudget) return cudaErrorInvalidValue;
-    const size_t sm = sizeof(Smem);
+cudaError_t launch_cand_select(const CandSelectArgs& in, cudaStream_t st) {
+    if (in.rows <= 0) return cudaSuccess;
+    if (in.budget > kFusedSelectMaxBudget) return cudaErrorInvalidValue;
+    CandSelectArgs a = in;
+    // the longest candidate range of the launch is [0, max_ctx - 1 - window]
+    const int64_t n_cand = a.max_ctx - a.window > 0 ? a.max_ctx - a.window : 0;
+    const int64_t words = (n_cand + 31) / 32;
+    a.map_words = words <= kMapWords ? static_cast<int>(words > 0 ? words : 1) : 0;
+    const size_t sm = sizeof(Smem) + (a.map_words > 0 ? 4 * static_cast<size_t>(a.map_words)
+                                                       : 4 * static_cast<size_t>(kFusedSelectMaxBudget));
     cudaError_t e = cudaFuncSetAttribute(cand_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(sm));
     if (e != cudaSuccess) return e;

@@ -67,6 +67,7 @@ struct CandSelectArgs {
     const int* cand_cnt;      // [rows][2] entries per segment
     const uint2* cand;        // [rows][2][cand_seg] (importance bits, position)
     int64_t cand_seg;
+    int map_words;            // set by launch_cand_select: bitmap words per CTA (0: position lists)
     int32_t* idx;
     int32_t* cnt;
     uint32_t* status;
