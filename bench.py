@@ -349,11 +349,36 @@ def run_prefill(args, ws_):
     }
 
 
+def run_decode_e4m3(args):
+    """The million-token e4m3 decode alone (its full-attention call and a sparse layer); with
+    --small one sequence at 655360 keys, still past the single-launch limit of 148 x 4096 keys,
+    so the same two-kernel path runs on a case small enough to profile."""
+    import kv_shared_b200 as hs
+    wl = synth.DECODE_1M_FP8
+    if args.small:
+        wl = synth.shrink(wl, batch=1, ctx=655360, needles=8)
+    blk = ConfigBlock(wl, seed=1004)
+    blk.full(); blk.sparse()
+    torch.cuda.synchronize()
+    if hs.hs2_last_status(blk.ws) != hs.HS2_OK:
+        raise RuntimeError(wl.name + ": device status " + hs.status_string(hs.hs2_last_status(blk.ws)))
+    stream = torch.cuda.current_stream()
+    full_ms = _time_graph(blk.full, stream, max(3, args.steps))
+    hbm, _, _ = _peaks()
+    return {"workload": wl.name, "batch": wl.batch, "ctx": wl.ctx,
+            "full_attn_select": {"ms": full_ms, "bytes_per_call": blk.cache_bytes(),
+                                 "hbm_frac": blk.cache_bytes() / (full_ms / 1e3) / 1e9 / hbm,
+                                 "launches": hs.hs2_full_attn_launches(blk.desc)},
+            "needle_recall": blk.recall(blk.idx.cpu(), blk.cnt.cpu())}
+
+
 def run_ours(args, ws_, rank, local):
     import kv_shared_b200 as hs
     if args.workload == "prefill":
         out = {"metric": METRIC, "prefill": run_prefill(args, ws_), "n_gpus": ws_, "data": "synthetic"}
         return out
+    if args.workload == "decode_e4m3":
+        return {"metric": METRIC, "decode_e4m3": run_decode_e4m3(args), "n_gpus": ws_, "data": "synthetic"}
     wl = _decode_workload(args)
     blk = DecodeBlock(wl, seed=1002 + rank)
     stream = torch.cuda.current_stream()
@@ -943,8 +968,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the 1M e4m3, sweep and tiny workloads")
-    ap.add_argument("--workload", choices=["all", "decode", "prefill"], default="all",
-                    help="all: decode headline + prefill leg")
+    ap.add_argument("--workload", choices=["all", "decode", "prefill", "decode_e4m3"], default="all",
+                    help="all: decode headline + prefill leg; decode_e4m3: the 1M-token e4m3 decode alone")
     ap.add_argument("--small", action="store_true",
                     help="reduced shapes of the same kernels (for profiler captures; not a bench value)")
     ap.add_argument("--prefill-steps", type=int, default=10)

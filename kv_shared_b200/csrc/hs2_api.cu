@@ -104,12 +104,20 @@ bool fused_prefill_select(const hs2_attn_desc* d, Path path) {
     return path == Path::TC && d->n_q > 1 && d->budget <= kFusedSelectMaxBudget;
 }
 
+// decode on tensor cores selects long rows through candidate lists built from its importance
+// rows (shorter ones fit the cluster select's shared memory, which is faster for them)
+bool list_decode_select(const hs2_attn_desc* d, Path path) {
+    return path == Path::TC && d->n_q == 1 && d->budget <= kFusedSelectMaxBudget && d->max_ctx >= kListSelectMinCtx;
+}
+
 // bytes after the status block needed by hs2_full_attn_select
 size_t full_region(const hs2_attn_desc* d, Path path, bool scores_in_ws) {
     const size_t rows = static_cast<size_t>(d->batch) * d->n_q;
     const bool fused = fused_prefill_select(d, path);
     size_t n = 0;
-    if (path == Path::TC && d->n_q == 1) n += a256(decode_ws_bytes(d->batch, d->max_ctx, d->kv_dtype == HS2_E4M3));
+    if (path == Path::TC && d->n_q == 1)
+        n += a256(decode_ws_bytes(d->batch, d->max_ctx, d->kv_dtype == HS2_E4M3)) +
+             (list_decode_select(d, path) ? a256(row_select_ws_bytes(d->batch, d->max_ctx)) : 0);
     if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q, d->max_ctx, fused, d->kv_dtype == HS2_E4M3));
     if (scores_in_ws && !fused) n += a256(sizeof(float) * rows * static_cast<size_t>(score_pitch(d)));
     return n;
@@ -164,9 +172,17 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     int64_t score_ld = desc->max_ctx;
     size_t used = 0;
     const bool fused = fused_prefill_select(desc, path);
-    if (path == Path::TC)
-        used = desc->n_q == 1 ? a256(decode_ws_bytes(desc->batch, desc->max_ctx, desc->kv_dtype == HS2_E4M3))
-                              : a256(prefill_ws_bytes(desc->batch, desc->n_q, desc->max_ctx, fused, kv8));
+    const bool list_sel = list_decode_select(desc, path);
+    uint8_t* sel_ws = nullptr;                           // decode: bins, counts, candidate lists
+    if (path == Path::TC && desc->n_q == 1) {
+        used = a256(decode_ws_bytes(desc->batch, desc->max_ctx, kv8));
+        if (list_sel) {
+            sel_ws = region + used;
+            used += a256(row_select_ws_bytes(desc->batch, desc->max_ctx));
+        }
+    } else if (path == Path::TC) {
+        used = a256(prefill_ws_bytes(desc->batch, desc->n_q, desc->max_ctx, fused, kv8));
+    }
     if (!score_buf && !fused) {
         score_buf = reinterpret_cast<float*>(region + used);
         score_ld = score_pitch(desc);
@@ -205,13 +221,14 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     sa.rows = desc->batch * desc->n_q; sa.n_q = desc->n_q; sa.q_pos0 = q_pos0; sa.max_ctx = desc->max_ctx;
     sa.scores = score_buf; sa.score_ld = score_ld; sa.window = desc->window; sa.budget = desc->budget;
     sa.block_size = 1; sa.idx_stride = desc->idx_stride; sa.idx = idx; sa.cnt = cnt; sa.status = status;
+    if (list_sel) return from_cuda(launch_row_select(sa, sel_ws, st));
     return from_cuda(launch_select(sa, st));
 }
 
 int32_t hs2_full_attn_launches(const hs2_attn_desc* desc) {
     Path path;
     if (check_desc(desc, &path) != HS2_OK) return 0;
-    int32_t n = 1;                                      // the selection
+    int32_t n = list_decode_select(desc, path) ? 4 : 1;   // the selection (decode: range, bins, lists, top-K)
     if (path == Path::F32) n += 1;
     else if (desc->n_q > 1) n += 2;                     // prefill: log-sum-exp pass, output pass
     else n += plan_decode(desc->batch, desc->max_ctx, desc->kv_dtype == HS2_E4M3).fused ? 1 : 3;  // or: 2 passes + merge

@@ -114,6 +114,15 @@ struct SelectArgs {
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
+// Token-level selection (block_size 1, budget <= kFusedSelectMaxBudget) from importance rows
+// through candidate lists: range, histogram and compaction passes over slices of every row,
+// then cand_select.  Scratch: row_select_ws_bytes (range, bins, counts, lists).  Decode calls
+// use it for rows longer than launch_select's clusters hold in shared memory (16 CTAs x 24576
+// keys): launch_select streams such rows from global memory twice, with few CTAs per row.
+constexpr int64_t kListSelectMinCtx = 16 * 24576 + 1;
+size_t row_select_ws_bytes(int rows, int64_t max_ctx);
+cudaError_t launch_row_select(const SelectArgs& a, void* ws, cudaStream_t st);
+
 // ---------------------------------------------------------------- sparse attention
 struct SparsePlan {
     int splits;

@@ -220,6 +220,41 @@ def test_decode_1m_fp8_full_size_sampled():
     _block_parity(synth.DECODE_1M_FP8, seed=1004, seqs=[3], device="cuda")
 
 
+def test_decode_long_rows_list_select():
+    # rows longer than the cluster select holds in shared memory take the candidate-list
+    # selection (range, fine bins, lists, top-K); ragged positions put short rows, rows
+    # below the window and rows with fewer candidates than the budget in the same call
+    wl = synth.shrink(synth.DECODE_128K, batch=6, ctx=400000, needles=16)
+    pos0 = np.array([0, 100, 1151, 5000, 393300, wl.ctx - 1])
+    _block_parity(wl, seed=1010, pos0=pos0, device="cuda")
+
+
+def test_decode_long_rows_all_equal_importance():
+    # zero keys: every logit 0 and every importance equal, so the lowest positions win; the
+    # whole row lands in one bin of the list selection, which narrows it in global memory
+    from hs2_check import check_selection
+    T = 400000
+    g = torch.Generator(device="cuda")
+    g.manual_seed(9)
+    q = torch.randn(1, 1, 16, 128, generator=g, device="cuda").to(torch.bfloat16)
+    k = torch.zeros(1, T, 128, dtype=torch.bfloat16, device="cuda")
+    v = torch.randn(1, T, 128, generator=g, device="cuda").to(torch.bfloat16)
+    desc = hs.make_desc(1, 1, 16, 128, max_ctx=T)
+    ws = hs.alloc_workspace(desc)
+    o = torch.empty_like(q)
+    idx = torch.empty(1, 1, desc.idx_stride, dtype=torch.int32, device="cuda")
+    cnt = torch.empty(1, 1, dtype=torch.int32, device="cuda")
+    q_pos0 = torch.tensor([T - 1], dtype=torch.int32, device="cuda")
+    hs.hs2_full_attn_select(desc, q, k, v, None, None, q_pos0, o, None, idx, cnt, None, ws)
+    assert hs.hs2_last_status(ws) == hs.HS2_OK
+    pos = np.array([T - 1])
+    _, _, sc = oracle.full_attn(q[0].double().cpu().numpy(), k[0].double().cpu().numpy(),
+                                v[0].double().cpu().numpy(), pos)
+    o_idx, o_cnt = oracle.select_rows(sc, pos, 128, 1024)
+    check_selection(idx[0].cpu().numpy(), cnt[0].cpu().numpy(), o_idx, o_cnt, sc, pos, 128)
+    np.testing.assert_array_equal(idx[0].cpu().numpy(), o_idx)
+
+
 @pytest.mark.parametrize("ctx", [4096, 32768, 262144, 1 << 20])   # 1M: two-kernel decode path
 def test_granularity_sweep_recall(ctx):
     tok = synth.sweep(ctx)

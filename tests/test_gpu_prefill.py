@@ -272,3 +272,14 @@ def test_fused_select_budgets(budget):
     k = torch.randn(ctx, 128, generator=g)
     v = torch.randn(ctx, 128, generator=g)
     _select_case(q, k, v, n_q, ctx, budget=budget)
+
+
+def test_fused_select_long_context_position_lists():
+    # rows with more than 262144 candidates: the selection keeps position lists and sorts
+    # them instead of using a bitmap of the candidate range
+    g = torch.Generator().manual_seed(14)
+    n_q, ctx = 6, 270000
+    q = torch.randn(n_q, 16, 128, generator=g)
+    k = torch.randn(ctx, 128, generator=g)
+    v = torch.randn(ctx, 128, generator=g)
+    _select_case(q, k, v, n_q, ctx)
