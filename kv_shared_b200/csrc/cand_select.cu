@@ -121,16 +121,16 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
         const int c = c0 + max(0, min(a.cand_cnt[2 * row + 1], segcap));
         auto entry = [&](int i) -> uint2 { return i < c0 ? seg0[i] : seg1[i - c0]; };
         auto entry_cs = [&](int i) -> uint2 { return i < c0 ? __ldcs(seg0 + i) : __ldcs(seg1 + (i - c0)); };
-        if (tid < kImpBins) sm.hist[tid] = a.hist[static_cast<size_t>(row) * kImpBins + tid];
+        for (int i = tid; i < kImpBins; i += CNT) sm.hist[i] = a.hist[static_cast<size_t>(row) * kImpBins + i];
         if (use_map)
             for (int i = tid; i < words; i += CNT) map[i] = 0u;
         if (tid == 0) { sm.nsel = 0; sm.nbnd[0] = 0; sm.nbnd[1] = 0; sm.cur = 0; sm.kand = ~0ull; sm.kor = 0ull; }
         __syncthreads();
         if (warp == 0) {                               // 1. the cutoff bin
-            uint32_t h[4];
+            uint32_t h[kImpPerLane];
+            int mine = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) h[j] = sm.hist[4 * lane + j];
-            const int mine = static_cast<int>(h[0] + h[1] + h[2] + h[3]);
+            for (int j = 0; j < kImpPerLane; ++j) { h[j] = sm.hist[kImpPerLane * lane + j]; mine += static_cast<int>(h[j]); }
             int above = mine;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
@@ -139,8 +139,8 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
             }
             int cum = above - mine, best = -1, best_cum = 0;
 #pragma unroll
-            for (int j = 3; j >= 0; --j) {
-                if (best < 0 && cum + static_cast<int>(h[j]) >= kg) { best = 4 * lane + j; best_cum = cum; }
+            for (int j = kImpPerLane - 1; j >= 0; --j) {
+                if (best < 0 && cum + static_cast<int>(h[j]) >= kg) { best = kImpPerLane * lane + j; best_cum = cum; }
                 cum += static_cast<int>(h[j]);
             }
             const int top = __reduce_max_sync(0xffffffffu, best);
@@ -153,7 +153,7 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
             } else if (lane == __ffs(own) - 1) {
                 sm.bstar = top;
                 sm.need = kg - best_cum;
-                sm.nb = static_cast<int>(h[top & 3]);
+                sm.nb = static_cast<int>(h[top % kImpPerLane]);
             }
         }
         __syncthreads();
@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(RNT) row_compact_kernel(RowListArgs a) {
     const int n_cand = row_candidates(a, row, kg);
     const int begin = blockIdx.x * a.slice, end = min(begin + a.slice, n_cand);
     if (kg <= 0 || begin >= end) return;
-    if (tid < kImpBins) ch[tid] = 0u;
+    for (int i = tid; i < kImpBins; i += RNT) ch[i] = 0u;
     // the cutoff fine bin: thread t sums bins 8t .. 8t + 7; suffix sums from the top
     constexpr int PER = kFine / RNT;
     const uint32_t* fr = a.fine + static_cast<size_t>(row) * kFine;
@@ -501,7 +501,8 @@ __global__ void __launch_bounds__(RNT) row_compact_kernel(RowListArgs a) {
         }
     });
     __syncthreads();
-    if (tid < kImpBins && ch[tid]) atomicAdd(a.hist + static_cast<size_t>(row) * kImpBins + tid, ch[tid]);
+    for (int i = tid; i < kImpBins; i += RNT)
+        if (ch[i]) atomicAdd(a.hist + static_cast<size_t>(row) * kImpBins + i, ch[i]);
 }
 
 }  // namespace

@@ -253,21 +253,23 @@ __device__ __forceinline__ float ex2(float x) {
 
 // ---------------------------------------------------------------- importance bins
 // Coarse bins of a non-negative fp32 importance value, used to find the selection
-// cutoff while the values stream out of the prefill kernel: four bins per octave (the
-// exponent and the top two mantissa bits), bin 0 holding everything below 2^-28 (zero
-// included), bin 127 everything from 2^3.75 up (importance never exceeds the head
+// cutoff while the values stream out of the prefill kernel: eight bins per octave (the
+// exponent and the top three mantissa bits), bin 0 holding everything below 2^-28 (zero
+// included), the last bin everything from 2^3.875 up (importance never exceeds the head
 // count, 16).  Bins are ordered like the values they hold.
-constexpr int kImpBins = 128;
-constexpr int kImpBinBase = (127 - 28) << 2;
+constexpr int kImpSub = 3;                                   // mantissa bits in a bin index
+constexpr int kImpBins = 32 << kImpSub;                      // 32 octaves
+constexpr int kImpPerLane = kImpBins / 32;                   // bins per lane in warp scans
+constexpr int kImpBinBase = (127 - 28) << kImpSub;
 
 __device__ __forceinline__ int imp_bin(float v) {
-    const int b = static_cast<int>(__float_as_uint(v) >> 21) - kImpBinBase;
+    const int b = static_cast<int>(__float_as_uint(v) >> (23 - kImpSub)) - kImpBinBase;
     return b < 0 ? 0 : (b > kImpBins - 1 ? kImpBins - 1 : b);
 }
 
 // smallest value of bin b (0 for bin 0)
 __device__ __forceinline__ float imp_bin_floor(int b) {
-    return b <= 0 ? 0.f : __uint_as_float(static_cast<uint32_t>(b + kImpBinBase) << 21);
+    return b <= 0 ? 0.f : __uint_as_float(static_cast<uint32_t>(b + kImpBinBase) << (23 - kImpSub));
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

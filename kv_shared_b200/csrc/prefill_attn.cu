@@ -449,7 +449,7 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
 // ones before it, and the lower position wins ties).  The bins count candidates only:
 // every key at or above the current thr is a candidate, so the counts from thr's bin
 // up are those of all keys seen.
-struct RowSel {
+struct __align__(16) RowSel {
     uint32_t hist[kImpBins];
     float thr;
 };
@@ -480,10 +480,12 @@ __device__ __forceinline__ void p2_candidates(float2 v, int k, int last_cand, Ro
 // (a warp reads the bins while others may still add to them: a stale count is smaller,
 // which only lowers the bound).
 __device__ __forceinline__ void p2_raise_threshold(RowSel& rs, int K, int lane) {
-    uint32_t h[4];
+    uint32_t h[kImpPerLane], mine = 0u;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) h[j] = *reinterpret_cast<volatile uint32_t*>(&rs.hist[4 * lane + j]);
-    const uint32_t mine = h[0] + h[1] + h[2] + h[3];
+    for (int j = 0; j < kImpPerLane; ++j) {
+        h[j] = *reinterpret_cast<volatile uint32_t*>(&rs.hist[kImpPerLane * lane + j]);
+        mine += h[j];
+    }
     uint32_t above = mine;                                     // suffix sum over lanes >= lane
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -493,9 +495,9 @@ __device__ __forceinline__ void p2_raise_threshold(RowSel& rs, int K, int lane) 
     uint32_t cum = above - mine;                               // counts of the lanes above
     int best = -1;
 #pragma unroll
-    for (int j = 3; j >= 0; --j) {
+    for (int j = kImpPerLane - 1; j >= 0; --j) {
         cum += h[j];
-        if (best < 0 && cum >= static_cast<uint32_t>(K)) best = 4 * lane + j;
+        if (best < 0 && cum >= static_cast<uint32_t>(K)) best = kImpPerLane * lane + j;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
@@ -740,16 +742,17 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             }
             if (crow && key0 <= last_cand) {
                 p2_candidates(sv, k, last_cand, rs, crow, ccount, lane);
-                if (kh == 0 && (i & 3) == 3) p2_raise_threshold(rs, a.budget, lane);
+                if (kh == 0 && (i & 1) == 1) p2_raise_threshold(rs, a.budget, lane);
             }
         }
         // the row's candidate count and bins, for the selection kernel
         named_sync(2, NSOFT);
         if (crow) {
             if (kh == 0) {
-                uint4 h;
-                h.x = rs.hist[4 * lane]; h.y = rs.hist[4 * lane + 1]; h.z = rs.hist[4 * lane + 2]; h.w = rs.hist[4 * lane + 3];
-                reinterpret_cast<uint4*>(a.hist + grow * kImpBins)[lane] = h;
+#pragma unroll
+                for (int j = 0; j < kImpPerLane; j += 4)
+                    reinterpret_cast<uint4*>(a.hist + grow * kImpBins)[lane * (kImpPerLane / 4) + j / 4] =
+                        *reinterpret_cast<const uint4*>(&rs.hist[kImpPerLane * lane + j]);
             }
             if (lane == 0) a.cand_cnt[2 * grow + kh] = ccount;
         }
