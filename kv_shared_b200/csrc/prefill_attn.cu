@@ -742,7 +742,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
             }
             if (crow && key0 <= last_cand) {
                 p2_candidates(sv, k, last_cand, rs, crow, ccount, lane);
-                if (kh == 0 && (i & 1) == 1) p2_raise_threshold(rs, a.budget, lane);
+                if (kh == 0 && (i & 3) == 3) p2_raise_threshold(rs, a.budget, lane);
             }
         }
         // the row's candidate count and bins, for the selection kernel

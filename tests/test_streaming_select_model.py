@@ -8,7 +8,7 @@ least K candidates at or above it.  The selection then takes the row's exact top
 desc, position asc) from the list alone.  Correct only if every key of the final top K is
 in the list and the bin counts are exact from the cutoff bin up; this file replays that
 protocol (two warps per row, 128-key tiles split in halves, the bound raised by one warp
-every second tile from the counts of the candidates appended so far, the kernel's bin
+every fourth tile from the counts of the candidates appended so far, the kernel's bin
 arithmetic on fp32 bit patterns) on random and adversarial rows and compares the result
 with a full sort.  It models the kernel's protocol, not its code; the GPU tests run the
 kernels themselves.
@@ -16,7 +16,7 @@ kernels themselves.
 import numpy as np
 from hypothesis import given, settings, strategies as st
 
-SUB = 3                      # mantissa bits in a bin index (8 bins per octave)
+SUB = 2                      # mantissa bits in a bin index (4 bins per octave)
 NBINS = 32 << SUB
 BASE = (127 - 28) << SUB
 
@@ -41,7 +41,7 @@ def raise_threshold(hist, K, thr):
     return thr
 
 
-def stream_candidates(v, last, K, raise_every=2):
+def stream_candidates(v, last, K, raise_every=4):
     """Pass 2's protocol for one row: returns the list (positions) and the bin counts."""
     n = v.size
     thr = np.float32(0.0) if K > 0 else np.float32(np.inf)
