@@ -98,7 +98,7 @@ __device__ __forceinline__ int block_excl_scan(int x, Smem& sm) {
     return before + incl - x;
 }
 
-__global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
+__global__ void __launch_bounds__(CNT, 5) cand_select_kernel(CandSelectArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
     uint32_t* map = reinterpret_cast<uint32_t*>(smem_raw + sizeof(Smem));     // bitmap mode
@@ -159,8 +159,9 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
         __syncthreads();
         const int bs = sm.bstar, nb = sm.nb;
         const bool bnd_smem = nb <= kBndCap;
-        // 2. mark the positions above bin b*, gather bin b*'s keys
-        constexpr int kLd = 8;                         // loads in flight per thread
+        // 2. mark the positions above bin b*, gather bin b*'s keys; a batch's appends take one
+        // shared counter update per warp (a per-entry update serialised the warps on it)
+        constexpr int kLd = 16;                        // loads in flight per thread
         unsigned long long kand = ~0ull, kor = 0ull;
         for (int base = 0; base < c; base += kLd * CNT) {
             uint2 e[kLd];
@@ -169,20 +170,47 @@ __global__ void __launch_bounds__(CNT) cand_select_kernel(CandSelectArgs a) {
                 const int i = base + u * CNT + tid;
                 e[u] = i < c ? entry_cs(i) : make_uint2(0u, 0x7fffffffu);
             }
+            uint32_t at_bs = 0u, above = 0u;           // bit u: entry u in bin b* / above it
 #pragma unroll
             for (int u = 0; u < kLd; ++u) {
                 const bool valid = base + u * CNT + tid < c;
                 const int bin = valid ? imp_bin(__uint_as_float(e[u].x)) : -1;
                 const int pos = static_cast<int>(e[u].y);
-                const bool hi = bin > bs;
-                if (use_map) {
-                    if (hi && pos < n_cand) atomicOr(&map[pos >> 5], 1u << (pos & 31));
-                } else {
-                    warp_append(hi, pos, sel, &sm.nsel, kFusedSelectMaxBudget);
+                if (bin > bs) {
+                    above |= 1u << u;
+                    if (use_map && pos < n_cand) atomicOr(&map[pos >> 5], 1u << (pos & 31));
                 }
-                warp_append(bin == bs && bnd_smem, sel_key(e[u]), sm.bnd[0], &sm.nbnd[0], kBndCap);
-                if (bin == bs) { kand &= sel_key(e[u]); kor |= sel_key(e[u]); }
+                if (bin == bs) {
+                    at_bs |= 1u << u;
+                    kand &= sel_key(e[u]);
+                    kor |= sel_key(e[u]);
+                }
             }
+            auto append = [&](uint32_t flags, int* count, int cap, auto value) {
+                const int n = __popc(flags);
+                int incl = n;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                if (__shfl_sync(0xffffffffu, incl, 31) == 0) return;
+                int base_w = 0;
+                if (lane == 31) base_w = atomicAdd(count, incl);
+                int off = __shfl_sync(0xffffffffu, base_w, 31) + incl - n;
+#pragma unroll
+                for (int u = 0; u < kLd; ++u)             // static indices: e[] stays in registers
+                    if (flags & (1u << u)) {
+                        if (off < cap) value(off, u);
+                        ++off;
+                    }
+            };
+            if (bnd_smem)
+                append(at_bs, &sm.nbnd[0], kBndCap,
+                       [&](int off, int u) { sm.bnd[0][off] = sel_key(e[u]); });
+            if (!use_map)
+                append(above, &sm.nsel, kFusedSelectMaxBudget,
+                       [&](int off, int u) { sel[off] = static_cast<int>(e[u].y); });
         }
         atomicAnd(&sm.kand, kand);
         atomicOr(&sm.kor, kor);

@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
         for (int s = 0; s < P1_STAGES; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
         for (int s = 0; s < 2; ++s)
             for (int h = 0; h < 2; ++h) { mbar_init(&s_full[s][h], 1); mbar_init(&s_empty[s][h], 8); }
-        for (int s = 0; s < SC_SLOTS; ++s) mbar_init(&sc_full[s], 1);
+        for (int s = 0; s < SC_SLOTS; ++s) mbar_init(&sc_full[s], 32);
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -243,13 +243,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
                     tma_load_2d(dst, &kmap, &k_full[s], 0, krow);
                     tma_load_2d(dst + BOX_BYTES, &kmap, &k_full[s], 64, krow);
                 }
-                if (KV8) {      // the tile's 128 key scales into ring slot i % SC_SLOTS
-                    reinterpret_cast<float4*>(ring + (i % SC_SLOTS) * KT)[lane] =
-                        __ldg(reinterpret_cast<const float4*>(a.ksc + krow) + lane);
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&sc_full[i % SC_SLOTS]);
+                if (KV8) {      // the tile's 128 key scales into ring slot i % SC_SLOTS, asynchronously:
+                                // each lane's copy arrives on the slot's barrier when it lands
+                    cp_async16(ring + (i % SC_SLOTS) * KT + 4 * lane, a.ksc + krow + 4 * lane);
+                    cp_async_arrive_noinc(&sc_full[i % SC_SLOTS]);
                 }
             }
+            if (KV8) asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight when the CTA leaves
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -557,7 +557,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
         for (int u = 0; u < NSB2; ++u) { mbar_init(&s_full[u], 1); mbar_init(&p_full[u], 16); }
         mbar_init(&q_tm, 16);
         mbar_init(&o_full, 1);
-        for (int s = 0; s < SC_SLOTS; ++s) mbar_init(&sc_full[s], 1);
+        for (int s = 0; s < SC_SLOTS; ++s) mbar_init(&sc_full[s], 32);
         fence_mbar_init();
         abort_flag = 0;
     }
@@ -585,12 +585,12 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
                         tma_load_2d(kst + s * TILE_BYTES, &kmap, &k_full[s], 0, krow);
                         tma_load_2d(kst + s * TILE_BYTES + BOX_BYTES, &kmap, &k_full[s], 64, krow);
                     }
-                    if (KV8) {  // the tile's 128 K and 128 V scales into ring slot t % SC_SLOTS
-                        float4* slot = reinterpret_cast<float4*>(ring + (t % SC_SLOTS) * 2 * KT);
-                        slot[lane] = __ldg(reinterpret_cast<const float4*>(a.ksc + krow) + lane);
-                        slot[32 + lane] = __ldg(reinterpret_cast<const float4*>(a.vsc + krow) + lane);
-                        __syncwarp();
-                        if (lane == 0) mbar_arrive(&sc_full[t % SC_SLOTS]);
+                    if (KV8) {  // the tile's 128 K and 128 V scales into ring slot t % SC_SLOTS,
+                                // asynchronously (each lane's copies arrive on the slot's barrier)
+                        float* slot = ring + (t % SC_SLOTS) * 2 * KT;
+                        cp_async16(slot + 4 * lane, a.ksc + krow + 4 * lane);
+                        cp_async16(slot + KT + 4 * lane, a.vsc + krow + 4 * lane);
+                        cp_async_arrive_noinc(&sc_full[t % SC_SLOTS]);
                     }
                 }
                 if (t >= 1) {
@@ -607,6 +607,7 @@ __global__ void __launch_bounds__(NT, 1) prefill_out_kernel(const __grid_constan
                     }
                 }
             }
+            if (KV8) asm volatile("cp.async.wait_all;" ::: "memory");   // no copy in flight when the CTA leaves
         }
     } else if (warp == 1) {
         if (lane == 0) {
