@@ -9,7 +9,7 @@
 // with 16-byte cp.async copies into shared memory (swizzled or padded so that
 // ldmatrix reads are conflict-free), all 16 heads are computed against each
 // gathered row once (mma.sync m16n8k16, M = the 16 heads), and the softmax stays
-// online in registers.  Few rows (decode): one 8-CTA cluster per row, the CTAs'
+// online in registers.  Few rows (decode): one 4-CTA cluster per row, the CTAs'
 // partials merged through distributed shared memory.  Many rows (prefill): one
 // CTA per row, or a few split CTAs per row whose partials (max, sum, O) the last
 // of them merges (semaphore counter, no spin).  e4m3 rows are converted to bf16
@@ -35,12 +35,13 @@ using sparse::Layout;
 using sparse::NT;
 using sparse::SUB;
 constexpr int kMaxSplits = 32;     // bound of the split count (shared-memory merge tables)
-constexpr int kCluster = 8;        // CTAs per query row in the cluster kernel
+constexpr int kCluster = 4;        // CTAs per query row in the cluster kernel
 constexpr int kWT = 16;            // selected entries per warp tile (cluster kernel)
-constexpr int kCW = 9;             // warps (= warp tiles) per CTA of the cluster kernel
-constexpr int kCEntries = kWT * kCW;               // 144 entries per CTA
-constexpr int kCNT = 32 * kCW;                     // 288 threads
-static_assert(H == 2 * kCluster, "each CTA of a cluster finalizes two heads");
+constexpr int kCW = 18;            // warps (= warp tiles) per CTA of the cluster kernel
+constexpr int kCEntries = kWT * kCW;               // 288 entries per CTA
+constexpr int kCNT = 32 * kCW;                     // 576 threads
+constexpr int kHPC = H / kCluster;                  // heads each CTA of a cluster finalizes
+static_assert(H % kCluster == 0, "the heads split evenly over a cluster");
 
 struct Params {
     int rows, n_q, idx_stride, splits, chunk;
@@ -257,8 +258,10 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
 // slice of shared memory), scores them against the 16 heads and forms its partial
 // (max, sum, O) with no CTA-wide barrier on the way.  The warps' partials are folded
 // into one per CTA with shared-memory float atomics, each CTA pushes its partial of
-// heads 2p, 2p + 1 into CTA p's shared memory (distributed shared memory stores),
-// and after one cluster barrier CTA p finalizes heads 2p, 2p + 1 from its own memory.
+// heads 4p .. 4p + 3 into CTA p's shared memory (distributed shared memory stores),
+// and after one cluster barrier CTA p finalizes those heads from its own memory.  Four
+// CTAs of 18 warps per row (one per SM) were faster than eight of 9 warps (two per SM):
+// 7.6 against 7.9 us per warm layer at 32 rows.
 template <bool KV8>
 struct CLayout {
     static constexpr int ROWB = KV8 ? 128 : 256;          // bytes per gathered row
@@ -268,8 +271,8 @@ struct CLayout {
     static constexpr int GATHER_END = kCW * (KV8 ? RAW : TILE);
     static constexpr int SLAB_BYTES = kCW * H * sparse::RP * 4;   // the warps' rescaled O, after the compute
     static constexpr int Q_OFF = GATHER_END > SLAB_BYTES ? GATHER_END : SLAB_BYTES;
-    static constexpr int RECV_OFF = Q_OFF + H * D * 2;    // [kCluster][2][D] f32 pushed partials
-    static constexpr int BYTES = RECV_OFF + kCluster * 2 * D * 4;
+    static constexpr int RECV_OFF = Q_OFF + H * D * 2;    // [kCluster][kHPC][D] f32 pushed partials
+    static constexpr int BYTES = RECV_OFF + kCluster * kHPC * D * 4;
 };
 
 // This warp's 16 gathered rows against the 16 heads: state `s` receives the tile's
@@ -408,14 +411,14 @@ __device__ __forceinline__ void attend_warp_tile_e4m3(uint32_t kb, uint32_t vb, 
 }
 
 template <bool KV8>
-__global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
+__global__ void __launch_bounds__(kCNT, (kCNT <= 288 ? 2 : 1)) sparse_cluster_kernel(Params a) {
     using CL = CLayout<KV8>;
     extern __shared__ uint8_t csm_raw[];
     uint8_t* csm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(csm_raw) + 127) & ~uintptr_t(127));
     uint8_t* qs = csm + CL::Q_OFF;                                    // [H][D] bf16, swz_off<16>
-    float* recv_o = reinterpret_cast<float*>(csm + CL::RECV_OFF);    // [kCluster][2][D]
+    float* recv_o = reinterpret_cast<float*>(csm + CL::RECV_OFF);    // [kCluster][kHPC][D]
     __shared__ float wm[kCW][H], wl[kCW][H], cmx[H], csum[H];
-    __shared__ float2 recv_ml[kCluster][2];
+    __shared__ float2 recv_ml[kCluster][kHPC];
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
@@ -535,7 +538,7 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
     }
     __syncthreads();
     asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
-    // ---- push heads 2p, 2p + 1 of this CTA's partial (weighted slab sum) to CTA p
+    // ---- push heads kHPC p .. kHPC p + kHPC - 1 of this CTA's partial (weighted slab sum) to CTA p
     for (int i = tid; i < H * D / 4; i += kCNT) {
         const int h = (4 * i) / D, d = (4 * i) % D;
         const float M = cmx[h];
@@ -550,14 +553,14 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
                 v.x += wt * u.x; v.y += wt * u.y; v.z += wt * u.z; v.w += wt * u.w;
             }
         }
-        float* dst = cluster.map_shared_rank(recv_o, h >> 1) + (rank * 2 + (h & 1)) * D + d;
+        float* dst = cluster.map_shared_rank(recv_o, h / kHPC) + (rank * kHPC + h % kHPC) * D + d;
         *reinterpret_cast<float4*>(dst) = v;
     }
-    if (tid < H) *cluster.map_shared_rank(&recv_ml[rank][tid & 1], tid >> 1) = make_float2(cmx[tid], csum[tid]);
+    if (tid < H) *cluster.map_shared_rank(&recv_ml[rank][tid % kHPC], tid / kHPC) = make_float2(cmx[tid], csum[tid]);
     cluster.sync();                                      // pushes complete and visible; none after it
-    // ---- finalize heads 2 rank, 2 rank + 1 from this CTA's own memory
-    if (tid < 2 * D) {
-        const int hh = tid / D, d = tid % D, h = 2 * rank + hh;
+    // ---- finalize heads kHPC rank .. kHPC rank + kHPC - 1 from this CTA's own memory
+    if (tid < kHPC * D) {
+        const int hh = tid / D, d = tid % D, h = kHPC * rank + hh;
         float M = -INFINITY;
 #pragma unroll
         for (int cc = 0; cc < kCluster; ++cc) M = fmaxf(M, recv_ml[cc][hh].x);
@@ -570,7 +573,7 @@ __global__ void __launch_bounds__(kCNT, 2) sparse_cluster_kernel(Params a) {
 #pragma unroll
         for (int cc = 0; cc < kCluster; ++cc) {
             const float mc = recv_ml[cc][hh].x;
-            if (mc != -INFINITY) acc += ex2(mc - M) * inv * recv_o[(cc * 2 + hh) * D + d];
+            if (mc != -INFINITY) acc += ex2(mc - M) * inv * recv_o[(cc * kHPC + hh) * D + d];
         }
         a.o[(static_cast<size_t>(row) * H + h) * D + d] = __float2bfloat16_rn(acc);
         if (a.lse && d == 0)
