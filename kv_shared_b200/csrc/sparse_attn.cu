@@ -12,9 +12,9 @@
 // online in registers.  Few rows (decode): one 4-CTA cluster per row, the CTAs'
 // partials merged through distributed shared memory.  Many rows (prefill): one
 // CTA per row, or a few split CTAs per row whose partials (max, sum, O) the last
-// of them merges (semaphore counter, no spin).  e4m3 rows are converted to bf16
-// in shared memory (exact) and their per-token scales folded into the logits and
-// into P.
+// of them merges (semaphore counter, no spin).  e4m3 rows feed f16 MMAs straight
+// from shared memory as gathered (exact conversion of each code pair in registers),
+// their per-token scales folded into the logits and into P.
 #include <mutex>
 
 #include <cooperative_groups.h>
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
     uint8_t* smem = sparse::align128(smem_raw);
     using WS = sparse::WarpSlot<KV8>;
     static_assert(4 * WS::BYTES == L::STAGE && 4 * WS::CVT == L::CVT, "four warps' slots make a sub-tile");
-    uint8_t* cvt = smem + STAGES * L::STAGE;               // e4m3 only: each warp's K bf16 then V bf16
+    uint8_t* cvt = smem + STAGES * L::STAGE;               // e4m3: room the warp merge below uses
     int* sidx = reinterpret_cast<int*>(cvt + L::CVT);      // [chunk] cache row per entry (-1 invalid)
     float* sks = reinterpret_cast<float*>(sidx + a.chunk); // [chunk] k scales (e4m3)
     float* svs = sks + a.chunk;                            // [chunk] v scales (e4m3)
@@ -145,13 +145,30 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
 
     // the queries (needed at the first sub-tile) and every index (and scale) of this CTA's
     // entries, loaded once up front, their latencies overlapped
+    // (e4m3: Q as f16 fragments in the e4m3 helpers' k order, divided by a power of two)
     uint32_t qa[8][4];
-    sparse::load_q(a.q + static_cast<size_t>(row) * H * D, qa, lane >> 2, lane & 3);
+    float qscale = 1.f;
+    if (KV8) qscale = load_q_frags_e4m3(a.q + static_cast<size_t>(row) * H * D, lane >> 2, lane & 3, qa);
+    else sparse::load_q(a.q + static_cast<size_t>(row) * H * D, qa, lane >> 2, lane & 3);
     load_entries<KV8>(a, row, e_begin, a.chunk, a.chunk, c, sidx, sks, svs, seq_base);
     __syncthreads();
+    // e4m3: P * v_scale enters the f16 MMAs times pscale, a power of two that brings the
+    // largest V scale of this CTA's entries to 2^14 (f16 keeps 2^-14 .. 65504 normal)
+    float pscale = 1.f;
+    if (KV8) {
+        float vmax = 0.f;
+        for (int e = tid; e < a.chunk; e += NT) vmax = fmaxf(vmax, svs[e]);
+        vmax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(vmax)));   // >= 0: bits order
+        if (lane == 0) wm[0][warp] = vmax;
+        __syncthreads();
+        vmax = fmaxf(fmaxf(wm[0][0], wm[0][1]), fmaxf(wm[0][2], wm[0][3]));
+        __syncthreads();
+        int ex = 0;
+        if (vmax > 0.f) frexpf(vmax, &ex);               // vmax < 2^ex
+        pscale = ldexpf(1.f, 14 - ex);
+    }
     // this warp's rows 16 warp .. 16 warp + 15 of every sub-tile, through its own STAGES slots
     uint8_t* wslots = smem + warp * STAGES * WS::BYTES;
-    uint8_t* wcvt = cvt + warp * WS::CVT;
     auto gather = [&](int i) {
         sparse::gather_warp_rows<KV8>(wslots + (i % STAGES) * WS::BYTES, sidx + i * SUB + warp * 16, a.k, a.v,
                                       seq_base, lane);
@@ -174,10 +191,10 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
         }
         __syncwarp();
         const int e = i * SUB + warp * 16;
-        sparse::attend_warp_rows<KV8>(wslots + (i % STAGES) * WS::BYTES, wcvt, sidx + e, sks + e, svs + e, qa, a.sc2,
-                                      stt, lane);
+        sparse::attend_warp_rows<KV8>(wslots + (i % STAGES) * WS::BYTES, sidx + e, sks + e, svs + e, qa,
+                                      a.sc2 * qscale, pscale, stt, lane);
     }
-    sparse::cta_reduce(stt, reinterpret_cast<float*>(smem), red_o, wm, wl, cm, cl, tid, warp, lane);
+    sparse::cta_reduce<KV8>(stt, reinterpret_cast<float*>(smem), red_o, wm, wl, cm, cl, tid, warp, lane, 1.f / pscale);
 
     if (a.splits == 1) {
         for (int i = tid; i < H * D / 4; i += NT) {

@@ -5,6 +5,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "e4m3_mma.cuh"
 
 namespace hs2 {
 namespace sparse {
@@ -94,63 +95,48 @@ __device__ __forceinline__ void gather_warp_rows(uint8_t* ws, const int* si, con
         const int r = u * RPI + lane / CH;
         const int j = si[r];
         const size_t off = (seq_base + (j >= 0 ? j : 0)) * L::ROWB + ch * 16;
-        const uint32_t d = r * L::ROWP + ch * 16;
+        // bf16: padded rows; e4m3: 128-byte rows with the chunk index XOR-ed by row % 8, the
+        // layout the f16 MMA helpers read
+        const uint32_t d = KV8 ? r * 128 + ((ch ^ (r & 7)) << 4) : r * L::ROWP + ch * 16;
         cp_async16_zfill(ws + d, k + off, j >= 0);
         cp_async16_zfill(ws + 16 * L::ROWP + d, v + off, j >= 0);
     }
 }
 
-// This warp's landed 16 rows (slot `ws`): e4m3 rows are first converted to bf16 in the
-// warp's `cvtw` (exact, swizzled layout), then they are scored against the 16 heads, the
-// online softmax advanced and P V added.  `si` / `sks` / `svs`: the rows' cache rows and
-// (e4m3) per-token scales.
+// This warp's landed 16 rows (slot `ws`) are scored against the 16 heads, the online
+// softmax advanced and P V added.  bf16 rows: bf16 MMAs on the padded rows.  e4m3 rows: f16
+// MMAs straight from the gathered codes (`qa` are Q's f16 fragments in the helpers' k order,
+// `sc2` already divided by Q's power-of-two scale); P times the V scale enters the f16 MMA
+// multiplied by `pscale` (a power of two that keeps the CTA's largest V scale at 2^14), and
+// O accumulates in the helpers' dim order (see pv_e4m3), pscale included.  `si` / `sks` /
+// `svs`: the rows' cache rows and (e4m3) per-token scales.
 template <bool KV8>
-__device__ __forceinline__ void attend_warp_rows(const uint8_t* ws, uint8_t* cvtw, const int* si, const float* sks,
-                                                 const float* svs, const uint32_t (&qa)[8][4], float sc2, State& s,
-                                                 int lane) {
+__device__ __forceinline__ void attend_warp_rows(const uint8_t* ws, const int* si, const float* sks,
+                                                 const float* svs, const uint32_t (&qa)[8][4], float sc2,
+                                                 float pscale, State& s, int lane) {
     using L = Layout<KV8>;
     const int t = lane & 3;
     const uint8_t* kt = ws;
     const uint8_t* vt = ws + 16 * L::ROWP;
-    // byte offset of 16-byte chunk ch of row r: padded rows as copied (bf16), the
-    // swizzled converted rows (e4m3)
-    auto off = [](int r, int ch) -> uint32_t {
-        return KV8 ? swz_off<16>(r, ch) : static_cast<uint32_t>(r * L::ROWP + ch * 16);
-    };
-    if (KV8) {
-#pragma unroll 2
-        for (int it = lane; it < 2 * 16 * 8; it += 32) {
-            const int half = it / (16 * 8), rr = (it / 8) % 16, c8 = it & 7;
-            const uint8_t* src = ws + half * 16 * L::ROWP + rr * L::ROWP + c8 * 16;
-            uint8_t* dst = cvtw + half * 16 * 256;
-            const uint4 in = *reinterpret_cast<const uint4*>(src);
-            const uint16_t* bb = reinterpret_cast<const uint16_t*>(&in);
-            uint4 lo, hi;
-            lo.x = e4m3x2_to_bf16x2(bb[0]); lo.y = e4m3x2_to_bf16x2(bb[1]);
-            lo.z = e4m3x2_to_bf16x2(bb[2]); lo.w = e4m3x2_to_bf16x2(bb[3]);
-            hi.x = e4m3x2_to_bf16x2(bb[4]); hi.y = e4m3x2_to_bf16x2(bb[5]);
-            hi.z = e4m3x2_to_bf16x2(bb[6]); hi.w = e4m3x2_to_bf16x2(bb[7]);
-            *reinterpret_cast<uint4*>(dst + swz_off<16>(rr, 2 * c8)) = lo;
-            *reinterpret_cast<uint4*>(dst + swz_off<16>(rr, 2 * c8 + 1)) = hi;
-        }
-        __syncwarp();
-        kt = cvtw;
-        vt = cvtw + 16 * 256;
-    }
+    auto off = [](int r, int ch) -> uint32_t { return static_cast<uint32_t>(r * L::ROWP + ch * 16); };
     // S = Q K^T for the warp's 16 rows
     float acc[2][4];
     const uint32_t kb = smem_u32(kt);
+    if (KV8) {
+        qk_e4m3(kb, 0, qa, acc, lane);
+    } else {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+        for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
-        const int r = nt * 8 + (lane & 7);
+            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.f;
+            const int r = nt * 8 + (lane & 7);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kb + off(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
-            mma_bf16(acc[nt], qa[2 * kk], b0, b1);
-            mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+            for (int kk = 0; kk < 4; ++kk) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kb + off(r, 4 * kk + (lane >> 3)), b0, b1, b2, b3);
+                mma_bf16(acc[nt], qa[2 * kk], b0, b1);
+                mma_bf16(acc[nt], qa[2 * kk + 1], b2, b3);
+            }
         }
     }
     float vf[2][2];
@@ -162,7 +148,7 @@ __device__ __forceinline__ void attend_warp_rows(const uint8_t* ws, uint8_t* cvt
         float f0 = sc2, f1 = sc2;
         if (KV8) {
             f0 *= sks[r0]; f1 *= sks[r0 + 1];
-            vf[nt][0] = svs[r0]; vf[nt][1] = svs[r0 + 1];
+            vf[nt][0] = svs[r0] * pscale; vf[nt][1] = svs[r0 + 1] * pscale;
         } else {
             vf[nt][0] = vf[nt][1] = 1.f;
         }
@@ -199,6 +185,14 @@ __device__ __forceinline__ void attend_warp_rows(const uint8_t* ws, uint8_t* cvt
         s.o[n][2] *= alpha[1]; s.o[n][3] *= alpha[1];
     }
     uint32_t pa[4];
+    if (KV8) {
+        pa[0] = pack_f16(pr[0][0] * vf[0][0], pr[0][1] * vf[0][1]);
+        pa[1] = pack_f16(pr[0][2] * vf[0][0], pr[0][3] * vf[0][1]);
+        pa[2] = pack_f16(pr[1][0] * vf[1][0], pr[1][1] * vf[1][1]);
+        pa[3] = pack_f16(pr[1][2] * vf[1][0], pr[1][3] * vf[1][1]);
+        pv_e4m3(smem_u32(vt), 0, pa, s.o, lane);
+        return;
+    }
     pa[0] = pack_bf16(pr[0][0] * vf[0][0], pr[0][1] * vf[0][1]);
     pa[1] = pack_bf16(pr[0][2] * vf[0][0], pr[0][3] * vf[0][1]);
     pa[2] = pack_bf16(pr[1][0] * vf[1][0], pr[1][1] * vf[1][1]);
@@ -216,9 +210,12 @@ __device__ __forceinline__ void attend_warp_rows(const uint8_t* ws, uint8_t* cvt
 
 // Reduces the four warps' states to this CTA's per-head (max, sum) in cm/cl and its
 // unnormalized O (rescaled to that max) in red_o[H][D].  `slabs` (Layout::SLABS bytes)
-// must be free shared memory (the drained stages); wm/wl are [4][H] scratch.
+// must be free shared memory (the drained stages); wm/wl are [4][H] scratch.  e4m3: O is in
+// pv_e4m3's dim order and carries the factor 1 / `oscale`, both undone here.
+template <bool KV8>
 __device__ __forceinline__ void cta_reduce(const State& s, float* slabs, float* red_o, float (*wm)[H],
-                                           float (*wl)[H], float* cm, float* cl, int tid, int warp, int lane) {
+                                           float (*wl)[H], float* cm, float* cl, int tid, int warp, int lane,
+                                           float oscale) {
     const int g = lane >> 2, t = lane & 3;
     float l2[2] = {s.l2[0], s.l2[1]};
 #pragma unroll
@@ -236,15 +233,23 @@ __device__ __forceinline__ void cta_reduce(const State& s, float* slabs, float* 
     for (int hh = 0; hh < 2; ++hh) {
         const int h = g + 8 * hh;
         const float M = fmaxf(fmaxf(wm[0][h], wm[1][h]), fmaxf(wm[2][h], wm[3][h]));
-        f[hh] = (M == -INFINITY) ? 0.f : ex2(s.m2[hh] - M);
+        f[hh] = (M == -INFINITY) ? 0.f : ex2(s.m2[hh] - M) * oscale;
     }
     // each warp's rescaled O goes to its own padded slab, then the four are summed
     float* slab = slabs + warp * H * RP;
 #pragma unroll
     for (int n = 0; n < 16; ++n) {
-        const int d = 8 * n + 2 * t;
-        *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(s.o[n][0] * f[0], s.o[n][1] * f[0]);
-        *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(s.o[n][2] * f[1], s.o[n][3] * f[1]);
+        if (KV8) {                                       // pv_e4m3's dim order
+            const int d = 32 * (n >> 2) + 16 * ((n >> 1) & 1) + 4 * t + (n & 1);
+            slab[g * RP + d] = s.o[n][0] * f[0];
+            slab[g * RP + d + 2] = s.o[n][1] * f[0];
+            slab[(g + 8) * RP + d] = s.o[n][2] * f[1];
+            slab[(g + 8) * RP + d + 2] = s.o[n][3] * f[1];
+        } else {
+            const int d = 8 * n + 2 * t;
+            *reinterpret_cast<float2*>(&slab[g * RP + d]) = make_float2(s.o[n][0] * f[0], s.o[n][1] * f[0]);
+            *reinterpret_cast<float2*>(&slab[(g + 8) * RP + d]) = make_float2(s.o[n][2] * f[1], s.o[n][3] * f[1]);
+        }
     }
     __syncthreads();
     for (int i = tid; i < H * D / 4; i += NT) {            // 16-byte slab reads (RP * 4 B is a multiple of 16)
