@@ -292,10 +292,13 @@ __global__ void __launch_bounds__(NT, 1) prefill_lse_kernel(const __grid_constan
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
             if (KV8) {          // logit = (q . code) * key scale, exact in the oracle's terms
+                const float2 z = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int j = 0; j < 32; j += 4) {
                     const float4 c = *reinterpret_cast<const float4*>(kscale + j);
-                    v[j] *= c.x; v[j + 1] *= c.y; v[j + 2] *= c.z; v[j + 3] *= c.w;
+                    const float2 p0 = fma2(make_float2(v[j], v[j + 1]), make_float2(c.x, c.y), z);
+                    const float2 p1 = fma2(make_float2(v[j + 2], v[j + 3]), make_float2(c.z, c.w), z);
+                    v[j] = p0.x; v[j + 1] = p0.y; v[j + 2] = p1.x; v[j + 3] = p1.y;
                 }
             }
             if (key0 + 31 > p) {
@@ -420,7 +423,7 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
         if (KV8) {
             const float2 k2 = *reinterpret_cast<const float2*>(sc + 8 * j + 2 * (t & 3));
             vs = *reinterpret_cast<const float2*>(sc + KT + 8 * j + 2 * (t & 3));
-            c2 = make_float2(sc2 * k2.x, sc2 * k2.y);
+            c2 = fma2(s2, k2, make_float2(0.f, 0.f));
         }
         const float2 xa = fma2(make_float2(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1])), c2, na);
         const float2 xb = fma2(make_float2(__uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])), c2, nb);
@@ -431,8 +434,10 @@ __device__ __forceinline__ void p2_chunk(const uint32_t (&r)[32], uint32_t p_tad
             if (k0 + 1 > p) { pa.y = 0.f; pb.y = 0.f; }
         }
         if (KV8) {
-            pk[2 * j] = pack_bf16(pa.x * vs.x, pa.y * vs.y);
-            pk[2 * j + 1] = pack_bf16(pb.x * vs.x, pb.y * vs.y);
+            const float2 z = make_float2(0.f, 0.f);
+            const float2 qa = fma2(pa, vs, z), qb = fma2(pb, vs, z);
+            pk[2 * j] = pack_bf16(qa.x, qa.y);
+            pk[2 * j + 1] = pack_bf16(qb.x, qb.y);
         } else {
             pk[2 * j] = pack_bf16(pa.x, pa.y);
             pk[2 * j + 1] = pack_bf16(pb.x, pb.y);
