@@ -35,13 +35,23 @@ using sparse::Layout;
 using sparse::NT;
 using sparse::SUB;
 constexpr int kMaxSplits = 32;     // bound of the split count (shared-memory merge tables)
-constexpr int kCluster = 4;        // CTAs per query row in the cluster kernel
 constexpr int kWT = 16;            // selected entries per warp tile (cluster kernel)
-constexpr int kCW = 18;            // warps (= warp tiles) per CTA of the cluster kernel
-constexpr int kCEntries = kWT * kCW;               // 288 entries per CTA
-constexpr int kCNT = 32 * kCW;                     // 576 threads
-constexpr int kHPC = H / kCluster;                  // heads each CTA of a cluster finalizes
-static_assert(H % kCluster == 0, "the heads split evenly over a cluster");
+constexpr int kClusterEntries = 1152;              // entries a cluster covers (72 warp tiles)
+
+// Shape of the cluster kernel: NC CTAs per query row, each of 72 / NC warps.  Few rows take
+// 8 CTAs of 9 warps (two per SM: a row spread over more SMs); enough rows to fill the GPU
+// take 4 CTAs of 18 warps (one per SM: fewer CTAs for each row to wait on).
+template <int NC>
+struct CShape {
+    static constexpr int kCluster = NC;
+    static constexpr int kCW = kClusterEntries / kWT / NC;    // warps per CTA
+    static constexpr int kCEntries = kWT * kCW;               // entries per CTA
+    static constexpr int kCNT = 32 * kCW;                     // threads per CTA
+    static constexpr int kHPC = H / NC;                       // heads each CTA finalizes
+    static_assert(H % NC == 0 && kCW * NC * kWT == kClusterEntries, "the work splits evenly");
+};
+// rows up to which a launch takes the 8-CTA shape (8 x 18 CTAs fit one wave on 148 SMs)
+constexpr int kWideClusterRows = 18;
 
 struct Params {
     int rows, n_q, idx_stride, splits, chunk;
@@ -279,8 +289,9 @@ __global__ void __launch_bounds__(NT, sparse::MIN_CTAS) sparse_kernel(Params a) 
 // and after one cluster barrier CTA p finalizes those heads from its own memory.  Four
 // CTAs of 18 warps per row (one per SM) were faster than eight of 9 warps (two per SM):
 // 7.6 against 7.9 us per warm layer at 32 rows.
-template <bool KV8>
+template <bool KV8, int NC>
 struct CLayout {
+    static constexpr int kCluster = CShape<NC>::kCluster, kCW = CShape<NC>::kCW, kHPC = CShape<NC>::kHPC;
     static constexpr int ROWB = KV8 ? 128 : 256;          // bytes per gathered row
     static constexpr int RAW = 2 * kWT * ROWB;            // one warp's gathered K then V rows
     static constexpr int TILE = 2 * kWT * 256;            // one warp's bf16 K then V tiles (= RAW)
@@ -427,9 +438,11 @@ __device__ __forceinline__ void attend_warp_tile_e4m3(uint32_t kb, uint32_t vb, 
     }
 }
 
-template <bool KV8>
-__global__ void __launch_bounds__(kCNT, (kCNT <= 288 ? 2 : 1)) sparse_cluster_kernel(Params a) {
-    using CL = CLayout<KV8>;
+template <bool KV8, int NC>
+__global__ void __launch_bounds__(CShape<NC>::kCNT, (CShape<NC>::kCNT <= 288 ? 2 : 1)) sparse_cluster_kernel(Params a) {
+    using CL = CLayout<KV8, NC>;
+    constexpr int kCluster = CShape<NC>::kCluster, kCW = CShape<NC>::kCW, kCEntries = CShape<NC>::kCEntries;
+    constexpr int kCNT = CShape<NC>::kCNT, kHPC = CShape<NC>::kHPC;
     extern __shared__ uint8_t csm_raw[];
     uint8_t* csm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(csm_raw) + 127) & ~uintptr_t(127));
     uint8_t* qs = csm + CL::Q_OFF;                                    // [H][D] bf16, swz_off<16>
@@ -640,23 +653,28 @@ cudaError_t launch_impl(const SparseArgs& sa, cudaStream_t st) {
     a.status = sa.status;
     cudaError_t e;
     if (pl.cluster) {
-        const size_t sm = CLayout<KV8>::BYTES + 128;
-        e = cudaFuncSetAttribute(sparse_cluster_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(sm));
-        if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t cfg{};
-        cfg.gridDim = dim3(kCluster, sa.rows);
-        cfg.blockDim = dim3(kCNT);
-        cfg.dynamicSmemBytes = sm;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = kCluster;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        return cudaLaunchKernelEx(&cfg, sparse_cluster_kernel<KV8>, a);
+        auto launch = [&](auto shape) -> cudaError_t {
+            constexpr int NC = decltype(shape)::kCluster;
+            auto kern = sparse_cluster_kernel<KV8, NC>;
+            const size_t sm = CLayout<KV8, NC>::BYTES + 128;
+            cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   static_cast<int>(sm));
+            if (err != cudaSuccess) return err;
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3(NC, sa.rows);
+            cfg.blockDim = dim3(CShape<NC>::kCNT);
+            cfg.dynamicSmemBytes = sm;
+            cfg.stream = st;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = NC;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            return cudaLaunchKernelEx(&cfg, kern, a);
+        };
+        return sa.rows <= kWideClusterRows ? launch(CShape<8>{}) : launch(CShape<4>{});
     }
     const size_t sm = smem_bytes<KV8>(pl.chunk);
     e = cudaFuncSetAttribute(sparse_kernel<KV8>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
@@ -671,10 +689,10 @@ SparsePlan plan_sparse(int rows, int idx_stride) {
     SparsePlan pl;
     pl.cluster = false;
     // few rows: one cluster of kCluster CTAs per row, merged on chip
-    if (rows <= num_sms() && idx_stride <= kCluster * kCEntries) {
+    if (rows <= num_sms() && idx_stride <= kClusterEntries) {
         pl.cluster = true;
-        pl.splits = kCluster;
-        pl.chunk = kCEntries;
+        pl.splits = rows <= kWideClusterRows ? CShape<8>::kCluster : CShape<4>::kCluster;
+        pl.chunk = kClusterEntries / pl.splits;
         return pl;
     }
     // enough CTAs to cover the SMs twice; one CTA per row when rows alone do
