@@ -370,224 +370,7 @@ __global__ void __launch_bounds__(CNT, 5) cand_select_kernel(CandSelectArgs a) {
     if (tid == 0) a.cnt[row] = kg + nwin;
 }
 
-// ---------------------------------------------------------------- lists from importance rows
-// Rows whose importance sits in memory (decode calls): the same candidate lists, built by
-// many CTAs per row in three passes over slices of the rows.
-//   1. range: the largest and smallest importance of the row's candidates (the values are
-//      non-negative, so their bit patterns order like them; the minimum is kept as the
-//      maximum of the complement, so every slot starts at zero);
-//   2. fine bins: 2048 bins on the 11 bits right below the bits that the row's range shares,
-//      so a row whose importance is nearly uniform is still resolved;
-//   3. compaction: the highest fine bin f* with K keys at or above it, and every key of bins
-//      >= f* appended to the row's list (warp-aggregated offsets), with its coarse bin
-//      (imp_bin) counted for cand_select_kernel.
-// The list holds every key whose value reaches the floor of f*, and at least K keys do, so the
-// row's K best are in it, and the coarse counts of the list are exact from the coarse bin that
-// the K-th best falls in upwards -- what cand_select_kernel reads.
-constexpr int RNT = 256;
-constexpr int kFineBits = 11;
-constexpr int kFine = 1 << kFineBits;
-
-struct RowListArgs {
-    int rows, n_q;
-    const int32_t* q_pos0;
-    int64_t max_ctx;
-    int window, budget;
-    const float* scores;
-    int64_t score_ld;
-    int slice;                   // keys per CTA
-    uint32_t* range;             // [rows][2]: max of ~bits (the minimum), max of bits; zero on entry
-    uint32_t* fine;              // [rows][kFine] fine bins, zero on entry
-    uint32_t* hist;              // [rows][kImpBins] coarse bins of the list, zero on entry
-    int* cand_cnt;               // [rows][2], zero on entry
-    uint2* cand;                 // [rows][2][cand_seg]
-    int64_t cand_seg;
-    uint32_t* status;
-};
-
-__device__ __forceinline__ int row_candidates(const RowListArgs& a, int row, int& kg) {
-    const int b = row / a.n_q, r = row % a.n_q;
-    const int p = checked_pos(a.q_pos0[b] + r, a.max_ctx, a.status);
-    const int n_cand = max(0, p - a.window + 1);
-    kg = min(a.budget, n_cand);
-    return n_cand;
-}
-
-// fine-bin mapping of a row: digit = (bits >> shift) - base
-__device__ __forceinline__ void fine_map(const RowListArgs& a, int row, int& shift, uint32_t& base) {
-    const uint32_t lo = ~__ldcg(a.range + 2 * row), hi = __ldcg(a.range + 2 * row + 1);
-    const uint32_t diff = lo ^ hi;
-    const int top = diff ? 32 - __clz(static_cast<int>(diff)) : 0;          // differing low bits
-    shift = top > kFineBits ? top - kFineBits : 0;
-    base = lo >> shift;
-}
-
-template <typename F>
-__device__ __forceinline__ void for_slice(const float* s, int begin, int end, F f) {
-    for (int base = begin; base < end; base += 4 * RNT) {
-        float v[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = base + u * RNT + threadIdx.x;
-            v[u] = i < end ? __ldcg(s + i) : -1.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) f(base + u * RNT + threadIdx.x, v[u]);
-    }
-}
-
-__global__ void __launch_bounds__(RNT) row_range_kernel(RowListArgs a) {
-    const int row = blockIdx.y, lane = threadIdx.x & 31;
-    int kg;
-    const int n_cand = row_candidates(a, row, kg);
-    const int begin = blockIdx.x * a.slice, end = min(begin + a.slice, n_cand);
-    if (kg <= 0 || begin >= end) return;
-    uint32_t nlo = 0u, hi = 0u;                         // max of ~bits, max of bits
-    for_slice(a.scores + static_cast<size_t>(row) * a.score_ld, begin, end, [&](int, float v) {
-        if (v >= 0.f) { nlo = max(nlo, ~__float_as_uint(v)); hi = max(hi, __float_as_uint(v)); }
-    });
-    nlo = __reduce_max_sync(0xffffffffu, nlo);
-    hi = __reduce_max_sync(0xffffffffu, hi);
-    if (lane == 0) {
-        atomicMax(a.range + 2 * row, nlo);
-        atomicMax(a.range + 2 * row + 1, hi);
-    }
-}
-
-__global__ void __launch_bounds__(RNT) row_hist_kernel(RowListArgs a) {
-    __shared__ uint32_t h[kFine];
-    const int row = blockIdx.y, tid = threadIdx.x;
-    int kg;
-    const int n_cand = row_candidates(a, row, kg);
-    const int begin = blockIdx.x * a.slice, end = min(begin + a.slice, n_cand);
-    if (kg <= 0 || begin >= end) return;
-    for (int i = tid; i < kFine; i += RNT) h[i] = 0u;
-    int shift;
-    uint32_t base;
-    fine_map(a, row, shift, base);
-    __syncthreads();
-    for_slice(a.scores + static_cast<size_t>(row) * a.score_ld, begin, end, [&](int, float v) {
-        if (v >= 0.f) atomicAdd(&h[min((__float_as_uint(v) >> shift) - base, static_cast<uint32_t>(kFine - 1))], 1u);
-    });
-    __syncthreads();
-    for (int i = tid; i < kFine; i += RNT)
-        if (h[i]) atomicAdd(a.fine + static_cast<size_t>(row) * kFine + i, h[i]);
-}
-
-__global__ void __launch_bounds__(RNT) row_compact_kernel(RowListArgs a) {
-    __shared__ int s_part[RNT / 32];
-    __shared__ int s_fstar;
-    __shared__ uint32_t ch[kImpBins];
-    const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
-    int kg;
-    const int n_cand = row_candidates(a, row, kg);
-    const int begin = blockIdx.x * a.slice, end = min(begin + a.slice, n_cand);
-    if (kg <= 0 || begin >= end) return;
-    for (int i = tid; i < kImpBins; i += RNT) ch[i] = 0u;
-    // the cutoff fine bin: thread t sums bins 8t .. 8t + 7; suffix sums from the top
-    constexpr int PER = kFine / RNT;
-    const uint32_t* fr = a.fine + static_cast<size_t>(row) * kFine;
-    int hb[PER], mine = 0;
-#pragma unroll
-    for (int j = 0; j < PER; ++j) { hb[j] = static_cast<int>(__ldcg(fr + PER * tid + j)); mine += hb[j]; }
-    // suffix sums: within the warp from the higher lanes, then the totals of the higher warps
-    int suf = mine;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += y;
-    }
-    if (lane == 0) s_part[tid >> 5] = suf;               // the warp's total
-    if (tid == 0) s_fstar = 0;
-    __syncthreads();
-    int above = suf - mine;                              // bins of the threads above this one
-    for (int w = (tid >> 5) + 1; w < RNT / 32; ++w) above += s_part[w];
-    int cum = above, best = -1;
-#pragma unroll
-    for (int j = PER - 1; j >= 0; --j) {
-        if (best < 0 && cum + hb[j] >= kg) best = PER * tid + j;
-        cum += hb[j];
-    }
-    if (best >= 0) atomicMax(&s_fstar, best);
-    int shift;
-    uint32_t base;
-    fine_map(a, row, shift, base);
-    __syncthreads();
-    const uint32_t fstar = static_cast<uint32_t>(s_fstar);
-    uint2* list = a.cand + static_cast<size_t>(row) * 2 * a.cand_seg;
-    int* count = a.cand_cnt + 2 * row;
-    for_slice(a.scores + static_cast<size_t>(row) * a.score_ld, begin, end, [&](int i, float v) {
-        const bool take = v >= 0.f && min((__float_as_uint(v) >> shift) - base, static_cast<uint32_t>(kFine - 1)) >= fstar;
-        const uint32_t m = __ballot_sync(0xffffffffu, take);
-        if (m == 0u) return;
-        int off = 0;
-        if (lane == __ffs(m) - 1) off = atomicAdd(count, __popc(m));
-        off = __shfl_sync(0xffffffffu, off, __ffs(m) - 1) + __popc(m & ((1u << lane) - 1u));
-        if (take) {
-            atomicAdd(&ch[imp_bin(v)], 1u);
-            if (off < a.cand_seg) list[off] = make_uint2(__float_as_uint(v), static_cast<uint32_t>(i));
-        }
-    });
-    __syncthreads();
-    for (int i = tid; i < kImpBins; i += RNT)
-        if (ch[i]) atomicAdd(a.hist + static_cast<size_t>(row) * kImpBins + i, ch[i]);
-}
-
 }  // namespace
-
-size_t row_select_ws_bytes(int rows, int64_t max_ctx) {
-    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t r = static_cast<size_t>(rows);
-    return al(sizeof(uint32_t) * 2 * r) + al(sizeof(uint32_t) * r * kFine) + al(sizeof(uint32_t) * r * kImpBins) +
-           al(sizeof(int) * 2 * r) + al(sizeof(uint2) * r * 2 * static_cast<size_t>(max_ctx > 0 ? max_ctx : 1));
-}
-
-cudaError_t launch_row_select(const SelectArgs& sa, void* ws, cudaStream_t st) {
-    if (sa.rows <= 0) return cudaSuccess;
-    if (sa.budget > kFusedSelectMaxBudget || sa.block_size != 1) return cudaErrorInvalidValue;
-    auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-    const size_t r = static_cast<size_t>(sa.rows);
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    RowListArgs a{};
-    a.rows = sa.rows; a.n_q = sa.n_q; a.q_pos0 = sa.q_pos0; a.max_ctx = sa.max_ctx;
-    a.window = sa.window; a.budget = sa.budget; a.scores = sa.scores; a.score_ld = sa.score_ld;
-    a.range = reinterpret_cast<uint32_t*>(w);
-    w += al(sizeof(uint32_t) * 2 * r);
-    a.fine = reinterpret_cast<uint32_t*>(w);
-    w += al(sizeof(uint32_t) * r * kFine);
-    a.hist = reinterpret_cast<uint32_t*>(w);
-    w += al(sizeof(uint32_t) * r * kImpBins);
-    a.cand_cnt = reinterpret_cast<int*>(w);
-    w += al(sizeof(int) * 2 * r);
-    a.cand = reinterpret_cast<uint2*>(w);
-    a.cand_seg = sa.max_ctx > 0 ? sa.max_ctx : 1;
-    a.status = sa.status;
-    // slices: about two CTAs per SM over all rows, at least 4096 keys each
-    const int64_t n_max = sa.max_ctx - sa.window > 0 ? sa.max_ctx - sa.window : 1;
-    int64_t slices = (2 * static_cast<int64_t>(num_sms()) + sa.rows - 1) / sa.rows;
-    const int64_t cap_slices = (n_max + 4095) / 4096;
-    if (slices > cap_slices) slices = cap_slices;
-    if (slices < 1) slices = 1;
-    if (slices > 65535) slices = 65535;
-    a.slice = static_cast<int>((n_max + slices - 1) / slices);
-    a.slice = (a.slice + 4 * RNT - 1) / (4 * RNT) * (4 * RNT);
-    slices = (n_max + a.slice - 1) / a.slice;
-    // range, bins and counts (adjacent) start at zero: one memset on the stream
-    cudaError_t e = cudaMemsetAsync(a.range, 0, reinterpret_cast<uint8_t*>(a.cand) - reinterpret_cast<uint8_t*>(a.range), st);
-    if (e != cudaSuccess) return e;
-    const dim3 grid(static_cast<unsigned>(slices), static_cast<unsigned>(sa.rows));
-    row_range_kernel<<<grid, RNT, 0, st>>>(a);
-    row_hist_kernel<<<grid, RNT, 0, st>>>(a);
-    row_compact_kernel<<<grid, RNT, 0, st>>>(a);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    CandSelectArgs cs{};
-    cs.rows = sa.rows; cs.n_q = sa.n_q; cs.q_pos0 = sa.q_pos0; cs.max_ctx = sa.max_ctx;
-    cs.window = sa.window; cs.budget = sa.budget; cs.idx_stride = sa.idx_stride;
-    cs.hist = a.hist; cs.cand_cnt = a.cand_cnt; cs.cand = a.cand; cs.cand_seg = a.cand_seg;
-    cs.idx = sa.idx; cs.cnt = sa.cnt; cs.status = sa.status;
-    return launch_cand_select(cs, st);
-}
 
 cudaError_t launch_cand_select(const CandSelectArgs& in, cudaStream_t st) {
     if (in.rows <= 0) return cudaSuccess;

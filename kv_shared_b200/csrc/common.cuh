@@ -150,6 +150,11 @@ __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, boo
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
                  ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 16 : 0) : "memory");
 }
+// 4-byte copy (for 4-byte-aligned sources); zero-filled when !valid
+__device__ __forceinline__ void cp_async4_zfill(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(valid ? 4 : 0) : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
@@ -277,6 +282,20 @@ __device__ __forceinline__ int imp_bin(float v) {
 // smallest value of bin b (0 for bin 0)
 __device__ __forceinline__ float imp_bin_floor(int b) {
     return b <= 0 ? 0.f : __uint_as_float(static_cast<uint32_t>(b + kImpBinBase) << (23 - kImpSub));
+}
+
+// Bin of a decode row's importance for its selection histogram: the fp32 bit pattern's top
+// bits (exponent and kDecHistShift's leading mantissa bits; values are non-negative, so the
+// bins order like the values), clamped into the histogram.
+constexpr int kDecHistShift = 21;                           // 4 bins per octave
+constexpr int kDecHistBins = 1 << (31 - kDecHistShift);     // every non-negative fp32 value
+constexpr int kDecFineBits = 11;                            // refinement of a cutoff bin
+constexpr int kDecFineBins = 1 << kDecFineBits;
+constexpr int kDecFineShift = kDecHistShift - kDecFineBits;
+constexpr int kDecHistRow = kDecHistBins + kDecFineBins;    // a row's coarse then fine counts
+__device__ __forceinline__ int dec_bin(uint32_t bits) {
+    const uint32_t b = bits >> kDecHistShift;
+    return b < static_cast<uint32_t>(kDecHistBins) ? static_cast<int>(b) : kDecHistBins - 1;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;

@@ -57,7 +57,38 @@ struct Params {
     float* scores;                  // [B][score_ld]
     int64_t score_ld;
     uint32_t* status;
+    int window;                     // candidates of a row for the selection: keys [0, p - window]
+    int* ghist;                     // [B][kDecHistRow] selection histogram (coarse, fine), or null
+    int* gctl;                      // [B][4] selection counters (zeroed with the histogram)
 };
+
+// Zeroes row b's selection histogram and counters (n threads from thread t), before any CTA
+// adds to them; each thread's stores are made visible before it goes on.
+__device__ __forceinline__ void zero_select_state(const Params& a, int b, int t, int n) {
+    for (int i = t; i < kDecHistRow; i += n) a.ghist[static_cast<size_t>(b) * kDecHistRow + i] = 0;
+    if (t < 4) a.gctl[4 * b + t] = 0;
+    __threadfence();
+}
+
+// Counts the candidate keys among a thread's four importance values into the shared-memory
+// histogram hs (keys below c_end = p - window + 1; valid[e] marks keys that exist).
+__device__ __forceinline__ void count_candidates(int* hs, const float (&sc)[4], const int (&key)[4],
+                                                 const bool (&valid)[4], int c_end) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        if (valid[e] && key[e] < c_end) atomicAdd(&hs[dec_bin(__float_as_uint(sc[e]))], 1);
+}
+
+// Adds a CTA's shared-memory histogram to row b's and clears it (threads t, t + n, ...).
+__device__ __forceinline__ void flush_hist(const Params& a, int* hs, int b, int t, int n) {
+    for (int i = t; i < kDecHistBins; i += n) {
+        const int c = hs[i];
+        if (c) {
+            atomicAdd(a.ghist + static_cast<size_t>(b) * kDecHistRow + i, c);
+            hs[i] = 0;
+        }
+    }
+}
 
 template <bool KV8>
 struct Layout {
@@ -110,6 +141,7 @@ __global__ void __launch_bounds__(NT) dec_qk_kernel(const __grid_constant__ CUte
         for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
+    if (a.ghist && split == 0) zero_select_state(a, b, tid, NT);   // dec_pv adds to it
     __syncthreads();
 
     auto issue = [&](int i, int s) {
@@ -258,6 +290,7 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
     uint8_t* smem = align1024(smem_raw);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE);
     float4* red_o4 = reinterpret_cast<float4*>(smem);              // [4][16][32] after the tiles
+    __shared__ int hs[kDecHistBins];                               // this CTA's selection counts
 
     const int b = blockIdx.y, split = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, g = lane >> 2, t = lane & 3;
@@ -272,6 +305,8 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
         for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
+    for (int i = tid; i < kDecHistBins; i += NT) hs[i] = 0;
+    const int c_end = p - a.window + 1;
     __syncthreads();
 
     auto issue = [&](int i, int s) {
@@ -421,6 +456,8 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
                 mma_bf16(o[2 * c + 1], pa, b2, b3);
             }
         }
+        // selection counts, after the MMAs so that they stay off the tile's path
+        if (a.ghist && g == 0) count_candidates(hs, sc, {kl, kl + 1, kh, kh + 1}, {v0, v1, v2, v3}, c_end);
         if (__syncthreads_or(!ok)) break;
         if (tid == 0 && i + STAGES < n_tiles) issue(i + STAGES, s);
     }
@@ -458,6 +495,7 @@ __global__ void __launch_bounds__(NT) dec_pv_kernel(const __grid_constant__ CUte
             *reinterpret_cast<float2*>(my + (h + 8) * D + d) = make_float2(sum.z, sum.w);
         }
     }
+    if (a.ghist) flush_hist(a, hs, b, tid, NT);      // every warp's counts are in (barriers above)
 }
 
 // O = sum of the split partials: CTA (row, group) = (blockIdx.x / 8, blockIdx.x % 8) takes
@@ -523,7 +561,7 @@ struct FusedLayout {
     // and read a stale tile.  An even depth keeps every stage within one group.
     static_assert(FS % 2 == 0, "the ring depth must be even (stage parity per consumer group)");
     static constexpr size_t VSC = KV8 ? kFusedMaxTiles * TILE * 4 : 0;   // V scales of the split
-    static constexpr size_t BYTES = 1024 + FS * Layout<KV8>::RAW + 2 * FS * 8 + 8 * H * D * 4 + VSC;
+    static constexpr size_t BYTES = 1024 + FS * Layout<KV8>::RAW + 2 * FS * 8 + 8 * H * D * 4 + VSC + kDecHistBins * 4;
 };
 
 __device__ __forceinline__ void bar_sync(int id, int n) {
@@ -563,6 +601,7 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
     uint64_t* empty = full + FS;
     float4* red_o4 = reinterpret_cast<float4*>(empty + FS);          // [8][16][32] O partials
     float* vsm = reinterpret_cast<float*>(red_o4 + 8 * 16 * 32);      // [64 tiles][64] (e4m3)
+    int* hs = reinterpret_cast<int*>(vsm + (KV8 ? kFusedMaxTiles * TILE : 0));   // selection counts
     __shared__ float red_m[8][H], red_l[8][H], red_v[8];
     __shared__ float2 lse_part[FCONS / H][H];
     __shared__ float lse_s[H];
@@ -589,6 +628,7 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
         fence_mbar_init();
         s_abort = 0;
     }
+    for (int i = tid; i < kDecHistBins; i += FNT) hs[i] = 0;
     umma::fence_before();
     __syncthreads();
     umma::fence_after();
@@ -646,11 +686,24 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[ld % FS]);
         };
+        // the selection state of this CTA's sequences is zeroed here, each split taking its share
+        // of every one of them: a split adds to a sequence's histogram only after that
+        // sequence's exchange, which every split reaches after this
+        if (a.ghist) {
+            for (int w = 0; w < nw; ++w) {
+                const int b = w * wb + group;
+                const int lo = split * kDecHistRow / a.splits, hi = (split + 1) * kDecHistRow / a.splits;
+                for (int i = lo + tid; i < hi; i += FCONS) a.ghist[static_cast<size_t>(b) * kDecHistRow + i] = 0;
+                if (split == 0 && tid < 4) a.gctl[4 * b + tid] = 0;
+            }
+            __threadfence();
+        }
         uint32_t wbase = 0;                       // loads of the earlier waves
         for (int w = 0; w < nw; ++w) {
             const int b = w * wb + group;
             int k_end;
             const int n_tiles = tiles_of(w, k_end);
+            const int c_end = checked_pos(a.q_pos0[b], a.max_ctx, nullptr) - a.window + 1;
 
             // ---- pass A: logits to tensor memory, running (max, sum) per head.  e4m3 keys:
             // f16 MMAs straight from the raw tile (Q in f16, k order permuted, scaled by
@@ -664,23 +717,28 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
             const float* ksc = KV8 ? a.k_scale + b * a.cap : nullptr;
             const float* vsc = KV8 ? a.v_scale + b * a.cap : nullptr;
             // e4m3: lane l of a warp holds the key scale (l < 16) or the V scale (l >= 16) of
-            // key l % 16 of its 16 keys of a tile: one coalesced load per tile, issued four of the
-            // group's tiles ahead so that the memory latency stays off the tile's path.  The V
-            // scales also go to shared memory for pass B (the same warp reads them back).
-            auto load_sc = [&](int i) -> float {
+            // key l % 16 of its 16 keys of a tile, copied asynchronously into the warp's ring of
+            // 8 slots (in the O-partial area, free during pass A) four of the group's tiles
+            // ahead, so that the memory latency stays off the tile's path.  The V scales also
+            // go to shared memory for pass B (the same warp reads them back).
+            float* sc_ring = reinterpret_cast<float*>(red_o4) + warp * 8 * 32;
+            auto issue_sc = [&](int i) {
                 const int key = k_begin + i * TILE + q * 16 + (lane & 15);
-                return (i < n_tiles && key < k_end) ? __ldg((lane < 16 ? ksc : vsc) + key) : 0.f;
+                const bool valid = i < n_tiles && key < k_end;
+                cp_async4_zfill(sc_ring + ((i >> 1) & 7) * 32 + lane, valid ? (lane < 16 ? ksc : vsc) + key : ksc,
+                                valid);
+                cp_async_commit();
             };
-            float sc_p[4] = {0.f, 0.f, 0.f, 0.f};
             if (KV8)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) sc_p[j] = load_sc(c + 2 * j);
+                for (int j = 0; j < 4; ++j) issue_sc(c + 2 * j);
             for (int i = c; i < n_tiles; i += 2) {
                 const uint32_t ld = wbase + i;
-                const float sc_cur = sc_p[0];
+                float sc_cur = 0.f;
                 if (KV8) {
-                    sc_p[0] = sc_p[1]; sc_p[1] = sc_p[2]; sc_p[2] = sc_p[3];
-                    sc_p[3] = load_sc(i + 8);
+                    issue_sc(i + 8);
+                    cp_async_wait<4>();
+                    sc_cur = sc_ring[((i >> 1) & 7) * 32 + lane];
                     if (lane >= 16) {
                         vmax = fmaxf(vmax, sc_cur);
                         vsm[i * TILE + q * 16 + (lane & 15)] = sc_cur;
@@ -746,6 +804,7 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                 release(ld);
             }
             umma::tmem_st_wait();
+            if (KV8) asm volatile("cp.async.wait_all;" ::: "memory");   // the ring is O-partial space again
             // ---- exchange: publish this split's (max, sum), wait for the other splits
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -901,6 +960,8 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                             mma_bf16(o[2 * cv + 1], pa, b2, b3);
                         }
                     }
+                    // selection counts, after the MMAs so that they stay off the tile's path
+                    if (a.ghist && g == 0) count_candidates(hs, sc, {kl, kl + 1, kh, kh + 1}, {v0, v1, v2, v3}, c_end);
                 }
                 release(ld);
             }
@@ -939,6 +1000,7 @@ __global__ void __launch_bounds__(FNT, 1) dec_fused_kernel(const __grid_constant
                 }
             }
             bar_sync(3, FCONS);
+            if (a.ghist) flush_hist(a, hs, b, tid, FCONS);   // the next wave's counts start after its exchange
             if (tid == 0 && !s_abort) {
                 __threadfence();                  // the CTA's partial, ordered by the barrier
                 atomicAdd(&cnt_o[b], 1);
@@ -1025,6 +1087,9 @@ cudaError_t launch_impl(const DecodeArgs& da, cudaStream_t st) {
     a.lse = da.lse;
     a.scores = da.scores; a.score_ld = da.score_ld;
     a.status = da.status;
+    a.window = da.window;
+    a.ghist = da.sel.hist;
+    a.gctl = da.sel.ctl;
 
     CUtensorMap kmap, vmap, smap;
     const uint64_t rows = static_cast<uint64_t>(da.batch) * da.cap;

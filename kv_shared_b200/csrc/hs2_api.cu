@@ -104,10 +104,11 @@ bool fused_prefill_select(const hs2_attn_desc* d, Path path) {
     return path == Path::TC && d->n_q > 1 && d->budget <= kFusedSelectMaxBudget;
 }
 
-// decode on tensor cores selects long rows through candidate lists built from its importance
-// rows (shorter ones fit the cluster select's shared memory, which is faster for them)
-bool list_decode_select(const hs2_attn_desc* d, Path path) {
-    return path == Path::TC && d->n_q == 1 && d->budget <= kFusedSelectMaxBudget && d->max_ctx >= kListSelectMinCtx;
+// decode on tensor cores selects long rows from the histograms its attention kernels build
+// while they write the importance rows (budgets up to kFusedSelectMaxBudget); shorter rows
+// fit the cluster select's shared memory, which is faster for them
+bool hist_decode_select(const hs2_attn_desc* d, Path path) {
+    return path == Path::TC && d->n_q == 1 && d->budget <= kFusedSelectMaxBudget && d->max_ctx >= kHistSelectMinCtx;
 }
 
 // bytes after the status block needed by hs2_full_attn_select
@@ -117,7 +118,7 @@ size_t full_region(const hs2_attn_desc* d, Path path, bool scores_in_ws) {
     size_t n = 0;
     if (path == Path::TC && d->n_q == 1)
         n += a256(decode_ws_bytes(d->batch, d->max_ctx, d->kv_dtype == HS2_E4M3)) +
-             (list_decode_select(d, path) ? a256(row_select_ws_bytes(d->batch, d->max_ctx)) : 0);
+             (hist_decode_select(d, path) ? a256(dec_select_ws_bytes(d->batch, d->budget)) : 0);
     if (path == Path::TC && d->n_q > 1) n += a256(prefill_ws_bytes(d->batch, d->n_q, d->max_ctx, fused, d->kv_dtype == HS2_E4M3));
     if (scores_in_ws && !fused) n += a256(sizeof(float) * rows * static_cast<size_t>(score_pitch(d)));
     return n;
@@ -172,13 +173,13 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     int64_t score_ld = desc->max_ctx;
     size_t used = 0;
     const bool fused = fused_prefill_select(desc, path);
-    const bool list_sel = list_decode_select(desc, path);
-    uint8_t* sel_ws = nullptr;                           // decode: bins, counts, candidate lists
+    const bool hist_sel = hist_decode_select(desc, path);
+    DecSelState sel{};                                   // decode: histograms, counters, lists
     if (path == Path::TC && desc->n_q == 1) {
         used = a256(decode_ws_bytes(desc->batch, desc->max_ctx, kv8));
-        if (list_sel) {
-            sel_ws = region + used;
-            used += a256(row_select_ws_bytes(desc->batch, desc->max_ctx));
+        if (hist_sel) {
+            sel = dec_select_state(region + used, desc->batch, desc->budget);
+            used += a256(dec_select_ws_bytes(desc->batch, desc->budget));
         }
     } else if (path == Path::TC) {
         used = a256(prefill_ws_bytes(desc->batch, desc->n_q, desc->max_ctx, fused, kv8));
@@ -214,6 +215,7 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
         a.q = q; a.k = k; a.v = v; a.k_scale = k_scale; a.v_scale = v_scale; a.kv8 = kv8;
         a.scale = scale; a.o = o; a.lse = lse; a.scores = score_buf; a.score_ld = score_ld;
         a.ws = region; a.status = status;
+        a.window = desc->window; a.sel = sel;
         e = launch_decode_full(a, st);
     }
     if (e != cudaSuccess) return HS2_ERR_CUDA;
@@ -221,14 +223,22 @@ hs2_status hs2_full_attn_select(const hs2_attn_desc* desc, const void* q, const 
     sa.rows = desc->batch * desc->n_q; sa.n_q = desc->n_q; sa.q_pos0 = q_pos0; sa.max_ctx = desc->max_ctx;
     sa.scores = score_buf; sa.score_ld = score_ld; sa.window = desc->window; sa.budget = desc->budget;
     sa.block_size = 1; sa.idx_stride = desc->idx_stride; sa.idx = idx; sa.cnt = cnt; sa.status = status;
-    if (list_sel) return from_cuda(launch_row_select(sa, sel_ws, st));
+    if (hist_sel) {
+        HistSelectArgs ha{};
+        ha.rows = desc->batch; ha.q_pos0 = q_pos0; ha.max_ctx = desc->max_ctx;
+        ha.window = desc->window; ha.budget = desc->budget; ha.idx_stride = desc->idx_stride;
+        ha.scores = score_buf; ha.score_ld = score_ld;
+        ha.hist = sel.hist; ha.ctl = sel.ctl; ha.above = sel.above; ha.tie = sel.tie;
+        ha.idx = idx; ha.cnt = cnt; ha.status = status;
+        return from_cuda(launch_hist_select(ha, st));
+    }
     return from_cuda(launch_select(sa, st));
 }
 
 int32_t hs2_full_attn_launches(const hs2_attn_desc* desc) {
     Path path;
     if (check_desc(desc, &path) != HS2_OK) return 0;
-    int32_t n = list_decode_select(desc, path) ? 4 : 1;   // the selection (decode: range, bins, lists, top-K)
+    int32_t n = 1;                                      // the selection
     if (path == Path::F32) n += 1;
     else if (desc->n_q > 1) n += 2;                     // prefill: log-sum-exp pass, output pass
     else n += plan_decode(desc->batch, desc->max_ctx, desc->kv_dtype == HS2_E4M3).fused ? 1 : 3;  // or: 2 passes + merge

@@ -30,6 +30,45 @@ struct DecodePlan {
 DecodePlan plan_decode(int batch, int64_t max_ctx, bool kv8);
 size_t decode_ws_bytes(int batch, int64_t max_ctx, bool kv8);   // logits + partials + counters
 
+// Token-level selection of a decode call (budget <= kFusedSelectMaxBudget): the attention
+// kernels count the candidate importances of each row into a histogram (bins dec_bin, built in
+// shared memory and added per CTA), and launch_hist_select takes the row's K best from the
+// bins above the cutoff bin and the best of that bin.  The histogram and the counters of a row
+// are zeroed by the attention kernels before they add to them.
+constexpr int kDecTieCap = 4096;          // cutoff-bin keys kept per row (more: passes over the row)
+struct DecSelState {
+    int* hist;                            // [B][kDecHistRow]: coarse bins, then the refinement's fine bins
+    int* ctl;                             // [B][4]: keys above the cutoff class, keys of it, CTAs done,
+                                          //         CTAs past the refinement count
+    int* above;                           // [B][budget] positions above the cutoff bin
+    unsigned long long* tie;              // [B][kDecTieCap] (importance bits, ~position)
+};
+size_t dec_select_ws_bytes(int batch, int budget);
+DecSelState dec_select_state(void* ws, int batch, int budget);
+// Rows at least this long take the histogram selection; shorter ones the cluster select of
+// launch_select, which holds them in shared memory (faster there than the histogram's
+// counting inside the attention kernel and its passes over the rows).
+constexpr int64_t kHistSelectMinCtx = 16 * 24576 + 1;
+
+struct HistSelectArgs {
+    int rows;                             // = batch (one query row per sequence)
+    const int32_t* q_pos0;
+    int64_t max_ctx;
+    int window, budget, idx_stride;
+    const float* scores;                  // [rows][score_ld]
+    int64_t score_ld;
+    int* hist;
+    int* ctl;
+    int* above;
+    unsigned long long* tie;
+    int slice;                            // keys per CTA (set by launch_hist_select)
+    bool vec4;                            // rows 16-byte aligned: float4 loads (set there too)
+    int32_t* idx;
+    int32_t* cnt;
+    uint32_t* status;
+};
+cudaError_t launch_hist_select(const HistSelectArgs& a, cudaStream_t st);
+
 struct DecodeArgs {
     int batch;
     int64_t cap;
@@ -48,6 +87,8 @@ struct DecodeArgs {
     int64_t score_ld;
     void* ws;                 // decode scratch (decode_ws_bytes)
     uint32_t* status;
+    int window;               // candidates of a row: keys [0, p - window]
+    DecSelState sel;          // selection histogram and counters (hist null: none built)
 };
 cudaError_t launch_decode_full(const DecodeArgs& a, cudaStream_t st);
 
@@ -114,14 +155,6 @@ struct SelectArgs {
 };
 cudaError_t launch_select(const SelectArgs& a, cudaStream_t st);
 
-// Token-level selection (block_size 1, budget <= kFusedSelectMaxBudget) from importance rows
-// through candidate lists: range, histogram and compaction passes over slices of every row,
-// then cand_select.  Scratch: row_select_ws_bytes (range, bins, counts, lists).  Decode calls
-// use it for rows longer than launch_select's clusters hold in shared memory (16 CTAs x 24576
-// keys): launch_select streams such rows from global memory twice, with few CTAs per row.
-constexpr int64_t kListSelectMinCtx = 16 * 24576 + 1;
-size_t row_select_ws_bytes(int rows, int64_t max_ctx);
-cudaError_t launch_row_select(const SelectArgs& a, void* ws, cudaStream_t st);
 
 // ---------------------------------------------------------------- sparse attention
 struct SparsePlan {

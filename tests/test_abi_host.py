@@ -66,7 +66,7 @@ def test_full_attn_launch_count(L):
     # the merge of the split partials) plus the selection through candidate lists (range,
     # bins, lists, top-K)
     assert hs.hs2_full_attn_launches(_desc(batch=32, max_ctx=131072)) == 2
-    assert hs.hs2_full_attn_launches(_desc(batch=4, max_ctx=1 << 20, kv_dtype=hs.HS2_E4M3)) == 7
+    assert hs.hs2_full_attn_launches(_desc(batch=4, max_ctx=1 << 20, kv_dtype=hs.HS2_E4M3)) == 4
     assert hs.hs2_full_attn_launches(_desc(batch=4, n_q=8192, max_ctx=65536 + 8192)) == 3
     f32 = _desc(heads=8, head_dim=64, q_dtype=hs.HS2_F32, kv_dtype=hs.HS2_F32, n_q=64, max_ctx=64)
     assert hs.hs2_full_attn_launches(f32) == 2

@@ -220,9 +220,8 @@ def test_decode_1m_fp8_full_size_sampled():
     _block_parity(synth.DECODE_1M_FP8, seed=1004, seqs=[3], device="cuda")
 
 
-def test_decode_long_rows_list_select():
-    # rows longer than the cluster select holds in shared memory take the candidate-list
-    # selection (range, fine bins, lists, top-K); ragged positions put short rows, rows
+def test_decode_long_rows_ragged():
+    # long rows (more splits than one wave's share) with ragged positions: short rows, rows
     # below the window and rows with fewer candidates than the budget in the same call
     wl = synth.shrink(synth.DECODE_128K, batch=6, ctx=400000, needles=16)
     pos0 = np.array([0, 100, 1151, 5000, 393300, wl.ctx - 1])
@@ -231,7 +230,7 @@ def test_decode_long_rows_list_select():
 
 def test_decode_long_rows_all_equal_importance():
     # zero keys: every logit 0 and every importance equal, so the lowest positions win; the
-    # whole row lands in one bin of the list selection, which narrows it in global memory
+    # whole row lands in one bin of the selection histogram, narrowed over the row in memory
     from hs2_check import check_selection
     T = 400000
     g = torch.Generator(device="cuda")
