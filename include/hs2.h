@@ -107,7 +107,9 @@ typedef struct {
  * Workspace bytes the three attention calls need for `desc` (the largest of the
  * three).  Decode (n_q = 1) and f32 descriptions select from importance rows: if
  * `scores_in_workspace` is non-zero they are kept in the workspace
- * ([batch][n_q][max_ctx] fp32) when the caller passes no scores buffer.  Prefill
+ * ([batch][n_q][max_ctx] fp32) when the caller passes no scores buffer.  Decode
+ * descriptions with max_ctx > 393216 and budget <= 4096 also hold the selection's
+ * per-sequence histograms and lists (about 45 KB + 4 * budget bytes per sequence).  Prefill
  * on the tensor-core path (n_q > 1, budget <= 4096) selects from candidate lists
  * that its second pass streams into the workspace (room for max_ctx + 128
  * (importance, position) pairs of 8 bytes per query row; in practice a few
