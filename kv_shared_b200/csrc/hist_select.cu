@@ -28,10 +28,10 @@ namespace hs2 {
 namespace {
 
 constexpr int HNT = 256;
-constexpr int kSortBuckets = 4096;            // buckets of the final counting sort
 constexpr int HWARPS = HNT / 32;
-constexpr int kBinsPerThread = kDecHistBins / HNT;
-static_assert(kDecHistBins % HNT == 0, "bins split evenly over the threads");
+constexpr int kSortBuckets = 4096;            // buckets of the final counting sort
+static_assert(kDecHistBins % HNT == 0 && kDecFineBins % HNT == 0 && kSortBuckets % HNT == 0,
+              "bins and buckets split evenly over the threads");
 
 struct HSmem {
     int wsum[HWARPS];
