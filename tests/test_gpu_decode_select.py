@@ -100,6 +100,10 @@ def test_e4m3_single_launch():
     _run("normal", 4, 300000, kv=hs.HS2_E4M3, seed=5)
 
 
+def test_e4m3_single_launch_long_rows():
+    _run("normal", 2, 450000, kv=hs.HS2_E4M3, seed=9)   # one launch, histogram selection
+
+
 def test_e4m3_two_kernel_path():
     _run("normal", 2, 1 << 20, kv=hs.HS2_E4M3, seed=6)
 
