@@ -63,14 +63,25 @@ def test_workspace_size_valid_and_invalid(L):
 def test_full_attn_launch_count(L):
     # host-side plan: decode contexts whose splits fit tensor memory take one launch plus
     # the selection; longer ones (1M keys: more than 148 x 4096) take three (two passes and
-    # the merge of the split partials) plus the selection through candidate lists (range,
-    # bins, lists, top-K)
+    # the merge of the split partials) plus the selection (one launch either way: the cluster
+    # select for rows up to 393216 keys, the selection from the histograms beyond)
     assert hs.hs2_full_attn_launches(_desc(batch=32, max_ctx=131072)) == 2
+    assert hs.hs2_full_attn_launches(_desc(batch=2, max_ctx=450000)) == 2
     assert hs.hs2_full_attn_launches(_desc(batch=4, max_ctx=1 << 20, kv_dtype=hs.HS2_E4M3)) == 4
     assert hs.hs2_full_attn_launches(_desc(batch=4, n_q=8192, max_ctx=65536 + 8192)) == 3
     f32 = _desc(heads=8, head_dim=64, q_dtype=hs.HS2_F32, kv_dtype=hs.HS2_F32, n_q=64, max_ctx=64)
     assert hs.hs2_full_attn_launches(f32) == 2
     assert hs.hs2_full_attn_launches(_desc(head_dim=96)) == 0
+
+
+def test_long_decode_workspace_holds_the_selection_state(L):
+    # rows of 393217 keys and more select from per-sequence histograms and lists in the
+    # workspace: 3072 counts, 4 counters, `budget` positions and 4096 8-byte keys per sequence
+    short = hs.hs2_workspace_size(_desc(batch=2, max_ctx=393216), False)
+    long_ = hs.hs2_workspace_size(_desc(batch=2, max_ctx=393217), False)
+    per_seq = 3072 * 4 + 4 * 4 + 1024 * 4 + 4096 * 8
+    assert long_ - short >= 2 * per_seq
+    assert long_ - short < 2 * per_seq + 8192
 
 
 def test_null_and_misaligned_arguments_are_rejected(L):
